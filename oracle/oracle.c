@@ -1,0 +1,260 @@
+/*
+ * FP64 CPU oracle for the W4A16 weight-only linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library; the product path (the
+ * CUDA library and its Python binding) never calls it and shares no code with
+ * it.  It is deliberately plain and slow: one straightforward loop per step of
+ * the method, every floating-point decision in binary64, rows spread over
+ * OpenMP threads and nothing else.
+ *
+ * What it computes (source pages, by title and section):
+ *  - "Axe Corsa 28B" model card, "How the Compression Works": asymmetric INT4,
+ *    each group of 128 consecutive weights has its own scale and zero point,
+ *    all 16 levels used; dequantisation w_hat = (q - z_g) * s_g with s_g a
+ *    BF16 scale and z_g an INT32 zero point ("What the Tensor Types Tell You");
+ *    activations stay BF16 and the dequantised weights feed the multiply.
+ *  - "Quantization I: int8, int4, the basics", Concept: round to a scale, a
+ *    zero point shifts the grid, clipping maps extremes to the boundary; the
+ *    products accumulate in higher precision.
+ *
+ * The forward quantisation formula did not survive in the pages' text; the
+ * reading implemented here is the plainest one the prose supports (min/max
+ * affine):
+ *   lo = min w, hi = max w over the group (FP32 compares)
+ *   s  = bf16_rne((hi - lo) / 15)                (difference and quotient in binary64)
+ *        if s == 0: s = bf16_rne(max(|lo|, |hi|)); if still 0: s = 1
+ *   z  = rint(-lo / s)                            (ties to even, not clamped)
+ *   q  = clamp(rint(w / s) + z, 0, 15)
+ * using the stored BF16 scale for z and q so the stored parameters reproduce
+ * the codes.  Codes are packed 8 per uint32 word, lowest K index in the lowest
+ * nibble.  Group index runs along K, per output row n.
+ *
+ * Parity status: quantise/pack/unpack/dequant are pinned by hand-worked
+ * groups, tie cases, grid round trips and invariants; the matmul by a library
+ * FP64 matmul of the dequantised weights and one-hot/constant inputs; the
+ * row renormalisation by its closed form (unit RMS) on tiny inputs.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_G 128
+
+enum {
+    ORC_OK = 0,
+    ORC_ERR_ARG = 1,
+    ORC_ERR_SHAPE = 3,
+    ORC_ERR_NONFINITE = 7,
+    ORC_ERR_ZERO_RANGE = 8,
+};
+
+int orc_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* BF16 bit pattern -> value (exact). */
+double orc_bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Binary64 -> nearest BF16 (8 significant bits, exponent range of binary32,
+ * ties to even), written from the definition: find the spacing of BF16 values
+ * around |x|, round |x| / spacing to an integer, scale back. */
+uint16_t orc_bf16_round(double x) {
+    if (isnan(x)) return 0x7FC0;
+    double a = fabs(x);
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    if (a == 0.0) return sign;
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80);
+    int e;
+    frexp(a, &e);              /* a = f 2^e, f in [0.5, 1): 2^(e-1) <= a < 2^e */
+    int lead = e - 1;          /* exponent of the leading bit */
+    if (lead < -126) lead = -126; /* below the normal range the spacing stays 2^-133 */
+    double spacing = ldexp(1.0, lead - 7);
+    double r = nearbyint(a / spacing) * spacing; /* a / spacing is exact (power of two) */
+    if (r > 0x1.FEp127) return (uint16_t)(sign | 0x7F80); /* overflow past the largest BF16 */
+    float rf = (float)r;       /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &rf, 4);
+    return (uint16_t)(sign | (uint16_t)((u >> 16) & 0x7FFF));
+}
+
+/* Quantise one group of G weights (steps above).  Returns a status code. */
+static int orc_quantize_group(const float* w, int64_t G, uint16_t* s_out, int32_t* z_out, uint8_t* q_out,
+                              uint8_t* clipped) {
+    float lo = w[0], hi = w[0];
+    for (int64_t i = 0; i < G; ++i) {
+        if (!isfinite(w[i])) return ORC_ERR_NONFINITE;
+        if (w[i] < lo) lo = w[i];
+        if (w[i] > hi) hi = w[i];
+    }
+    uint16_t sb = orc_bf16_round(((double)hi - (double)lo) / 15.0);
+    if (orc_bf16_value(sb) == 0.0) {
+        double m = fabs((double)lo) > fabs((double)hi) ? fabs((double)lo) : fabs((double)hi);
+        sb = orc_bf16_round(m);
+        if (orc_bf16_value(sb) == 0.0) sb = 0x3F80; /* 1.0 */
+    }
+    double s = orc_bf16_value(sb);
+    double z = nearbyint(-(double)lo / s);
+    if (z > 2147483647.0 || z < -2147483648.0) return ORC_ERR_ZERO_RANGE;
+    for (int64_t i = 0; i < G; ++i) {
+        double t = nearbyint((double)w[i] / s) + z;
+        int clip = (t < 0.0) || (t > 15.0);
+        if (t < 0.0) t = 0.0;
+        if (t > 15.0) t = 15.0;
+        q_out[i] = (uint8_t)t;
+        if (clipped) clipped[i] = (uint8_t)clip;
+    }
+    *s_out = sb;
+    *z_out = (int32_t)z;
+    return ORC_OK;
+}
+
+/* Pack codes[N][K] (values 0..15) into qweight[N][K/8]: nibble i of word j
+ * holds the code of k = 8j + i. */
+void orc_pack_codes(const uint8_t* codes, int64_t N, int64_t K, uint32_t* qweight) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < K / 8; ++j) {
+            uint32_t word = 0;
+            for (int i = 0; i < 8; ++i) word |= ((uint32_t)(codes[n * K + 8 * j + i] & 15u)) << (4 * i);
+            qweight[n * (K / 8) + j] = word;
+        }
+}
+
+/* W fp32 [N][K] -> qweight u32 [N][K/8], scales bf16 [N][K/128], zeros i32 [N][K/128].
+ * clipped (nullable) u8 [N][K]: 1 where rint(w/s)+z fell outside [0, 15]. */
+int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
+                      int32_t* zeros, uint8_t* clipped) {
+    if (!W || !qweight || !scales || !zeros || N < 1 || K < 1) return ORC_ERR_ARG;
+    if (K % ORC_G) return ORC_ERR_SHAPE;
+    const int64_t ng = K / ORC_G;
+    int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t n = 0; n < N; ++n) {
+        uint8_t q[ORC_G];
+        for (int64_t g = 0; g < ng; ++g) {
+            const float* w = W + n * K + g * ORC_G;
+            uint8_t* cl = clipped ? clipped + n * K + g * ORC_G : NULL;
+            int st = orc_quantize_group(w, ORC_G, &scales[n * ng + g], &zeros[n * ng + g], q, cl);
+            if (st != ORC_OK) {
+#pragma omp critical
+                { if (status == ORC_OK) status = st; }
+                memset(q, 0, sizeof q);
+                scales[n * ng + g] = 0;
+                zeros[n * ng + g] = 0;
+            }
+            for (int j = 0; j < ORC_G / 8; ++j) {
+                uint32_t word = 0;
+                for (int i = 0; i < 8; ++i) word |= ((uint32_t)q[8 * j + i]) << (4 * i);
+                qweight[n * (K / 8) + g * (ORC_G / 8) + j] = word;
+            }
+        }
+    }
+    return status;
+}
+
+/* qweight -> codes u8 [N][K]. */
+void orc_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) codes[n * K + k] = (uint8_t)((qweight[n * (K / 8) + k / 8] >> (4 * (k % 8))) & 15u);
+}
+
+/* Exact dequantised weight of one element: (q - z) * s, exact in binary64. */
+static double orc_w_hat(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t K,
+                        int64_t n, int64_t k) {
+    int64_t ng = K / ORC_G;
+    uint32_t q = (qweight[n * (K / 8) + k / 8] >> (4 * (k % 8))) & 15u;
+    int64_t g = k / ORC_G;
+    return ((double)q - (double)zeros[n * ng + g]) * orc_bf16_value(scales[n * ng + g]);
+}
+
+/* W_hat f64 [N][K]. */
+void orc_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                 double* W_hat) {
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) W_hat[n * K + k] = orc_w_hat(qweight, scales, zeros, K, n, k);
+}
+
+/* W_hat rounded to BF16 (nearest, ties to even) [N][K]. */
+void orc_dequant_bf16(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N,
+                      int64_t K, uint16_t* out) {
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) out[n * K + k] = orc_bf16_round(orc_w_hat(qweight, scales, zeros, K, n, k));
+}
+
+/* Y_ref[i][j] = sum_k x[m_i][k] * w_hat[n_j][k] in binary64 (unrounded), for
+ * the listed token rows m_i and output columns n_j.  X is BF16 bits [M][K]. */
+void orc_linear_sampled(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                        const int32_t* zeros, int64_t N, const int64_t* m_idx, int64_t n_m, const int64_t* n_idx,
+                        int64_t n_n, double* Y) {
+    (void)M;
+    (void)N;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t j = 0; j < n_n; ++j) {
+        int64_t n = n_idx[j];
+        double w[ORC_G];
+        for (int64_t i = 0; i < n_m; ++i) Y[i * n_n + j] = 0.0;
+        for (int64_t k0 = 0; k0 < K; k0 += ORC_G) {
+            for (int64_t t = 0; t < ORC_G; ++t) w[t] = orc_w_hat(qweight, scales, zeros, K, n, k0 + t);
+            for (int64_t i = 0; i < n_m; ++i) {
+                const uint16_t* x = X + m_idx[i] * K + k0;
+                double acc = 0.0;
+                for (int64_t t = 0; t < ORC_G; ++t) acc += orc_bf16_value(x[t]) * w[t];
+                Y[i * n_n + j] += acc;
+            }
+        }
+    }
+}
+
+/* Full Y_ref [M][N] in binary64. */
+void orc_linear(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                const int32_t* zeros, int64_t N, double* Y) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        double w[ORC_G];
+        for (int64_t m = 0; m < M; ++m) Y[m * N + n] = 0.0;
+        for (int64_t k0 = 0; k0 < K; k0 += ORC_G) {
+            for (int64_t t = 0; t < ORC_G; ++t) w[t] = orc_w_hat(qweight, scales, zeros, K, n, k0 + t);
+            for (int64_t m = 0; m < M; ++m) {
+                const uint16_t* x = X + m * K + k0;
+                double acc = 0.0;
+                for (int64_t t = 0; t < ORC_G; ++t) acc += orc_bf16_value(x[t]) * w[t];
+                Y[m * N + n] += acc;
+            }
+        }
+    }
+}
+
+/* Row renormalisation between chained layers (the decode-stack workload):
+ * out[m][:] = bf16_rne(y[m][:] / sqrt(mean_j y[m][j]^2)), y read as BF16
+ * bits [M][N]; exact[m][j] (nullable) receives the unrounded quotient.
+ * A zero row stays zero. */
+void orc_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, double* exact) {
+    for (int64_t m = 0; m < M; ++m) {
+        double ss = 0.0;
+        for (int64_t j = 0; j < N; ++j) {
+            double v = orc_bf16_value(y[m * N + j]);
+            ss += v * v;
+        }
+        double rms = sqrt(ss / (double)N);
+        for (int64_t j = 0; j < N; ++j) {
+            double v = orc_bf16_value(y[m * N + j]);
+            double r = rms > 0.0 ? v / rms : 0.0;
+            if (exact) exact[m * N + j] = r;
+            out[m * N + j] = orc_bf16_round(r);
+        }
+    }
+}
