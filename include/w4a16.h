@@ -1,0 +1,169 @@
+/*
+ * w4a16 -- weight-only INT4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * Y[M,N] (bf16) = X[M,K] (bf16) . W_hat^T,  W_hat[n,k] = (q[n,k] - z[n,g]) * s[n,g],  g = k / 128
+ *
+ * Operation: "Axe Corsa 28B" model card, "How the Compression Works"
+ * (asymmetric INT4, one scale and one zero point per group of 128
+ * consecutive weights, dequantisation w_hat = (q - z_g) * s_g inside the
+ * matrix multiply, BF16 activations never quantised) and "What the Tensor
+ * Types Tell You" (BF16 scales, INT32 zero points, two codes per byte);
+ * "Quantization I: int8, int4, the basics", Concept (dequantise tile by tile
+ * inside the multiply so only the packed codes cross the memory bus;
+ * accumulate in higher precision -- FP32 here).
+ *
+ * Conventions for every entry point
+ *  - All tensors are row-major and contiguous.  Element types are given by
+ *    the pointer types; BF16 values are passed as their 16-bit patterns
+ *    (uint16_t).
+ *  - Layouts: W fp32 [N][K]; qweight uint32 [N][K/8] with the code of
+ *    k = 8j + i in bits 4i..4i+3 of word j (lowest K index in the lowest
+ *    nibble); scales bf16 [N][K/128]; zeros int32 [N][K/128]; X bf16 [M][K];
+ *    Y bf16 [M][N].  K must be a multiple of 128; M, N >= 1.
+ *  - Pointers named "device" are CUDA device pointers owned by the caller;
+ *    the library keeps no reference after the call returns and allocates no
+ *    device memory.  Every base pointer must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous on that stream; nothing synchronises the host.
+ *  - Arguments are validated on the host before any launch; a failed check
+ *    returns a status code and launches nothing.  Errors raised by the CUDA
+ *    runtime at launch map to W4A16_ERR_CUDA.  The device must be sm_100
+ *    (checked once per device, cached).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define W4A16_GROUP 128
+
+#if defined(__GNUC__)
+#define W4A16_API __attribute__((visibility("default")))
+#else
+#define W4A16_API
+#endif
+
+typedef enum {
+    W4A16_OK = 0,
+    W4A16_ERR_ARG = 1,        /* null pointer, negative or zero size, unknown option */
+    W4A16_ERR_ALIGN = 2,      /* a base pointer is not 16-byte aligned */
+    W4A16_ERR_SHAPE = 3,      /* K not a multiple of 128, or a size beyond the supported range */
+    W4A16_ERR_DEVICE = 4,     /* no CUDA device, or the current device is not sm_100 */
+    W4A16_ERR_WORKSPACE = 5,  /* workspace missing or smaller than w4a16_workspace_bytes() */
+    W4A16_ERR_CUDA = 6,       /* the CUDA runtime reported an error at launch */
+    W4A16_ERR_NONFINITE = 7,  /* (device status word) a weight group holds NaN or Inf */
+    W4A16_ERR_ZERO_RANGE = 8  /* (device status word) a zero point does not fit in int32 */
+} w4a16_status;
+
+/* Kernel family selection for w4a16_linear_path(). */
+typedef enum {
+    W4A16_PATH_AUTO = 0,    /* decode GEMV for small M, tensor-core GEMM for large M */
+    W4A16_PATH_DECODE = 1,  /* split-K GEMV: register dequantisation, any M (tiles of 32 tokens) */
+    W4A16_PATH_PREFILL = 2  /* TMA + tcgen05/TMEM GEMM on BF16 tiles dequantised in shared memory */
+} w4a16_path;
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+W4A16_API const char* w4a16_status_string(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+W4A16_API int w4a16_version(void);
+
+/*
+ * Quantise and pack (offline step; "Axe Corsa 28B" model card, "How the
+ * Compression Works": each group of 128 consecutive weights along K gets a
+ * scale and a zero point, asymmetric, all 16 levels used).  Per row n and
+ * group g, in binary64:
+ *   lo, hi = min, max of the group; s = bf16_rne((hi - lo) / 15)
+ *   (if s == 0: s = bf16_rne(max(|lo|, |hi|)); if still 0: s = 1)
+ *   z = rint(-lo / s) (ties to even, not clamped); q = clamp(rint(w / s) + z, 0, 15)
+ * The stored BF16 scale is the one used for z and q.
+ *   W          device, fp32 [N][K]                       (read)
+ *   qweight    device, uint32 [N][K/8]                    (written)
+ *   scales     device, bf16 bits [N][K/128]               (written)
+ *   zeros      device, int32 [N][K/128]                   (written)
+ *   dev_status device, one int32                          (written: cleared on the stream, then
+ *              set to W4A16_ERR_NONFINITE / W4A16_ERR_ZERO_RANGE if a group fails; the failing
+ *              group's outputs are unspecified).  Read it after the stream completes.
+ * Returns a host-side status (argument, device or launch errors only).
+ */
+W4A16_API int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
+                        int32_t* zeros, int32_t* dev_status, void* stream);
+
+/*
+ * Bytes of device workspace w4a16_linear() needs for this shape (0 if none).
+ * The workspace holds FP32 split-K partial sums and per-tile arrival counters.
+ * The counter area must be zero before its first use (w4a16_workspace_init);
+ * each completed call leaves it zero again, so one workspace can be reused by
+ * calls that are ordered on one stream.  Calls that may run concurrently need
+ * separate workspaces.
+ */
+W4A16_API size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* Zero a workspace (enqueues a memset of `bytes` on `stream`). */
+W4A16_API int w4a16_workspace_init(void* workspace, size_t bytes, void* stream);
+
+/*
+ * The W4A16 linear layer (the hot path).  Dequantises each weight tile on
+ * the fly -- codes unpacked and (q - z) formed in registers, the BF16 scale
+ * applied per group to the FP32 partial sums -- so only packed codes and
+ * per-group metadata are read from memory.  Accumulation is FP32; Y is
+ * rounded to BF16 (nearest, ties to even) once at the end.
+ *   X         device, bf16 bits [M][K]
+ *   qweight   device, uint32 [N][K/8];  scales device, bf16 bits [N][K/128];
+ *   zeros     device, int32 [N][K/128]
+ *   Y         device, bf16 bits [M][N] (written; must not overlap the inputs)
+ *   workspace device, >= w4a16_workspace_bytes(M, N, K) bytes (NULL allowed when that is 0)
+ */
+W4A16_API int w4a16_linear(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                 const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* As w4a16_linear() with an explicit kernel family (enum w4a16_path). */
+W4A16_API int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                      const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                      int path, void* stream);
+
+/*
+ * Unpack codes ("What the Tensor Types Tell You": two INT4 codes per byte;
+ * the word layout above).  codes: device, uint8 [N][K], values 0..15.
+ * Test and inspection use.
+ */
+W4A16_API int w4a16_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, void* stream);
+
+/*
+ * Materialise W_hat = (q - z) * s rounded to BF16 (nearest, ties to even):
+ * W_hat device, bf16 bits [N][K].  This is the offline dequantisation the
+ * pages call an anti-pattern for inference ("Quantization I", Concept);
+ * provided for tests and for the unfused comparison only.
+ */
+W4A16_API int w4a16_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                  uint16_t* W_hat, void* stream);
+
+/*
+ * Row renormalisation used between chained layers of the decode-stack
+ * workload (not part of the method): out[m][:] = bf16_rne(y[m][:] / rms(y[m][:]))
+ * with the sum of squares in FP32; a zero row stays zero.
+ *   y, out device, bf16 bits [M][N] (out may equal y).
+ */
+W4A16_API int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, void* stream);
+
+/*
+ * Diagnostic: synchronise the current device, then read and clear its fault
+ * word.  Returns 0 when no kernel gave up a bounded wait since the last
+ * call, a positive site code when one did (its outputs are then invalid),
+ * or -1 if the device could not be queried.  Kernels never trap or spin
+ * forever: a pipeline wait that exceeds about two seconds records its site
+ * here and the kernel returns.
+ */
+W4A16_API int w4a16_device_fault(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

@@ -10,10 +10,9 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
-    config.addinivalue_line("markers", "slow: full-size workload case")
 
 
-def gpu_available() -> bool:
+def _cuda_available() -> bool:
     try:
         import torch
         return torch.cuda.is_available()
@@ -21,9 +20,22 @@ def gpu_available() -> bool:
         return False
 
 
+def pytest_collection_modifyitems(config, items):
+    if _cuda_available():
+        return
+    skip = pytest.mark.skip(reason="no CUDA device in this environment")
+    for item in items:
+        if "gpu" in item.keywords:
+            item.add_marker(skip)
+
+
 @pytest.fixture(scope="session")
 def cuda_lib():
-    """The product binding, loaded from the in-tree shared library."""
+    """The product binding, loaded from the in-tree shared library (built if stale)."""
+    import synth
     import weight_only_int4_linear_b200 as w4
+    from weight_only_int4_linear_b200 import build as w4build
+    w4build.build()
+    synth.build_device()
     w4.load()
     return w4

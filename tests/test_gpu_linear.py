@@ -1,0 +1,168 @@
+"""GPU W4A16 linear layer against the FP64 oracle, element by element, under
+the stated tolerance: max |Y - Y_ref| <= 2^-7 |Y_ref| + 1e-3 rms(Y_ref) and
+relative Frobenius error <= 5e-3.
+
+Small cases compare every output; the workloads' full sizes compare sampled
+output rows (the oracle packs and multiplies just those rows, which are
+independent) computed in the same launch configuration the benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_int4_linear_b200 as w4
+from synth import workloads
+from tests._parity import (assert_close, bf16_dev_to_f64, bits_to_dev_bf16, dev_weights, oracle_pack_rows,
+                           sample_rows)
+
+pytestmark = pytest.mark.gpu
+
+PATHS = [w4.PATH_DECODE]
+
+
+def run_linear(X_bits: np.ndarray, pw, path=w4.PATH_AUTO) -> torch.Tensor:
+    M, K = X_bits.shape
+    X = bits_to_dev_bf16(X_bits)
+    Y = torch.full((M, pw.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nbytes = w4.workspace_bytes(M, pw.N, K)
+    ws = torch.zeros(max(nbytes, 1), dtype=torch.uint8, device="cuda")
+    w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y, ws if nbytes else None, path=path)
+    torch.cuda.synchronize()
+    return Y
+
+
+def packed_from_host(W: np.ndarray):
+    pw = w4.PackedWeight.from_float(torch.from_numpy(np.ascontiguousarray(W)).cuda())
+    torch.cuda.synchronize()
+    assert int(pw.status.item()) == 0
+    return pw
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (1, 33, 256), (3, 130, 384), (8, 256, 1024), (9, 200, 512),
+                                   (16, 129, 2048), (17, 64, 640), (32, 384, 1152), (33, 100, 256),
+                                   (70, 150, 768)])
+def test_small_shapes_all_outputs(cuda_lib, M, N, K, path):
+    W = synth.weights_f32(M * 1000 + N, synth.TAG_W, N, K)
+    X = synth.activations_bf16(M + 7, M, K)
+    pw = packed_from_host(W)
+    st, qw, sc, z = oracle.quantize_pack(W)
+    Y = run_linear(X, pw, path)
+    assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), f"M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_one_hot_inputs_pick_weight_columns(cuda_lib, path):
+    """x = e_k must give Y[:, n] = bf16(w_hat[n][k]) exactly: pins nibble order,
+    group indexing and scale/zero addressing through the GPU path."""
+    N, K = 96, 512
+    W = synth.weights_f32(5, synth.TAG_W, N, K)
+    W[:9] += np.float32(0.25)  # negative zero points on some rows
+    pw = packed_from_host(W)
+    st, qw, sc, z = oracle.quantize_pack(W)
+    ks = [0, 1, 4, 7, 8, 15, 16, 31, 127, 128, 129, 255, 300, 511]
+    X = np.zeros((len(ks), K), dtype=np.uint16)
+    for i, k in enumerate(ks):
+        X[i, k] = 0x3F80
+    Y = run_linear(X, pw, path)
+    wh_bits = oracle.dequant_bf16(qw, sc, z, K)
+    got = Y.view(torch.int16).cpu().numpy().view(np.uint16)
+    for i, k in enumerate(ks):
+        np.testing.assert_array_equal(got[i], wh_bits[:, k], err_msg=f"k={k}")
+
+
+def test_constant_inputs(cuda_lib):
+    """A constant row restricted to one group sums that group's w_hat."""
+    N, K = 64, 384
+    W = synth.weights_f32(6, synth.TAG_W, N, K)
+    pw = packed_from_host(W)
+    st, qw, sc, z = oracle.quantize_pack(W)
+    X = np.zeros((2, K), dtype=np.uint16)
+    X[0, 128:256] = 0x4000  # 2.0
+    X[1, :] = 0xBF80        # -1.0
+    Y = bf16_dev_to_f64(run_linear(X, pw))
+    wh = oracle.dequant(qw, sc, z, K)
+    assert_close(Y, np.stack([2.0 * wh[:, 128:256].sum(1), -wh.sum(1)]), "constant rows")
+
+
+def test_single_gemv_full(cuda_lib):
+    case = workloads.single_gemv()[0]
+    pw = packed_from_host(synth.weights_f32(case.w_seed, case.w_tag, case.N, case.K))
+    X = synth.activations_bf16(case.x_seed, case.M, case.K)
+    st, qw, sc, z = oracle.quantize_pack(synth.weights_f32(case.w_seed, case.w_tag, case.N, case.K))
+    Y = run_linear(X, pw)
+    stats = assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), case.name)
+    # the final BF16 rounding of Y alone contributes ~1.7e-3 relative Frobenius error
+    assert stats["rel_fro"] < 2.5e-3
+
+
+def _device_packed(case):
+    W = dev_weights(case.w_seed, case.w_tag, case.N, case.K)
+    pw = w4.PackedWeight.from_float(W)
+    torch.cuda.synchronize()
+    del W
+    assert int(pw.status.item()) == 0
+    return pw
+
+
+@pytest.mark.parametrize("case", workloads.decode_5120() + workloads.small_batch_8192(),
+                         ids=lambda c: f"{c.workload}-{c.name}")
+def test_decode_workloads_sampled_rows(cuda_lib, case):
+    pw = _device_packed(case)
+    X = synth.activations_bf16(case.x_seed, case.M, case.K)
+    Y = run_linear(X, pw)
+    rows = sample_rows(case.N, 192, case.w_seed)
+    qw, sc, z = oracle_pack_rows(case, rows)
+    ref = oracle.linear(X, qw, sc, z)  # [M, len(rows)]
+    got = bf16_dev_to_f64(Y)[:, rows]
+    assert_close(got, ref, f"{case.workload}/{case.name}")
+    assert np.all(np.isfinite(bf16_dev_to_f64(Y)))
+
+
+@pytest.mark.parametrize("case", workloads.prefill_8192(ms=[512]), ids=lambda c: f"{c.workload}-{c.name}")
+def test_prefill_workloads_sampled(cuda_lib, case):
+    pw = _device_packed(case)
+    X = synth.activations_bf16(case.x_seed, case.M, case.K)
+    Y = bf16_dev_to_f64(run_linear(X, pw))
+    rows = sample_rows(case.N, 64, case.w_seed)
+    qw, sc, z = oracle_pack_rows(case, rows)
+    m_idx = sample_rows(case.M, 48, case.x_seed)
+    ref = oracle.linear_sampled(X, qw, sc, z, m_idx, np.arange(rows.size))
+    assert_close(Y[np.ix_(m_idx, rows)], ref, f"{case.workload}/{case.name}")
+
+
+def test_workspace_reuse_and_errors(cuda_lib):
+    N, K, M = 512, 4096, 1
+    W = synth.weights_f32(9, synth.TAG_W, N, K)
+    pw = packed_from_host(W)
+    X = bits_to_dev_bf16(synth.activations_bf16(9, M, K))
+    nbytes = w4.workspace_bytes(M, N, K)
+    assert nbytes > 0  # small N splits K across CTAs
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    Y1 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    Y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y1, ws)
+    w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))  # deterministic split-K order
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y1, ws[: nbytes - 256])
+    assert e.value.status == w4.ERR_WORKSPACE
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y1, None)
+    assert e.value.status == w4.ERR_WORKSPACE
+
+
+def test_renorm_rows(cuda_lib):
+    rng = np.random.default_rng(4)
+    y = torch.from_numpy(rng.standard_normal((3, 28672)).astype(np.float32) * 5).to(torch.bfloat16).cuda()
+    y[2].zero_()
+    out = torch.empty_like(y)
+    w4.renorm_rows(y, out)
+    torch.cuda.synchronize()
+    ref_bits, exact = oracle.renorm(y.view(torch.int16).cpu().numpy().view(np.uint16))
+    got = out.view(torch.int16).cpu().numpy().view(np.uint16).astype(np.int32)
+    # FP32 sum of squares vs FP64: at most one BF16 ulp apart, almost always equal
+    assert np.max(np.abs(got - ref_bits.astype(np.int32))) <= 1
+    assert np.mean(got != ref_bits) < 1e-3

@@ -1,0 +1,159 @@
+// C-ABI entry points of the w4a16 library: host-side validation, device
+// checks and kernel dispatch.  No entry point allocates device memory or
+// synchronises the host.
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace w4a16 {
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_device_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 rejected
+std::atomic<int> g_num_sms[kMaxDevices];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return W4A16_ERR_DEVICE;
+    }
+    if (dev >= kMaxDevices) return W4A16_ERR_DEVICE;
+    int state = g_device_ok[dev].load(std::memory_order_acquire);
+    if (state == 0) {
+        int major = 0, minor = 0, sms = 0;
+        bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+                  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+                  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+        ok = ok && major == 10 && minor == 0;
+        if (ok) g_num_sms[dev].store(sms, std::memory_order_relaxed);
+        state = ok ? 1 : 2;
+        g_device_ok[dev].store(state, std::memory_order_release);
+    }
+    return state == 1 ? W4A16_OK : W4A16_ERR_DEVICE;
+}
+
+// Shape limits: indices inside the kernels are 32-bit for M, N, K and 64-bit
+// for element offsets.
+constexpr int64_t kMaxDim = (int64_t)1 << 30;
+
+int check_shape(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || N < 1 || K < 1) return W4A16_ERR_ARG;
+    if (K % kGroup != 0) return W4A16_ERR_SHAPE;
+    if (M > kMaxDim || N > kMaxDim || K > kMaxDim) return W4A16_ERR_SHAPE;
+    return W4A16_OK;
+}
+}  // namespace
+
+int num_sms_current() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    const int s = g_num_sms[dev].load(std::memory_order_relaxed);
+    return s > 0 ? s : 148;
+}
+
+}  // namespace w4a16
+
+using namespace w4a16;
+
+extern "C" {
+
+const char* w4a16_status_string(int status) {
+    switch (status) {
+        case W4A16_OK: return "ok";
+        case W4A16_ERR_ARG: return "invalid argument (null pointer, non-positive size or unknown option)";
+        case W4A16_ERR_ALIGN: return "a base pointer is not 16-byte aligned";
+        case W4A16_ERR_SHAPE: return "unsupported shape (K must be a multiple of 128; sizes up to 2^30)";
+        case W4A16_ERR_DEVICE: return "no usable device: the current CUDA device must be sm_100 (B200)";
+        case W4A16_ERR_WORKSPACE: return "workspace missing or smaller than w4a16_workspace_bytes()";
+        case W4A16_ERR_CUDA: return "the CUDA runtime reported an error at launch";
+        case W4A16_ERR_NONFINITE: return "a weight group holds NaN or Inf";
+        case W4A16_ERR_ZERO_RANGE: return "a zero point does not fit in int32";
+        default: return "unknown status";
+    }
+}
+
+int w4a16_version(void) { return 100; }
+
+int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
+                        int32_t* dev_status, void* stream) {
+    if (!W || !qweight || !scales || !zeros || !dev_status) return W4A16_ERR_ARG;
+    int st = check_shape(1, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+        (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+        return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    return launch_quantize_pack(W, N, K, qweight, scales, zeros, dev_status, (cudaStream_t)stream);
+}
+
+size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (check_shape(M, N, K) != W4A16_OK) return 0;
+    check_device();  // caches the SM count the plan depends on
+    return plan_decode(M, N, K, num_sms_current()).workspace_bytes();
+}
+
+int w4a16_workspace_init(void* workspace, size_t bytes, void* stream) {
+    if (bytes == 0) return W4A16_OK;
+    if (!workspace) return W4A16_ERR_ARG;
+    if (check_device() != W4A16_OK) return W4A16_ERR_DEVICE;
+    return cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                      const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                      int path, void* stream) {
+    if (!X || !qweight || !scales || !zeros || !Y) return W4A16_ERR_ARG;
+    if (path < W4A16_PATH_AUTO || path > W4A16_PATH_PREFILL) return W4A16_ERR_ARG;
+    int st = check_shape(M, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y))
+        return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    const DecodePlan plan = plan_decode(M, N, K, num_sms_current());
+    const size_t need = plan.workspace_bytes();
+    if (need > 0 && (!workspace || workspace_bytes < need)) return W4A16_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return W4A16_ERR_ALIGN;
+    if (path == W4A16_PATH_PREFILL) return W4A16_ERR_ARG;  // tensor-core path not built in this version
+    return launch_decode(X, M, K, qweight, scales, zeros, N, Y, workspace, plan, (cudaStream_t)stream);
+}
+
+int w4a16_linear(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                 const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+    return w4a16_linear_path(X, M, K, qweight, scales, zeros, N, Y, workspace, workspace_bytes, W4A16_PATH_AUTO,
+                             stream);
+}
+
+int w4a16_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, void* stream) {
+    if (!qweight || !codes) return W4A16_ERR_ARG;
+    int st = check_shape(1, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(qweight) || !aligned16(codes)) return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    return launch_unpack(qweight, N, K, codes, (cudaStream_t)stream);
+}
+
+int w4a16_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                  uint16_t* W_hat, void* stream) {
+    if (!qweight || !scales || !zeros || !W_hat) return W4A16_ERR_ARG;
+    int st = check_shape(1, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(W_hat)) return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    return launch_dequant(qweight, scales, zeros, N, K, W_hat, (cudaStream_t)stream);
+}
+
+int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, void* stream) {
+    if (!y || !out) return W4A16_ERR_ARG;
+    if (M < 1 || N < 1) return W4A16_ERR_ARG;
+    if (M > kMaxDim || N > kMaxDim) return W4A16_ERR_SHAPE;
+    int st = check_device();
+    if (st != W4A16_OK) return st;
+    return launch_renorm(y, M, N, out, (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+// Shared device/host helpers of the w4a16 CUDA library (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/w4a16.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "w4a16 targets sm_100a (Blackwell) only"
+#endif
+
+namespace w4a16 {
+
+constexpr int kGroup = W4A16_GROUP;  // weights per quantisation group along K
+constexpr int kWordsPerGroup = kGroup / 8;
+
+// BF16 bit pattern -> float (exact).
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+
+// float -> BF16 bits, round to nearest, ties to even (NaN kept quiet).
+__device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x0040u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+// binary64 -> BF16 bits, one rounding (nearest, ties to even), by integer
+// arithmetic on the binary64 encoding.
+__device__ __forceinline__ uint16_t double_to_bf16_bits(double x) {
+    uint64_t b = (uint64_t)__double_as_longlong(x);
+    uint32_t sign = (uint32_t)(b >> 63) << 15;
+    uint64_t mag = b & 0x7FFFFFFFFFFFFFFFull;
+    if (mag == 0) return (uint16_t)sign;
+    if (mag >= 0x7FF0000000000000ull) return (uint16_t)(sign | (mag > 0x7FF0000000000000ull ? 0x7FC0u : 0x7F80u));
+    uint32_t r;
+    if (mag < 0x3810000000000000ull) {  // below 2^-126: BF16 subnormal spacing 2^-133
+        double scaled = __longlong_as_double((long long)mag) * 0x1.0p133;
+        r = (uint32_t)__double2ll_rn(scaled);  // <= 128; 128 is the smallest normal's encoding
+    } else {
+        uint64_t keep = mag >> 45;
+        uint64_t rest = mag & ((1ull << 45) - 1ull);
+        keep += (rest > (1ull << 44) || (rest == (1ull << 44) && (keep & 1ull))) ? 1ull : 0ull;
+        int64_t e = (int64_t)(keep >> 7) - 1023 + 127;
+        r = (e >= 255) ? 0x7F80u : (uint32_t)(((uint64_t)e << 7) | (keep & 0x7Full));
+    }
+    return (uint16_t)(sign | r);
+}
+
+__host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace w4a16
+
+// Host-side launch helpers (defined in api.cu).
+namespace w4a16 {
+int launch_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
+                         int32_t* dev_status, cudaStream_t stream);
+int launch_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, cudaStream_t stream);
+int launch_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                   uint16_t* out, cudaStream_t stream);
+int launch_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, cudaStream_t stream);
+
+struct DecodePlan {
+    int nt;           // token tiles of 8 per launch (1, 2 or 4: up to 32 tokens)
+    int row_tiles;    // 128-row tiles along N
+    int grid;         // persistent CTAs
+    int units_base;   // each CTA streams units_base (+1 for the first units_rem CTAs) units
+    int units_rem;
+    int max_slots;    // partial-sum slots per row tile
+    size_t ws_xp_bytes, ws_xs_bytes, ws_partial_bytes, ws_counter_bytes;
+    size_t workspace_bytes() const;
+};
+DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms);
+int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                  const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, const DecodePlan& plan,
+                  cudaStream_t stream);
+int num_sms_current();
+}  // namespace w4a16

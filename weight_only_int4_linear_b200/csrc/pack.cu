@@ -1,0 +1,173 @@
+// Offline and inspection kernels: quantise + pack, unpack, BF16 dequantisation,
+// and the row renormalisation used between chained layers.
+//
+// Quantise + pack follows the "Axe Corsa 28B" model card, "How the Compression
+// Works" (asymmetric INT4, one scale and one zero point per 128 consecutive
+// weights, all 16 levels used) under the min/max affine reading documented in
+// include/w4a16.h.  Every decision that sets a code or a stored parameter is
+// taken in binary64 with IEEE division and round-half-even, so the packed
+// output is bit-exact with any correct implementation of the same reading.
+#include "common.cuh"
+
+namespace w4a16 {
+
+// One warp per group of 128 weights: lane l holds w[4l .. 4l+3].
+__global__ void __launch_bounds__(256) quantize_pack_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+                                                            uint32_t* __restrict__ qweight,
+                                                            uint16_t* __restrict__ scales,
+                                                            int32_t* __restrict__ zeros, int32_t* status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t ng = K / kGroup;
+    const int64_t total = N * ng;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t grp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; grp < total; grp += warps) {
+        const int64_t n = grp / ng, g = grp % ng;
+        const float4 v = reinterpret_cast<const float4*>(W + n * K + g * kGroup)[lane];
+        const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+        if (!__all_sync(0xFFFFFFFFu, finite)) {
+            if (lane == 0) {
+                atomicCAS(status, 0, (int)W4A16_ERR_NONFINITE);
+                scales[grp] = 0;
+                zeros[grp] = 0;
+            }
+            if ((lane & 1) == 0) qweight[n * (K / 8) + g * kWordsPerGroup + lane / 2] = 0u;
+            continue;
+        }
+        float lo = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
+        float hi = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+        }
+        uint16_t sb = double_to_bf16_bits(__ddiv_rn(__dsub_rn((double)hi, (double)lo), 15.0));
+        if ((sb & 0x7FFFu) == 0) {
+            sb = double_to_bf16_bits(fmax(fabs((double)lo), fabs((double)hi)));
+            if ((sb & 0x7FFFu) == 0) sb = 0x3F80u;  // 1.0
+        }
+        const double s = (double)bf16_bits_to_float(sb);
+        const double z = rint(__ddiv_rn(-(double)lo, s));
+        if (z > 2147483647.0 || z < -2147483648.0) {
+            if (lane == 0) {
+                atomicCAS(status, 0, (int)W4A16_ERR_ZERO_RANGE);
+                scales[grp] = 0;
+                zeros[grp] = 0;
+            }
+            if ((lane & 1) == 0) qweight[n * (K / 8) + g * kWordsPerGroup + lane / 2] = 0u;
+            continue;
+        }
+        const float w4[4] = {v.x, v.y, v.z, v.w};
+        uint32_t half = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            double t = __dadd_rn(rint(__ddiv_rn((double)w4[i], s)), z);
+            t = fmin(fmax(t, 0.0), 15.0);
+            half |= ((uint32_t)t) << (4 * i);
+        }
+        // word j = codes of lanes 2j (low half) and 2j+1 (high half)
+        const uint32_t upper = __shfl_down_sync(0xFFFFFFFFu, half, 1);
+        if ((lane & 1) == 0) qweight[n * (K / 8) + g * kWordsPerGroup + lane / 2] = half | (upper << 16);
+        if (lane == 0) {
+            scales[grp] = sb;
+            zeros[grp] = (int32_t)z;
+        }
+    }
+}
+
+// One thread per packed word -> 8 codes.
+__global__ void unpack_kernel(const uint32_t* __restrict__ qweight, int64_t words, uint8_t* __restrict__ codes) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t w = qweight[i];
+        uint2 out;
+        out.x = (w & 0xFu) | ((w >> 4) & 0xFu) << 8 | ((w >> 8) & 0xFu) << 16 | ((w >> 12) & 0xFu) << 24;
+        out.y = ((w >> 16) & 0xFu) | ((w >> 20) & 0xFu) << 8 | ((w >> 24) & 0xFu) << 16 | ((w >> 28) & 0xFu) << 24;
+        reinterpret_cast<uint2*>(codes)[i] = out;
+    }
+}
+
+// One thread per packed word -> 8 BF16 values of (q - z) * s (exact product in
+// binary64, one rounding to BF16).
+__global__ void dequant_kernel(const uint32_t* __restrict__ qweight, const uint16_t* __restrict__ scales,
+                               const int32_t* __restrict__ zeros, int64_t words, int64_t words_per_row,
+                               uint16_t* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i / words_per_row, j = i % words_per_row;
+        const int64_t grp = n * (words_per_row / kWordsPerGroup) + j / kWordsPerGroup;
+        const double s = (double)bf16_bits_to_float(scales[grp]);
+        const double z = (double)zeros[grp];
+        const uint32_t w = qweight[i];
+        uint32_t packed[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const double lo = ((double)((w >> (8 * p)) & 0xFu) - z) * s;
+            const double hi = ((double)((w >> (8 * p + 4)) & 0xFu) - z) * s;
+            packed[p] = (uint32_t)double_to_bf16_bits(lo) | ((uint32_t)double_to_bf16_bits(hi) << 16);
+        }
+        reinterpret_cast<uint4*>(out)[i] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+}
+
+// One CTA per row: sum of squares in FP32, then y / sqrt(mean) rounded to BF16.
+__global__ void __launch_bounds__(256) renorm_kernel(const uint16_t* __restrict__ y, int64_t N,
+                                                     uint16_t* __restrict__ out) {
+    const uint16_t* row = y + (int64_t)blockIdx.x * N;
+    uint16_t* orow = out + (int64_t)blockIdx.x * N;
+    float ss = 0.f;
+    for (int64_t j = threadIdx.x; j < N; j += blockDim.x) {
+        const float v = bf16_bits_to_float(row[j]);
+        ss = fmaf(v, v, ss);
+    }
+    __shared__ float red[32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float t = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+        if (threadIdx.x == 0) red[0] = t;
+    }
+    __syncthreads();
+    const float rms = sqrtf(red[0] / (float)N);
+    for (int64_t j = threadIdx.x; j < N; j += blockDim.x) {
+        const float v = bf16_bits_to_float(row[j]);
+        orow[j] = float_to_bf16_bits(rms > 0.f ? v / rms : 0.f);
+    }
+}
+
+static int grid_for(int64_t items, int threads) {
+    int64_t blocks = ceil_div(items, threads);
+    const int64_t cap = (int64_t)num_sms_current() * 32;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+int launch_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
+                         int32_t* dev_status, cudaStream_t stream) {
+    if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), stream) != cudaSuccess) return W4A16_ERR_CUDA;
+    const int64_t groups = N * (K / kGroup);
+    quantize_pack_kernel<<<grid_for(groups * 32, 256), 256, 0, stream>>>(W, N, K, qweight, scales, zeros, dev_status);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+int launch_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, cudaStream_t stream) {
+    const int64_t words = N * (K / 8);
+    unpack_kernel<<<grid_for(words, 256), 256, 0, stream>>>(qweight, words, codes);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+int launch_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                   uint16_t* out, cudaStream_t stream) {
+    const int64_t words = N * (K / 8);
+    dequant_kernel<<<grid_for(words, 256), 256, 0, stream>>>(qweight, scales, zeros, words, K / 8, out);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+int launch_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, cudaStream_t stream) {
+    renorm_kernel<<<(unsigned)M, 256, 0, stream>>>(y, N, out);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+}  // namespace w4a16
