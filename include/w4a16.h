@@ -153,6 +153,35 @@ W4A16_API int w4a16_dequant(const uint32_t* qweight, const uint16_t* scales, con
 W4A16_API int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, void* stream);
 
 /*
+ * The linear layer without a caller-provided workspace.  (The source pages
+ * describe no such entry point; it exists for callers that cannot allocate.)
+ * Some callers may not allocate device memory once they run -- a serving loop
+ * that reserved all of HBM at start-up, a framework whose allocator owns the
+ * device, code that cannot reach cudaMalloc where it calls this library.  This
+ * variant of the decode path (split-K GEMV, any M in token tiles of 32) keeps
+ * its scratch -- prepared X, split-K partial sums, arrival counters -- in one
+ * file-scope device array of w4a16_noalloc_scratch_bytes() bytes (16 MiB) that
+ * every process loading the library holds on each GPU it uses until exit.  It
+ * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ *  - Arguments, layouts and results are those of w4a16_linear().
+ *  - A problem whose scratch (w4a16_workspace_bytes(M, N, K)) exceeds the
+ *    array returns W4A16_ERR_WORKSPACE and launches nothing.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents; each call clears the counters it needs before launching.
+ *    Calls that may overlap on the GPU (different streams, concurrent host
+ *    threads without ordering) race on the array: order them on one stream.
+ */
+W4A16_API int w4a16_linear_noalloc(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight,
+                                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y,
+                                   void* stream);
+
+/* Size of the built-in scratch array w4a16_linear_noalloc() uses, in bytes. */
+W4A16_API size_t w4a16_noalloc_scratch_bytes(void);
+
+/*
  * Diagnostic: synchronise the current device, then read and clear its fault
  * word.  Returns 0 when no kernel gave up a bounded wait since the last
  * call, a positive site code when one did (its outputs are then invalid),

@@ -54,6 +54,8 @@ SIGNATURES = {
     "w4a16_dequant": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "w4a16_renorm_rows": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_device_fault": (_int, []),
+    "w4a16_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
+    "w4a16_noalloc_scratch_bytes": (_sz, []),
 }
 
 
@@ -153,6 +155,25 @@ def linear(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: 
         _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N,
         _dev(Y, "Y", torch.bfloat16, (M, N)), ws_ptr, ws_bytes, path, _stream(stream))
     _check("w4a16_linear", st)
+
+
+def linear_noalloc(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                   Y: torch.Tensor, stream=None) -> None:
+    """w4a16_linear_noalloc: the decode-path linear layer using the library's built-in
+    device scratch array instead of a workspace (for callers that cannot allocate)."""
+    M, K = X.shape
+    N = qweight.shape[0]
+    st = load().w4a16_linear_noalloc(
+        _dev(X, "X", torch.bfloat16), M, K,
+        _dev(qweight, "qweight", torch.int32, (N, K // 8)),
+        _dev(scales, "scales", torch.bfloat16, (N, K // GROUP)),
+        _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N,
+        _dev(Y, "Y", torch.bfloat16, (M, N)), _stream(stream))
+    _check("w4a16_linear_noalloc", st)
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(load().w4a16_noalloc_scratch_bytes())
 
 
 def unpack(qweight: torch.Tensor, K: int, codes: torch.Tensor, stream=None) -> None:
