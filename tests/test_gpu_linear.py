@@ -18,7 +18,7 @@ from tests._parity import (assert_close, bf16_dev_to_f64, bits_to_dev_bf16, dev_
 
 pytestmark = pytest.mark.gpu
 
-PATHS = [w4.PATH_DECODE]
+PATHS = [w4.PATH_DECODE, w4.PATH_PREFILL]
 
 
 def run_linear(X_bits: np.ndarray, pw, path=w4.PATH_AUTO) -> torch.Tensor:
@@ -120,7 +120,7 @@ def test_decode_workloads_sampled_rows(cuda_lib, case):
     assert np.all(np.isfinite(bf16_dev_to_f64(Y)))
 
 
-@pytest.mark.parametrize("case", workloads.prefill_8192(ms=[512]), ids=lambda c: f"{c.workload}-{c.name}")
+@pytest.mark.parametrize("case", workloads.prefill_8192(), ids=lambda c: f"{c.workload}-{c.name}")
 def test_prefill_workloads_sampled(cuda_lib, case):
     pw = _device_packed(case)
     X = synth.activations_bf16(case.x_seed, case.M, case.K)

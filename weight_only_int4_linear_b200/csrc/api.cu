@@ -93,7 +93,10 @@ int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight,
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
     if (check_shape(M, N, K) != W4A16_OK) return 0;
     check_device();  // caches the SM count the plan depends on
-    return plan_decode(M, N, K, num_sms_current()).workspace_bytes();
+    // enough for every kernel family (the decode need is independent of M beyond 32 tokens)
+    const size_t dec = plan_decode(M, N, K, num_sms_current()).workspace_bytes();
+    const size_t pre = prefill_workspace_bytes(M, K);
+    return dec > pre ? dec : pre;
 }
 
 int w4a16_workspace_init(void* workspace, size_t bytes, void* stream) {
@@ -113,11 +116,12 @@ int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* q
     if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y))
         return W4A16_ERR_ALIGN;
     if ((st = check_device()) != W4A16_OK) return st;
+    const bool prefill = path == W4A16_PATH_PREFILL || (path == W4A16_PATH_AUTO && M >= kPrefillMinM);
     const DecodePlan plan = plan_decode(M, N, K, num_sms_current());
-    const size_t need = plan.workspace_bytes();
+    const size_t need = prefill ? prefill_workspace_bytes(M, K) : plan.workspace_bytes();
     if (need > 0 && (!workspace || workspace_bytes < need)) return W4A16_ERR_WORKSPACE;
     if (need > 0 && !aligned16(workspace)) return W4A16_ERR_ALIGN;
-    if (path == W4A16_PATH_PREFILL) return W4A16_ERR_ARG;  // tensor-core path not built in this version
+    if (prefill) return launch_prefill(X, M, K, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
     return launch_decode(X, M, K, qweight, scales, zeros, N, Y, workspace, plan, (cudaStream_t)stream);
 }
 

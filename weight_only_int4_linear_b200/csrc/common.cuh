@@ -76,4 +76,10 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
                   const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, const DecodePlan& plan,
                   cudaStream_t stream);
 int num_sms_current();
+
+// Prefill (tensor-core GEMM) path for large M.
+constexpr int64_t kPrefillMinM = 64;  // W4A16_PATH_AUTO switches to the GEMM at this many tokens
+size_t prefill_workspace_bytes(int64_t M, int64_t K);
+int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                   const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, cudaStream_t stream);
 }  // namespace w4a16

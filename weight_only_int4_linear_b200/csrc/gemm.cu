@@ -1,0 +1,410 @@
+// Prefill path of the W4A16 linear layer: a persistent, warp-specialised
+// tcgen05 GEMM for large M.
+//
+// The weights are dequantised tile by tile on chip and never written back:
+// packed codes arrive by TMA, dequantiser warps expand them to BF16 operand
+// tiles in shared memory, and the 5th-generation tensor cores multiply them
+// with BF16 X tiles ("Weight-Only Quantization and Mixed Precision",
+// section 7: fused read, unpack, dequantise and matmul, asynchronous copies
+// overlapping the math; "Quantization I: int8, int4, the basics", Concept:
+// dequantise tile by tile inside the multiply, accumulate in higher precision).
+//
+// Arithmetic: per group g of 128 weights along K,
+//   Y[m][n] += s[n][g] * ( sum_k (128 + q[n][k]) x[m][k]  -  (128 + z[n][g]) xsum[m][g] )
+// with (128 + q) exact in BF16 (0x4300 | q, one lop3 per two codes), the inner
+// sum on the tensor cores into a per-group FP32 accumulator in tensor memory,
+// and the fold in FP32 by the epilogue warps.  The BF16 scale never enters a
+// rounded operand; the only rounding besides FP32 summation is the final BF16
+// rounding of Y.
+//
+// Tile: 128 weight rows (MMA M) x 256 tokens (MMA N, swap-AB so the per-row
+// scale is a per-thread constant in the fold).  K advances in stages of 64
+// (half a group).  MMA K order inside each 8-block of K is (0,4,1,5,2,6,3,7):
+// that is the order a lop3 pair extraction yields, and X is prepared in it.
+//
+// Warps (512 threads):
+//   0-3   dequantise: thread = weight row; 8 packed words -> one 128-byte
+//         row of the 128B-swizzled K-major A tile
+//   4-11  fold + epilogue: warp w reads TMEM lane quadrant w % 4, token
+//         columns 128 * ((w - 4) / 4) ... + 127; totals live in registers
+//   12    TMA: X tile (256 x 64, 128-byte swizzle) and code tile (128 x 8
+//         words, 32-byte swizzle) per stage
+//   13    MMA issue: four tcgen05.mma (128 x 256 x 16) per stage
+//   14-15 idle
+// Accumulators: two 256-column TMEM buffers, one per group in flight, so the
+// fold of group g overlaps the MMAs of group g + 1.
+#include "common.cuh"
+#include "sm100.cuh"
+
+#include <mutex>
+
+namespace w4a16 {
+namespace {
+
+constexpr int kPBM = 128;                      // weight rows per tile
+constexpr int kPBN = 256;                      // tokens per tile
+constexpr int kPBK = 64;                       // K per stage
+constexpr int kPStages = 4;
+constexpr int kPXBytes = kPBN * kPBK * 2;      // 32 KB
+constexpr int kPABytes = kPBM * kPBK * 2;      // 16 KB
+constexpr int kPCodeBytes = kPBM * kPBK / 2;   // 4 KB
+constexpr int kPStageBytes = kPXBytes + kPABytes + kPCodeBytes;  // 52 KB (1024-aligned)
+constexpr size_t kPSmem = (size_t)kPStages * kPStageBytes + 1024;
+constexpr int kPThreads = 512;
+constexpr uint32_t kPIdesc = idesc_bf16_f32(kPBM, kPBN);
+
+struct PrefillArgs {
+    const uint16_t* scales;
+    const int32_t* zeros;
+    const float* xsT;  // [G][Mp]: per-group sums of X, Mp = M rounded up to a multiple of 4
+    uint16_t* Y;
+    int* fault;
+    int M, N, K, G, Mp;
+    int m_tiles, n_tiles;
+    int tiles_base, tiles_rem;  // CTA b runs tiles_base (+1 for the first tiles_rem CTAs) consecutive tiles
+};
+
+__device__ __forceinline__ uint32_t magic_pair(uint32_t w) {
+    uint32_t r;
+    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(w));  // (w & m) | c
+    return r;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint4 permute_block(uint4 v) {
+    uint4 o;
+    o.x = __byte_perm(v.x, v.z, 0x5410);  // x0, x4
+    o.y = __byte_perm(v.x, v.z, 0x7632);  // x1, x5
+    o.z = __byte_perm(v.y, v.w, 0x5410);  // x2, x6
+    o.w = __byte_perm(v.y, v.w, 0x7632);  // x3, x7
+    return o;
+}
+
+// X -> Xp (each 8-block reordered (0,4,1,5,2,6,3,7)) and xsT[g][m] = sum of the group
+// (row stride Mp, a multiple of 4 so the fold can read float4s).
+__global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __restrict__ X, int M, int K, int Mp,
+                                                           uint16_t* __restrict__ Xp, float* __restrict__ xsT) {
+    pdl_launch_dependents();
+    const int G = K / kGroup;
+    const int64_t units = (int64_t)M * G * 16;  // multiple of 16
+    for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x; u0 < units; u0 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t u = u0 + threadIdx.x;
+        const bool active = u < units;
+        const int64_t mg = u >> 4;  // (m, g) pair, g fastest
+        const int blk = (int)(u & 15);
+        const int m = (int)(mg / G), g = (int)(mg - (int64_t)m * G);
+        float sum = 0.f;
+        if (active) {
+            const int64_t off = (int64_t)m * K + (int64_t)g * kGroup + blk * 8;
+            const uint4 v = *reinterpret_cast<const uint4*>(X + off);
+            *reinterpret_cast<uint4*>(Xp + off) = permute_block(v);
+            sum = (bf16lo(v.x) + bf16hi(v.x)) + (bf16lo(v.y) + bf16hi(v.y)) + (bf16lo(v.z) + bf16hi(v.z)) +
+                  (bf16lo(v.w) + bf16hi(v.w));
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (active && blk == 0) xsT[(int64_t)g * Mp + m] = sum;
+    }
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tx,
+                                                               const __grid_constant__ CUtensorMap tq,
+                                                               const PrefillArgs a) {
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t full[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
+    __shared__ uint32_t s_tmem;
+    const uint32_t raw = smem_u32(smem_raw);
+    unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x;
+    const int t_first = b * a.tiles_base + min(b, a.tiles_rem);
+    const int ntiles = a.tiles_base + (b < a.tiles_rem ? 1 : 0);
+    const int G = a.G;
+    const int stages_per_tile = 2 * G;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&afull[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&mdone[i], 1);
+            mbar_init(&dfree[i], 8);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0) tmem_alloc(&s_tmem, 512);
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const int wg = warp >> 2;
+
+    // register split (launch: 512 x 128 = 65536): 4 x 32 x (72 + 56 + 192 + 192) = 65536
+    if (wg == 3) {  // ------------------------------------------------ TMA + MMA
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
+        if (warp == 12 && lane == 0) {
+            prefetch_tmap(&tx);
+            prefetch_tmap(&tq);
+            pdl_wait_primary();  // X comes from the preparation kernel
+            int it = 0;
+            for (int tt = 0; tt < ntiles; ++tt) {
+                const int tile = t_first + tt;
+                const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+                for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
+                    const int s = it % kPStages;
+                    if (it >= kPStages && !mbar_wait(&empty[s], ((it / kPStages) - 1) & 1, a.fault, 61)) goto done_tma;
+                    unsigned char* st = ring + s * kPStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kPXBytes + kPCodeBytes);
+                    tma_load_2d(st, &tx, ks * kPBK, mt * kPBN, &full[s]);
+                    tma_load_2d(st + kPXBytes + kPABytes, &tq, ks * (kPBK / 8), nt * kPBM, &full[s]);
+                }
+            }
+        done_tma:
+            // copies in flight land before the CTA may exit
+            for (int i = max(0, it - kPStages); i < it; ++i) mbar_wait(&full[i % kPStages], (i / kPStages) & 1, a.fault, 62);
+        } else if (warp == 13 && lane == 0) {
+            int it = 0, gc = 0;
+            for (int tt = 0; tt < ntiles; ++tt) {
+                for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
+                    const int s = it % kPStages;
+                    const int half = ks & 1;
+                    const int dbuf = gc & 1;
+                    if (half == 0 && gc >= 2 && !mbar_wait(&dfree[dbuf], ((gc >> 1) - 1) & 1, a.fault, 71)) goto done_mma;
+                    if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 72)) goto done_mma;
+                    if (!mbar_wait(&afull[s], (it / kPStages) & 1, a.fault, 73)) goto done_mma;
+                    tc_fence_after();
+                    const uint32_t xaddr = smem_u32(ring + s * kPStageBytes);
+                    const uint32_t aaddr = xaddr + kPXBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kPBK / 16; ++kk) {
+                        umma_ss(tmem + dbuf * kPBN, sw128_kmajor_desc(aaddr + kk * 32), sw128_kmajor_desc(xaddr + kk * 32),
+                                kPIdesc, half > 0 || kk > 0);
+                    }
+                    umma_commit(&empty[s]);
+                    if (half == 1) {
+                        umma_commit(&mdone[dbuf]);
+                        ++gc;
+                    }
+                }
+            }
+        done_mma:;
+        }
+    } else if (wg == 0) {  // ------------------------------------ dequantisers
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+        const int r = threadIdx.x;  // weight row within the tile
+        // codes tile: 32 bytes per row, 32-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 2) & 1)
+        const int csw = (r >> 2) & 1;
+        int it = 0;
+        for (int tt = 0; tt < ntiles; ++tt) {
+            for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
+                const int s = it % kPStages;
+                if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 81)) goto done_dq;
+                unsigned char* st = ring + s * kPStageBytes;
+                const unsigned char* codes = st + kPXBytes + kPABytes + r * 32;
+                const uint4 c0 = *reinterpret_cast<const uint4*>(codes + 16 * csw);
+                const uint4 c1 = *reinterpret_cast<const uint4*>(codes + 16 * (1 - csw));
+                const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                // A row r: 128 bytes, 16-byte chunk j (word j) stored at chunk j ^ (r % 8)
+                unsigned char* arow = st + kPXBytes + r * 128;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint32_t x = w[j];
+                    const uint4 v = make_uint4(magic_pair(x), magic_pair(x >> 4), magic_pair(x >> 8), magic_pair(x >> 12));
+                    *reinterpret_cast<uint4*>(arow + 16 * (j ^ (r & 7))) = v;
+                }
+                fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&afull[s]);
+            }
+        }
+    done_dq:;
+    } else {  // -------------------------------------------- fold + epilogue (wg 1, 2)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 192;");
+        const int quad = warp & 3;
+        const int colh = (warp - 4) >> 2;            // token half of the tile
+        const int row = quad * 32 + lane;            // weight row within the tile = TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
+        float T[128];
+#pragma unroll
+        for (int j = 0; j < 128; ++j) T[j] = 0.f;
+        int gc = 0;
+        bool aborted = false;
+        for (int tt = 0; tt < ntiles; ++tt) {
+            const int tile = t_first + tt;
+            const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+            const int n = nt * kPBM + row;
+            const int m0 = mt * kPBN + colh * 128;
+            for (int g = 0; g < G; ++g, ++gc) {
+                float sv = 0.f, cz = 0.f;
+                if (n < a.N) {
+                    sv = bf16_bits_to_float(__ldg(a.scales + (int64_t)n * G + g));
+                    cz = 128.f + (float)__ldg(a.zeros + (int64_t)n * G + g);
+                }
+                const float* xs = a.xsT + (int64_t)g * a.Mp + m0;
+                const int dbuf = gc & 1;
+                if (!aborted && !mbar_wait(&mdone[dbuf], (gc >> 1) & 1, a.fault, 91)) aborted = true;
+                if (!aborted) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint32_t d[16];
+                        tmem_ld16(tl + dbuf * kPBN + colh * 128 + cc * 16, d);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const int mcol = m0 + cc * 16 + 4 * j4;
+                            // xsT rows hold Mp >= M values (the padding is never read past Mp)
+                            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f);
+                            if (mcol < a.Mp) xv = __ldg(reinterpret_cast<const float4*>(xs + cc * 16 + 4 * j4));
+                            const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j = cc * 16 + 4 * j4 + e;
+                                T[j] = fmaf(sv, fmaf(-cz, xq[e], __uint_as_float(d[4 * j4 + e])), T[j]);
+                            }
+                        }
+                    }
+                    tc_fence_before();
+                }
+                __syncwarp();
+                if (lane == 0 && !aborted) mbar_arrive(&dfree[dbuf]);
+            }
+            // epilogue: this thread's row n, tokens m0 .. m0 + 127
+            if (n < a.N) {
+#pragma unroll
+                for (int j = 0; j < 128; ++j) {
+                    const int m = m0 + j;
+                    if (m < a.M) a.Y[(int64_t)m * a.N + n] = float_to_bf16_bits(T[j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 128; ++j) T[j] = 0.f;
+        }
+    }
+    // teardown: all roles done; every MMA was waited on by the fold warps
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+std::mutex g_ptmap_mu;
+struct PTmap {
+    const void* ptr;
+    int64_t rows, cols;
+    int kind;
+    CUtensorMap map;
+};
+PTmap g_ptmaps[64];
+int g_ptmap_next = 0;
+
+bool prefill_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensorMap* out) {
+    std::lock_guard<std::mutex> lk(g_ptmap_mu);
+    for (auto& e : g_ptmaps)
+        if (e.ptr == ptr && e.rows == rows && e.cols == cols && e.kind == kind) {
+            *out = e.map;
+            return true;
+        }
+    PTmap& e = g_ptmaps[g_ptmap_next];
+    bool ok;
+    if (kind == 0)  // prepared X: bf16 [M][K], box 64 x 256, 128-byte swizzle
+        ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
+                            (uint64_t)cols * 2, kPBK, kPBN, CU_TENSOR_MAP_SWIZZLE_128B);
+    else  // packed weights: uint32 [N][K/8], box 8 words x 128 rows, 32-byte swizzle
+        ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, ptr, (uint64_t)cols, (uint64_t)rows,
+                            (uint64_t)cols * 4, kPBK / 8, kPBM, CU_TENSOR_MAP_SWIZZLE_32B);
+    if (!ok) return false;
+    e.ptr = ptr;
+    e.rows = rows;
+    e.cols = cols;
+    e.kind = kind;
+    g_ptmap_next = (g_ptmap_next + 1) % 64;
+    *out = e.map;
+    return true;
+}
+
+size_t align256p(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+size_t prefill_workspace_bytes(int64_t M, int64_t K) {
+    const int64_t Mp = (M + 3) & ~(int64_t)3;
+    return align256p((size_t)M * K * 2) + align256p((size_t)(K / kGroup) * Mp * 4);
+}
+
+int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                   const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, cudaStream_t stream) {
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem) !=
+            cudaSuccess)
+            return W4A16_ERR_CUDA;
+        attr = true;
+    }
+    int* fault = fault_word();
+    if (!fault) return W4A16_ERR_CUDA;
+    char* ws = reinterpret_cast<char*>(workspace);
+    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
+    float* xsT = reinterpret_cast<float*>(ws + align256p((size_t)M * K * 2));
+    CUtensorMap tx, tq;
+    if (!prefill_tmap(0, Xp, M, K, &tx) || !prefill_tmap(1, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
+
+    const int G = (int)(K / kGroup);
+    const int64_t units = M * G * 16;
+    int pgrid = (int)ceil_div(units, 256);
+    if (pgrid > num_sms_current() * 16) pgrid = num_sms_current() * 16;
+    const int Mp = (int)((M + 3) & ~(int64_t)3);
+    if (Mp > M && cudaMemsetAsync(xsT, 0, (size_t)G * Mp * 4, stream) != cudaSuccess) return W4A16_ERR_CUDA;
+    prefill_prep_kernel<<<pgrid, 256, 0, stream>>>(X, (int)M, (int)K, Mp, Xp, xsT);
+    if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
+
+    PrefillArgs args;
+    args.scales = scales;
+    args.zeros = zeros;
+    args.xsT = xsT;
+    args.Y = Y;
+    args.fault = fault;
+    args.M = (int)M;
+    args.N = (int)N;
+    args.K = (int)K;
+    args.G = G;
+    args.Mp = Mp;
+    args.m_tiles = (int)ceil_div(M, kPBN);
+    args.n_tiles = (int)ceil_div(N, kPBM);
+    const int tiles = args.m_tiles * args.n_tiles;
+    int grid = num_sms_current();
+    if (grid > tiles) grid = tiles;
+    args.tiles_base = tiles / grid;
+    args.tiles_rem = tiles % grid;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPThreads);
+    cfg.dynamicSmemBytes = kPSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr1[1];
+    attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr1[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr1;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel, tx, tq, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+}  // namespace w4a16
