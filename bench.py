@@ -131,8 +131,14 @@ def setup_layers(cases, torch, w4, stream):
     return layers
 
 
+PREFILL_MIN_M = 64  # the library's automatic path choice: M >= 64 takes the tensor-core GEMM
+
+
 def launches_per_call(c) -> int:
-    """Our kernels per linear call: X preparation + GEMV per 32-token chunk."""
+    """Our kernels per linear call: X preparation + GEMM (M >= 64), else
+    X preparation + GEMV per 32-token chunk."""
+    if c.M >= PREFILL_MIN_M:
+        return 2
     return 2 * ((c.M + 31) // 32)
 
 
@@ -442,6 +448,27 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(spec: str, repeats: int = 4):
+    """Run one layer of a workload a few times (for an ncu capture; no timing)."""
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    w4.load()
+    wl, name = spec.split(":")
+    cases = {"decode": workloads.decode_5120(), "small": workloads.small_batch_8192(),
+             "prefill": workloads.prefill_8192()}[wl]
+    case = [c for c in cases if c.name == name][0]
+    stream = torch.cuda.Stream()
+    L = setup_layers([case], torch, w4, stream)[0]
+    with torch.cuda.stream(stream):
+        for _ in range(repeats):
+            _linear_call(w4, L, w4.PATH_AUTO)
+    torch.cuda.synchronize()
+    fault = w4.device_fault()
+    print(json.dumps({"profiled": spec, "repeats": repeats, "fault": fault}))
+    if fault:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,7 +481,12 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture of this build")
+    ap.add_argument("--profile", default=None,
+                    help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096): run it a few times, untimed")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args.profile)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

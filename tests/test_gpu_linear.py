@@ -166,3 +166,35 @@ def test_renorm_rows(cuda_lib):
     # FP32 sum of squares vs FP64: at most one BF16 ulp apart, almost always equal
     assert np.max(np.abs(got - ref_bits.astype(np.int32))) <= 1
     assert np.mean(got != ref_bits) < 1e-3
+
+
+def _groups_with_zero_points(N, K, zs, seed):
+    """Weights whose group g of row n has scale 1/16 and zero point
+    zs[(n + g) % len(zs)]: the group is rescaled onto [lo, lo + 15/16] with
+    lo = -z/16, so (hi - lo)/15 = 1/16 exactly and z = rint(-lo/s)."""
+    W = synth.weights_f32(seed, synth.TAG_W, N, K).astype(np.float64).reshape(N, K // 128, 128)
+    lo_w = W.min(axis=2, keepdims=True)
+    hi_w = W.max(axis=2, keepdims=True)
+    z = np.array([[zs[(n + g) % len(zs)] for g in range(K // 128)] for n in range(N)], dtype=np.float64)
+    lo = (-z / 16.0)[:, :, None]
+    W = lo + (W - lo_w) / (hi_w - lo_w) * (15.0 / 16.0)
+    return W.reshape(N, K).astype(np.float32), z.astype(np.int64)
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("M", [1, 8, 70])
+def test_zero_points_far_outside_the_code_range(cuda_lib, M, path):
+    """One-signed groups have zero points far from 0..15 (here up to +-2000):
+    the kernels take a different branch for |z| > 128; both sides of that
+    boundary, and z = +-128 on it, must match the oracle."""
+    zs = [0, 7, 15, 127, 128, 129, -127, -128, -129, 300, -300, 2000, -2000, 64]
+    N, K = 130, 1024
+    W, z_expect = _groups_with_zero_points(N, K, zs, 77)
+    st, qw, sc, z = oracle.quantize_pack(W)
+    assert st == oracle.OK
+    np.testing.assert_array_equal(z, z_expect)
+    pw = packed_from_host(W)
+    assert torch.equal(pw.zeros.cpu(), torch.from_numpy(z.astype(np.int32)))
+    X = synth.activations_bf16(900 + M, M, K)
+    Y = run_linear(X, pw, path)
+    assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), f"M={M}")

@@ -10,12 +10,15 @@
 // dequantise tile by tile inside the multiply, accumulate in higher precision).
 //
 // Arithmetic: per group g of 128 weights along K,
-//   Y[m][n] += s[n][g] * ( sum_k (128 + q[n][k]) x[m][k]  -  (128 + z[n][g]) xsum[m][g] )
-// with (128 + q) exact in BF16 (0x4300 | q, one lop3 per two codes), the inner
-// sum on the tensor cores into a per-group FP32 accumulator in tensor memory,
-// and the fold in FP32 by the epilogue warps.  The BF16 scale never enters a
-// rounded operand; the only rounding besides FP32 summation is the final BF16
-// rounding of Y.
+//   Y[m][n] += s[n][g] * sum_k (q[n][k] - c) x[m][k]  -  s[n][g] (z[n][g] - c) xsum[m][g]
+// The dequantiser forms (128 + q) in BF16 (0x4300 | q, one lop3 per two codes)
+// and subtracts (128 + c) with one packed BF16 subtract, exact because both
+// are integers of magnitude <= 256: c = z whenever |z| <= 128 (every group
+// whose range straddles zero), else c = 0.  The inner sum runs on the tensor
+// cores into a per-group FP32 accumulator in tensor memory; the fold is one
+// FP32 FMA per element, T += s * D, plus the xsum term for the rare rows with
+// c != z.  The BF16 scale never enters a rounded operand; the only rounding
+// besides FP32 summation is the final BF16 rounding of Y.
 //
 // Tile: 128 weight rows (MMA M) x 256 tokens (MMA N, swap-AB so the per-row
 // scale is a per-thread constant in the fold).  K advances in stages of 64
@@ -67,6 +70,13 @@ struct PrefillArgs {
 __device__ __forceinline__ uint32_t magic_pair(uint32_t w) {
     uint32_t r;
     asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(w));  // (w & m) | c
+    return r;
+}
+
+// (a - b) on BF16 pairs; exact here (integers of magnitude <= 256).
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 
@@ -127,6 +137,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
     __shared__ uint32_t s_tmem;
+    __shared__ __align__(16) float s_xs[2][kPBN];  // per-group X sums of the tile's tokens, by group parity
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
 
@@ -212,7 +223,16 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         const int csw = (r >> 2) & 1;
         int it = 0;
         for (int tt = 0; tt < ntiles; ++tt) {
+            const int nt = (t_first + tt) / a.m_tiles;
+            const int n = nt * kPBM + r;
+            uint32_t zc2 = 0x43004300u;  // (128 + c) as a BF16 pair
             for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
+                if ((ks & 1) == 0) {
+                    const int z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + (ks >> 1)) : 0;
+                    const int c = (z >= -128 && z <= 128) ? z : 0;
+                    const uint32_t cb = __float_as_uint(128.f + (float)c) >> 16;  // exact: |128 + c| <= 256
+                    zc2 = cb | (cb << 16);
+                }
                 const int s = it % kPStages;
                 if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 81)) goto done_dq;
                 unsigned char* st = ring + s * kPStageBytes;
@@ -225,7 +245,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const uint32_t x = w[j];
-                    const uint4 v = make_uint4(magic_pair(x), magic_pair(x >> 4), magic_pair(x >> 8), magic_pair(x >> 12));
+                    const uint4 v = make_uint4(sub_bf16x2(magic_pair(x), zc2), sub_bf16x2(magic_pair(x >> 4), zc2),
+                                               sub_bf16x2(magic_pair(x >> 8), zc2), sub_bf16x2(magic_pair(x >> 12), zc2));
                     *reinterpret_cast<uint4*>(arow + 16 * (j ^ (r & 7))) = v;
                 }
                 fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
@@ -239,24 +260,47 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         const int quad = warp & 3;
         const int colh = (warp - 4) >> 2;            // token half of the tile
         const int row = quad * 32 + lane;            // weight row within the tile = TMEM lane
+        const int hl = quad * 32 + lane;             // thread index within this token half (0..127)
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         float T[128];
 #pragma unroll
         for (int j = 0; j < 128; ++j) T[j] = 0.f;
         int gc = 0;
         bool aborted = false;
+        // loads for the next group are issued one group ahead
+        auto load_meta = [&](int tt, int g, float& sv, float& zv, float& xv) {
+            sv = 0.f;
+            zv = 0.f;
+            xv = 0.f;
+            if (tt >= ntiles) return;
+            const int tile = t_first + tt;
+            const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+            const int n = nt * kPBM + row;
+            const int m = mt * kPBN + colh * 128 + hl;
+            if (n < a.N) {
+                sv = bf16_bits_to_float(__ldg(a.scales + (int64_t)n * G + g));
+                zv = (float)__ldg(a.zeros + (int64_t)n * G + g);
+            }
+            if (m < a.M) xv = __ldg(a.xsT + (int64_t)g * a.Mp + m);
+        };
+        float nsv, nzv, nxv;
+        load_meta(0, 0, nsv, nzv, nxv);
         for (int tt = 0; tt < ntiles; ++tt) {
             const int tile = t_first + tt;
             const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
             const int n = nt * kPBM + row;
             const int m0 = mt * kPBN + colh * 128;
             for (int g = 0; g < G; ++g, ++gc) {
-                float sv = 0.f, cz = 0.f;
-                if (n < a.N) {
-                    sv = bf16_bits_to_float(__ldg(a.scales + (int64_t)n * G + g));
-                    cz = 128.f + (float)__ldg(a.zeros + (int64_t)n * G + g);
-                }
-                const float* xs = a.xsT + (int64_t)g * a.Mp + m0;
+                const float sv = nsv, zv = nzv;
+                s_xs[gc & 1][colh * 128 + hl] = nxv;
+                if (g + 1 < G) load_meta(tt, g + 1, nsv, nzv, nxv);
+                else load_meta(tt + 1, 0, nsv, nzv, nxv);
+                // rows whose zero point was not subtracted by the dequantiser (|z| > 128) fold
+                // - s (z - c) xsum with c = 0; the X sums of this half's tokens are in s_xs
+                const float zr = (zv >= -128.f && zv <= 128.f) ? 0.f : zv;
+                named_barrier_sync(2 + colh, 128);
+                const bool need_xs = __any_sync(0xFFFFFFFFu, zr != 0.f);
+                const float* xs = &s_xs[gc & 1][colh * 128];
                 const int dbuf = gc & 1;
                 if (!aborted && !mbar_wait(&mdone[dbuf], (gc >> 1) & 1, a.fault, 91)) aborted = true;
                 if (!aborted) {
@@ -266,17 +310,19 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                         uint32_t d[16];
                         tmem_ld16(tl + dbuf * kPBN + colh * 128 + cc * 16, d);
                         tmem_wait_ld();
+                        if (!need_xs) {
 #pragma unroll
-                        for (int j4 = 0; j4 < 4; ++j4) {
-                            const int mcol = m0 + cc * 16 + 4 * j4;
-                            // xsT rows hold Mp >= M values (the padding is never read past Mp)
-                            float4 xv = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (mcol < a.Mp) xv = __ldg(reinterpret_cast<const float4*>(xs + cc * 16 + 4 * j4));
-                            const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
+                            for (int e = 0; e < 16; ++e) T[cc * 16 + e] = fmaf(sv, __uint_as_float(d[e]), T[cc * 16 + e]);
+                        } else {
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int j = cc * 16 + 4 * j4 + e;
-                                T[j] = fmaf(sv, fmaf(-cz, xq[e], __uint_as_float(d[4 * j4 + e])), T[j]);
+                            for (int j4 = 0; j4 < 4; ++j4) {
+                                const float4 xv = *reinterpret_cast<const float4*>(xs + cc * 16 + 4 * j4);
+                                const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int j = cc * 16 + 4 * j4 + e;
+                                    T[j] = fmaf(sv, fmaf(-zr, xq[e], __uint_as_float(d[4 * j4 + e])), T[j]);
+                                }
                             }
                         }
                     }
