@@ -38,7 +38,7 @@ constexpr int kXsStride = 32;  // tokens per group row of xsum
 constexpr int kMaxTokens = 32;  // tokens per launch
 
 struct DecodeArgs {
-    const uint16_t* Xp;  // [Mc][K] BF16, 8-blocks reordered (0,4,1,5,2,6,3,7)
+    const uint16_t* Xp;  // [Mc][K] BF16, 8-blocks reordered (0,4,1,5,2,6,3,7); the input X itself for M = 1
     const float* xs;     // [G][32] per-group sums of X (zero for tokens >= Mc)
     const uint16_t* scales;
     const int32_t* zeros;
@@ -87,21 +87,11 @@ __device__ __forceinline__ uint4 permute_block(uint4 v) {
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// X -> per-group sums xs, plus the operand layout the GEMV reads:
-//  * tensor-core kernels: BF16 Xp with each 8-block reordered (0,4,1,5,2,6,3,7);
-//  * CUDA-core kernel (fp32_layout): FP32 x_k * 16^-e, e = (0,1,2,3,4,2,3,4)[k mod 8],
-//    as pairs (0,1), (2,5), (3,6), (4,7) of every 8-block, one 144-byte block per
-//    quarter group (32 values + 16 bytes padding so the four quarter readers of a
-//    warp hit distinct banks), then a 32-byte extras block per group:
-//    [xsum, xoff_0..3, 0, 0, 0] with xoff_c = sum over quarter c of
-//    2048 (x_3 + x_6) + 128 (x_4 + x_7) per 8-block (the 2^23 offsets that the
-//    GEMV leaves in its high-position products, removed per quarter instead).
-// Lets the GEMV launch early (PDL).
-constexpr int kQuarterFloats = 36;                       // 32 values + 4 padding
-constexpr int kGroupXfBytes = 4 * kQuarterFloats * 4 + 32;  // 576 + extras = 608 B per group
-
+// X -> per-group sums xs and the B operand of the tensor-core kernels: BF16 Xp
+// with each 8-block reordered (0,4,1,5,2,6,3,7).  Lets the GEMV launch early
+// (PDL).
 __global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict__ X, int M, int K, uint16_t* __restrict__ Xp,
-                                                     float* __restrict__ xs, int fp32_layout) {
+                                                     float* __restrict__ xs) {
     pdl_launch_dependents();
     const int G = K / kGroup;
     const int64_t units = (int64_t)kXsStride * G * 16;  // multiple of 32
@@ -111,42 +101,17 @@ __global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict_
         const int m = (int)(u / (G * 16));
         const int rem = (int)(u - (int64_t)m * G * 16);
         const int g = rem >> 4, blk = rem & 15;
-        float sum = 0.f, off = 0.f;
+        float sum = 0.f;
         if (active && m < M) {
             const int64_t xoff = (int64_t)m * K + (int64_t)g * kGroup + blk * 8;
             const uint4 v = *reinterpret_cast<const uint4*>(X + xoff);
-            const float f[8] = {bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y),
-                                bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w)};
-            if (fp32_layout) {
-                // word blk of the group: quarter blk / 4, 32 bytes per word inside it
-                float* dst = reinterpret_cast<float*>(reinterpret_cast<char*>(Xp) + ((int64_t)m * G + g) * kGroupXfBytes) +
-                             (blk >> 2) * kQuarterFloats + 8 * (blk & 3);
-                reinterpret_cast<float4*>(dst)[0] = make_float4(f[0], f[1] * 0x1p-4f, f[2] * 0x1p-8f, f[5] * 0x1p-8f);
-                reinterpret_cast<float4*>(dst)[1] =
-                    make_float4(f[3] * 0x1p-12f, f[6] * 0x1p-12f, f[4] * 0x1p-16f, f[7] * 0x1p-16f);
-                off = 2048.f * (f[3] + f[6]) + 128.f * (f[4] + f[7]);
-            } else {
-                *reinterpret_cast<uint4*>(Xp + xoff) = permute_block(v);
-            }
-            sum = (f[0] + f[1]) + (f[2] + f[3]) + (f[4] + f[5]) + (f[6] + f[7]);
+            *reinterpret_cast<uint4*>(Xp + xoff) = permute_block(v);
+            sum = ((bf16lo(v.x) + bf16hi(v.x)) + (bf16lo(v.y) + bf16hi(v.y))) +
+                  ((bf16lo(v.z) + bf16hi(v.z)) + (bf16lo(v.w) + bf16hi(v.w)));
         }
 #pragma unroll
         for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        // quarter sums of the offsets: lanes 4q..4q+3 of each 16-lane half hold quarter q
-        off += __shfl_xor_sync(0xFFFFFFFFu, off, 1);
-        off += __shfl_xor_sync(0xFFFFFFFFu, off, 2);
         if (active && blk == 0) xs[(int64_t)g * kXsStride + m] = sum;
-        if (active && fp32_layout && m < M) {
-            float* ext = reinterpret_cast<float*>(reinterpret_cast<char*>(Xp) + ((int64_t)m * G + g) * kGroupXfBytes +
-                                                  4 * kQuarterFloats * 4);
-            if (blk == 0) {
-                ext[0] = sum;
-                ext[5] = 0.f;
-                ext[6] = 0.f;
-                ext[7] = 0.f;
-            }
-            if ((blk & 3) == 0) ext[1 + (blk >> 2)] = off;
-        }
     }
 }
 
@@ -477,81 +442,121 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 //
 // At M = 1 a tensor-core MMA would waste most of its columns and each MMA
 // instruction costs about a hundred cycles however small, so the dot product
-// runs on the FP32 pipes.  Per packed word: one lop3 per code places its
-// nibble in the mantissa of 2^23 (bits 4e, e = 0..4; codes 5-7 after one
-// shift), giving 2^23 + 16^e q; packed FP32 FMAs (fma.f32x2) multiply by
-// x * 16^-e (prepared once per call, exact).  For the low positions (e <= 2)
-// a packed subtract removes 2^23 first; for e = 3, 4 the product keeps
-// 2^(23-4e) x, which is small next to q x and is removed once per quarter
-// group with the prepared offset sum.  Per group, each thread adds
-// s * (its partial sum) to each of its rows, and one of the four threads
-// sharing the group subtracts s * z * xsum.
+// runs on the integer dot-product units (dp4a: four 8-bit x 8-bit products
+// added to a 32-bit accumulator), which take four codes per instruction with
+// no conversion.  Codes become bytes with two logical ops per word:
+// w & 0x0F0F0F0F holds codes 0, 2, 4, 6 and (w >> 4) & 0x0F0F0F0F codes
+// 1, 3, 5, 7.  X is expanded exactly into integers per group: with E the
+// exponent of the group's largest |x|, x_int = x * 2^(22 - E) is a signed
+// integer below 2^23 in magnitude (exact for every x within 2^15 of the
+// group maximum, which a BF16 significand of 8 bits needs; smaller values are
+// rounded at 2^(E - 22), far below FP32 accumulation error), split into three
+// byte planes x_int = 65536 p2 + 256 p1 + p0 (p2 signed).  The inner sums
+// sum_k q_k p_k are exact in int32; per group and row they are combined in
+// FP32 as s * 2^(E - 22) * (sum_k q_k x_int_k - z * sum_k x_int_k).
 //
-// CTA: warp 4 drives TMA (codes of 128 rows x one group with the 64-byte
-// swizzle, the matching 128 x 8 scales and 128 x 4 zero points, the scaled X
-// and its extras) into a 4-stage ring; warps 0-3 compute, thread t taking
-// words 4c..4c+3 (c = t % 4) of rows t/4 + 32i, i = 0..3.  Up to four CTAs
-// share an SM.
-constexpr int kCcWarps = 4;
-constexpr int kCcThreads = (kCcWarps + 1) * 32;
+// X of one group in the layout the kernel reads (400 bytes): four 96-byte
+// quarter blocks (words 4c..4c+3), each word as six 32-bit registers
+// [P0e, P1e, P2e, P0o, P1o, P2o] where Ppe holds plane p of x at k = 0, 2, 4,
+// 6 of the word and Ppo at k = 1, 3, 5, 7 (one byte each), then
+// [sum_k x_int_k (int32), 2^(E - 22) (FP32), -, -].  The 96-byte stride puts
+// the four quarters a warp reads at once in distinct banks.
+constexpr int kQuarterBytes = 96;
+constexpr int kGroupXiBytes = 4 * kQuarterBytes + 16;  // 400 B per group
+
+// The CTA streams units (128 rows x one group) through a 4-stage ring:
+//  * warp 4 (one thread) drives TMA: the codes of each unit (8 KB, 64-byte
+//    swizzle) and, once per block of 8 groups of a row tile, that block's
+//    128 x 8 scales and 128 x 8 zero points into one of two metadata slots;
+//  * warp 5 prepares X for each unit's group straight from the BF16 input
+//    (byte planes, the integer group sum and the group's power of two), so
+//    the call is a single launch;
+//  * warps 0-3 compute, thread t taking words 4c..4c+3 (c = t % 4) of rows
+//    t/4 + 32 i, i = 0..3.
+// Up to four CTAs share an SM.
+constexpr int kCcWarps = 4;                             // compute warps
+constexpr int kCcTmaWarp = kCcWarps;                    // warp 4
+constexpr int kCcXWarp = kCcWarps + 1;                  // warp 5
+constexpr int kCcThreads = (kCcWarps + 2) * 32;
 constexpr int kCcStages = 4;
 constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
-constexpr int kCcScOff = kCcCodeBytes;                  // scales box: 128 rows x 8 groups (BF16)
-constexpr int kCcZeOff = kCcScOff + kRowsPerCta * 16;   // zeros box: 128 rows x 4 groups (int32)
-constexpr int kCcXOff = kCcZeOff + kRowsPerCta * 16;    // scaled FP32 X of the group + extras (608 B)
-constexpr int kCcExtOff = kCcXOff + 4 * kQuarterFloats * 4;
-constexpr int kCcStageBytes = 13 * 1024;                // keeps stages 1024-aligned
-constexpr size_t kCcSmem = (size_t)kCcStages * kCcStageBytes + 1024;
-static_assert(kCcXOff + kGroupXfBytes <= kCcStageBytes, "stage layout");
+constexpr int kCcXOff = kCcCodeBytes;                   // X planes of the group + extras (400 B)
+constexpr int kCcExtOff = kCcXOff + 4 * kQuarterBytes;
+constexpr int kCcStageBytes = 9 * 1024;                 // keeps stages 1024-aligned
+constexpr int kCcMetaGroups = 8;                        // groups per metadata block
+constexpr int kCcScBytes = kRowsPerCta * kCcMetaGroups * 2;  // 128 rows x 8 BF16 scales
+constexpr int kCcZeBytes = kRowsPerCta * kCcMetaGroups * 4;  // 128 rows x 8 int32 zero points
+constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;   // one slot, 6 KB
+constexpr int kCcMetaOff = kCcStages * kCcStageBytes;   // two slots after the ring
+constexpr size_t kCcSmem = (size_t)kCcMetaOff + 2 * kCcMetaBytes + 1024;
+static_assert(kCcXOff + kGroupXiBytes <= kCcStageBytes, "stage layout");
+// A metadata slot is rewritten two blocks later.  Blocks are aligned to 8
+// groups inside a row tile (the kernel needs G % 8 == 0), so the block in
+// between has 8 units; with at most kCcStages units in flight, every unit of
+// the older block has been released by then.
+static_assert(kCcStages <= kCcMetaGroups, "metadata slot reuse");
 
-// acc (two FP32 lanes) (+)= sum over one packed word of q_k * x_k (plus the
-// 2^(23-4e) x offsets of the e = 3, 4 positions).  xp0..xp3 are the scaled X
-// pairs (0,1), (2,5), (3,6), (4,7); m2 holds (2^23, 2^23).
-#define W4A16_WORD_DOT_BODY(FIRST_FMA)                                    \
-    "{\n\t"                                                                \
-    ".reg .b32 h, a0, a1, a2, a5, a3, a6, a4, a7;\n\t"                     \
-    ".reg .b64 v0, v1, v2, v3;\n\t"                                        \
-    "shr.b32 h, %1, 12;\n\t"                                               \
-    "lop3.b32 a0, %1, 0x0000000F, 0x4B000000, 0xEA;\n\t"                   \
-    "lop3.b32 a1, %1, 0x000000F0, 0x4B000000, 0xEA;\n\t"                   \
-    "lop3.b32 a2, %1, 0x00000F00, 0x4B000000, 0xEA;\n\t"                   \
-    "lop3.b32 a5, h, 0x00000F00, 0x4B000000, 0xEA;\n\t"                    \
-    "lop3.b32 a3, %1, 0x0000F000, 0x4B000000, 0xEA;\n\t"                   \
-    "lop3.b32 a6, h, 0x0000F000, 0x4B000000, 0xEA;\n\t"                    \
-    "lop3.b32 a4, %1, 0x000F0000, 0x4B000000, 0xEA;\n\t"                   \
-    "lop3.b32 a7, h, 0x000F0000, 0x4B000000, 0xEA;\n\t"                    \
-    "mov.b64 v0, {a0, a1};\n\t"                                            \
-    "mov.b64 v1, {a2, a5};\n\t"                                            \
-    "mov.b64 v2, {a3, a6};\n\t"                                            \
-    "mov.b64 v3, {a4, a7};\n\t"                                            \
-    "sub.rn.f32x2 v0, v0, %6;\n\t"                                         \
-    "sub.rn.f32x2 v1, v1, %6;\n\t" FIRST_FMA                              \
-    "fma.rn.f32x2 %0, v1, %3, %0;\n\t"                                     \
-    "fma.rn.f32x2 %0, v2, %4, %0;\n\t"                                     \
-    "fma.rn.f32x2 %0, v3, %5, %0;\n\t"                                     \
-    "}"
-
-// acc (two FP32 lanes) (+)= sum over one packed word of q_k * x_k (plus the
-// 2^(23-4e) x offsets of the e = 3, 4 positions).  xp0..xp3 are the scaled X
-// pairs (0,1), (2,5), (3,6), (4,7); m2 holds (2^23, 2^23).  FIRST starts acc.
-template <bool FIRST>
-__device__ __forceinline__ void word_dot(unsigned long long& acc, uint32_t w, unsigned long long xp0,
-                                         unsigned long long xp1, unsigned long long xp2, unsigned long long xp3,
-                                         unsigned long long m2) {
-    if (FIRST)
-        asm(W4A16_WORD_DOT_BODY("mul.rn.f32x2 %0, v0, %2;\n\t")
-            : "=l"(acc)
-            : "r"(w), "l"(xp0), "l"(xp1), "l"(xp2), "l"(xp3), "l"(m2));
-    else
-        asm(W4A16_WORD_DOT_BODY("fma.rn.f32x2 %0, v0, %2, %0;\n\t")
-            : "+l"(acc)
-            : "r"(w), "l"(xp0), "l"(xp1), "l"(xp2), "l"(xp3), "l"(m2));
+__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
 }
 
-__device__ __forceinline__ float lanes_sum(unsigned long long v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-    return lo + hi;
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// 2^e as FP32 for e in [-149, 127] (subnormal below -126).
+__device__ __forceinline__ float pow2f(int e) {
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
+}
+
+// One warp writes group g's X in the layout above: lane 2w + h holds values
+// 4h..4h+3 of word w.
+__device__ __forceinline__ void prep_group_x(const uint16_t* __restrict__ X, int g, unsigned char* dst, int lane) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(X + (int64_t)g * kGroup + lane * 4));
+    const uint32_t bits[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
+    uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
+    amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+    const int ef = (int)(amax >> 7);            // biased exponent of the largest |x| (0: zero or subnormal)
+    const int E = ef == 0 ? -127 : ef - 127;    // every |x| of the group is below 2^(E + 1)
+    const int k = 22 - E;                       // in [-105, 149]
+    const int k1 = min(k, 127);
+    const float s1 = pow2f(k1), s2 = pow2f(k - k1);  // exact scalings, |x * 2^k| < 2^23
+    int xi[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xi[i] = __float2int_rn(__uint_as_float(bits[i] << 16) * s1 * s2);
+    // planes of this lane's values: plane p of x_i is byte p of xi (plane 2 signed)
+    uint32_t m[3];
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+        const uint32_t b0 = ((uint32_t)xi[0] >> (8 * p)) & 0xFFu, b1 = ((uint32_t)xi[1] >> (8 * p)) & 0xFFu;
+        const uint32_t b2 = ((uint32_t)xi[2] >> (8 * p)) & 0xFFu, b3 = ((uint32_t)xi[3] >> (8 * p)) & 0xFFu;
+        m[p] = b0 | (b2 << 8) | (b1 << 16) | (b3 << 24);  // [even half | odd half]
+    }
+    const int h = lane & 1, w = lane >> 1;
+    uint32_t* out = reinterpret_cast<uint32_t*>(dst + (w >> 2) * kQuarterBytes + (w & 3) * 24 + h * 12);
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+        const uint32_t pm = __shfl_xor_sync(0xFFFFFFFFu, m[p], 1);
+        // h = 0 assembles the even register (its values 0, 2 then the partner's 4, 6),
+        // h = 1 the odd one (the partner's 1, 3 then its own 5, 7)
+        out[p] = h ? __byte_perm(pm, m[p], 0x7632) : __byte_perm(m[p], pm, 0x5410);
+    }
+    const int sum = __reduce_add_sync(0xFFFFFFFFu, (xi[0] + xi[1]) + (xi[2] + xi[3]));  // |sum| < 2^30
+    if (lane == 0) {
+        int* ext = reinterpret_cast<int*>(dst + 4 * kQuarterBytes);
+        ext[0] = sum;
+        reinterpret_cast<float*>(ext)[1] = pow2f(E - 22);
+    }
+}
+
+// All lanes wait; the warp gives up together if any lane's wait ran out.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, int parity, int* fault, int site) {
+    const bool ok = mbar_wait(bar, parity, fault, site);
+    return __all_sync(0xFFFFFFFFu, ok);
 }
 
 __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
@@ -563,7 +568,9 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
     __shared__ int s_last;
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    unsigned char* meta = ring + kCcMetaOff;
 
+    pdl_launch_dependents();  // the next call may start its weight loads as this grid's CTAs retire
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
     const int64_t u_first = (int64_t)b * a.units_base + min(b, a.units_rem);
@@ -572,48 +579,54 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCcStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 2);  // TMA thread (with the transaction bytes) + X warp
             mbar_init(&empty[s], kCcWarps);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == kCcWarps) {  // ---------------------------------------------- TMA
+    if (warp == kCcTmaWarp) {  // ------------------------------------------- TMA
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tsc);
             prefetch_tmap(&tze);
-            constexpr uint32_t kTx = kCcCodeBytes + 2 * kRowsPerCta * 16 + kGroupXfBytes;
-            const char* xf = reinterpret_cast<const char*>(a.Xp);
-            const int pre = min(kCcStages, nunits);
+            // the weights need nothing from the preceding kernel: no PDL wait here
             UnitCursor cur(u_first, G);
-            for (int i = 0; i < pre; ++i, cur.next(G)) {  // the weights need nothing from the preparation kernel
-                unsigned char* st = ring + i * kCcStageBytes;
-                mbar_arrive_expect_tx(&full[i], kTx);
-                tma_load_2d(st, &tq, cur.g * kWordsPerGroup, cur.tile * kRowsPerCta, &full[i]);
-                tma_load_2d(st + kCcScOff, &tsc, cur.g & ~7, cur.tile * kRowsPerCta, &full[i]);
-                tma_load_2d(st + kCcZeOff, &tze, cur.g & ~3, cur.tile * kRowsPerCta, &full[i]);
-            }
-            pdl_wait_primary();  // scaled X and its extras come from the preparation kernel
-            UnitCursor cx(u_first, G);
-            for (int i = 0; i < pre; ++i, cx.next(G))
-                bulk_load(ring + i * kCcStageBytes + kCcXOff, xf + (int64_t)cx.g * kGroupXfBytes, kGroupXfBytes,
-                          &full[i]);
-            int issued = pre;
-            for (int i = pre; i < nunits; ++i, cur.next(G)) {
+            int mb = -1, issued = 0;
+            for (int i = 0; i < nunits; ++i, cur.next(G)) {
                 const int s = i % kCcStages;
-                if (!mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) break;
+                if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) break;
+                const bool new_block = i == 0 || (cur.g & (kCcMetaGroups - 1)) == 0;
+                if (new_block) ++mb;
                 unsigned char* st = ring + s * kCcStageBytes;
-                mbar_arrive_expect_tx(&full[s], kTx);
+                mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (new_block ? kCcMetaBytes : 0));
                 tma_load_2d(st, &tq, cur.g * kWordsPerGroup, cur.tile * kRowsPerCta, &full[s]);
-                tma_load_2d(st + kCcScOff, &tsc, cur.g & ~7, cur.tile * kRowsPerCta, &full[s]);
-                tma_load_2d(st + kCcZeOff, &tze, cur.g & ~3, cur.tile * kRowsPerCta, &full[s]);
-                bulk_load(st + kCcXOff, xf + (int64_t)cur.g * kGroupXfBytes, kGroupXfBytes, &full[s]);
+                if (new_block) {
+                    unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
+                    const int g8 = cur.g & ~(kCcMetaGroups - 1);
+                    tma_load_2d(ms, &tsc, g8, cur.tile * kRowsPerCta, &full[s]);
+                    tma_load_2d(ms + kCcScBytes, &tze, g8, cur.tile * kRowsPerCta, &full[s]);
+                }
                 ++issued;
             }
+            // no copy may still be in flight when the CTA exits
             for (int i = max(0, issued - kCcStages); i < issued; ++i)
                 mbar_wait(&full[i % kCcStages], (i / kCcStages) & 1, a.fault, 52);
+        }
+        return;
+    }
+
+    if (warp == kCcXWarp) {  // ------------------------------------------ X warp
+        pdl_wait_primary();  // X may come from the preceding kernel
+        const uint16_t* X = a.Xp;
+        UnitCursor cur(u_first, G);
+        for (int i = 0; i < nunits; ++i, cur.next(G)) {
+            const int s = i % kCcStages;
+            if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
+            prep_group_x(X, cur.g, ring + s * kCcStageBytes + kCcXOff, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[s]);
         }
         return;
     }
@@ -625,7 +638,6 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
     // the 64-byte swizzle of the codes tile: logical chunk c of row r sits at chunk c ^ ((r >> 1) & 3);
     // (r >> 1) & 3 is the same for the four rows rg + 32 i
     const int code_off = rg * 64 + 16 * (c ^ ((rg >> 1) & 3));
-    const int meta_off = rg * 16;
     float y[4] = {0.f, 0.f, 0.f, 0.f};
     int cur_tile = -1;
     bool aborted = false;
@@ -677,17 +689,18 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         for (int i = 0; i < 4; ++i) y[i] = 0.f;
     };
 
-    const unsigned long long m2 = 0x4B0000004B000000ull;
     UnitCursor uc(u_first, G);
+    int mb = -1;
     for (int i = 0; i < nunits; ++i, uc.next(G)) {
         const int tile = uc.tile, g = uc.g;
+        if (i == 0 || (g & (kCcMetaGroups - 1)) == 0) ++mb;
         if (tile != cur_tile) {
             if (cur_tile >= 0) flush(cur_tile);
             cur_tile = tile;
         }
         if (aborted) continue;
         const int s = i % kCcStages;
-        if (!mbar_wait(&full[s], (i / kCcStages) & 1, a.fault, 53)) {
+        if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 53)) {
             aborted = true;
             continue;
         }
@@ -695,34 +708,54 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         uint4 w[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) w[r] = *reinterpret_cast<const uint4*>(st + code_off + 2048 * r);
-        const ulonglong2* xq = reinterpret_cast<const ulonglong2*>(st + kCcXOff + c * kQuarterFloats * 4);
-        ulonglong2 xw[8];
+        // X planes of words 4c..4c+3: word j's registers at xr[6j .. 6j+5]
+        uint32_t xr[24];
+        const uint4* xq = reinterpret_cast<const uint4*>(st + kCcXOff + c * kQuarterBytes);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) xw[j] = xq[j];
-        const float* ext = reinterpret_cast<const float*>(st + kCcExtOff);
-        const float xsum = ext[0], xoff = ext[1 + c];
-        const unsigned char* scb = st + kCcScOff + meta_off + 2 * (g & 7);
-        const unsigned char* zeb = st + kCcZeOff + meta_off + 4 * (g & 3);
+        for (int j = 0; j < 6; ++j) {
+            const uint4 v = xq[j];
+            xr[4 * j] = v.x;
+            xr[4 * j + 1] = v.y;
+            xr[4 * j + 2] = v.z;
+            xr[4 * j + 3] = v.w;
+        }
+        const int* ext = reinterpret_cast<const int*>(st + kCcExtOff);
+        const int xsum = ext[0];
+        const float xscale = __int_as_float(ext[1]);
+        // this block's metadata (loaded with its first unit, which this warp has already waited for)
+        const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
+        const unsigned char* scb = ms + rg * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1));
+        const unsigned char* zeb = ms + kCcScBytes + rg * (kCcMetaGroups * 4) + 4 * (g & (kCcMetaGroups - 1));
         float sv[4], zv[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             // rows past N were zero-filled by TMA: s = 0 folds them away
-            sv[r] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(scb + 512 * r));
-            zv[r] = (float)*reinterpret_cast<const int32_t*>(zeb + 512 * r);
+            sv[r] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(scb + 32 * kCcMetaGroups * 2 * r));
+            zv[r] = (float)*reinterpret_cast<const int32_t*>(zeb + 32 * kCcMetaGroups * 4 * r);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
-        const float corr = (c == 0) ? xsum : 0.f;
+        const float corr = (c == 0) ? (float)xsum : 0.f;  // one thread of four folds the zero point
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            unsigned long long acc;
-            word_dot<true>(acc, w[r].x, xw[0].x, xw[0].y, xw[1].x, xw[1].y, m2);
-            word_dot<false>(acc, w[r].y, xw[2].x, xw[2].y, xw[3].x, xw[3].y, m2);
-            word_dot<false>(acc, w[r].z, xw[4].x, xw[4].y, xw[5].x, xw[5].y, m2);
-            word_dot<false>(acc, w[r].w, xw[6].x, xw[6].y, xw[7].x, xw[7].y, m2);
-            // y += s * (sum q x + offsets - xoff  -  [one thread of four] z xsum)
-            y[r] = fmaf(sv[r], fmaf(-zv[r], corr, lanes_sum(acc) - xoff), y[r]);
+            const uint32_t wr[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
+            int p0 = 0, p1 = 0, p2 = 0;  // sum_k q_k * plane_p(x_k) over this thread's 32 codes
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t ce = wr[j] & 0x0F0F0F0Fu, co = (wr[j] >> 4) & 0x0F0F0F0Fu;  // codes 0,2,4,6 / 1,3,5,7
+                p0 = dp4a_uu(ce, xr[6 * j], p0);
+                p1 = dp4a_uu(ce, xr[6 * j + 1], p1);
+                p2 = dp4a_us(ce, xr[6 * j + 2], p2);
+                p0 = dp4a_uu(co, xr[6 * j + 3], p0);
+                p1 = dp4a_uu(co, xr[6 * j + 4], p1);
+                p2 = dp4a_us(co, xr[6 * j + 5], p2);
+            }
+            // sum q x_int = 65536 p2 + (256 p1 + p0): the bracket is exact in int32 (< 2^25),
+            // the rest is FP32 with one rounding per step
+            const float qx = fmaf((float)p2, 65536.f, (float)(p1 * 256 + p0));
+            // y += s 2^(E-22) (sum q x_int  -  [one thread of four] z sum x_int)
+            y[r] = fmaf(sv[r] * xscale, fmaf(-zv[r], corr, qx), y[r]);
         }
     }
     if (cur_tile >= 0) flush(cur_tile);
@@ -792,9 +825,9 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     else if (kind == 2)  // scales: bf16 [rows = N][cols = G], box = 8 groups x 128 rows
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 2, 8, kRowsPerCta);
-    else if (kind == 3)  // zeros: int32 [rows = N][cols = G], box = 4 groups x 128 rows
+    else if (kind == 3)  // zeros: int32 [rows = N][cols = G], box = 8 groups x 128 rows
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_INT32, ptr, (uint64_t)cols, (uint64_t)rows,
-                            (uint64_t)cols * 4, 4, kRowsPerCta);
+                            (uint64_t)cols * 4, kCcMetaGroups, kRowsPerCta);
     else  // prepared X: bf16 [rows = Mc][cols = K], box = 64 x NTOK (kind), 128-byte swizzle
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 2, 64, (uint32_t)kind, CU_TENSOR_MAP_SWIZZLE_128B);
@@ -858,8 +891,9 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.units_base = (int)(units / grid);
     p.units_rem = (int)(units % grid);
     p.max_slots = (int)((G - 1) / p.units_base + 2);
-    p.ws_xp_bytes = align256(p.nt == 1 ? (size_t)G * kGroupXfBytes : (size_t)Mc * K * 2);
-    p.ws_xs_bytes = align256((size_t)G * kXsStride * 4);
+    // the single-token kernel prepares X itself
+    p.ws_xp_bytes = p.nt == 1 ? 0 : align256((size_t)Mc * K * 2);
+    p.ws_xs_bytes = p.nt == 1 ? 0 : align256((size_t)G * kXsStride * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
     p.ws_counter_bytes = align256((size_t)p.row_tiles * 4);
     return p;
@@ -884,13 +918,15 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
         const int Mc = (int)((M - m0) < kMaxTokens ? (M - m0) : kMaxTokens);
         CUtensorMap tx;
         if (plan.nt > 1 && !cached_tmap(plan.nt, Xp, Mc, K, &tx)) return W4A16_ERR_CUDA;
-        const int64_t prep_units = (int64_t)kXsStride * G * 16;
-        int prep_grid = (int)ceil_div(prep_units, 256);
-        if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
-        prep_x_kernel<<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, Xp, xs, plan.nt == 1 ? 1 : 0);
-        if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
+        if (plan.nt > 1) {
+            const int64_t prep_units = (int64_t)kXsStride * G * 16;
+            int prep_grid = (int)ceil_div(prep_units, 256);
+            if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
+            prep_x_kernel<<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, Xp, xs);
+            if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
+        }
         DecodeArgs args;
-        args.Xp = Xp;
+        args.Xp = plan.nt == 1 ? X + m0 * K : Xp;  // the single-token kernel reads X as given
         args.xs = xs;
         args.scales = scales;
         args.zeros = zeros;
