@@ -331,21 +331,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 #pragma unroll
             for (int m = 0; m < NTOK; ++m)
                 if (m < M) part[m * kRowsPerCta + row_local] = acc[m];
-            __threadfence();
             named_barrier_sync(1, kFoldWarps * 32);
-            if (threadIdx.x == 0) {
-                const int prev = atomicAdd(&a.counters[tile], 1);
-                s_last = (prev == nseg - 1);
-            }
+            if (threadIdx.x == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
             named_barrier_sync(1, kFoldWarps * 32);
             if (s_last) {
-                __threadfence();
                 const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
                 const float* pb = a.partial + (int64_t)tile * a.max_slots * M * kRowsPerCta;
                 for (int idx = threadIdx.x; idx < M * rows; idx += kFoldWarps * 32) {
                     const int m = idx / rows, rl = idx - m * rows;
-                    float sum = 0.f;
-                    for (int sl = 0; sl < nseg; ++sl) sum += __ldcg(pb + ((int64_t)sl * M + m) * kRowsPerCta + rl);
+                    const float sum = sum_slots(pb + (int64_t)m * kRowsPerCta + rl, (int64_t)M * kRowsPerCta, nseg);
                     a.Y[(int64_t)m * N + tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
                 }
                 if (threadIdx.x == 0) a.counters[tile] = 0;
@@ -665,22 +659,14 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 4; ++i) part[rg + 32 * i] = y[i];
             }
-            __threadfence();
             named_barrier_sync(1, kCcWarps * 32);
-            if (t == 0) {
-                const int prev = atomicAdd(&a.counters[tile], 1);
-                s_last = (prev == nseg - 1);
-            }
+            if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
             named_barrier_sync(1, kCcWarps * 32);
             if (s_last) {
-                __threadfence();
                 const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
                 const float* pb = a.partial + (int64_t)tile * a.max_slots * kRowsPerCta;
-                for (int rl = t; rl < rows; rl += kCcWarps * 32) {
-                    float sum = 0.f;
-                    for (int sl = 0; sl < nseg; ++sl) sum += __ldcg(pb + (int64_t)sl * kRowsPerCta + rl);
-                    a.Y[tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
-                }
+                for (int rl = t; rl < rows; rl += kCcWarps * 32)
+                    a.Y[tile * kRowsPerCta + rl] = float_to_bf16_bits(sum_slots(pb + rl, kRowsPerCta, nseg));
                 if (t == 0) a.counters[tile] = 0;
             }
             named_barrier_sync(1, kCcWarps * 32);

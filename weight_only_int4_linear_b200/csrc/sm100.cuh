@@ -89,6 +89,27 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 
 // Programmatic dependent launch: let the next kernel on the stream start its
 // prologue, and wait for the previous kernel's results.
+// Split-K arrival: returns the counter's previous value.  Release orders the
+// CTA's partial-sum stores (made CTA-visible by the barrier before it) ahead
+// of the increment; acquire lets the last arriver read every other CTA's.
+__device__ __forceinline__ int arrive_acq_rel_gpu(int* counter) {
+    int prev;
+    asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
+    return prev;
+}
+
+// Sum of nseg partial values p[0], p[stride], ... in a fixed order, with up
+// to four L2 loads in flight.
+__device__ __forceinline__ float sum_slots(const float* p, int64_t stride, int nseg) {
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < nseg; s0 += 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (s0 + j < nseg) s4[j] += __ldcg(p + (s0 + j) * stride);
+    }
+    return (s4[0] + s4[1]) + (s4[2] + s4[3]);
+}
+
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
