@@ -38,6 +38,32 @@ METRIC = "W4A16 effective weight GB/s (% HBM peak) at M=1; TFLOP/s (% BF16 peak)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (read + write) per launch of the dominant kernels, from one ncu capture each
+# (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
+# so each carries the sha256 of that source file; after any change it reads as null.
+NCU_TRAFFIC = {
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154175232 + dram__bytes_write.sum 3229440
+    ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
+                                      "sha256": "5da302d446d84ba505dec75ea1a4bf8be443db1d55ab8fe547c84f976303a262",
+                                      "bytes": 157404672},
+    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 7776783872 + write 468124928
+    ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
+                                          "sha256": "1a3ec3cf5010e7434b861f412d54b3c9b7baec54e4659889d58d6f1695c8823b",
+                                          "bytes": 8244908800},
+}
+
+
+def ncu_traffic(kernel: str, layer: str):
+    import hashlib
+    rec = NCU_TRAFFIC.get((kernel, layer))
+    if not rec or rec["bytes"] is None:
+        return None
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["sha256"]:
+            return None
+    return rec["bytes"]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -45,6 +71,22 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def max_over_ranks(x: float, device: str) -> float:
+    """Max of a per-rank float over the process group (device time of the slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(bytes_per_step_per_rank: float, steps: int, ms: float, world: int) -> float:
+    """GB/s of the whole job: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_step_per_rank * steps / (ms * 1e-3) / 1e9
 
 
 def dist_env():
@@ -135,39 +177,14 @@ PREFILL_MIN_M = 64  # the library's automatic path choice: M >= 64 takes the ten
 
 
 def launches_per_call(c) -> int:
-    """Our kernels per linear call: X preparation + GEMM (M >= 64), else
-    X preparation + GEMV per 32-token chunk."""
+    """Our kernels per linear call: X preparation + GEMM (M >= 64); one
+    single-token GEMV (M = 1, K/128 a multiple of 8, X prepared inside it);
+    else X preparation + GEMV per 32-token chunk."""
     if c.M >= PREFILL_MIN_M:
         return 2
+    if c.M == 1 and (c.K // 128) % 8 == 0:
+        return 1
     return 2 * ((c.M + 31) // 32)
-
-
-class ExternalEvents:
-    """CUDA events recorded as external event nodes inside a captured graph, so
-    each replay times the kernels between them (cudaEventRecordExternal)."""
-
-    def __init__(self, n):
-        from cuda.bindings import runtime as rt
-        self.rt = rt
-        self.ev = []
-        for _ in range(n):
-            err, e = rt.cudaEventCreate()
-            assert int(err) == 0, err
-            self.ev.append(e)
-
-    def record(self, i, stream_handle):
-        err, = self.rt.cudaEventRecordWithFlags(self.ev[i], self.rt.cudaStream_t(stream_handle),
-                                                 self.rt.cudaEventRecordExternal)
-        assert int(err) == 0, err
-
-    def elapsed(self, i, j):
-        err, ms = self.rt.cudaEventElapsedTime(self.ev[i], self.ev[j])
-        assert int(err) == 0, err
-        return ms
-
-    def close(self):
-        for e in self.ev:
-            self.rt.cudaEventDestroy(e)
 
 
 def _linear_call(w4, L, path):
@@ -218,32 +235,50 @@ def time_steps(layers, steps, warmup, torch, w4, stream, path, block=50):
     return total_ms
 
 
-def time_per_layer(layers, torch, w4, stream, path, steps=20, replays=5):
-    """Mean device time of each layer's call inside the real step sequence
-    (external event nodes around every call of a captured multi-step graph)."""
-    n = len(layers)
-    ev = ExternalEvents(2 * n * steps)
+def time_layer_alone(c, torch, w4, stream, min_calls=200):
+    """Device time of one call of layer `c` (CUDA events on the launching
+    stream): back-to-back calls replayed from a CUDA graph, each call reading a
+    different copy of the packed weights, rotating through enough copies that
+    their codes exceed 3x L2.  Returns (us per call, copies)."""
+    W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
+    synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+    copies = max(1, min(32, -(-3 * L2_BYTES // c.code_bytes)))
+    pws = [w4.PackedWeight.from_float(W, stream=stream) for _ in range(copies)]
+    torch.cuda.synchronize()
+    del W
+    if any(int(pw.status.item()) != 0 for pw in pws):
+        raise RuntimeError(f"packing failed for {c.name}")
+    xb = synth.activations_bf16(c.x_seed, c.M, c.K)
+    X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+    nb = w4.workspace_bytes(c.M, c.N, c.K)
+    ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device="cuda")
+    passes = max(1, -(-min_calls // copies)) if c.M < 512 else 1
 
     def body():
-        h = torch.cuda.current_stream().cuda_stream
-        for s in range(steps):
-            for i, L in enumerate(layers):
-                ev.record(2 * (s * n + i), h)
-                _linear_call(w4, L, path)
-                ev.record(2 * (s * n + i) + 1, h)
-
+        for _ in range(passes):
+            for pw in pws:
+                w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y, ws)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            body()
+    torch.cuda.synchronize()
     g = capture(torch, stream, body)
-    times = [[] for _ in range(n)]
-    for _ in range(replays):
-        with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
             g.replay()
-        torch.cuda.synchronize()
-        for s in range(1, steps):  # first step of a replay follows the idle host gap
-            for i in range(n):
-                times[i].append(ev.elapsed(2 * (s * n + i), 2 * (s * n + i) + 1))
-    del g
-    ev.close()
-    return [statistics.mean(t) for t in times]
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * passes * copies)
+    del g, pws, X, Y, ws
+    torch.cuda.empty_cache()
+    return us, copies
 
 
 def time_e2e(layers, steps, warmup, torch, w4, stream, path):
@@ -271,6 +306,110 @@ def time_e2e(layers, steps, warmup, torch, w4, stream, path):
     h2d = sum(L["X"].numel() * 2 for L in layers)
     d2h = sum(L["Y"].numel() * 2 for L in layers)
     return start.elapsed_time(end), h2d, d2h
+
+
+# ----------------------------------------------------------------------------------------------
+# the 80-layer decode stack (hidden 8192, M = 1), all packed weights resident
+# ----------------------------------------------------------------------------------------------
+
+STACK_LAYERS = 80
+STACK_DOWN_IN = 28672  # down reads the first half of gate+up's output, renormalised
+
+
+def build_stack(torch, w4, stream, n_layers=STACK_LAYERS):
+    """Packed weights of layers 0 .. n_layers-1 (seed = layer index), generated and packed on the device."""
+    cases0 = workloads.stack_layer(0)
+    Wtmp = torch.empty(max(c.N * c.K for c in cases0), dtype=torch.float32, device="cuda")
+    layers = []
+    for layer in range(n_layers):
+        mats = []
+        for c in workloads.stack_layer(layer):
+            synth.fill_weights_device(c.w_seed, c.w_tag, Wtmp.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+            mats.append(w4.PackedWeight.from_float(Wtmp[: c.N * c.K].view(c.N, c.K), stream=stream))
+        layers.append(mats)
+    torch.cuda.synchronize()
+    del Wtmp
+    for layer, mats in enumerate(layers):
+        for pw in mats:
+            if int(pw.status.item()) != 0:
+                raise RuntimeError(f"packing failed in stack layer {layer}")
+    return layers
+
+
+class StackBuffers:
+    def __init__(self, torch, w4, layers):
+        qkv, o, gu, down = layers[0]
+        bf = dict(dtype=torch.bfloat16, device="cuda")
+        self.h = [torch.empty((1, qkv.K), **bf), torch.empty((1, qkv.K), **bf)]
+        self.y_qkv = torch.empty((1, qkv.N), **bf)
+        self.y_o = torch.empty((1, o.N), **bf)
+        self.y_gu = torch.empty((1, gu.N), **bf)
+        self.u = torch.empty((1, STACK_DOWN_IN), **bf)
+        self.y_down = torch.empty((1, down.N), **bf)
+        nb = max(w4.workspace_bytes(1, pw.N, pw.K) for pw in layers[0])
+        self.ws = torch.zeros(max(nb, 256), dtype=torch.uint8, device="cuda")
+
+
+def stack_step(w4, layers, buf, record=()):
+    """One decode step through the stack from buf.h[0]: per layer qkv, o and
+    gate+up read the hidden state h; down reads u = renorm(gate+up[:, :28672]);
+    the next hidden state is renorm(down).  Returns (final h, {layer: copies of
+    that layer's inputs and outputs} for the layers in `record`)."""
+    h = buf.h[0]
+    rec = {}
+    for layer, (p_qkv, p_o, p_gu, p_down) in enumerate(layers):
+        w4.linear(h, p_qkv.qweight, p_qkv.scales, p_qkv.zeros, buf.y_qkv, buf.ws)
+        w4.linear(h, p_o.qweight, p_o.scales, p_o.zeros, buf.y_o, buf.ws)
+        w4.linear(h, p_gu.qweight, p_gu.scales, p_gu.zeros, buf.y_gu, buf.ws)
+        w4.renorm_rows(buf.y_gu[:, :STACK_DOWN_IN], buf.u)
+        w4.linear(buf.u, p_down.qweight, p_down.scales, p_down.zeros, buf.y_down, buf.ws)
+        h_next = buf.h[(layer + 1) % 2]
+        w4.renorm_rows(buf.y_down, h_next)
+        if layer in record:
+            rec[layer] = {"h": h.clone(), "qkv": buf.y_qkv.clone(), "o_proj": buf.y_o.clone(),
+                          "gate_up": buf.y_gu.clone(), "u": buf.u.clone(), "down": buf.y_down.clone()}
+        h = h_next
+    return h, rec
+
+
+def run_stack(torch, w4, stream, steps):
+    """Aggregate weight GB/s of the 80-layer stack: one step = 320 linear calls + 160 renorms, replayed
+    from a CUDA graph; the step starts from the same X each time."""
+    layers = build_stack(torch, w4, stream)
+    buf = StackBuffers(torch, w4, layers)
+    c0 = workloads.stack_layer(0)
+    x0 = torch.from_numpy(synth.activations_bf16(c0[0].x_seed, 1, c0[0].K).view(np.int16)).cuda().view(torch.bfloat16)
+    code_bytes = sum(pw.N * pw.K // 2 for mats in layers for pw in mats)
+
+    def body():
+        buf.h[0].copy_(x0)
+        stack_step(w4, layers, buf)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            body()
+    torch.cuda.synchronize()
+    g = capture(torch, stream, body)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(steps):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    fault = w4.device_fault()
+    del g, layers, buf
+    torch.cuda.empty_cache()
+    if fault:
+        raise RuntimeError(f"a kernel gave up a bounded wait (site {fault}) in the stack")
+    return {"value": code_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "workload": "decode_stack_80x8192",
+            "ms_per_step": ms, "steps": steps, "packed_code_bytes": code_bytes,
+            "launches_per_step": STACK_LAYERS * (4 + 2),
+            "note": "aggregate packed-code GB/s over 80 layers x {qkv, o, gate+up, down} chained on one "
+                    "stream with the renorm kernels between them (their time included)"}
 
 
 def cpu_baseline(cases, budget_s=12.0):
@@ -326,27 +465,25 @@ def run_ours(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         total_ms = time_steps(layers, args.steps, args.warmup, torch, w4, stream, w4.PATH_AUTO)
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * code_bytes * args.steps / (total_ms * 1e-3) / 1e9
-    per_layer = time_per_layer(layers, torch, w4, stream, w4.PATH_AUTO)
-    fault = w4.device_fault()
-    if fault != 0:
-        raise RuntimeError(f"a kernel gave up a bounded wait (site {fault}); results invalid")
-
-    # dominant kernel: the largest layer (gate+up)
-    dom = max(range(len(cases)), key=lambda i: cases[i].code_bytes)
-    dom_ms = per_layer[dom]
-    dom_gbs = cases[dom].code_bytes / (dom_ms * 1e-3) / 1e9
-    dom_all = (cases[dom].code_bytes + cases[dom].meta_bytes) / (dom_ms * 1e-3) / 1e9
+    total_ms = max_over_ranks(total_ms, "cuda")
+    value = whole_job_rate(code_bytes, args.steps, total_ms, world)
 
     # end to end through the public API with host buffers
     e2e_ms, h2d, d2h = time_e2e(layers, args.steps, args.warmup, torch, w4, stream, w4.PATH_AUTO)
-    e2e_value = world * code_bytes * args.steps / (e2e_ms * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(e2e_ms, "cuda")
+    e2e_value = whole_job_rate(code_bytes, args.steps, e2e_ms, world)
     del layers
     torch.cuda.empty_cache()
+
+    # each layer's kernel alone (an M = 1 call is one launch); dominant kernel: gate+up
+    per_layer = [time_layer_alone(c, torch, w4, stream)[0] for c in cases]
+    dom = max(range(len(cases)), key=lambda i: cases[i].code_bytes)
+    dom_us = per_layer[dom]
+    dom_gbs = cases[dom].code_bytes / dom_us / 1e3
+    dom_all = (cases[dom].code_bytes + cases[dom].meta_bytes) / dom_us / 1e3
+    fault = w4.device_fault()
+    if fault != 0:
+        raise RuntimeError(f"a kernel gave up a bounded wait (site {fault}); results invalid")
 
     # prefill layer set at M = 4096 (hidden-8192 shapes)
     prefill = None
@@ -354,19 +491,27 @@ def run_ours(args):
         pcases = workloads.prefill_8192(ms=[4096])
         players = setup_layers(pcases, torch, w4, stream)
         p_ms = time_steps(players, args.prefill_steps, 1, torch, w4, stream, w4.PATH_AUTO, block=1)
-        p_layer = time_per_layer(players, torch, w4, stream, w4.PATH_AUTO, steps=2, replays=2)
+        del players
+        torch.cuda.empty_cache()
         flops = sum(c.flops for c in pcases)
         tflops = flops * args.prefill_steps / (p_ms * 1e-3) / 1e12
         pdom = max(range(len(pcases)), key=lambda i: pcases[i].flops)
-        pdom_tf = pcases[pdom].flops / (p_layer[pdom] * 1e-3) / 1e12
+        pdom_us = time_layer_alone(pcases[pdom], torch, w4, stream)[0]  # X preparation + GEMM
+        pdom_tf = pcases[pdom].flops / pdom_us / 1e6
         prefill = {"value": tflops, "unit": "TFLOP/s", "workload": "prefill_hidden8192_m4096",
                    "ms_per_step": p_ms / args.prefill_steps, "steps": args.prefill_steps,
                    "frac_of_bf16_peak": tflops / peaks["bf16_tflops"],
-                   "roofline": {"bound": "tensor", "kernel": f"linear {pcases[pdom].name}",
+                   "roofline": {"bound": "tensor", "kernel": f"prefill_kernel on {pcases[pdom].name} "
+                                                             f"({pcases[pdom].K}x{pcases[pdom].N}, M={pcases[pdom].M})",
                                 "achieved": pdom_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                "frac": pdom_tf / peaks["bf16_tflops"], "peak_source": peak_src}}
-        del players
-        torch.cuda.empty_cache()
+                                "frac": pdom_tf / peaks["bf16_tflops"],
+                                "traffic": ncu_traffic("prefill_kernel", pcases[pdom].name),
+                                "per_call_us": pdom_us, "timed": "whole call: X preparation (about 2% of it) + GEMM",
+                                "peak_source": peak_src}}
+
+    stack = None
+    if not args.no_stack:
+        stack = run_stack(torch, w4, stream, args.stack_steps)
 
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
@@ -401,13 +546,16 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": f"decode GEMV on {cases[dom].name} "
                                                 f"({cases[dom].K}x{cases[dom].N})",
                      "achieved": dom_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": dom_gbs / peaks["hbm_gbs"], "traffic": args.traffic,
-                     "achieved_all_bytes": dom_all, "per_launch_ms": dom_ms,
+                     "frac": dom_gbs / peaks["hbm_gbs"],
+                     "traffic": args.traffic if args.traffic is not None else ncu_traffic("decode_cc_kernel",
+                                                                                         cases[dom].name),
+                     "achieved_all_bytes": dom_all, "per_launch_us": dom_us,
                      "algorithmic_bytes_per_launch": cases[dom].code_bytes, "peak_source": peak_src},
-        "per_layer_ms": {c.name: ms for c, ms in zip(cases, per_layer)},
+        "per_layer_us": {c.name: us for c, us in zip(cases, per_layer)},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         "prefill": prefill,
+        "stack": stack,
         "gpu_launches": launches,
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
@@ -420,30 +568,67 @@ def run_ours(args):
 # ----------------------------------------------------------------------------------------------
 
 def run_reference(args):
+    """The reference arm: the FP64 oracle, as it stands, on the host cores.  A
+    step is one pass over a bounded sample of the decode step (the first rows
+    of each of the four layers), sized so that warm-up + timed steps take about
+    --ref-seconds in all.  Under torch.distributed.run only rank 0 runs."""
     world, rank, _ = dist_env()
     if rank != 0:
         return
+    import oracle
     cases = workloads.decode_5120()
-    cpu, dt = cpu_baseline(cases, budget_s=max(5.0, min(60.0, args.cpu_budget)))
-    steps_equiv = cpu["value"]
+
+    def sample(rows_per_layer):
+        out = []
+        for c in cases:
+            rows = np.arange(min(rows_per_layer, c.N), dtype=np.int64)
+            W = synth.weight_rows_f32(c.w_seed, c.w_tag, c.K, rows)
+            st, qw, sc, z = oracle.quantize_pack(W)
+            out.append((synth.activations_bf16(c.x_seed, c.M, c.K), qw, sc, z, rows.size * c.K // 2))
+        return out
+
+    def step(smp):
+        for X, qw, sc, z, _ in smp:
+            oracle.linear(X, qw, sc, z)
+
+    probe_rows = 256
+    smp = sample(probe_rows)
+    t0 = time.perf_counter()
+    step(smp)
+    t_probe = time.perf_counter() - t0
+    per_step = args.ref_seconds / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(4096, probe_rows * per_step / max(t_probe, 1e-6))))
+    smp = sample(rows)
+    for _ in range(args.warmup):
+        step(smp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step(smp)
+    dt = time.perf_counter() - t0
+    nbytes = sum(x[4] for x in smp)
+    value = nbytes * args.steps / dt / 1e9
+    sample_desc = (f"first {rows} output rows of each of the {len(cases)} layers ({', '.join(c.name for c in cases)}), "
+                   f"M=1, packed by the oracle; {args.steps} timed steps of one pass each in {dt:.2f} s; "
+                   f"GB/s of packed code bytes")
     line = {
         "impl": "reference",
         "metric": METRIC,
-        "value": steps_equiv,
+        "value": value,
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": sum(c.code_bytes for c in cases) / (cpu["value"] * 1e9) * 1e3,
+        "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (same seeded workload)",
         "config": {"workload": "decode_hidden5120_m1", "M": 1, "shapes_KxN": [[c.K, c.N] for c in cases],
-                   "group": 128},
-        "cpu_baseline": cpu,
-        "e2e": {"value": cpu["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                   "group": 128, "sample_rows_per_layer": rows},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample_desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
@@ -469,6 +654,32 @@ def run_profile(spec: str, repeats: int = 4):
         raise SystemExit(1)
 
 
+def run_sweep(which: str):
+    """Per-layer device time of every workload shape (one JSON line each): each
+    call reads a different copy of the packed weights, rotating through enough
+    copies that their codes exceed 3x L2, replayed from a CUDA graph."""
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    w4.load()
+    stream = torch.cuda.Stream()
+    peaks, peak_src = load_peaks()
+    sets = {"single_gemv": workloads.single_gemv(), "decode": workloads.decode_5120(),
+            "small": workloads.small_batch_8192(), "prefill": workloads.prefill_8192()}
+    names = list(sets) if which == "all" else which.split(",")
+    for wl in names:
+        for c in sets[wl]:
+            us, copies = time_layer_alone(c, torch, w4, stream)
+            fault = w4.device_fault()
+            line = {"sweep": c.workload, "layer": c.name, "M": c.M, "K": c.K, "N": c.N, "us_per_call": us,
+                    "code_gbs": c.code_bytes / us / 1e3, "all_bytes_gbs": (c.code_bytes + c.meta_bytes) / us / 1e3,
+                    "tflops": c.flops / us / 1e6, "frac_hbm": c.code_bytes / us / 1e3 / peaks["hbm_gbs"],
+                    "frac_bf16": c.flops / us / 1e6 / peaks["bf16_tflops"], "weight_copies": copies,
+                    "fault": fault}
+            print(json.dumps(line), flush=True)
+            if fault:
+                raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -477,13 +688,22 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--prefill-steps", type=int, default=3)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--stack-steps", type=int, default=20)
+    ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="reference arm: approximate host seconds for warm-up + timed steps")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture of this build")
     ap.add_argument("--profile", default=None,
                     help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096): run it a few times, untimed")
+    ap.add_argument("--sweep", default=None,
+                    help="all, or a comma list of single_gemv, decode, small, prefill: per-layer times, one line each")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args.sweep)
+        return
     if args.profile:
         run_profile(args.profile)
         return

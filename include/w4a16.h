@@ -96,11 +96,14 @@ W4A16_API int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t
 
 /*
  * Bytes of device workspace w4a16_linear() needs for this shape (0 if none).
- * The workspace holds FP32 split-K partial sums and per-tile arrival counters.
- * The counter area must be zero before its first use (w4a16_workspace_init);
- * each completed call leaves it zero again, so one workspace can be reused by
- * calls that are ordered on one stream.  Calls that may run concurrently need
- * separate workspaces.
+ * The workspace starts with a 256 KB area of split-K arrival counters, then
+ * holds prepared activations and FP32 split-K partial sums.  The counter area
+ * must be zero before its first use (w4a16_workspace_init); every completed
+ * call leaves it zero again and no call writes anything else there, so one
+ * workspace, sized for the largest shape, can be shared by calls of any
+ * shapes that are ordered on one stream.  Exception: a decode call with
+ * N > 8,388,608 keeps counters beyond that area and needs a workspace of its
+ * own.  Calls that may run concurrently need separate workspaces.
  */
 W4A16_API size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 

@@ -154,6 +154,36 @@ def test_workspace_reuse_and_errors(cuda_lib):
     assert e.value.status == w4.ERR_WORKSPACE
 
 
+def test_one_workspace_shared_by_shapes_and_paths(cuda_lib):
+    """Calls of different shapes and paths, ordered on one stream, share one
+    workspace initialised once: each call must leave the split-K counters the
+    next one relies on at zero, whatever it writes elsewhere."""
+    shapes = [(1, 384, 8192), (1, 256, 28672), (3, 384, 8192), (70, 256, 1024), (1, 384, 8192), (1, 256, 28672),
+              (17, 640, 2048), (1, 384, 8192)]
+    packed, inputs, refs = {}, {}, {}
+    for M, N, K in shapes:
+        if (N, K) not in packed:
+            W = synth.weights_f32(N + K, synth.TAG_W, N, K)
+            packed[(N, K)] = (packed_from_host(W), oracle.quantize_pack(W)[1:])
+        if (M, N, K) not in inputs:
+            inputs[(M, N, K)] = synth.activations_bf16(M + K, M, K)
+            qw, sc, z = packed[(N, K)][1]
+            refs[(M, N, K)] = oracle.linear(inputs[(M, N, K)], qw, sc, z)
+    nbytes = max(w4.workspace_bytes(M, N, K) for M, N, K in shapes)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    w4.workspace_init(ws)
+    outs = []
+    for M, N, K in shapes:
+        pw = packed[(N, K)][0]
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        w4.linear(bits_to_dev_bf16(inputs[(M, N, K)]), pw.qweight, pw.scales, pw.zeros, Y, ws)
+        outs.append(Y)
+    torch.cuda.synchronize()
+    for (M, N, K), Y in zip(shapes, outs):
+        assert_close(bf16_dev_to_f64(Y), refs[(M, N, K)], f"shared workspace M={M} N={N} K={K}")
+    assert w4.device_fault() == 0
+
+
 def test_renorm_rows(cuda_lib):
     rng = np.random.default_rng(4)
     y = torch.from_numpy(rng.standard_normal((3, 28672)).astype(np.float32) * 5).to(torch.bfloat16).cuda()

@@ -218,10 +218,17 @@ class PackedWeight:
 
     @classmethod
     def from_float(cls, W: torch.Tensor, stream=None) -> "PackedWeight":
+        """Pack W on `stream` (a torch.cuda.Stream, or None for the current one);
+        the status word is cleared on that stream before the kernel runs."""
         N, K = W.shape
-        pw = cls(N, K, device=W.device)
-        status = torch.zeros(1, dtype=torch.int32, device=W.device)
-        quantize_pack(W, pw.qweight, pw.scales, pw.zeros, status, stream)
+        if stream is None:
+            stream = torch.cuda.current_stream(W.device)
+        if not isinstance(stream, torch.cuda.Stream):
+            raise TypeError("stream must be a torch.cuda.Stream or None")
+        with torch.cuda.stream(stream):
+            pw = cls(N, K, device=W.device)
+            status = torch.zeros(1, dtype=torch.int32, device=W.device)
+            quantize_pack(W, pw.qweight, pw.scales, pw.zeros, status, stream)
         pw.status = status
         return pw
 

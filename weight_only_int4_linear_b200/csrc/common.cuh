@@ -61,6 +61,14 @@ int launch_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_
                    uint16_t* out, cudaStream_t stream);
 int launch_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, cudaStream_t stream);
 
+// Every workspace starts with the decode path's split-K arrival counters, at
+// the same place for every shape: each call leaves its counters zero and no
+// call writes anything else below kCounterBytes, so calls of any shapes and
+// paths ordered on one stream can share one workspace (row tiles up to
+// kSharedCounterTiles, i.e. N up to 8,388,608).
+constexpr int64_t kSharedCounterTiles = 65536;
+constexpr size_t kCounterBytes = (size_t)kSharedCounterTiles * 4;  // 256 KB
+
 struct DecodePlan {
     int nt;           // token tiles of 8 per launch (1, 2 or 4: up to 32 tokens)
     int row_tiles;    // 128-row tiles along N
@@ -68,7 +76,8 @@ struct DecodePlan {
     int units_base;   // each CTA streams units_base (+1 for the first units_rem CTAs) units
     int units_rem;
     int max_slots;    // partial-sum slots per row tile
-    size_t ws_xp_bytes, ws_xs_bytes, ws_partial_bytes, ws_counter_bytes;
+    // workspace layout: [counters][Xp][xs][partials]
+    size_t ws_counter_bytes, ws_xp_bytes, ws_xs_bytes, ws_partial_bytes;
     size_t workspace_bytes() const;
 };
 DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms);

@@ -392,7 +392,8 @@ size_t align256p(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t prefill_workspace_bytes(int64_t M, int64_t K) {
     const int64_t Mp = (M + 3) & ~(int64_t)3;
-    return align256p((size_t)M * K * 2) + align256p((size_t)(K / kGroup) * Mp * 4);
+    // the decode path's counter area stays untouched at the front (shared workspaces)
+    return kCounterBytes + align256p((size_t)M * K * 2) + align256p((size_t)(K / kGroup) * Mp * 4);
 }
 
 int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
@@ -406,7 +407,7 @@ int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qwei
     }
     int* fault = fault_word();
     if (!fault) return W4A16_ERR_CUDA;
-    char* ws = reinterpret_cast<char*>(workspace);
+    char* ws = reinterpret_cast<char*>(workspace) + kCounterBytes;
     uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
     float* xsT = reinterpret_cast<float*>(ws + align256p((size_t)M * K * 2));
     CUtensorMap tx, tq;

@@ -881,7 +881,7 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.ws_xp_bytes = p.nt == 1 ? 0 : align256((size_t)Mc * K * 2);
     p.ws_xs_bytes = p.nt == 1 ? 0 : align256((size_t)G * kXsStride * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
-    p.ws_counter_bytes = align256((size_t)p.row_tiles * 4);
+    p.ws_counter_bytes = align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
     return p;
 }
 
@@ -895,10 +895,10 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
     int* fault = fault_word();
     if (!fault) return W4A16_ERR_CUDA;
     char* ws = reinterpret_cast<char*>(workspace);
-    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws);
-    float* xs = reinterpret_cast<float*>(ws + plan.ws_xp_bytes);
-    float* partial = reinterpret_cast<float*>(ws + plan.ws_xp_bytes + plan.ws_xs_bytes);
-    int* counters = reinterpret_cast<int*>(ws + plan.ws_xp_bytes + plan.ws_xs_bytes + plan.ws_partial_bytes);
+    int* counters = reinterpret_cast<int*>(ws);
+    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws + plan.ws_counter_bytes);
+    float* xs = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes);
+    float* partial = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes + plan.ws_xs_bytes);
     const int G = (int)(K / kGroup);
     for (int64_t m0 = 0; m0 < M; m0 += kMaxTokens) {
         const int Mc = (int)((M - m0) < kMaxTokens ? (M - m0) : kMaxTokens);

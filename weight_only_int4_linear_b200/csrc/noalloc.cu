@@ -93,7 +93,7 @@ extern "C" int w4a16_linear_noalloc(const uint16_t* X, int64_t M, int64_t K, con
     if (!scratch) return st;
     cudaStream_t s = (cudaStream_t)stream;
     // the buffer keeps the previous call's contents: the arrival counters must start at zero
-    char* counters = static_cast<char*>(scratch) + plan.ws_xp_bytes + plan.ws_xs_bytes + plan.ws_partial_bytes;
-    if (cudaMemsetAsync(counters, 0, plan.ws_counter_bytes, s) != cudaSuccess) return W4A16_ERR_CUDA;
+    // counters lead the layout; only this call's row tiles need clearing
+    if (cudaMemsetAsync(scratch, 0, (size_t)plan.row_tiles * 4, s) != cudaSuccess) return W4A16_ERR_CUDA;
     return launch_decode(X, M, K, qweight, scales, zeros, N, Y, scratch, plan, s);
 }
