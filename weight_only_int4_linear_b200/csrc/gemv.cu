@@ -468,16 +468,26 @@ constexpr int kGroupXiBytes = 4 * kQuarterBytes + 16;  // 400 B per group
 //  * warps 0-3 compute, thread t taking words 4c..4c+3 (c = t % 4) of rows
 //    t/4 + 32 i, i = 0..3.
 // Up to four CTAs share an SM.
-constexpr int kCcWarps = 4;                             // compute warps
+#ifndef W4A16_CC_WARPS
+#define W4A16_CC_WARPS 4
+#endif
+#ifndef W4A16_CC_STAGES
+#define W4A16_CC_STAGES 4
+#endif
+constexpr int kCcWarps = W4A16_CC_WARPS;                // compute warps
+constexpr int kCcRowStep = kCcWarps * 8;                // rows rg + kCcRowStep * i of one thread
+constexpr int kCcRows = kRowsPerCta / kCcRowStep;       // rows per thread
+static_assert(kCcRows * kCcRowStep == kRowsPerCta && kCcRowStep % 8 == 0, "row split");
 constexpr int kCcTmaWarp = kCcWarps;                    // warp 4
 constexpr int kCcXWarp = kCcWarps + 1;                  // warp 5
 constexpr int kCcThreads = (kCcWarps + 2) * 32;
-constexpr int kCcStages = 4;
+constexpr int kCcStages = W4A16_CC_STAGES;
 constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
 constexpr int kCcXOff = kCcCodeBytes;                   // X planes of the group + extras (400 B)
 constexpr int kCcExtOff = kCcXOff + 4 * kQuarterBytes;
 constexpr int kCcStageBytes = 9 * 1024;                 // keeps stages 1024-aligned
 constexpr int kCcMetaGroups = 8;                        // groups per metadata block
+constexpr int kXAhead = 6;                              // X warp: loads in flight, in units
 constexpr int kCcScBytes = kRowsPerCta * kCcMetaGroups * 2;  // 128 rows x 8 BF16 scales
 constexpr int kCcZeBytes = kRowsPerCta * kCcMetaGroups * 4;  // 128 rows x 8 int32 zero points
 constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;   // one slot, 6 KB
@@ -507,10 +517,13 @@ __device__ __forceinline__ float pow2f(int e) {
     return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
 }
 
-// One warp writes group g's X in the layout above: lane 2w + h holds values
-// 4h..4h+3 of word w.
-__device__ __forceinline__ void prep_group_x(const uint16_t* __restrict__ X, int g, unsigned char* dst, int lane) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(X + (int64_t)g * kGroup + lane * 4));
+// This lane's four BF16 values of group g: lane 2w + h holds values 4h..4h+3 of word w.
+__device__ __forceinline__ uint2 load_group_x(const uint16_t* __restrict__ X, int g, int lane) {
+    return __ldg(reinterpret_cast<const uint2*>(X + (int64_t)g * kGroup + lane * 4));
+}
+
+// One warp writes a group's X (its lanes' values v from load_group_x) in the layout above.
+__device__ __forceinline__ void prep_group_x(const uint2 v, unsigned char* dst, int lane) {
     const uint32_t bits[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
     uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
     amax = __reduce_max_sync(0xFFFFFFFFu, amax);
@@ -614,11 +627,19 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
     if (warp == kCcXWarp) {  // ------------------------------------------ X warp
         pdl_wait_primary();  // X may come from the preceding kernel
         const uint16_t* X = a.Xp;
-        UnitCursor cur(u_first, G);
-        for (int i = 0; i < nunits; ++i, cur.next(G)) {
+        // loads run kXAhead units ahead of the preparation, so L2 latency is paid once, not per unit
+        uint2 q[kXAhead];
+        UnitCursor cl(u_first, G);
+#pragma unroll
+        for (int j = 0; j < kXAhead; ++j, cl.next(G)) q[j] = j < nunits ? load_group_x(X, cl.g, lane) : make_uint2(0, 0);
+        for (int i = 0; i < nunits; ++i, cl.next(G)) {
+            const uint2 v = q[0];
+#pragma unroll
+            for (int j = 0; j + 1 < kXAhead; ++j) q[j] = q[j + 1];
+            q[kXAhead - 1] = i + kXAhead < nunits ? load_group_x(X, cl.g, lane) : make_uint2(0, 0);
             const int s = i % kCcStages;
             if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
-            prep_group_x(X, cur.g, ring + s * kCcStageBytes + kCcXOff, lane);
+            prep_group_x(v, ring + s * kCcStageBytes + kCcXOff, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         }
@@ -628,17 +649,19 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
     // ---------------------------------------------------- compute warps 0-3
     const int t = threadIdx.x;
     const int c = t & 3;   // words 4c..4c+3 of the group
-    const int rg = t >> 2; // rows rg + 32 i
+    const int rg = t >> 2; // rows rg + kCcRowStep i
     // the 64-byte swizzle of the codes tile: logical chunk c of row r sits at chunk c ^ ((r >> 1) & 3);
-    // (r >> 1) & 3 is the same for the four rows rg + 32 i
+    // (r >> 1) & 3 is the same for all rows rg + kCcRowStep i (kCcRowStep % 8 == 0)
     const int code_off = rg * 64 + 16 * (c ^ ((rg >> 1) & 3));
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    float y[kCcRows];
+#pragma unroll
+    for (int i = 0; i < kCcRows; ++i) y[i] = 0.f;
     int cur_tile = -1;
     bool aborted = false;
 
     auto flush = [&](int tile) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // reduce over the four threads of each row
+        for (int i = 0; i < kCcRows; ++i) {  // reduce over the four threads of each row
             y[i] += __shfl_xor_sync(0xFFFFFFFFu, y[i], 1);
             y[i] += __shfl_xor_sync(0xFFFFFFFFu, y[i], 2);
         }
@@ -647,8 +670,8 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         if (first == last) {
             if (c == 0) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int n = tile * kRowsPerCta + rg + 32 * i;
+                for (int i = 0; i < kCcRows; ++i) {
+                    const int n = tile * kRowsPerCta + rg + kCcRowStep * i;
                     if (n < N) a.Y[n] = float_to_bf16_bits(y[i]);
                 }
             }
@@ -657,7 +680,7 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
             float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * kRowsPerCta;
             if (c == 0) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) part[rg + 32 * i] = y[i];
+                for (int i = 0; i < kCcRows; ++i) part[rg + kCcRowStep * i] = y[i];
             }
             named_barrier_sync(1, kCcWarps * 32);
             if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
@@ -672,7 +695,7 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
             named_barrier_sync(1, kCcWarps * 32);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) y[i] = 0.f;
+        for (int i = 0; i < kCcRows; ++i) y[i] = 0.f;
     };
 
     UnitCursor uc(u_first, G);
@@ -691,9 +714,9 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
             continue;
         }
         const unsigned char* st = ring + s * kCcStageBytes;
-        uint4 w[4];
+        uint4 w[kCcRows];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) w[r] = *reinterpret_cast<const uint4*>(st + code_off + 2048 * r);
+        for (int r = 0; r < kCcRows; ++r) w[r] = *reinterpret_cast<const uint4*>(st + code_off + 64 * kCcRowStep * r);
         // X planes of words 4c..4c+3: word j's registers at xr[6j .. 6j+5]
         uint32_t xr[24];
         const uint4* xq = reinterpret_cast<const uint4*>(st + kCcXOff + c * kQuarterBytes);
@@ -712,19 +735,19 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
         const unsigned char* scb = ms + rg * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1));
         const unsigned char* zeb = ms + kCcScBytes + rg * (kCcMetaGroups * 4) + 4 * (g & (kCcMetaGroups - 1));
-        float sv[4], zv[4];
+        float sv[kCcRows], zv[kCcRows];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < kCcRows; ++r) {
             // rows past N were zero-filled by TMA: s = 0 folds them away
-            sv[r] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(scb + 32 * kCcMetaGroups * 2 * r));
-            zv[r] = (float)*reinterpret_cast<const int32_t*>(zeb + 32 * kCcMetaGroups * 4 * r);
+            sv[r] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(scb + kCcRowStep * kCcMetaGroups * 2 * r));
+            zv[r] = (float)*reinterpret_cast<const int32_t*>(zeb + kCcRowStep * kCcMetaGroups * 4 * r);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
         const float corr = (c == 0) ? (float)xsum : 0.f;  // one thread of four folds the zero point
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int r = 0; r < kCcRows; ++r) {
             const uint32_t wr[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
             int p0 = 0, p1 = 0, p2 = 0;  // sum_k q_k * plane_p(x_k) over this thread's 32 codes
 #pragma unroll
