@@ -40,7 +40,8 @@ def packed_from_host(W: np.ndarray):
 
 
 @pytest.mark.parametrize("path", PATHS)
-@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (1, 33, 256), (3, 130, 384), (8, 256, 1024), (9, 200, 512),
+@pytest.mark.parametrize("M,N,K", [(1, 16, 128), (1, 33, 256), (2, 130, 1024), (2, 72, 384), (3, 130, 384),
+                                   (8, 256, 1024), (9, 200, 512),
                                    (16, 129, 2048), (17, 64, 640), (32, 384, 1152), (33, 100, 256),
                                    (70, 150, 768)])
 def test_small_shapes_all_outputs(cuda_lib, M, N, K, path):

@@ -70,7 +70,8 @@ constexpr int64_t kSharedCounterTiles = 65536;
 constexpr size_t kCounterBytes = (size_t)kSharedCounterTiles * 4;  // 256 KB
 
 struct DecodePlan {
-    int nt;           // token tiles of 8 per launch (1, 2 or 4: up to 32 tokens)
+    int cc_tokens;    // > 0: the integer CUDA-core kernel for this many tokens (M <= 2)
+    int nt;           // tensor-core kernel: MMA N (16 or 32 tokens per launch); 1 with cc_tokens
     int row_tiles;    // 128-row tiles along N
     int grid;         // persistent CTAs
     int units_base;   // each CTA streams units_base (+1 for the first units_rem CTAs) units

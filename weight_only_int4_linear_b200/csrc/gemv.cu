@@ -483,8 +483,8 @@ constexpr int kCcXWarp = kCcWarps + 1;                  // warp 5
 constexpr int kCcThreads = (kCcWarps + 2) * 32;
 constexpr int kCcStages = W4A16_CC_STAGES;
 constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
-constexpr int kCcXOff = kCcCodeBytes;                   // X planes of the group + extras (400 B)
-constexpr int kCcExtOff = kCcXOff + 4 * kQuarterBytes;
+constexpr int kCcMaxTokens = 2;                         // tokens per launch of the integer kernel
+constexpr int kCcXOff = kCcCodeBytes;                   // X planes of the group, per token (400 B each)
 constexpr int kCcStageBytes = 9 * 1024;                 // keeps stages 1024-aligned
 constexpr int kCcMetaGroups = 8;                        // groups per metadata block
 constexpr int kXAhead = 6;                              // X warp: loads in flight, in units
@@ -493,7 +493,7 @@ constexpr int kCcZeBytes = kRowsPerCta * kCcMetaGroups * 4;  // 128 rows x 8 int
 constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;   // one slot, 6 KB
 constexpr int kCcMetaOff = kCcStages * kCcStageBytes;   // two slots after the ring
 constexpr size_t kCcSmem = (size_t)kCcMetaOff + 2 * kCcMetaBytes + 1024;
-static_assert(kCcXOff + kGroupXiBytes <= kCcStageBytes, "stage layout");
+static_assert(kCcXOff + kCcMaxTokens * kGroupXiBytes <= kCcStageBytes, "stage layout");
 // A metadata slot is rewritten two blocks later.  Blocks are aligned to 8
 // groups inside a row tile (the kernel needs G % 8 == 0), so the block in
 // between has 8 units; with at most kCcStages units in flight, every unit of
@@ -566,7 +566,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, int parity, int* fault,
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
-__global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
+template <int NT>
+#ifndef W4A16_CC2_MIN_BLOCKS
+#define W4A16_CC2_MIN_BLOCKS 3
+#endif
+__global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
                                                                const __grid_constant__ CUtensorMap tsc,
                                                                const __grid_constant__ CUtensorMap tze,
                                                                const DecodeArgs a) {
@@ -628,18 +632,27 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         pdl_wait_primary();  // X may come from the preceding kernel
         const uint16_t* X = a.Xp;
         // loads run kXAhead units ahead of the preparation, so L2 latency is paid once, not per unit
-        uint2 q[kXAhead];
+        uint2 q[kXAhead][NT];
         UnitCursor cl(u_first, G);
 #pragma unroll
-        for (int j = 0; j < kXAhead; ++j, cl.next(G)) q[j] = j < nunits ? load_group_x(X, cl.g, lane) : make_uint2(0, 0);
-        for (int i = 0; i < nunits; ++i, cl.next(G)) {
-            const uint2 v = q[0];
+        for (int j = 0; j < kXAhead; ++j, cl.next(G))
 #pragma unroll
-            for (int j = 0; j + 1 < kXAhead; ++j) q[j] = q[j + 1];
-            q[kXAhead - 1] = i + kXAhead < nunits ? load_group_x(X, cl.g, lane) : make_uint2(0, 0);
+            for (int m = 0; m < NT; ++m)
+                q[j][m] = j < nunits && m < a.M ? load_group_x(X + (int64_t)m * a.K, cl.g, lane) : make_uint2(0, 0);
+        for (int i = 0; i < nunits; ++i, cl.next(G)) {
+            uint2 v[NT];
+#pragma unroll
+            for (int m = 0; m < NT; ++m) {
+                v[m] = q[0][m];
+#pragma unroll
+                for (int j = 0; j + 1 < kXAhead; ++j) q[j][m] = q[j + 1][m];
+                q[kXAhead - 1][m] = i + kXAhead < nunits && m < a.M ? load_group_x(X + (int64_t)m * a.K, cl.g, lane)
+                                                                      : make_uint2(0, 0);
+            }
             const int s = i % kCcStages;
             if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
-            prep_group_x(v, ring + s * kCcStageBytes + kCcXOff, lane);
+#pragma unroll
+            for (int m = 0; m < NT; ++m) prep_group_x(v[m], ring + s * kCcStageBytes + kCcXOff + m * kGroupXiBytes, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         }
@@ -653,18 +666,22 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
     // the 64-byte swizzle of the codes tile: logical chunk c of row r sits at chunk c ^ ((r >> 1) & 3);
     // (r >> 1) & 3 is the same for all rows rg + kCcRowStep i (kCcRowStep % 8 == 0)
     const int code_off = rg * 64 + 16 * (c ^ ((rg >> 1) & 3));
-    float y[kCcRows];
+    float y[kCcRows][NT];
 #pragma unroll
-    for (int i = 0; i < kCcRows; ++i) y[i] = 0.f;
+    for (int i = 0; i < kCcRows; ++i)
+#pragma unroll
+        for (int m = 0; m < NT; ++m) y[i][m] = 0.f;
     int cur_tile = -1;
     bool aborted = false;
 
     auto flush = [&](int tile) {
 #pragma unroll
-        for (int i = 0; i < kCcRows; ++i) {  // reduce over the four threads of each row
-            y[i] += __shfl_xor_sync(0xFFFFFFFFu, y[i], 1);
-            y[i] += __shfl_xor_sync(0xFFFFFFFFu, y[i], 2);
-        }
+        for (int i = 0; i < kCcRows; ++i)  // reduce over the four threads of each row
+#pragma unroll
+            for (int m = 0; m < NT; ++m) {
+                y[i][m] += __shfl_xor_sync(0xFFFFFFFFu, y[i][m], 1);
+                y[i][m] += __shfl_xor_sync(0xFFFFFFFFu, y[i][m], 2);
+            }
         const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
         const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
         if (first == last) {
@@ -672,30 +689,43 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < kCcRows; ++i) {
                     const int n = tile * kRowsPerCta + rg + kCcRowStep * i;
-                    if (n < N) a.Y[n] = float_to_bf16_bits(y[i]);
+#pragma unroll
+                    for (int m = 0; m < NT; ++m)
+                        if (n < N && m < a.M) a.Y[(int64_t)m * N + n] = float_to_bf16_bits(y[i][m]);
                 }
             }
         } else {
             const int slot = b - first, nseg = last - first + 1;
-            float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * kRowsPerCta;
+            float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * a.M * kRowsPerCta;
             if (c == 0) {
 #pragma unroll
-                for (int i = 0; i < kCcRows; ++i) part[rg + kCcRowStep * i] = y[i];
+                for (int i = 0; i < kCcRows; ++i)
+#pragma unroll
+                    for (int m = 0; m < NT; ++m)
+                        if (m < a.M) part[m * kRowsPerCta + rg + kCcRowStep * i] = y[i][m];
             }
             named_barrier_sync(1, kCcWarps * 32);
             if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
             named_barrier_sync(1, kCcWarps * 32);
             if (s_last) {
                 const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
-                const float* pb = a.partial + (int64_t)tile * a.max_slots * kRowsPerCta;
-                for (int rl = t; rl < rows; rl += kCcWarps * 32)
-                    a.Y[tile * kRowsPerCta + rl] = float_to_bf16_bits(sum_slots(pb + rl, kRowsPerCta, nseg));
+                const float* pb = a.partial + (int64_t)tile * a.max_slots * a.M * kRowsPerCta;
+#pragma unroll
+                for (int m = 0; m < NT; ++m) {
+                    if (m >= a.M) break;
+                    for (int rl = t; rl < rows; rl += kCcWarps * 32) {
+                        const float sum = sum_slots(pb + (int64_t)m * kRowsPerCta + rl, (int64_t)a.M * kRowsPerCta, nseg);
+                        a.Y[(int64_t)m * N + tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
+                    }
+                }
                 if (t == 0) a.counters[tile] = 0;
             }
             named_barrier_sync(1, kCcWarps * 32);
         }
 #pragma unroll
-        for (int i = 0; i < kCcRows; ++i) y[i] = 0.f;
+        for (int i = 0; i < kCcRows; ++i)
+#pragma unroll
+            for (int m = 0; m < NT; ++m) y[i][m] = 0.f;
     };
 
     UnitCursor uc(u_first, G);
@@ -717,20 +747,26 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         uint4 w[kCcRows];
 #pragma unroll
         for (int r = 0; r < kCcRows; ++r) w[r] = *reinterpret_cast<const uint4*>(st + code_off + 64 * kCcRowStep * r);
-        // X planes of words 4c..4c+3: word j's registers at xr[6j .. 6j+5]
-        uint32_t xr[24];
-        const uint4* xq = reinterpret_cast<const uint4*>(st + kCcXOff + c * kQuarterBytes);
+        // X planes of words 4c..4c+3 of token m: word j's registers at xr[m][6j .. 6j+5]
+        uint32_t xr[NT][24];
+        int xsum[NT];
+        float xscale[NT];
 #pragma unroll
-        for (int j = 0; j < 6; ++j) {
-            const uint4 v = xq[j];
-            xr[4 * j] = v.x;
-            xr[4 * j + 1] = v.y;
-            xr[4 * j + 2] = v.z;
-            xr[4 * j + 3] = v.w;
+        for (int m = 0; m < NT; ++m) {
+            const unsigned char* xg = st + kCcXOff + m * kGroupXiBytes;
+            const uint4* xq = reinterpret_cast<const uint4*>(xg + c * kQuarterBytes);
+#pragma unroll
+            for (int j = 0; j < 6; ++j) {
+                const uint4 v = xq[j];
+                xr[m][4 * j] = v.x;
+                xr[m][4 * j + 1] = v.y;
+                xr[m][4 * j + 2] = v.z;
+                xr[m][4 * j + 3] = v.w;
+            }
+            const int* ext = reinterpret_cast<const int*>(xg + 4 * kQuarterBytes);
+            xsum[m] = ext[0];
+            xscale[m] = __int_as_float(ext[1]);
         }
-        const int* ext = reinterpret_cast<const int*>(st + kCcExtOff);
-        const int xsum = ext[0];
-        const float xscale = __int_as_float(ext[1]);
         // this block's metadata (loaded with its first unit, which this warp has already waited for)
         const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
         const unsigned char* scb = ms + rg * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1));
@@ -745,26 +781,34 @@ __global__ void __launch_bounds__(kCcThreads) decode_cc_kernel(const __grid_cons
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
-        const float corr = (c == 0) ? (float)xsum : 0.f;  // one thread of four folds the zero point
 #pragma unroll
         for (int r = 0; r < kCcRows; ++r) {
             const uint32_t wr[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
-            int p0 = 0, p1 = 0, p2 = 0;  // sum_k q_k * plane_p(x_k) over this thread's 32 codes
+            int p0[NT], p1[NT], p2[NT];  // sum_k q_k * plane_p(x_k) over this thread's 32 codes, per token
+#pragma unroll
+            for (int m = 0; m < NT; ++m) p0[m] = p1[m] = p2[m] = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint32_t ce = wr[j] & 0x0F0F0F0Fu, co = (wr[j] >> 4) & 0x0F0F0F0Fu;  // codes 0,2,4,6 / 1,3,5,7
-                p0 = dp4a_uu(ce, xr[6 * j], p0);
-                p1 = dp4a_uu(ce, xr[6 * j + 1], p1);
-                p2 = dp4a_us(ce, xr[6 * j + 2], p2);
-                p0 = dp4a_uu(co, xr[6 * j + 3], p0);
-                p1 = dp4a_uu(co, xr[6 * j + 4], p1);
-                p2 = dp4a_us(co, xr[6 * j + 5], p2);
+#pragma unroll
+                for (int m = 0; m < NT; ++m) {
+                    p0[m] = dp4a_uu(ce, xr[m][6 * j], p0[m]);
+                    p1[m] = dp4a_uu(ce, xr[m][6 * j + 1], p1[m]);
+                    p2[m] = dp4a_us(ce, xr[m][6 * j + 2], p2[m]);
+                    p0[m] = dp4a_uu(co, xr[m][6 * j + 3], p0[m]);
+                    p1[m] = dp4a_uu(co, xr[m][6 * j + 4], p1[m]);
+                    p2[m] = dp4a_us(co, xr[m][6 * j + 5], p2[m]);
+                }
             }
-            // sum q x_int = 65536 p2 + (256 p1 + p0): the bracket is exact in int32 (< 2^25),
-            // the rest is FP32 with one rounding per step
-            const float qx = fmaf((float)p2, 65536.f, (float)(p1 * 256 + p0));
-            // y += s 2^(E-22) (sum q x_int  -  [one thread of four] z sum x_int)
-            y[r] = fmaf(sv[r] * xscale, fmaf(-zv[r], corr, qx), y[r]);
+#pragma unroll
+            for (int m = 0; m < NT; ++m) {
+                // sum q x_int = 65536 p2 + (256 p1 + p0): the bracket is exact in int32 (< 2^25),
+                // the rest is FP32 with one rounding per step
+                const float qx = fmaf((float)p2[m], 65536.f, (float)(p1[m] * 256 + p0[m]));
+                // y += s 2^(E-22) (sum q x_int  -  [one thread of four] z sum x_int)
+                const float corr = (c == 0) ? (float)xsum[m] : 0.f;
+                y[r][m] = fmaf(sv[r] * xscale[m], fmaf(-zv[r], corr, qx), y[r][m]);
+            }
         }
     }
     if (cur_tile >= 0) flush(cur_tile);
@@ -787,14 +831,16 @@ int occupancy_nt() {
     return occ;
 }
 
+template <int NT>
 int occupancy_cc() {
     static int occ = 0;
     if (occ == 0) {
-        if (cudaFuncSetAttribute(decode_cc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCcSmem) !=
+        if (cudaFuncSetAttribute(decode_cc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCcSmem) !=
             cudaSuccess)
             return 0;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel, kCcThreads, kCcSmem) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel<NT>, kCcThreads, kCcSmem) !=
+                cudaSuccess ||
             o < 1)
             return 0;
         occ = o;
@@ -802,8 +848,10 @@ int occupancy_cc() {
     return occ;
 }
 
-int occupancy(int ntok) {
-    if (ntok == 1) return occupancy_cc();
+// cc_tokens > 0: the integer CUDA-core kernel for that many tokens; else the tensor-core kernel with MMA N = ntok
+int occupancy(int cc_tokens, int ntok) {
+    if (cc_tokens == 1) return occupancy_cc<1>();
+    if (cc_tokens == 2) return occupancy_cc<2>();
     return ntok == 16 ? occupancy_nt<16>() : occupancy_nt<32>();
 }
 
@@ -850,6 +898,7 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     return true;
 }
 
+template <int NT>
 int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& tze, const DecodeArgs& args, int grid,
               cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
@@ -862,7 +911,8 @@ int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_cc_kernel, tq, tsc, tze, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, decode_cc_kernel<NT>, tq, tsc, tze, args) == cudaSuccess ? W4A16_OK
+                                                                                              : W4A16_ERR_CUDA;
 }
 
 template <int NTOK>
@@ -888,11 +938,13 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     DecodePlan p{};
     const int64_t Mc = M < kMaxTokens ? M : kMaxTokens;
     const int64_t G = K / kGroup;
-    // 1: CUDA-core kernel (needs 16-byte metadata rows: G % 8 == 0); else tensor-core MMA N
-    p.nt = (Mc == 1 && G % 8 == 0) ? 1 : (Mc <= 16 ? 16 : 32);
+    // the integer CUDA-core kernel for M <= kCcMaxTokens (needs 16-byte metadata rows: G % 8 == 0);
+    // else the tensor-core kernel with MMA N = 16 or 32
+    p.cc_tokens = (M <= kCcMaxTokens && G % 8 == 0) ? (int)M : 0;
+    p.nt = p.cc_tokens ? 1 : (Mc <= 16 ? 16 : 32);
     p.row_tiles = (int)ceil_div(N, kRowsPerCta);
     const int64_t units = (int64_t)p.row_tiles * G;
-    int occ = occupancy(p.nt);
+    int occ = occupancy(p.cc_tokens, p.nt);
     if (occ < 1) occ = 1;
     int64_t grid = (int64_t)occ * num_sms;
     if (grid > units) grid = units;
@@ -900,9 +952,9 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.units_base = (int)(units / grid);
     p.units_rem = (int)(units % grid);
     p.max_slots = (int)((G - 1) / p.units_base + 2);
-    // the single-token kernel prepares X itself
-    p.ws_xp_bytes = p.nt == 1 ? 0 : align256((size_t)Mc * K * 2);
-    p.ws_xs_bytes = p.nt == 1 ? 0 : align256((size_t)G * kXsStride * 4);
+    // the integer kernel prepares X itself
+    p.ws_xp_bytes = p.cc_tokens ? 0 : align256((size_t)Mc * K * 2);
+    p.ws_xs_bytes = p.cc_tokens ? 0 : align256((size_t)G * kXsStride * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
     p.ws_counter_bytes = align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
     return p;
@@ -926,8 +978,8 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
     for (int64_t m0 = 0; m0 < M; m0 += kMaxTokens) {
         const int Mc = (int)((M - m0) < kMaxTokens ? (M - m0) : kMaxTokens);
         CUtensorMap tx;
-        if (plan.nt > 1 && !cached_tmap(plan.nt, Xp, Mc, K, &tx)) return W4A16_ERR_CUDA;
-        if (plan.nt > 1) {
+        if (!plan.cc_tokens && !cached_tmap(plan.nt, Xp, Mc, K, &tx)) return W4A16_ERR_CUDA;
+        if (!plan.cc_tokens) {
             const int64_t prep_units = (int64_t)kXsStride * G * 16;
             int prep_grid = (int)ceil_div(prep_units, 256);
             if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
@@ -935,7 +987,7 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
             if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
         }
         DecodeArgs args;
-        args.Xp = plan.nt == 1 ? X + m0 * K : Xp;  // the single-token kernel reads X as given
+        args.Xp = plan.cc_tokens ? X + m0 * K : Xp;  // the integer kernel reads X as given
         args.xs = xs;
         args.scales = scales;
         args.zeros = zeros;
@@ -951,11 +1003,12 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
         args.units_rem = plan.units_rem;
         args.max_slots = plan.max_slots;
         CUtensorMap tsc, tze;
-        if (plan.nt == 1 && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze)))
+        if (plan.cc_tokens && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze)))
             return W4A16_ERR_CUDA;
-        const int st = plan.nt == 1    ? launch_cc(tq, tsc, tze, args, plan.grid, stream)
-                       : plan.nt == 16 ? launch_tc<16>(tq, tx, args, plan.grid, stream)
-                                       : launch_tc<32>(tq, tx, args, plan.grid, stream);
+        const int st = plan.cc_tokens == 1   ? launch_cc<1>(tq, tsc, tze, args, plan.grid, stream)
+                       : plan.cc_tokens == 2 ? launch_cc<2>(tq, tsc, tze, args, plan.grid, stream)
+                       : plan.nt == 16       ? launch_tc<16>(tq, tx, args, plan.grid, stream)
+                                             : launch_tc<32>(tq, tx, args, plan.grid, stream);
         if (st != W4A16_OK) return st;
     }
     return W4A16_OK;
