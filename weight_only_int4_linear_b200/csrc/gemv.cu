@@ -34,7 +34,6 @@ namespace {
 
 constexpr int kRowsPerCta = 128;
 constexpr int kStageWords = kRowsPerCta * kWordsPerGroup;  // 2048 words = 8 KB
-constexpr int kXsStride = 32;  // tokens per group row of xsum
 constexpr int kMaxTokens = 32;  // tokens per launch
 
 struct DecodeArgs {
@@ -69,88 +68,137 @@ struct UnitCursor {
     }
 };
 
-__device__ __forceinline__ uint32_t magic_pair(uint32_t w) {
-    uint32_t r;
-    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(w));  // (w & m) | c
-    return r;
-}
-
-__device__ __forceinline__ uint4 permute_block(uint4 v) {
-    uint4 o;
-    o.x = __byte_perm(v.x, v.z, 0x5410);  // x0, x4
-    o.y = __byte_perm(v.x, v.z, 0x7632);  // x1, x5
-    o.z = __byte_perm(v.y, v.w, 0x5410);  // x2, x6
-    o.w = __byte_perm(v.y, v.w, 0x7632);  // x3, x7
-    return o;
-}
-
-__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// X -> per-group sums xs and the B operand of the tensor-core kernels: BF16 Xp
-// with each 8-block reordered (0,4,1,5,2,6,3,7).  Lets the GEMV launch early
-// (PDL).
-__global__ void __launch_bounds__(256) prep_x_kernel(const uint16_t* __restrict__ X, int M, int K, uint16_t* __restrict__ Xp,
-                                                     float* __restrict__ xs) {
-    pdl_launch_dependents();
-    const int G = K / kGroup;
-    const int64_t units = (int64_t)kXsStride * G * 16;  // multiple of 32
-    for (int64_t u0 = (int64_t)blockIdx.x * blockDim.x; u0 < units; u0 += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t u = u0 + threadIdx.x;
-        const bool active = u < units;
-        const int m = (int)(u / (G * 16));
-        const int rem = (int)(u - (int64_t)m * G * 16);
-        const int g = rem >> 4, blk = rem & 15;
-        float sum = 0.f;
-        if (active && m < M) {
-            const int64_t xoff = (int64_t)m * K + (int64_t)g * kGroup + blk * 8;
-            const uint4 v = *reinterpret_cast<const uint4*>(X + xoff);
-            *reinterpret_cast<uint4*>(Xp + xoff) = permute_block(v);
-            sum = ((bf16lo(v.x) + bf16hi(v.x)) + (bf16lo(v.y) + bf16hi(v.y))) +
-                  ((bf16lo(v.z) + bf16hi(v.z)) + (bf16lo(v.w) + bf16hi(v.w)));
-        }
-#pragma unroll
-        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        if (active && blk == 0) xs[(int64_t)g * kXsStride + m] = sum;
-    }
+// 2^e as FP32 for e in [-149, 127] (subnormal below -126).
+__device__ __forceinline__ float pow2f(int e) {
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
 }
 
 // --------------------------------------------------------------------------
-// Tensor-core decode kernel (tcgen05 / TMEM), one persistent CTA per SM.
+// Tensor-core decode kernel (tcgen05, 8-bit integer MMA), one persistent CTA
+// per SM, for 2 <= M <= 32 tokens per launch.
 //
-// Per unit (128 weight rows x one group): a dequantiser warp set (4 warps, one
-// weight row per thread = one TMEM lane) turns the row's 16 packed words into
-// 64 BF16 pairs (128 + q) and stores them with tcgen05.st as the A operand
-// (128 x 128 BF16 = 64 columns) in tensor memory.  Column 4w + j holds codes
-// j and j + 4 of word w; the prepared X uses the matching K order, so the B
-// operand (NTOK tokens x 128, K-major) is a plain 128-byte-swizzled TMA tile.
-// One thread issues eight tcgen05.mma (M = 128, N = NTOK, K = 16) per unit
-// into its own TMEM accumulator; the fold warps read it back and apply
-// acc += s * (D - (128 + z) * xsum).
+// The codes are the A operand as unsigned bytes, exactly: per packed word,
+// w & 0x0F0F0F0F holds codes 0, 2, 4, 6 and (w >> 4) & 0x0F0F0F0F codes
+// 1, 3, 5, 7, and a dequantiser thread stores its row's 32 such words into
+// tensor memory (K order (0,2,4,6,1,3,5,7) in every 8-block).  X is the B
+// operand as signed bytes: per group and token, x_int = x * 2^(21 - E) (E the
+// exponent of the group's largest |x|; exact for every x within 2^14 of it,
+// smaller values rounded at 2^(E - 21)) is written in balanced base 256,
+// x_int = 65536 d2 + 256 d1 + d0 with every digit in [-128, 127], and the
+// three digit planes of NTOK tokens are the 3 NTOK rows of B.  One
+// tcgen05.mma kind::i8 (M = 128, N = 3 NTOK, K = 32) thus takes 32 codes of
+// every row against all planes of all tokens, with exact int32 sums; a unit
+// (128 rows x one group) is four MMAs, half the instructions of BF16 operands.
+// The fold warps combine the planes and apply scale and zero point in FP32:
+//   acc += s 2^(E - 21) (65536 D2 + 256 D1 + D0 - z sum_k x_int).
 //
-// Warp roles (448 threads): 0-3 fold (TMEM lane quadrants 0-3, also the row
-// tile epilogue), 4-7 and 8-11 dequantise even and odd units, 12 issues the
-// MMAs, 13 drives TMA.  Rings: shared-memory stages (codes, X tile, xsum),
-// 4 A buffers and 8 (NTOK = 16) or 4 (NTOK = 32) accumulators, each with a
-// full/free mbarrier pair, so loads, dequantisation, MMAs and folds overlap.
+// Warp roles (448 threads): 0-7 fold (warp w: TMEM lane quadrant w % 4, half
+// w / 4 of the tokens; also the row tile epilogue), 8-11 dequantise, 12 issues
+// the MMAs, 13 drives TMA.  Rings:
+// shared-memory stages (codes, X planes, per token X sums and scales), 4 A
+// buffers and 8 (NTOK = 16) or 4 (NTOK = 32) accumulators, each with a
+// full/free mbarrier pair.
+
+// X planes of one launch, prepared by prep_x8_kernel: for group g, row
+// p NTOK + m of the B tile holds digit plane p of token m (128 bytes, MMA K
+// order); xs holds per group [sum_k x_int (FP32) for each token, then
+// 2^(E - 21) for each token].
 template <int NTOK>
 struct TcCfg {
-    static constexpr int kXBlockBytes = NTOK * 128;  // 64 BF16 of K for NTOK tokens
-    static constexpr int kXBytes = 2 * kXBlockBytes;  // one group of K
-    static constexpr int kCodeOff = kXBytes;
-    static constexpr int kXsOff = kXBytes + kStageWords * 4;
-    static constexpr int kStageBytes = kXsOff + 1024;  // xsum slot, keeps stages 1024-aligned
-    static constexpr int kStages = NTOK == 16 ? 12 : 10;
+    static constexpr int kBRows = 3 * NTOK;                  // MMA N
+    static constexpr int kBBytes = kBRows * 128;             // one group of K, 128-byte swizzle
+    static constexpr int kCodeOff = kBBytes;                 // 1024-aligned
+    static constexpr int kXsOff = kCodeOff + kStageWords * 4;
+    static constexpr int kXsBytes = 2 * NTOK * 4;
+    static constexpr int kStageBytes = (kXsOff + kXsBytes + 1023) & ~1023;
+    static constexpr int kStages = (220 * 1024) / kStageBytes;
     static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;  // + alignment slack
-    static constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr int kNumA = 4;                  // A buffers of 64 columns at 0..255
-    static constexpr int kNumD = NTOK == 16 ? 8 : 4;  // accumulators at 256..383
-    static constexpr uint32_t kColD = 256;
+    static constexpr int kACols = 32;                        // 128 rows x 128 bytes
+    static constexpr int kNumA = 4;                          // A buffers at 0..127
+    static constexpr uint32_t kColD = kNumA * kACols;
+    static constexpr int kNumD = (512 - kNumA * kACols) / kBRows;  // accumulators of kBRows columns
 };
 
-constexpr int kFoldWarps = 4;
-constexpr int kDqWarps = 8;
+// Instruction descriptor, kind::i8: A unsigned 8-bit, B signed 8-bit, D s32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_u8s8_s32(int M, int N) {
+    return (2u << 4)                          // D format: S32
+           | (0u << 7)                        // A format: unsigned 8-bit
+           | (1u << 10)                       // B format: signed 8-bit
+           | ((uint32_t)(N >> 3) << 17)       // N / 8
+           | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// D[tmem] (+)= A[tmem] x B[smem desc]; kind::i8, int32 accumulate.
+__device__ __forceinline__ void umma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
+
+// One warp per (group g, token m < NTOK): lane l holds x at k = 4l .. 4l + 3 (word w = l / 2,
+// half h = l % 2).  Tokens m >= M get zero planes.
+template <int NTOK>
+__global__ void __launch_bounds__(256) prep_x8_kernel(const uint16_t* __restrict__ X, int M, int K,
+                                                      uint8_t* __restrict__ planes, float* __restrict__ xs) {
+    pdl_launch_dependents();
+    const int G = K / kGroup;
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)G * NTOK;
+    for (int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; wid < warps;
+         wid += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int g = (int)(wid / NTOK), m = (int)(wid - (int64_t)g * NTOK);
+        uint32_t bits[4] = {0u, 0u, 0u, 0u};
+        if (m < M) {
+            const uint2 v = __ldg(reinterpret_cast<const uint2*>(X + (int64_t)m * K + (int64_t)g * kGroup + lane * 4));
+            bits[0] = v.x & 0xFFFFu;
+            bits[1] = v.x >> 16;
+            bits[2] = v.y & 0xFFFFu;
+            bits[3] = v.y >> 16;
+        }
+        uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
+        amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+        const int ef = (int)(amax >> 7);
+        const int E = ef == 0 ? -127 : ef - 127;  // every |x| of the group is below 2^(E + 1)
+        const int kx = 21 - E;                    // in [-106, 148]
+        const int k1 = min(kx, 127);
+        const float s1 = pow2f(k1), s2 = pow2f(kx - k1);  // exact scalings, |x * 2^kx| < 2^22
+        int xi[4];
+        uint32_t dg[3] = {0u, 0u, 0u};  // this lane's digit bytes per plane, as (i0, i2, i1, i3)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            xi[i] = __float2int_rn(__uint_as_float(bits[i] << 16) * s1 * s2);
+            const int d0 = ((xi[i] + 128) & 255) - 128;
+            const int t = (xi[i] - d0) >> 8;
+            const int d1 = ((t + 128) & 255) - 128;
+            const int d2 = (t - d1) >> 8;
+            const int pos = (i & 1) ? 16 + 8 * (i >> 1) : 8 * (i >> 1);  // i0 -> 0, i2 -> 8, i1 -> 16, i3 -> 24
+            dg[0] |= (uint32_t)(d0 & 255) << pos;
+            dg[1] |= (uint32_t)(d1 & 255) << pos;
+            dg[2] |= (uint32_t)(d2 & 255) << pos;
+        }
+        // word w's 8 MMA-order bytes: [h0.i0, h0.i2, h1.i0, h1.i2, h0.i1, h0.i3, h1.i1, h1.i3]
+        const int h = lane & 1, w = lane >> 1;
+#pragma unroll
+        for (int p = 0; p < 3; ++p) {
+            const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, dg[p], 1);
+            const uint32_t lo = h ? other : dg[p], hi = h ? dg[p] : other;  // halves of lanes h = 0 and 1
+            const uint32_t out = h ? __byte_perm(lo, hi, 0x7632) : __byte_perm(lo, hi, 0x5410);
+            *reinterpret_cast<uint32_t*>(planes + ((int64_t)g * 3 * NTOK + p * NTOK + m) * 128 + 8 * w + 4 * h) = out;
+        }
+        const int sum = __reduce_add_sync(0xFFFFFFFFu, (xi[0] + xi[1]) + (xi[2] + xi[3]));  // |sum| < 2^29
+        if (lane == 0) {
+            xs[(int64_t)g * 2 * NTOK + m] = (float)sum;
+            xs[(int64_t)g * 2 * NTOK + NTOK + m] = pow2f(E - 21);
+        }
+    }
+}
+
+constexpr int kFoldWarps = 8;                    // two per TMEM lane quadrant, each with half the tokens
+constexpr int kDqWarps = 4;
 constexpr int kMmaWarp = kFoldWarps + kDqWarps;  // 12
 constexpr int kTmaWarp = kMmaWarp + 1;           // 13
 constexpr int kTcThreads = (kTmaWarp + 1) * 32;  // 448
@@ -162,6 +210,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     using C = TcCfg<NTOK>;
     constexpr int S = C::kStages;
     constexpr int NA = C::kNumA, ND = C::kNumD;
+    constexpr uint32_t kIdesc = idesc_u8s8_s32(128, C::kBRows);
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[S], empty[S], afull[NA], afree[NA], mdone[ND], dfree[ND];
     __shared__ uint32_t s_tmem;
@@ -180,7 +229,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 4 + 1 + kFoldWarps);  // dequantiser set, MMA commit, fold warps (xsum)
+            mbar_init(&empty[s], 4 + 1 + kFoldWarps);  // dequantiser set, MMA commit, fold warps (X sums)
         }
         for (int i = 0; i < NA; ++i) {
             mbar_init(&afull[i], 4);
@@ -202,22 +251,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tx);
+            constexpr uint32_t kTx = C::kBBytes + kStageWords * 4 + C::kXsBytes;
             const int pre = min(S, nunits);
             // the weights do not depend on the preparation kernel: start streaming them at once
             UnitCursor cur(u_first, G);
             for (int i = 0; i < pre; ++i, cur.next(G)) {
-                mbar_arrive_expect_tx(&full[i], C::kStageBytes - 1024 + 128);
+                mbar_arrive_expect_tx(&full[i], kTx);
                 tma_load_2d(ring + i * C::kStageBytes + C::kCodeOff, &tq, cur.g * kWordsPerGroup,
                             cur.tile * kRowsPerCta, &full[i]);
             }
-            pdl_wait_primary();  // X and xsum come from the preparation kernel
+            pdl_wait_primary();  // X planes come from the preparation kernel
             UnitCursor cx(u_first, G);
             for (int i = 0; i < pre; ++i, cx.next(G)) {
                 const int g = cx.g;
                 unsigned char* st = ring + i * C::kStageBytes;
-                tma_load_2d(st, &tx, g * kGroup, 0, &full[i]);
-                tma_load_2d(st + C::kXBlockBytes, &tx, g * kGroup + 64, 0, &full[i]);
-                bulk_load(st + C::kXsOff, a.xs + (int64_t)g * kXsStride, 128, &full[i]);
+                tma_load_2d(st, &tx, 0, g * C::kBRows, &full[i]);
+                bulk_load(st + C::kXsOff, a.xs + (int64_t)g * 2 * NTOK, C::kXsBytes, &full[i]);
             }
             int issued = pre;
             for (int i = pre; i < nunits; ++i, cur.next(G)) {
@@ -225,11 +274,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
                 if (!mbar_wait(&empty[s], ((i / S) - 1) & 1, a.fault, 21)) break;
                 const int tile = cur.tile, g = cur.g;
                 unsigned char* st = ring + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], C::kStageBytes - 1024 + 128);
+                mbar_arrive_expect_tx(&full[s], kTx);
                 tma_load_2d(st + C::kCodeOff, &tq, g * kWordsPerGroup, tile * kRowsPerCta, &full[s]);
-                tma_load_2d(st, &tx, g * kGroup, 0, &full[s]);
-                tma_load_2d(st + C::kXBlockBytes, &tx, g * kGroup + 64, 0, &full[s]);
-                bulk_load(st + C::kXsOff, a.xs + (int64_t)g * kXsStride, 128, &full[s]);
+                tma_load_2d(st, &tx, 0, g * C::kBRows, &full[s]);
+                bulk_load(st + C::kXsOff, a.xs + (int64_t)g * 2 * NTOK, C::kXsBytes, &full[s]);
                 ++issued;
             }
             // every copy issued must land before the CTA may exit
@@ -246,12 +294,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
                 if (i >= ND && !mbar_wait(&dfree[di], ((i / ND) - 1) & 1, a.fault, 32)) break;
                 if (!mbar_wait(&full[s], (i / S) & 1, a.fault, 33)) break;
                 tc_fence_after();
-                const uint32_t xaddr = smem_u32(ring + s * C::kStageBytes);
+                const uint32_t baddr = smem_u32(ring + s * C::kStageBytes);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bdesc = sw128_kmajor_desc(xaddr + (kk >> 2) * C::kXBlockBytes + (kk & 3) * 32);
-                    umma_ts(tmem + C::kColD + di * NTOK, tmem + ai * 64 + kk * 8, bdesc, C::kIdesc, kk > 0);
-                }
+                for (int kk = 0; kk < 4; ++kk)  // K = 32 bytes per MMA: 32 bytes along the swizzled row
+                    umma_ts_i8(tmem + C::kColD + di * C::kBRows, tmem + ai * C::kACols + kk * 8,
+                               sw128_kmajor_desc(baddr + kk * 32), kIdesc, kk > 0);
                 umma_commit(&afree[ai]);
                 umma_commit(&mdone[di]);
                 umma_commit(&empty[s]);
@@ -262,41 +309,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     }
 
     if (warp >= kFoldWarps) {  // ---------------------------------- dequantisers
-        const int set = (warp - kFoldWarps) >> 2;         // 0: even units, 1: odd units
-        const int quad = warp & 3;                        // TMEM lane quadrant
+        const int quad = warp & 3;                        // TMEM lane quadrant (warps 8-11: 0-3)
         const int row_local = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const int sw = (row_local >> 1) & 3;              // 64-byte swizzle of the codes tile
-        for (int i = set; i < nunits; i += 2) {
+        for (int i = 0; i < nunits; ++i) {
             const int s = i % S, ai = i % NA;
             if (i >= NA && !mbar_wait(&afree[ai], ((i / NA) - 1) & 1, a.fault, 41)) break;
             if (!mbar_wait(&full[s], (i / S) & 1, a.fault, 42)) break;
             // logical 16-byte chunk q of row r sits at chunk q ^ ((r >> 1) & 3): conflict-free reads
             const unsigned char* codes = ring + s * C::kStageBytes + C::kCodeOff + row_local * 64;
-            uint32_t w[16];
+            uint32_t pr[32];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const uint4 v = *reinterpret_cast<const uint4*>(codes + 16 * (q ^ sw));
-                w[4 * q] = v.x;
-                w[4 * q + 1] = v.y;
-                w[4 * q + 2] = v.z;
-                w[4 * q + 3] = v.w;
+                const uint32_t wq[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    pr[2 * (4 * q + j)] = wq[j] & 0x0F0F0F0Fu;             // codes 0, 2, 4, 6
+                    pr[2 * (4 * q + j) + 1] = (wq[j] >> 4) & 0x0F0F0F0Fu;  // codes 1, 3, 5, 7
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pr[32];
-#pragma unroll
-                for (int ww = 0; ww < 8; ++ww) {
-                    const uint32_t x = w[8 * half + ww];
-                    pr[4 * ww + 0] = magic_pair(x);
-                    pr[4 * ww + 1] = magic_pair(x >> 4);
-                    pr[4 * ww + 2] = magic_pair(x >> 8);
-                    pr[4 * ww + 3] = magic_pair(x >> 12);
-                }
-                tmem_st32(tl + ai * 64 + half * 32, pr);
-            }
+            tmem_st32(tl + ai * C::kACols, pr);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -305,13 +341,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         return;
     }
 
-    // ------------------------------------------------------- fold warps 0-3
-    const int row_local = warp * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    // ------------------------------------------------------- fold warps 0-7
+    constexpr int TH = NTOK / 2;                  // tokens per fold thread
+    const int quad = warp & 3, th = warp >> 2;    // lane quadrant, token half
+    const int row_local = quad * 32 + lane;
+    const int m_base = th * TH;
+    const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const int N = a.N, M = a.M;
-    float acc[NTOK];
+    float acc[TH];
 #pragma unroll
-    for (int m = 0; m < NTOK; ++m) acc[m] = 0.f;
+    for (int m = 0; m < TH; ++m) acc[m] = 0.f;
     bool aborted = false;
     int cur_tile = -1;
 
@@ -322,15 +361,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         if (first == last) {
             if (n < N) {
 #pragma unroll
-                for (int m = 0; m < NTOK; ++m)
-                    if (m < M) a.Y[(int64_t)m * N + n] = float_to_bf16_bits(acc[m]);
+                for (int e = 0; e < TH; ++e)
+                    if (m_base + e < M) a.Y[(int64_t)(m_base + e) * N + n] = float_to_bf16_bits(acc[e]);
             }
         } else {
             const int slot = b - first, nseg = last - first + 1;
             float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * M * kRowsPerCta;
 #pragma unroll
-            for (int m = 0; m < NTOK; ++m)
-                if (m < M) part[m * kRowsPerCta + row_local] = acc[m];
+            for (int e = 0; e < TH; ++e)
+                if (m_base + e < M) part[(m_base + e) * kRowsPerCta + row_local] = acc[e];
             named_barrier_sync(1, kFoldWarps * 32);
             if (threadIdx.x == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
             named_barrier_sync(1, kFoldWarps * 32);
@@ -347,20 +386,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             named_barrier_sync(1, kFoldWarps * 32);
         }
 #pragma unroll
-        for (int m = 0; m < NTOK; ++m) acc[m] = 0.f;
+        for (int e = 0; e < TH; ++e) acc[e] = 0.f;
     };
 
-    // scale and 128 + zero of this thread's row, one unit ahead
-    auto load_meta = [&](int j, int tile, int g, float& sv, float& zv) {
-        sv = 0.f;
-        zv = 0.f;
-        if (j < nunits) {
-            const int n = tile * kRowsPerCta + row_local;
-            if (n < N) {
-                sv = bf16_bits_to_float(__ldg(a.scales + (int64_t)n * G + g));
-                zv = 128.f + (float)__ldg(a.zeros + (int64_t)n * G + g);
-            }
-        }
+    // scale and zero point of this thread's row, one unit ahead
+    // raw loads, converted only when used, so that nothing waits on them before then; the row is
+    // clamped into the matrix (rows past N, and units past the last, are masked at use)
+    auto load_meta = [&](int tile, int g, uint32_t& sraw, int& zraw) {
+        const int n = min(tile * kRowsPerCta + row_local, N - 1);
+        sraw = __ldg(a.scales + (int64_t)n * G + g);
+        zraw = __ldg(a.zeros + (int64_t)n * G + g);
     };
 
     auto fold_unit = [&](int j, int tile, float sv, float zv) {
@@ -375,46 +410,64 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             return;
         }
         tc_fence_after();
-        uint32_t d0[16], d1[16];
-        tmem_ld16(tl + C::kColD + di * NTOK, d0);
-        if (NTOK == 32) tmem_ld16(tl + C::kColD + di * NTOK + 16, d1);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dfree[di]);
         const float* xs = reinterpret_cast<const float*>(ring + s * C::kStageBytes + C::kXsOff);
+        const uint32_t dcol = tl + C::kColD + di * C::kBRows + m_base;
+        // integer -> FP32 by the 2^23 + 2^22 magic (exact for |v| < 2^22; every plane sum is)
+        auto to_f = [](uint32_t v) { return __int_as_float((int)v + 0x4B400000) - 12582912.f; };
 #pragma unroll
-        for (int q = 0; q < NTOK / 4; ++q) {
-            if (4 * q < M) {
-                const float4 xv = *reinterpret_cast<const float4*>(xs + 4 * q);
-                const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
+        for (int h = 0; h < TH / 8; ++h) {  // 8 tokens at a time: their three digit planes
+            uint32_t d0[8], d1[8], d2[8];
+            tmem_ld8(dcol + h * 8, d0);
+            tmem_ld8(dcol + NTOK + h * 8, d1);
+            tmem_ld8(dcol + 2 * NTOK + h * 8, d2);
+            tmem_wait_ld();
+            if (h + 1 == TH / 8) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&dfree[di]);
+            }
+            if (m_base + h * 8 >= M) continue;  // padding tokens only
+            const float4 xs0 = *reinterpret_cast<const float4*>(xs + m_base + h * 8);
+            const float4 xs1 = *reinterpret_cast<const float4*>(xs + m_base + h * 8 + 4);
+            const float4 xc0 = *reinterpret_cast<const float4*>(xs + NTOK + m_base + h * 8);
+            const float4 xc1 = *reinterpret_cast<const float4*>(xs + NTOK + m_base + h * 8 + 4);
+            const float xsum[8] = {xs0.x, xs0.y, xs0.z, xs0.w, xs1.x, xs1.y, xs1.z, xs1.w};
+            const float xsc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int m = 4 * q + e;
-                    const uint32_t dm = m < 16 ? d0[m & 15] : d1[m & 15];
-                    acc[m] = fmaf(sv, fmaf(-zv, xq[e], __uint_as_float(dm)), acc[m]);
-                }
+            for (int e = 0; e < 8; ++e) {
+                // sum q x_int = 65536 D2 + 256 D1 + D0
+                const float qx = fmaf(to_f(d2[e]), 65536.f, fmaf(to_f(d1[e]), 256.f, to_f(d0[e])));
+                acc[h * 8 + e] = fmaf(sv * xsc[e], fmaf(-zv, xsum[e], qx), acc[h * 8 + e]);
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // xsum read
+        if (lane == 0) mbar_arrive(&empty[s]);  // X sums and scales read
     };
 
-    // two cursors: `fc` at the unit being folded, `mc` one unit ahead for the metadata loads
+    // metadata loads run kMetaAhead units ahead of the folds (scattered 2- and 4-byte loads of L2
+    // latency): unit j's scale and zero point live in slot j % kMetaAhead of a register ring
+    constexpr int kMetaAhead = 4;
     UnitCursor fc(u_first, G), mc(u_first, G);
-    float s0, z0, s1, z1;
-    load_meta(0, mc.tile, mc.g, s0, z0);
-    mc.next(G);
-    for (int j = 0; j < nunits; j += 2) {
-        load_meta(j + 1, mc.tile, mc.g, s1, z1);
+    uint32_t sr[kMetaAhead];
+    int zr[kMetaAhead];
+#pragma unroll
+    for (int u = 0; u < kMetaAhead; ++u) {
+        load_meta(mc.tile, mc.g, sr[u], zr[u]);
         mc.next(G);
-        fold_unit(j, fc.tile, s0, z0);
-        fc.next(G);
-        if (j + 1 < nunits) {
-            load_meta(j + 2, mc.tile, mc.g, s0, z0);
-            mc.next(G);
-            fold_unit(j + 1, fc.tile, s1, z1);
-            fc.next(G);
+    }
+    for (int j0 = 0; j0 < nunits; j0 += kMetaAhead) {
+#pragma unroll
+        for (int u = 0; u < kMetaAhead; ++u) {
+            const int j = j0 + u;
+            if (j < nunits) {
+                const bool row_ok = fc.tile * kRowsPerCta + row_local < N;
+                const float sv = row_ok ? bf16_bits_to_float((uint16_t)sr[u]) : 0.f;
+                const float zv = (float)zr[u];
+                load_meta(mc.tile, mc.g, sr[u], zr[u]);
+                mc.next(G);
+                fold_unit(j, fc.tile, sv, zv);
+                fc.next(G);
+            }
         }
     }
     if (cur_tile >= 0) flush(cur_tile);
@@ -510,11 +563,6 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
     int d;
     asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
     return d;
-}
-
-// 2^e as FP32 for e in [-149, 127] (subnormal below -126).
-__device__ __forceinline__ float pow2f(int e) {
-    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
 }
 
 // This lane's four BF16 values of group g: lane 2w + h holds values 4h..4h+3 of word w.
@@ -885,9 +933,9 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     else if (kind == 3)  // zeros: int32 [rows = N][cols = G], box = 8 groups x 128 rows
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_INT32, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 4, kCcMetaGroups, kRowsPerCta);
-    else  // prepared X: bf16 [rows = Mc][cols = K], box = 64 x NTOK (kind), 128-byte swizzle
-        ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
-                            (uint64_t)cols * 2, 64, (uint32_t)kind, CU_TENSOR_MAP_SWIZZLE_128B);
+    else  // X digit planes: uint8 [rows = G * 3 NTOK][cols = 128], box = 128 x 3 NTOK (kind = NTOK), 128-byte swizzle
+        ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, ptr, (uint64_t)cols, (uint64_t)rows,
+                            (uint64_t)cols, 128, (uint32_t)(3 * kind), CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return false;
     e.ptr = ptr;
     e.rows = rows;
@@ -952,9 +1000,10 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.units_base = (int)(units / grid);
     p.units_rem = (int)(units % grid);
     p.max_slots = (int)((G - 1) / p.units_base + 2);
-    // the integer kernel prepares X itself
-    p.ws_xp_bytes = p.cc_tokens ? 0 : align256((size_t)Mc * K * 2);
-    p.ws_xs_bytes = p.cc_tokens ? 0 : align256((size_t)G * kXsStride * 4);
+    // the CUDA-core kernel prepares X itself; the tensor-core kernel reads X digit planes and
+    // per-token sums and scales prepared per launch
+    p.ws_xp_bytes = p.cc_tokens ? 0 : align256((size_t)G * 3 * p.nt * 128);
+    p.ws_xs_bytes = p.cc_tokens ? 0 : align256((size_t)G * 2 * p.nt * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
     p.ws_counter_bytes = align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
     return p;
@@ -971,23 +1020,27 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
     if (!fault) return W4A16_ERR_CUDA;
     char* ws = reinterpret_cast<char*>(workspace);
     int* counters = reinterpret_cast<int*>(ws);
-    uint16_t* Xp = reinterpret_cast<uint16_t*>(ws + plan.ws_counter_bytes);
+    uint8_t* planes = reinterpret_cast<uint8_t*>(ws + plan.ws_counter_bytes);
     float* xs = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes);
     float* partial = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes + plan.ws_xs_bytes);
     const int G = (int)(K / kGroup);
     for (int64_t m0 = 0; m0 < M; m0 += kMaxTokens) {
         const int Mc = (int)((M - m0) < kMaxTokens ? (M - m0) : kMaxTokens);
         CUtensorMap tx;
-        if (!plan.cc_tokens && !cached_tmap(plan.nt, Xp, Mc, K, &tx)) return W4A16_ERR_CUDA;
+        if (!plan.cc_tokens && !cached_tmap(plan.nt, planes, (int64_t)G * 3 * plan.nt, 128, &tx))
+            return W4A16_ERR_CUDA;
         if (!plan.cc_tokens) {
-            const int64_t prep_units = (int64_t)kXsStride * G * 16;
-            int prep_grid = (int)ceil_div(prep_units, 256);
+            const int64_t prep_threads = (int64_t)G * plan.nt * 32;
+            int prep_grid = (int)ceil_div(prep_threads, 256);
             if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
-            prep_x_kernel<<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, Xp, xs);
+            if (plan.nt == 16)
+                prep_x8_kernel<16><<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, planes, xs);
+            else
+                prep_x8_kernel<32><<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, planes, xs);
             if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
         }
         DecodeArgs args;
-        args.Xp = plan.cc_tokens ? X + m0 * K : Xp;  // the integer kernel reads X as given
+        args.Xp = X + m0 * K;  // read by the CUDA-core kernel; the tensor-core kernel reads the planes
         args.xs = xs;
         args.scales = scales;
         args.zeros = zeros;
