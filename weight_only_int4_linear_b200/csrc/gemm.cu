@@ -52,14 +52,21 @@ constexpr int kPXBytes = kPBN * kPBK * 2;      // 32 KB
 constexpr int kPABytes = kPBM * kPBK * 2;      // 16 KB
 constexpr int kPCodeBytes = kPBM * kPBK / 2;   // 4 KB
 constexpr int kPStageBytes = kPXBytes + kPABytes + kPCodeBytes;  // 52 KB (1024-aligned)
-constexpr size_t kPSmem = (size_t)kPStages * kPStageBytes + 1024;
+// Per-group metadata ring, read by the fold warps: slot = group count % kPMetaSlots holds the 128 rows'
+// (scale, zero point) as FP32 pairs, written by the dequantisers, and the X sums of the tile's 256
+// tokens, copied by TMA.
+constexpr int kPMetaSlots = 8;
+constexpr int kPMetaSzBytes = kPBM * 8;
+constexpr int kPMetaBytes = kPMetaSzBytes + kPBN * 4;  // 2 KB
+constexpr int kPMetaOff = kPStages * kPStageBytes;
+constexpr size_t kPSmem = (size_t)kPMetaOff + kPMetaSlots * kPMetaBytes + 1024;
 constexpr int kPThreads = 512;
 constexpr uint32_t kPIdesc = idesc_bf16_f32(kPBM, kPBN);
 
 struct PrefillArgs {
     const uint16_t* scales;
     const int32_t* zeros;
-    const float* xsT;  // [G][Mp]: per-group sums of X, Mp = M rounded up to a multiple of 4
+    const float* xsT;  // [G][Mp]: per-group sums of X, Mp = M rounded up to a multiple of 256 (zero past M)
     uint16_t* Y;
     int* fault;
     int M, N, K, G, Mp;
@@ -93,7 +100,7 @@ __device__ __forceinline__ uint4 permute_block(uint4 v) {
 }
 
 // X -> Xp (each 8-block reordered (0,4,1,5,2,6,3,7)) and xsT[g][m] = sum of the group
-// (row stride Mp, a multiple of 4 so the fold can read float4s).
+// (row stride Mp, a multiple of the 256-token tile so one bulk copy per group and tile reads it).
 __global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __restrict__ X, int M, int K, int Mp,
                                                            uint16_t* __restrict__ Xp, float* __restrict__ xsT) {
     pdl_launch_dependents();
@@ -136,10 +143,11 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                                                                const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
+    __shared__ __align__(8) uint64_t metafull[kPMetaSlots], metafree[kPMetaSlots];
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(16) float s_xs[2][kPBN];  // per-group X sums of the tile's tokens, by group parity
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+    unsigned char* meta = ring + kPMetaOff;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
@@ -157,6 +165,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         for (int i = 0; i < 2; ++i) {
             mbar_init(&mdone[i], 1);
             mbar_init(&dfree[i], 8);
+        }
+        for (int i = 0; i < kPMetaSlots; ++i) {
+            mbar_init(&metafull[i], 4);  // the dequantiser warps, after the TMA copy of the X sums landed
+            mbar_init(&metafree[i], 8);  // the fold warps
         }
         fence_mbar_init();
     }
@@ -181,9 +193,17 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     const int s = it % kPStages;
                     if (it >= kPStages && !mbar_wait(&empty[s], ((it / kPStages) - 1) & 1, a.fault, 61)) goto done_tma;
                     unsigned char* st = ring + s * kPStageBytes;
-                    mbar_arrive_expect_tx(&full[s], kPXBytes + kPCodeBytes);
+                    const bool first_half = (ks & 1) == 0;  // a group starts: its X sums go to the metadata ring
+                    const int gi = it >> 1, slot = gi % kPMetaSlots;
+                    if (first_half && gi >= kPMetaSlots &&
+                        !mbar_wait(&metafree[slot], ((gi / kPMetaSlots) - 1) & 1, a.fault, 63))
+                        goto done_tma;
+                    mbar_arrive_expect_tx(&full[s], kPXBytes + kPCodeBytes + (first_half ? kPBN * 4 : 0));
                     tma_load_2d(st, &tx, ks * kPBK, mt * kPBN, &full[s]);
                     tma_load_2d(st + kPXBytes + kPABytes, &tq, ks * (kPBK / 8), nt * kPBM, &full[s]);
+                    if (first_half)
+                        bulk_load(meta + slot * kPMetaBytes + kPMetaSzBytes,
+                                  a.xsT + (int64_t)(ks >> 1) * a.Mp + mt * kPBN, kPBN * 4, &full[s]);
                 }
             }
         done_tma:
@@ -227,14 +247,27 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             const int n = nt * kPBM + r;
             uint32_t zc2 = 0x43004300u;  // (128 + c) as a BF16 pair
             for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
-                if ((ks & 1) == 0) {
-                    const int z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + (ks >> 1)) : 0;
+                const bool first_half = (ks & 1) == 0;
+                int z = 0;
+                uint32_t sraw = 0;
+                if (first_half) {
+                    z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + (ks >> 1)) : 0;
+                    sraw = n < a.N ? __ldg(a.scales + (int64_t)n * G + (ks >> 1)) : 0;
                     const int c = (z >= -128 && z <= 128) ? z : 0;
                     const uint32_t cb = __float_as_uint(128.f + (float)c) >> 16;  // exact: |128 + c| <= 256
                     zc2 = cb | (cb << 16);
                 }
                 const int s = it % kPStages;
                 if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 81)) goto done_dq;
+                if (first_half) {
+                    // this row's scale and zero point for the fold warps; the stage's full barrier also
+                    // covered the TMA copy of the group's X sums into the same slot
+                    const int gi = it >> 1, slot = gi % kPMetaSlots;
+                    reinterpret_cast<float2*>(meta + slot * kPMetaBytes)[r] =
+                        make_float2(bf16_bits_to_float((uint16_t)sraw), (float)z);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&metafull[slot]);
+                }
                 unsigned char* st = ring + s * kPStageBytes;
                 const unsigned char* codes = st + kPXBytes + kPABytes + r * 32;
                 const uint4 c0 = *reinterpret_cast<const uint4*>(codes + 16 * csw);
@@ -267,43 +300,24 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         for (int j = 0; j < 128; ++j) T[j] = 0.f;
         int gc = 0;
         bool aborted = false;
-        // loads for the next group are issued one group ahead
-        auto load_meta = [&](int tt, int g, float& sv, float& zv, float& xv) {
-            sv = 0.f;
-            zv = 0.f;
-            xv = 0.f;
-            if (tt >= ntiles) return;
-            const int tile = t_first + tt;
-            const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
-            const int n = nt * kPBM + row;
-            const int m = mt * kPBN + colh * 128 + hl;
-            if (n < a.N) {
-                sv = bf16_bits_to_float(__ldg(a.scales + (int64_t)n * G + g));
-                zv = (float)__ldg(a.zeros + (int64_t)n * G + g);
-            }
-            if (m < a.M) xv = __ldg(a.xsT + (int64_t)g * a.Mp + m);
-        };
-        float nsv, nzv, nxv;
-        load_meta(0, 0, nsv, nzv, nxv);
         for (int tt = 0; tt < ntiles; ++tt) {
             const int tile = t_first + tt;
             const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
             const int n = nt * kPBM + row;
             const int m0 = mt * kPBN + colh * 128;
             for (int g = 0; g < G; ++g, ++gc) {
-                const float sv = nsv, zv = nzv;
-                s_xs[gc & 1][colh * 128 + hl] = nxv;
-                if (g + 1 < G) load_meta(tt, g + 1, nsv, nzv, nxv);
-                else load_meta(tt + 1, 0, nsv, nzv, nxv);
-                // rows whose zero point was not subtracted by the dequantiser (|z| > 128) fold
-                // - s (z - c) xsum with c = 0; the X sums of this half's tokens are in s_xs
-                const float zr = (zv >= -128.f && zv <= 128.f) ? 0.f : zv;
-                named_barrier_sync(2 + colh, 128);
-                const bool need_xs = __any_sync(0xFFFFFFFFu, zr != 0.f);
-                const float* xs = &s_xs[gc & 1][colh * 128];
-                const int dbuf = gc & 1;
+                const int slot = gc % kPMetaSlots, dbuf = gc & 1;
+                if (!aborted && !mbar_wait(&metafull[slot], (gc / kPMetaSlots) & 1, a.fault, 92)) aborted = true;
                 if (!aborted && !mbar_wait(&mdone[dbuf], (gc >> 1) & 1, a.fault, 91)) aborted = true;
                 if (!aborted) {
+                    const unsigned char* ms = meta + slot * kPMetaBytes;
+                    const float2 sz = reinterpret_cast<const float2*>(ms)[row];  // rows past N: scale 0
+                    const float sv = sz.x, zv = sz.y;
+                    // rows whose zero point was not subtracted by the dequantiser (|z| > 128) fold
+                    // - s (z - c) xsum with c = 0, the X sums of this half's tokens from the ring
+                    const float zr = (zv >= -128.f && zv <= 128.f) ? 0.f : zv;
+                    const bool need_xs = __any_sync(0xFFFFFFFFu, zr != 0.f);
+                    const float* xs = reinterpret_cast<const float*>(ms + kPMetaSzBytes) + colh * 128;
                     tc_fence_after();
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc) {
@@ -329,7 +343,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     tc_fence_before();
                 }
                 __syncwarp();
-                if (lane == 0 && !aborted) mbar_arrive(&dfree[dbuf]);
+                if (lane == 0 && !aborted) {
+                    mbar_arrive(&dfree[dbuf]);
+                    mbar_arrive(&metafree[slot]);
+                }
             }
             // epilogue: this thread's row n, tokens m0 .. m0 + 127
             if (n < a.N) {
@@ -391,7 +408,7 @@ size_t align256p(size_t x) { return (x + 255) & ~(size_t)255; }
 }  // namespace
 
 size_t prefill_workspace_bytes(int64_t M, int64_t K) {
-    const int64_t Mp = (M + 3) & ~(int64_t)3;
+    const int64_t Mp = (M + kPBN - 1) / kPBN * kPBN;
     // the decode path's counter area stays untouched at the front (shared workspaces)
     return kCounterBytes + align256p((size_t)M * K * 2) + align256p((size_t)(K / kGroup) * Mp * 4);
 }
@@ -417,7 +434,7 @@ int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qwei
     const int64_t units = M * G * 16;
     int pgrid = (int)ceil_div(units, 256);
     if (pgrid > num_sms_current() * 16) pgrid = num_sms_current() * 16;
-    const int Mp = (int)((M + 3) & ~(int64_t)3);
+    const int Mp = (int)((M + kPBN - 1) / kPBN * kPBN);
     if (Mp > M && cudaMemsetAsync(xsT, 0, (size_t)G * Mp * 4, stream) != cudaSuccess) return W4A16_ERR_CUDA;
     prefill_prep_kernel<<<pgrid, 256, 0, stream>>>(X, (int)M, (int)K, Mp, Xp, xsT);
     if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
