@@ -25,7 +25,7 @@
 // (half a group).  MMA K order inside each 8-block of K is (0,4,1,5,2,6,3,7):
 // that is the order a lop3 pair extraction yields, and X is prepared in it.
 //
-// Warps (512 threads):
+// Warps (512 threads with 8 fold warps):
 //   0-3   dequantise: thread = weight row; 8 packed words -> one 128-byte
 //         row of the 128B-swizzled K-major A tile
 //   4-11  fold + epilogue: warp w reads TMEM lane quadrant w % 4, token
@@ -60,7 +60,24 @@ constexpr int kPMetaSzBytes = kPBM * 8;
 constexpr int kPMetaBytes = kPMetaSzBytes + kPBN * 4;  // 2 KB
 constexpr int kPMetaOff = kPStages * kPStageBytes;
 constexpr size_t kPSmem = (size_t)kPMetaOff + kPMetaSlots * kPMetaBytes + 1024;
-constexpr int kPThreads = 512;
+#ifndef W4A16_PF_FOLD_WARPS
+#define W4A16_PF_FOLD_WARPS 8
+#endif
+constexpr int kPFoldWarps = W4A16_PF_FOLD_WARPS;          // 8 or 16 (2 or 4 per TMEM lane quadrant)
+constexpr int kPFoldParts = kPFoldWarps / 4;              // token column slices per lane quadrant
+constexpr int kPFoldCols = kPBN / kPFoldParts;            // token columns per fold thread: 128 or 64
+constexpr int kPThreads = (4 + kPFoldWarps + 4) * 32;     // dequant warpgroup, fold warpgroups, TMA/MMA warpgroup
+constexpr int kPTmaWarp = 4 + kPFoldWarps, kPMmaWarp = kPTmaWarp + 1;
+// register split: every warp starts with the launch share (65536 / threads, a multiple of 8);
+// setmaxnreg moves registers from the dequantisers and the TMA/MMA warpgroup to the fold warps
+constexpr int kPRegsLaunch = (65536 / kPThreads) & ~7;
+constexpr int kPRegsDequant = 56;
+constexpr int kPRegsIssue = kPFoldWarps == 16 ? 40 : 72;
+constexpr int kPRegsFold = kPFoldWarps == 16 ? 96 : 192;
+static_assert(32 * (4 * kPRegsDequant + 4 * kPRegsIssue + kPFoldWarps * kPRegsFold) <= kPRegsLaunch * kPThreads,
+              "setmaxnreg split exceeds the registers the block is launched with");
+static_assert(kPFoldWarps == 8 || kPFoldWarps == 16, "fold warps");
+constexpr int kPLdCols = kPFoldWarps == 16 ? 8 : 16;    // TMEM columns per fold load
 constexpr uint32_t kPIdesc = idesc_bf16_f32(kPBM, kPBN);
 
 struct PrefillArgs {
@@ -126,6 +143,9 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __res
     }
 }
 
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[8]) { tmem_ld8(taddr, r); }
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16(taddr, r); }
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
@@ -164,11 +184,11 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&mdone[i], 1);
-            mbar_init(&dfree[i], 8);
+            mbar_init(&dfree[i], kPFoldWarps);
         }
         for (int i = 0; i < kPMetaSlots; ++i) {
             mbar_init(&metafull[i], 4);  // the dequantiser warps, after the TMA copy of the X sums landed
-            mbar_init(&metafree[i], 8);  // the fold warps
+            mbar_init(&metafree[i], kPFoldWarps);  // the fold warps
         }
         fence_mbar_init();
     }
@@ -179,9 +199,9 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     const int wg = warp >> 2;
 
     // register split (launch: 512 x 128 = 65536): 4 x 32 x (72 + 56 + 192 + 192) = 65536
-    if (wg == 3) {  // ------------------------------------------------ TMA + MMA
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;");
-        if (warp == 12 && lane == 0) {
+    if (wg == 1 + kPFoldParts) {  // ------------------------------------------------ TMA + MMA
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPRegsIssue));
+        if (warp == kPTmaWarp && lane == 0) {
             prefetch_tmap(&tx);
             prefetch_tmap(&tq);
             pdl_wait_primary();  // X comes from the preparation kernel
@@ -209,7 +229,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         done_tma:
             // copies in flight land before the CTA may exit
             for (int i = max(0, it - kPStages); i < it; ++i) mbar_wait(&full[i % kPStages], (i / kPStages) & 1, a.fault, 62);
-        } else if (warp == 13 && lane == 0) {
+        } else if (warp == kPMmaWarp && lane == 0) {
             int it = 0, gc = 0;
             for (int tt = 0; tt < ntiles; ++tt) {
                 for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
@@ -237,7 +257,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         done_mma:;
         }
     } else if (wg == 0) {  // ------------------------------------ dequantisers
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPRegsDequant));
         const int r = threadIdx.x;  // weight row within the tile
         // codes tile: 32 bytes per row, 32-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 2) & 1)
         const int csw = (r >> 2) & 1;
@@ -289,22 +309,22 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         }
     done_dq:;
     } else {  // -------------------------------------------- fold + epilogue (wg 1, 2)
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 192;");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPRegsFold));
         const int quad = warp & 3;
-        const int colh = (warp - 4) >> 2;            // token half of the tile
+        const int colh = (warp - 4) >> 2;            // token column slice of the tile (kPFoldCols wide)
         const int row = quad * 32 + lane;            // weight row within the tile = TMEM lane
         const int hl = quad * 32 + lane;             // thread index within this token half (0..127)
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
-        float T[128];
+        float T[kPFoldCols];
 #pragma unroll
-        for (int j = 0; j < 128; ++j) T[j] = 0.f;
+        for (int j = 0; j < kPFoldCols; ++j) T[j] = 0.f;
         int gc = 0;
         bool aborted = false;
         for (int tt = 0; tt < ntiles; ++tt) {
             const int tile = t_first + tt;
             const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
             const int n = nt * kPBM + row;
-            const int m0 = mt * kPBN + colh * 128;
+            const int m0 = mt * kPBN + colh * kPFoldCols;
             for (int g = 0; g < G; ++g, ++gc) {
                 const int slot = gc % kPMetaSlots, dbuf = gc & 1;
                 if (!aborted && !mbar_wait(&metafull[slot], (gc / kPMetaSlots) & 1, a.fault, 92)) aborted = true;
@@ -317,24 +337,25 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     // - s (z - c) xsum with c = 0, the X sums of this half's tokens from the ring
                     const float zr = (zv >= -128.f && zv <= 128.f) ? 0.f : zv;
                     const bool need_xs = __any_sync(0xFFFFFFFFu, zr != 0.f);
-                    const float* xs = reinterpret_cast<const float*>(ms + kPMetaSzBytes) + colh * 128;
+                    const float* xs = reinterpret_cast<const float*>(ms + kPMetaSzBytes) + colh * kPFoldCols;
                     tc_fence_after();
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint32_t d[16];
-                        tmem_ld16(tl + dbuf * kPBN + colh * 128 + cc * 16, d);
+                    for (int cc = 0; cc < kPFoldCols / kPLdCols; ++cc) {
+                        uint32_t d[kPLdCols];
+                        tmem_ldn(tl + dbuf * kPBN + colh * kPFoldCols + cc * kPLdCols, d);
                         tmem_wait_ld();
                         if (!need_xs) {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) T[cc * 16 + e] = fmaf(sv, __uint_as_float(d[e]), T[cc * 16 + e]);
+                            for (int e = 0; e < kPLdCols; ++e)
+                                T[cc * kPLdCols + e] = fmaf(sv, __uint_as_float(d[e]), T[cc * kPLdCols + e]);
                         } else {
 #pragma unroll
-                            for (int j4 = 0; j4 < 4; ++j4) {
-                                const float4 xv = *reinterpret_cast<const float4*>(xs + cc * 16 + 4 * j4);
+                            for (int j4 = 0; j4 < kPLdCols / 4; ++j4) {
+                                const float4 xv = *reinterpret_cast<const float4*>(xs + cc * kPLdCols + 4 * j4);
                                 const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                                 for (int e = 0; e < 4; ++e) {
-                                    const int j = cc * 16 + 4 * j4 + e;
+                                    const int j = cc * kPLdCols + 4 * j4 + e;
                                     T[j] = fmaf(sv, fmaf(-zr, xq[e], __uint_as_float(d[4 * j4 + e])), T[j]);
                                 }
                             }
@@ -348,16 +369,16 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     mbar_arrive(&metafree[slot]);
                 }
             }
-            // epilogue: this thread's row n, tokens m0 .. m0 + 127
+            // epilogue: this thread's row n, tokens m0 .. m0 + kPFoldCols - 1
             if (n < a.N) {
 #pragma unroll
-                for (int j = 0; j < 128; ++j) {
+                for (int j = 0; j < kPFoldCols; ++j) {
                     const int m = m0 + j;
                     if (m < a.M) a.Y[(int64_t)m * a.N + n] = float_to_bf16_bits(T[j]);
                 }
             }
 #pragma unroll
-            for (int j = 0; j < 128; ++j) T[j] = 0.f;
+            for (int j = 0; j < kPFoldCols; ++j) T[j] = 0.f;
         }
     }
     // teardown: all roles done; every MMA was waited on by the fold warps
