@@ -42,10 +42,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154175232 + dram__bytes_write.sum 3229440
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154158336 + dram__bytes_write.sum 3895808
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "5da302d446d84ba505dec75ea1a4bf8be443db1d55ab8fe547c84f976303a262",
-                                      "bytes": 157404672},
+                                      "sha256": "9554bfba3140cbce3c38f82262265fbb6f864eafdc2b675f881a481c837ca938",
+                                      "bytes": 158054144},
     # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 7776783872 + write 468124928
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
                                           "sha256": "1a3ec3cf5010e7434b861f412d54b3c9b7baec54e4659889d58d6f1695c8823b",
