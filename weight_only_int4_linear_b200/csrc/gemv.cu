@@ -538,15 +538,18 @@ constexpr int kCcStages = W4A16_CC_STAGES;
 constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
 constexpr int kCcMaxTokens = 2;                         // tokens per launch of the integer kernel
 constexpr int kCcXOff = kCcCodeBytes;                   // X planes of the group, per token (400 B each)
-constexpr int kCcStageBytes = 9 * 1024;                 // keeps stages 1024-aligned
+// codes + X planes of NT tokens, 512-aligned (the 64-byte swizzle's span)
+template <int NT>
+__host__ __device__ constexpr int cc_stage_bytes() { return (kCcCodeBytes + NT * kGroupXiBytes + 511) / 512 * 512; }
 constexpr int kCcMetaGroups = 8;                        // groups per metadata block
 constexpr int kXAhead = 6;                              // X warp: loads in flight, in units
 constexpr int kCcScBytes = kRowsPerCta * kCcMetaGroups * 2;  // 128 rows x 8 BF16 scales
 constexpr int kCcZeBytes = kRowsPerCta * kCcMetaGroups * 4;  // 128 rows x 8 int32 zero points
 constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;   // one slot, 6 KB
-constexpr int kCcMetaOff = kCcStages * kCcStageBytes;   // two slots after the ring
-constexpr size_t kCcSmem = (size_t)kCcMetaOff + 2 * kCcMetaBytes + 1024;
-static_assert(kCcXOff + kCcMaxTokens * kGroupXiBytes <= kCcStageBytes, "stage layout");
+template <int NT>
+__host__ __device__ constexpr int cc_meta_off() { return kCcStages * cc_stage_bytes<NT>(); }  // two slots after the ring
+template <int NT>
+__host__ __device__ constexpr size_t cc_smem() { return (size_t)cc_meta_off<NT>() + 2 * kCcMetaBytes + 512; }  // + alignment slack
 // A metadata slot is rewritten two blocks later.  Blocks are aligned to 8
 // groups inside a row tile (the kernel needs G % 8 == 0), so the block in
 // between has 8 units; with at most kCcStages units in flight, every unit of
@@ -626,8 +629,9 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
     __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages];
     __shared__ int s_last;
     const uint32_t raw = smem_u32(smem_raw);
-    unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    unsigned char* meta = ring + kCcMetaOff;
+    unsigned char* ring = smem_raw + ((512u - (raw & 511u)) & 511u);  // 512-aligned stages
+    constexpr int kStageBytes = cc_stage_bytes<NT>();
+    unsigned char* meta = ring + cc_meta_off<NT>();
 
     pdl_launch_dependents();  // the next call may start its weight loads as this grid's CTAs retire
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -658,7 +662,7 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
                 if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) break;
                 const bool new_block = i == 0 || (cur.g & (kCcMetaGroups - 1)) == 0;
                 if (new_block) ++mb;
-                unsigned char* st = ring + s * kCcStageBytes;
+                unsigned char* st = ring + s * kStageBytes;
                 mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (new_block ? kCcMetaBytes : 0));
                 tma_load_2d(st, &tq, cur.g * kWordsPerGroup, cur.tile * kRowsPerCta, &full[s]);
                 if (new_block) {
@@ -700,7 +704,7 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             const int s = i % kCcStages;
             if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
 #pragma unroll
-            for (int m = 0; m < NT; ++m) prep_group_x(v[m], ring + s * kCcStageBytes + kCcXOff + m * kGroupXiBytes, lane);
+            for (int m = 0; m < NT; ++m) prep_group_x(v[m], ring + s * kStageBytes + kCcXOff + m * kGroupXiBytes, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         }
@@ -791,7 +795,7 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             aborted = true;
             continue;
         }
-        const unsigned char* st = ring + s * kCcStageBytes;
+        const unsigned char* st = ring + s * kStageBytes;
         uint4 w[kCcRows];
 #pragma unroll
         for (int r = 0; r < kCcRows; ++r) w[r] = *reinterpret_cast<const uint4*>(st + code_off + 64 * kCcRowStep * r);
@@ -883,11 +887,11 @@ template <int NT>
 int occupancy_cc() {
     static int occ = 0;
     if (occ == 0) {
-        if (cudaFuncSetAttribute(decode_cc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCcSmem) !=
+        if (cudaFuncSetAttribute(decode_cc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cc_smem<NT>()) !=
             cudaSuccess)
             return 0;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel<NT>, kCcThreads, kCcSmem) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel<NT>, kCcThreads, cc_smem<NT>()) !=
                 cudaSuccess ||
             o < 1)
             return 0;
@@ -952,7 +956,7 @@ int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kCcThreads);
-    cfg.dynamicSmemBytes = kCcSmem;
+    cfg.dynamicSmemBytes = cc_smem<NT>();
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
