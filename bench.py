@@ -42,14 +42,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154158336 + dram__bytes_write.sum 3895808
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154180864 + dram__bytes_write.sum 3161856
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "9554bfba3140cbce3c38f82262265fbb6f864eafdc2b675f881a481c837ca938",
-                                      "bytes": 158054144},
-    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 7776783872 + write 468124928
+                                      "sha256": "5e152d4c9e9ee49728f656f5dd80c24d05c7cafb98d86172bb6159a6971d9599",
+                                      "bytes": 157342720},
+    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 8114076160 + write 467899392
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
-                                          "sha256": "1a3ec3cf5010e7434b861f412d54b3c9b7baec54e4659889d58d6f1695c8823b",
-                                          "bytes": 8244908800},
+                                          "sha256": "3b52599ece11483a5179dcf5ffeb0f59761808106138dd5d2dc8c73291b30e73",
+                                          "bytes": 8581975552},
 }
 
 
@@ -634,19 +634,21 @@ def run_reference(args):
 
 
 def run_profile(spec: str, repeats: int = 4):
-    """Run one layer of a workload a few times (for an ncu capture; no timing)."""
+    """Run one layer of a workload a few times, or (layer "all") the whole layer set, for an ncu
+    capture; no timing."""
     import torch
     import weight_only_int4_linear_b200 as w4
     w4.load()
     wl, name = spec.split(":")
     cases = {"decode": workloads.decode_5120(), "small": workloads.small_batch_8192(),
-             "prefill": workloads.prefill_8192()}[wl]
-    case = [c for c in cases if c.name == name][0]
+             "prefill": workloads.prefill_8192(ms=[4096])}[wl]
+    chosen = cases if name == "all" else [c for c in cases if c.name == name]
     stream = torch.cuda.Stream()
-    L = setup_layers([case], torch, w4, stream)[0]
+    layers = setup_layers(chosen, torch, w4, stream)
     with torch.cuda.stream(stream):
         for _ in range(repeats):
-            _linear_call(w4, L, w4.PATH_AUTO)
+            for L in layers:
+                _linear_call(w4, L, w4.PATH_AUTO)
     torch.cuda.synchronize()
     fault = w4.device_fault()
     print(json.dumps({"profiled": spec, "repeats": repeats, "fault": fault}))
@@ -697,7 +699,8 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture of this build")
     ap.add_argument("--profile", default=None,
-                    help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096): run it a few times, untimed")
+                    help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096, decode:all): run it a few "
+                         "times, untimed")
     ap.add_argument("--sweep", default=None,
                     help="all, or a comma list of single_gemv, decode, small, prefill: per-layer times, one line each")
     args = ap.parse_args()
