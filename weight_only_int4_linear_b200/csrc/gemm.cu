@@ -20,19 +20,31 @@
 // c != z.  The BF16 scale never enters a rounded operand; the only rounding
 // besides FP32 summation is the final BF16 rounding of Y.
 //
-// Tile: 128 weight rows (MMA M) x 256 tokens (MMA N, swap-AB so the per-row
-// scale is a per-thread constant in the fold).  K advances in stages of 64
-// (half a group).  MMA K order inside each 8-block of K is (0,4,1,5,2,6,3,7):
-// that is the order a lop3 pair extraction yields, and X is prepared in it.
+// Tile: 256 weight rows (MMA M) x 256 tokens (MMA N, swap-AB so the per-row
+// scale is a per-thread constant in the fold), computed by a cluster of two
+// CTAs with the pair MMA (tcgen05.mma.cta_group::2): each CTA dequantises its
+// own 128 weight rows into its shared memory, holds half of the tile's X rows
+// (the MMA exchanges the B halves between the pair), and receives its 128
+// rows of the FP32 accumulator in its own tensor memory.  Per CTA this halves
+// the X bytes that TMA writes and the MMA reads from shared memory against a
+// one-CTA 128 x 256 tile, which leaves room for six stages.  Rank 0 issues
+// the MMAs; both CTAs' dequantiser and fold warps arrive on rank 0's barriers
+// (mapa + remote mbarrier arrive), and its commits arrive on both CTAs'
+// barriers (multicast commit).  No TMA load is multicast.  K advances in
+// stages of 64 (half a group).  MMA K order inside each 8-block of K is
+// (0,4,1,5,2,6,3,7): that is the order a lop3 pair extraction yields, and X
+// is prepared in it.  (Built with W4A16_PF_CTAS=1 the same kernel runs one
+// CTA per 128 x 256 tile with cta_group::1.)
 //
-// Warps (512 threads with 8 fold warps):
+// Warps (512 threads per CTA with 8 fold warps):
 //   0-3   dequantise: thread = weight row; 8 packed words -> one 128-byte
 //         row of the 128B-swizzled K-major A tile
 //   4-11  fold + epilogue: warp w reads TMEM lane quadrant w % 4, token
-//         columns 128 * ((w - 4) / 4) ... + 127; totals live in registers
-//   12    TMA: X tile (256 x 64, 128-byte swizzle) and code tile (128 x 8
-//         words, 32-byte swizzle) per stage
-//   13    MMA issue: four tcgen05.mma (128 x 256 x 16) per stage
+//         columns 128 * ((w - 4) / 4) ... + 127; totals live in registers;
+//         T += s * D as packed FP32 FMAs (fma.rn.f32x2)
+//   12    TMA: this CTA's X half (128 x 64, 128-byte swizzle) and code tile
+//         (128 x 8 words, 32-byte swizzle) per stage
+//   13    MMA issue (rank 0): four tcgen05.mma (256 x 256 x 16) per stage
 //   14-15 idle
 // Accumulators: two 256-column TMEM buffers, one per group in flight, so the
 // fold of group g overlaps the MMAs of group g + 1.
@@ -44,22 +56,36 @@
 namespace w4a16 {
 namespace {
 
-constexpr int kPBM = 128;                      // weight rows per tile
+#ifndef W4A16_PF_CTAS
+#define W4A16_PF_CTAS 2
+#endif
+constexpr int kPCtas = W4A16_PF_CTAS;          // CTAs per MMA: 1 (cta_group::1) or a 2-CTA cluster (cta_group::2)
+static_assert(kPCtas == 1 || kPCtas == 2, "CTAs per MMA");
+constexpr int kPBM = 128;                      // weight rows per CTA (the MMA covers kPBM * kPCtas)
 constexpr int kPBN = 256;                      // tokens per tile
+constexpr int kPBNc = kPBN / kPCtas;           // tokens whose X tile this CTA holds (B split along N)
 constexpr int kPBK = 64;                       // K per stage
-constexpr int kPStages = 4;
-constexpr int kPXBytes = kPBN * kPBK * 2;      // 32 KB
+#ifndef W4A16_PF_STAGES
+#define W4A16_PF_STAGES (kPCtas == 2 ? 6 : 4)
+#endif
+constexpr int kPStages = W4A16_PF_STAGES;
+constexpr int kPXBytes = kPBNc * kPBK * 2;     // 32 KB (1 CTA) or 16 KB (2 CTAs)
 constexpr int kPABytes = kPBM * kPBK * 2;      // 16 KB
 constexpr int kPCodeBytes = kPBM * kPBK / 2;   // 4 KB
-constexpr int kPStageBytes = kPXBytes + kPABytes + kPCodeBytes;  // 52 KB (1024-aligned)
+constexpr int kPStageBytes = kPXBytes + kPABytes + kPCodeBytes;  // 52 KB or 36 KB (1024-aligned)
+static_assert(kPStageBytes % 1024 == 0, "stage alignment");
 // Per-group metadata ring, read by the fold warps: slot = group count % kPMetaSlots holds the 128 rows'
 // (scale, zero point) as FP32 pairs, written by the dequantisers, and the X sums of the tile's 256
 // tokens, copied by TMA.
-constexpr int kPMetaSlots = 8;
+#ifndef W4A16_PF_META_SLOTS
+#define W4A16_PF_META_SLOTS (kPCtas == 2 ? 4 : 8)
+#endif
+constexpr int kPMetaSlots = W4A16_PF_META_SLOTS;
 constexpr int kPMetaSzBytes = kPBM * 8;
 constexpr int kPMetaBytes = kPMetaSzBytes + kPBN * 4;  // 2 KB
 constexpr int kPMetaOff = kPStages * kPStageBytes;
 constexpr size_t kPSmem = (size_t)kPMetaOff + kPMetaSlots * kPMetaBytes + 1024;
+static_assert(kPSmem + 512 <= 232448, "shared memory per CTA");
 #ifndef W4A16_PF_FOLD_WARPS
 #define W4A16_PF_FOLD_WARPS 8
 #endif
@@ -78,7 +104,11 @@ static_assert(32 * (4 * kPRegsDequant + 4 * kPRegsIssue + kPFoldWarps * kPRegsFo
               "setmaxnreg split exceeds the registers the block is launched with");
 static_assert(kPFoldWarps == 8 || kPFoldWarps == 16, "fold warps");
 constexpr int kPLdCols = kPFoldWarps == 16 ? 8 : 16;    // TMEM columns per fold load
-constexpr uint32_t kPIdesc = idesc_bf16_f32(kPBM, kPBN);
+#ifndef W4A16_PF_LD_BATCH
+#define W4A16_PF_LD_BATCH 1
+#endif
+constexpr int kPLdBatch = W4A16_PF_LD_BATCH;            // fold loads in flight per wait
+constexpr uint32_t kPIdesc = idesc_bf16_f32(kPBM * kPCtas, kPBN);
 
 struct PrefillArgs {
     const uint16_t* scales;
@@ -87,8 +117,8 @@ struct PrefillArgs {
     uint16_t* Y;
     int* fault;
     int M, N, K, G, Mp;
-    int m_tiles, n_tiles;
-    int tiles_base, tiles_rem;  // CTA b runs tiles_base (+1 for the first tiles_rem CTAs) consecutive tiles
+    int m_tiles, n_tiles;       // tiles of 256 tokens x (128 x CTAs per MMA) weight rows
+    int tiles_base, tiles_rem;  // MMA unit (CTA or cluster) b runs tiles_base (+1 for the first tiles_rem) consecutive tiles
 };
 
 __device__ __forceinline__ uint32_t magic_pair(uint32_t w) {
@@ -143,6 +173,19 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __res
     }
 }
 
+// (t0, t1) = fma(s, d0, t0), fma(s, d1, t1) as one packed FP32 instruction (each lane a correctly
+// rounded fused multiply-add: the same bits as two fmaf calls).
+__device__ __forceinline__ void fma2_bcast(float& t0, float& t1, float s, uint32_t d0, uint32_t d1) {
+    asm("{\n\t.reg .b64 sa, da, ta;\n\t"
+        "mov.b64 sa, {%2, %2};\n\t"
+        "mov.b64 da, {%3, %4};\n\t"
+        "mov.b64 ta, {%0, %1};\n\t"
+        "fma.rn.f32x2 ta, sa, da, ta;\n\t"
+        "mov.b64 {%0, %1}, ta;\n\t}"
+        : "+f"(t0), "+f"(t1)
+        : "f"(s), "r"(d0), "r"(d1));
+}
+
 __device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[8]) { tmem_ld8(taddr, r); }
 __device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16(taddr, r); }
 
@@ -158,19 +201,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// Arrive on the MMA-issuing CTA's barrier (rank 0 of the cluster; this CTA with one CTA per MMA).
+__device__ __forceinline__ void arrive_issuer(uint64_t* bar) {
+    if constexpr (kPCtas == 2)
+        mbar_arrive_cluster(bar, 0);
+    else
+        mbar_arrive(bar);
+}
+
+
 __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tx,
                                                                const __grid_constant__ CUtensorMap tq,
                                                                const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
-    __shared__ __align__(8) uint64_t metafull[kPMetaSlots], metafree[kPMetaSlots];
+    __shared__ __align__(8) uint64_t full[kPStages], cfull[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
+    __shared__ __align__(8) uint64_t metafull[kPMetaSlots], metafree[kPMetaSlots], drained;
     __shared__ uint32_t s_tmem;
     const uint32_t raw = smem_u32(smem_raw);
+    // identical offsets in both CTAs of a cluster: the pair MMA reads the peer's tiles at this CTA's offsets
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
     unsigned char* meta = ring + kPMetaOff;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.x;
+    const uint32_t rank = kPCtas == 2 ? cluster_ctarank() : 0u;
+    const int b = blockIdx.x / kPCtas;  // MMA unit: this CTA or its cluster
     const int t_first = b * a.tiles_base + min(b, a.tiles_rem);
     const int ntiles = a.tiles_base + (b < a.tiles_rem ? 1 : 0);
     const int G = a.G;
@@ -178,26 +232,37 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&afull[s], 4);
+            mbar_init(&full[s], 1);   // X tile
+            mbar_init(&cfull[s], 1);  // codes tile (and, at a group's first stage, the group's X sums)
+            mbar_init(&afull[s], 4 * kPCtas);  // the dequantiser warps of every CTA of the MMA
             mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&mdone[i], 1);
-            mbar_init(&dfree[i], kPFoldWarps);
+            mbar_init(&dfree[i], kPFoldWarps * kPCtas);  // the fold warps of every CTA of the MMA
         }
         for (int i = 0; i < kPMetaSlots; ++i) {
             mbar_init(&metafull[i], 4);  // the dequantiser warps, after the TMA copy of the X sums landed
             mbar_init(&metafree[i], kPFoldWarps);  // the fold warps
         }
+        mbar_init(&drained, 1);
         fence_mbar_init();
     }
-    if (warp == 0) tmem_alloc(&s_tmem, 512);
-    __syncthreads();
+    __syncwarp();
+    if (warp == 0) {
+        if constexpr (kPCtas == 2)
+            tmem_alloc_pair(&s_tmem, 512);
+        else
+            tmem_alloc(&s_tmem, 512);
+    }
+    // barriers initialised and the TMEM base known in every CTA before any (remote) arrival
+    if constexpr (kPCtas == 2)
+        cluster_sync();
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     const int wg = warp >> 2;
-
     // register split (launch: 512 x 128 = 65536): 4 x 32 x (72 + 56 + 192 + 192) = 65536
     if (wg == 1 + kPFoldParts) {  // ------------------------------------------------ TMA + MMA
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPRegsIssue));
@@ -219,8 +284,9 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                         !mbar_wait(&metafree[slot], ((gi / kPMetaSlots) - 1) & 1, a.fault, 63))
                         goto done_tma;
                     mbar_arrive_expect_tx(&full[s], kPXBytes + kPCodeBytes + (first_half ? kPBN * 4 : 0));
-                    tma_load_2d(st, &tx, ks * kPBK, mt * kPBN, &full[s]);
-                    tma_load_2d(st + kPXBytes + kPABytes, &tq, ks * (kPBK / 8), nt * kPBM, &full[s]);
+                    tma_load_2d(st, &tx, ks * kPBK, mt * kPBN + (int)rank * kPBNc, &full[s]);
+                    tma_load_2d(st + kPXBytes + kPABytes, &tq, ks * (kPBK / 8), (nt * kPCtas + (int)rank) * kPBM,
+                                &full[s]);
                     if (first_half)
                         bulk_load(meta + slot * kPMetaBytes + kPMetaSzBytes,
                                   a.xsT + (int64_t)(ks >> 1) * a.Mp + mt * kPBN, kPBN * 4, &full[s]);
@@ -229,7 +295,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         done_tma:
             // copies in flight land before the CTA may exit
             for (int i = max(0, it - kPStages); i < it; ++i) mbar_wait(&full[i % kPStages], (i / kPStages) & 1, a.fault, 62);
-        } else if (warp == kPMmaWarp && lane == 0) {
+        } else if (warp == kPMmaWarp && lane == 0 && rank == 0) {
+            // afull[s] also stands for full[s] and cfull[s]: every dequantiser warp waited on its CTA's copies
             int it = 0, gc = 0;
             for (int tt = 0; tt < ntiles; ++tt) {
                 for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
@@ -237,34 +304,45 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     const int half = ks & 1;
                     const int dbuf = gc & 1;
                     if (half == 0 && gc >= 2 && !mbar_wait(&dfree[dbuf], ((gc >> 1) - 1) & 1, a.fault, 71)) goto done_mma;
-                    if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 72)) goto done_mma;
                     if (!mbar_wait(&afull[s], (it / kPStages) & 1, a.fault, 73)) goto done_mma;
                     tc_fence_after();
                     const uint32_t xaddr = smem_u32(ring + s * kPStageBytes);
                     const uint32_t aaddr = xaddr + kPXBytes;
 #pragma unroll
                     for (int kk = 0; kk < kPBK / 16; ++kk) {
-                        umma_ss(tmem + dbuf * kPBN, sw128_kmajor_desc(aaddr + kk * 32), sw128_kmajor_desc(xaddr + kk * 32),
-                                kPIdesc, half > 0 || kk > 0);
+                        const uint64_t ad = sw128_kmajor_desc(aaddr + kk * 32), bd = sw128_kmajor_desc(xaddr + kk * 32);
+                        if constexpr (kPCtas == 2)
+                            umma_ss_pair(tmem + dbuf * kPBN, ad, bd, kPIdesc, half > 0 || kk > 0);
+                        else
+                            umma_ss(tmem + dbuf * kPBN, ad, bd, kPIdesc, half > 0 || kk > 0);
                     }
-                    umma_commit(&empty[s]);
-                    if (half == 1) {
-                        umma_commit(&mdone[dbuf]);
-                        ++gc;
+                    if constexpr (kPCtas == 2) {
+                        umma_commit_pair(&empty[s], 0x3);
+                        if (half == 1) umma_commit_pair(&mdone[dbuf], 0x3);
+                    } else {
+                        umma_commit(&empty[s]);
+                        if (half == 1) umma_commit(&mdone[dbuf]);
                     }
+                    if (half == 1) ++gc;
                 }
             }
-        done_mma:;
+        done_mma:
+            // every MMA issued (also on an early exit) completes before the teardown
+            if constexpr (kPCtas == 2)
+                umma_commit_pair(&drained, 0x1);
+            else
+                umma_commit(&drained);
+            mbar_wait(&drained, 0, a.fault, 74);
         }
     } else if (wg == 0) {  // ------------------------------------ dequantisers
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPRegsDequant));
-        const int r = threadIdx.x;  // weight row within the tile
+        const int r = threadIdx.x;  // weight row within this CTA's 128
         // codes tile: 32 bytes per row, 32-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 2) & 1)
         const int csw = (r >> 2) & 1;
         int it = 0;
         for (int tt = 0; tt < ntiles; ++tt) {
             const int nt = (t_first + tt) / a.m_tiles;
-            const int n = nt * kPBM + r;
+            const int n = (nt * kPCtas + (int)rank) * kPBM + r;
             uint32_t zc2 = 0x43004300u;  // (128 + c) as a BF16 pair
             for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
                 const bool first_half = (ks & 1) == 0;
@@ -280,7 +358,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                 const int s = it % kPStages;
                 if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 81)) goto done_dq;
                 if (first_half) {
-                    // this row's scale and zero point for the fold warps; the stage's full barrier also
+                    // this row's scale and zero point for the fold warps; the stage's codes barrier also
                     // covered the TMA copy of the group's X sums into the same slot
                     const int gi = it >> 1, slot = gi % kPMetaSlots;
                     reinterpret_cast<float2*>(meta + slot * kPMetaBytes)[r] =
@@ -304,7 +382,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                 }
                 fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[s]);
+                if (lane == 0) arrive_issuer(&afull[s]);
             }
         }
     done_dq:;
@@ -312,8 +390,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPRegsFold));
         const int quad = warp & 3;
         const int colh = (warp - 4) >> 2;            // token column slice of the tile (kPFoldCols wide)
-        const int row = quad * 32 + lane;            // weight row within the tile = TMEM lane
-        const int hl = quad * 32 + lane;             // thread index within this token half (0..127)
+        const int row = quad * 32 + lane;            // weight row within this CTA's 128 = TMEM lane
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         float T[kPFoldCols];
 #pragma unroll
@@ -323,7 +400,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         for (int tt = 0; tt < ntiles; ++tt) {
             const int tile = t_first + tt;
             const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
-            const int n = nt * kPBM + row;
+            const int n = (nt * kPCtas + (int)rank) * kPBM + row;
             const int m0 = mt * kPBN + colh * kPFoldCols;
             for (int g = 0; g < G; ++g, ++gc) {
                 const int slot = gc % kPMetaSlots, dbuf = gc & 1;
@@ -340,23 +417,29 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     const float* xs = reinterpret_cast<const float*>(ms + kPMetaSzBytes) + colh * kPFoldCols;
                     tc_fence_after();
 #pragma unroll
-                    for (int cc = 0; cc < kPFoldCols / kPLdCols; ++cc) {
-                        uint32_t d[kPLdCols];
-                        tmem_ldn(tl + dbuf * kPBN + colh * kPFoldCols + cc * kPLdCols, d);
+                    for (int cc = 0; cc < kPFoldCols / (kPLdCols * kPLdBatch); ++cc) {
+                        uint32_t d[kPLdBatch][kPLdCols];
+#pragma unroll
+                        for (int bt = 0; bt < kPLdBatch; ++bt)
+                            tmem_ldn(tl + dbuf * kPBN + colh * kPFoldCols + (cc * kPLdBatch + bt) * kPLdCols, d[bt]);
                         tmem_wait_ld();
-                        if (!need_xs) {
 #pragma unroll
-                            for (int e = 0; e < kPLdCols; ++e)
-                                T[cc * kPLdCols + e] = fmaf(sv, __uint_as_float(d[e]), T[cc * kPLdCols + e]);
-                        } else {
+                        for (int bt = 0; bt < kPLdBatch; ++bt) {
+                            const int j0 = (cc * kPLdBatch + bt) * kPLdCols;
+                            if (!need_xs) {
 #pragma unroll
-                            for (int j4 = 0; j4 < kPLdCols / 4; ++j4) {
-                                const float4 xv = *reinterpret_cast<const float4*>(xs + cc * kPLdCols + 4 * j4);
-                                const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
+                                for (int e = 0; e < kPLdCols; e += 2)
+                                    fma2_bcast(T[j0 + e], T[j0 + e + 1], sv, d[bt][e], d[bt][e + 1]);
+                            } else {
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int j = cc * kPLdCols + 4 * j4 + e;
-                                    T[j] = fmaf(sv, fmaf(-zr, xq[e], __uint_as_float(d[4 * j4 + e])), T[j]);
+                                for (int j4 = 0; j4 < kPLdCols / 4; ++j4) {
+                                    const float4 xv = *reinterpret_cast<const float4*>(xs + j0 + 4 * j4);
+                                    const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const int j = j0 + 4 * j4 + e;
+                                        T[j] = fmaf(sv, fmaf(-zr, xq[e], __uint_as_float(d[bt][4 * j4 + e])), T[j]);
+                                    }
                                 }
                             }
                         }
@@ -365,7 +448,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                 }
                 __syncwarp();
                 if (lane == 0 && !aborted) {
-                    mbar_arrive(&dfree[dbuf]);
+                    arrive_issuer(&dfree[dbuf]);
                     mbar_arrive(&metafree[slot]);
                 }
             }
@@ -381,11 +464,18 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             for (int j = 0; j < kPFoldCols; ++j) T[j] = 0.f;
         }
     }
-    // teardown: all roles done; every MMA was waited on by the fold warps
-    __syncthreads();
+    // teardown: every role done, every MMA complete (drained), no arrival still bound for the peer
+    __syncwarp();
+    if constexpr (kPCtas == 2)
+        cluster_sync();
+    else
+        __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        if constexpr (kPCtas == 2)
+            tmem_dealloc_pair(tmem, 512);
+        else
+            tmem_dealloc(tmem, 512);
     }
 }
 
@@ -408,9 +498,9 @@ bool prefill_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtenso
         }
     PTmap& e = g_ptmaps[g_ptmap_next];
     bool ok;
-    if (kind == 0)  // prepared X: bf16 [M][K], box 64 x 256, 128-byte swizzle
+    if (kind == 0)  // prepared X: bf16 [M][K], box 64 x (this CTA's tokens), 128-byte swizzle
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
-                            (uint64_t)cols * 2, kPBK, kPBN, CU_TENSOR_MAP_SWIZZLE_128B);
+                            (uint64_t)cols * 2, kPBK, kPBNc, CU_TENSOR_MAP_SWIZZLE_128B);
     else  // packed weights: uint32 [N][K/8], box 8 words x 128 rows, 32-byte swizzle
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 4, kPBK / 8, kPBM, CU_TENSOR_MAP_SWIZZLE_32B);
@@ -425,6 +515,26 @@ bool prefill_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtenso
 }
 
 size_t align256p(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// MMA units of the prefill kernel that fit on the current device at once (cached per device).
+int prefill_resident_units(const cudaLaunchConfig_t& cfg) {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache[dev] > 0) return cache[dev];
+    int units = 0;
+    if constexpr (kPCtas == 1) {
+        units = num_sms_current();
+    } else {
+        cudaLaunchConfig_t q = cfg;
+        q.gridDim = dim3((unsigned)(kPCtas * num_sms_current()));
+        if (cudaOccupancyMaxActiveClusters(&units, prefill_kernel, &q) != cudaSuccess) return -1;
+    }
+    cache[dev] = units;
+    return units;
+}
 
 }  // namespace
 
@@ -472,23 +582,30 @@ int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qwei
     args.G = G;
     args.Mp = Mp;
     args.m_tiles = (int)ceil_div(M, kPBN);
-    args.n_tiles = (int)ceil_div(N, kPBM);
+    args.n_tiles = (int)ceil_div(N, kPBM * kPCtas);
     const int tiles = args.m_tiles * args.n_tiles;
-    int grid = num_sms_current();
-    if (grid > tiles) grid = tiles;
-    args.tiles_base = tiles / grid;
-    args.tiles_rem = tiles % grid;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kPThreads);
     cfg.dynamicSmemBytes = kPSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr1[1];
-    attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr1[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr1;
-    cfg.numAttrs = 1;
+    cudaLaunchAttribute attrs[2];
+    attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[0].val.programmaticStreamSerializationAllowed = 1;
+    attrs[1].id = cudaLaunchAttributeClusterDimension;
+    attrs[1].val.clusterDim.x = kPCtas;
+    attrs[1].val.clusterDim.y = 1;
+    attrs[1].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 2;
+    // persistent: one MMA unit (CTA or 2-CTA cluster) per resident slot, so that every unit runs
+    // in the first wave (a cluster needs two free SMs of one GPC, which not every SM count allows)
+    int mma_units = prefill_resident_units(cfg);
+    if (mma_units <= 0) return W4A16_ERR_CUDA;
+    if (mma_units > tiles) mma_units = tiles;
+    args.tiles_base = tiles / mma_units;
+    args.tiles_rem = tiles % mma_units;
+    cfg.gridDim = dim3((unsigned)(mma_units * kPCtas));
     return cudaLaunchKernelEx(&cfg, prefill_kernel, tx, tq, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
