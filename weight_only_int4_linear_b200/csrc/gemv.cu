@@ -2,22 +2,25 @@
 // (up to 32 tokens per launch).
 //
 // Only the packed codes (0.5 byte per weight) and the per-group scale and zero
-// point cross the memory bus: each code is turned into a BF16 operand on chip
-// and consumed at once ("Quantization I: int8, int4, the basics", Concept:
-// dequantise tile by tile inside the multiply; "Weight-Only Quantization and
-// Mixed Precision", section 7: one read of the packed INT4 weights, unpack
-// with bit operations, asynchronous copies overlapping the math, nothing
-// written back).
+// point cross the memory bus; each code is consumed on chip straight from its
+// packed word ("Quantization I: int8, int4, the basics", Concept: dequantise
+// tile by tile inside the multiply; "Weight-Only Quantization and Mixed
+// Precision", section 7: one read of the packed INT4 weights, unpack with bit
+// operations, asynchronous copies overlapping the math, nothing written back).
 //
-// Arithmetic per group g of 128 weights of row n and token m:
-//   sum_k (q - z) s x  =  s * ( sum_k (128 + q) x  -  (128 + z) * sum_k x ).
-// (128 + q) is exact in BF16 and comes out of a packed word with one lop3 per
-// two codes (0x4300 | q encodes 128 + q).  The inner sums run on the 5th-gen
-// tensor cores (tcgen05.mma, BF16 in, FP32 accumulate in tensor memory); the
-// fold s * (P - (128 + z) * xsum) is applied in FP32 once per group, with
-// xsum = sum_k x prepared alongside X.  The BF16 scale is never folded into a
-// rounded operand, so the only rounding besides FP32 summation is the final
-// BF16 rounding of Y.
+// Arithmetic per group g of 128 weights of row n and token m, exact in integers:
+//   sum_k (q - z) s x  =  s 2^(-k) ( sum_k q x_int  -  z sum_k x_int ),
+// x_int = x 2^k an integer (k from the exponent of the group's largest |x|).
+// The codes q stay unsigned bytes (w & 0x0F0F0F0F, (w >> 4) & 0x0F0F0F0F); x_int
+// is split into three byte planes, so sum_k q x_int is three exact int32 dot
+// products, combined and scaled in FP32 once per group.  The BF16 scale is never
+// folded into a rounded operand.  Three kernels:
+//   * M <= 2: decode_cc_kernel, the dot products as mma.sync m16n8k32 (codes u8 x
+//     balanced X digits s8, or dp4a on unsigned/signed byte planes in the
+//     W4A16_CC_MMA=0 build) in the warps' registers, X prepared inside the kernel;
+//   * 3 <= M <= 32 per launch: decode_tc_kernel, tcgen05.mma kind::i8 with the
+//     codes in tensor memory and the digit planes of all tokens as B;
+//   * prep_x8_kernel: the digit planes for the tensor-core kernel.
 //
 // Work decomposition: a unit is 128 weight rows x one group (8 KB of codes).
 // Units are numbered row tile by row tile and dealt out to a persistent grid
@@ -611,6 +614,72 @@ __device__ __forceinline__ void prep_group_x(const uint2 v, unsigned char* dst, 
     }
 }
 
+#ifndef W4A16_CC_MMA
+#define W4A16_CC_MMA 1
+#endif
+// 1: the integer dot products run as mma.sync m16n8k32 (codes u8 x balanced X digits s8, int32
+// accumulate) on the warp's registers; 0: as dp4a on X byte planes.
+constexpr bool kCcMma = W4A16_CC_MMA != 0;
+
+// mma.sync m16n8k32, A 16 x 32 unsigned bytes (row-major fragments), B 32 x 8 signed bytes
+// (column-major fragments), D (+)= int32: exact integer dot products.
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One warp writes token m's balanced base-256 digits of group g (its lanes' values v from
+// load_group_x) as the B operand rows of the MMA layout: row n = p NT + m (digit plane p) holds
+// 128 bytes, word w's codes 0,2,4,6 at 8w and codes 1,3,5,7 at 8w + 4, the order in which
+// w & 0x0F0F0F0F and (w >> 4) & 0x0F0F0F0F hold the codes.  x_int = x 2^(21 - E), E the exponent
+// of the group's largest |x| (exact for every x within 2^14 of it, smaller values rounded at
+// 2^(E - 21)), = 65536 d2 + 256 d1 + d0 with every digit in [-128, 127].  After the 3 NT rows:
+// per token (sum_k x_int as FP32, 2^(E - 21)).
+template <int NT>
+__device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst, int lane, int m) {
+    const uint32_t bits[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
+    uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
+    amax = __reduce_max_sync(0xFFFFFFFFu, amax);
+    const int ef = (int)(amax >> 7);
+    const int E = ef == 0 ? -127 : ef - 127;  // every |x| of the group is below 2^(E + 1)
+    const int kx = 21 - E;                    // in [-106, 148]
+    const int k1 = min(kx, 127);
+    const float s1 = pow2f(k1), s2 = pow2f(kx - k1);  // exact scalings, |x * 2^kx| < 2^22
+    int xi[4];
+    uint32_t dg[3] = {0u, 0u, 0u};  // this lane's digit bytes per plane, as (i0, i2, i1, i3)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        xi[i] = __float2int_rn(__uint_as_float(bits[i] << 16) * s1 * s2);
+        const int d0 = ((xi[i] + 128) & 255) - 128;
+        const int t = (xi[i] - d0) >> 8;
+        const int d1 = ((t + 128) & 255) - 128;
+        const int d2 = (t - d1) >> 8;
+        const int pos = (i & 1) ? 16 + 8 * (i >> 1) : 8 * (i >> 1);  // i0 -> 0, i2 -> 8, i1 -> 16, i3 -> 24
+        dg[0] |= (uint32_t)(d0 & 255) << pos;
+        dg[1] |= (uint32_t)(d1 & 255) << pos;
+        dg[2] |= (uint32_t)(d2 & 255) << pos;
+    }
+    // lane (w, h) holds codes 4h .. 4h + 3 of word w; h = 0 assembles the even-code register
+    // (its codes 0, 2, the partner's 4, 6), h = 1 the odd one (the partner's 1, 3, its own 5, 7)
+    const int h = lane & 1, w = lane >> 1;
+#pragma unroll
+    for (int p = 0; p < 3; ++p) {
+        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, dg[p], 1);
+        const uint32_t lo = h ? other : dg[p], hi = h ? dg[p] : other;
+        const uint32_t out = h ? __byte_perm(lo, hi, 0x7632) : __byte_perm(lo, hi, 0x5410);
+        *reinterpret_cast<uint32_t*>(dst + (p * NT + m) * 128 + 8 * w + 4 * h) = out;
+    }
+    const int sum = __reduce_add_sync(0xFFFFFFFFu, (xi[0] + xi[1]) + (xi[2] + xi[3]));  // |sum| < 2^29
+    if (lane == 0) {
+        float* ext = reinterpret_cast<float*>(dst + 3 * NT * 128);
+        ext[2 * m] = (float)sum;
+        ext[2 * m + 1] = pow2f(E - 21);
+    }
+}
+
 // All lanes wait; the warp gives up together if any lane's wait ran out.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, int parity, int* fault, int site) {
     const bool ok = mbar_wait(bar, parity, fault, site);
@@ -704,7 +773,12 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             const int s = i % kCcStages;
             if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
 #pragma unroll
-            for (int m = 0; m < NT; ++m) prep_group_x(v[m], ring + s * kStageBytes + kCcXOff + m * kGroupXiBytes, lane);
+            for (int m = 0; m < NT; ++m) {
+                if constexpr (kCcMma)
+                    prep_group_x8<NT>(v[m], ring + s * kStageBytes + kCcXOff, lane, m);
+                else
+                    prep_group_x(v[m], ring + s * kStageBytes + kCcXOff + m * kGroupXiBytes, lane);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         }
@@ -713,6 +787,148 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
 
     // ---------------------------------------------------- compute warps 0-3
     const int t = threadIdx.x;
+    if constexpr (kCcMma) {
+        // Warp w takes rows 32 w .. 32 w + 31 as two 16-row MMA blocks.  Lane (g8, tig) = (lane / 4,
+        // lane % 4) holds, per block, rows g8 and g8 + 8 of its A fragments and words 4 tig .. 4 tig + 3
+        // of each (one 16-byte chunk of the codes tile); MMA j takes word 4 tig + j of every lane, so
+        // its K = 32 codes are words j, 4 + j, 8 + j, 12 + j, and the lane's B fragments are the same
+        // words of digit plane n = g8.  After a unit, D column n = p NT + m of a row is
+        // sum_k q_k d_p(x_k) of token m; lane tig = m gathers its three planes and folds the row.
+        const int g8 = lane >> 2, tig = lane & 3;
+        const int mt = tig < NT ? tig : NT - 1;  // the token this lane folds (lanes tig < NT)
+        const bool owner = tig < NT && tig < a.M;
+        auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        int cur_tile = -1;
+        bool aborted = false;
+
+        auto flush = [&](int tile) {
+            const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
+            const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
+            if (first == last) {
+                if (owner) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int n = tile * kRowsPerCta + rrow(k);
+                        if (n < N) a.Y[(int64_t)mt * N + n] = float_to_bf16_bits(y[k]);
+                    }
+                }
+            } else {
+                const int slot = b - first, nseg = last - first + 1;
+                float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * a.M * kRowsPerCta;
+                if (owner) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) part[mt * kRowsPerCta + rrow(k)] = y[k];
+                }
+                named_barrier_sync(1, kCcWarps * 32);
+                if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
+                named_barrier_sync(1, kCcWarps * 32);
+                if (s_last) {
+                    const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
+                    const float* pb = a.partial + (int64_t)tile * a.max_slots * a.M * kRowsPerCta;
+#pragma unroll
+                    for (int m = 0; m < NT; ++m) {
+                        if (m >= a.M) break;
+                        for (int rl = t; rl < rows; rl += kCcWarps * 32) {
+                            const float sum = sum_slots(pb + (int64_t)m * kRowsPerCta + rl, (int64_t)a.M * kRowsPerCta, nseg);
+                            a.Y[(int64_t)m * N + tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
+                        }
+                    }
+                    if (t == 0) a.counters[tile] = 0;
+                }
+                named_barrier_sync(1, kCcWarps * 32);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) y[k] = 0.f;
+        };
+
+        UnitCursor uc(u_first, G);
+        int mb = -1;
+        for (int i = 0; i < nunits; ++i, uc.next(G)) {
+            const int tile = uc.tile, g = uc.g;
+            if (i == 0 || (g & (kCcMetaGroups - 1)) == 0) ++mb;
+            if (tile != cur_tile) {
+                if (cur_tile >= 0) flush(cur_tile);
+                cur_tile = tile;
+            }
+            if (aborted) continue;
+            const int s = i % kCcStages;
+            if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 53)) {
+                aborted = true;
+                continue;
+            }
+            const unsigned char* st = ring + s * kStageBytes;
+            // codes: chunk tig of each row, 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3))
+            uint4 cw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = rrow(k);
+                cw[k] = *reinterpret_cast<const uint4*>(st + r * 64 + 16 * (tig ^ ((r >> 1) & 3)));
+            }
+            uint32_t bx[8];
+            if (g8 < 3 * NT) {
+                const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + g8 * 128 + tig * 32);
+                const uint4 u0 = xp[0], u1 = xp[1];
+                bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
+                bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) bx[j] = 0u;
+            }
+            const float* ext = reinterpret_cast<const float*>(st + kCcXOff + 3 * NT * 128);
+            const float xsum = ext[2 * mt], xscale = ext[2 * mt + 1];
+            // this block's metadata (loaded with its first unit, which this warp has already waited for);
+            // rows past N were zero-filled by TMA: s = 0 folds them away
+            const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
+            float sv[4], zv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = rrow(k);
+                sv[k] = bf16_bits_to_float(
+                    *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
+                zv[k] = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
+                                                                 4 * (g & (kCcMetaGroups - 1)));
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb) {
+                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
+                int d[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_u8s8(d, w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
+                             (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
+                // lane tig holds columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    int P0, P1, P2;
+                    if constexpr (NT == 1) {  // planes 0, 1 at lane tig 0, plane 2 at lane tig 1
+                        P0 = d[2 * h];
+                        P1 = d[2 * h + 1];
+                        P2 = __shfl_sync(0xFFFFFFFFu, d[2 * h], lane | 1);
+                    } else {  // column p NT + m: token 0 planes at (0,0), (1,0), (2,0); token 1 at (0,1), (1,1), (2,1)
+                        const int own = tig == 0 ? d[2 * h] : d[2 * h + 1];
+                        const int x = __shfl_xor_sync(0xFFFFFFFFu, tig == 0 ? d[2 * h + 1] : d[2 * h], 1);
+                        const int t0 = __shfl_sync(0xFFFFFFFFu, d[2 * h], (lane & ~3) | 2);
+                        const int t1 = __shfl_sync(0xFFFFFFFFu, d[2 * h + 1], (lane & ~3) | 2);
+                        P0 = tig == 0 ? own : x;
+                        P1 = tig == 0 ? x : own;
+                        P2 = tig == 0 ? t0 : t1;
+                    }
+                    // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26),
+                    // the rest FP32 with one rounding per step
+                    const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+                    const int k = 2 * rb + h;
+                    y[k] = fmaf(sv[k] * xscale, fmaf(-zv[k], xsum, qx), y[k]);
+                }
+            }
+        }
+        if (cur_tile >= 0) flush(cur_tile);
+        return;
+    }
     const int c = t & 3;   // words 4c..4c+3 of the group
     const int rg = t >> 2; // rows rg + kCcRowStep i
     // the 64-byte swizzle of the codes tile: logical chunk c of row r sits at chunk c ^ ((r >> 1) & 3);

@@ -127,15 +127,20 @@ __device__ __forceinline__ int arrive_acq_rel_gpu(int* counter) {
 }
 
 // Sum of nseg partial values p[0], p[stride], ... in a fixed order, with up
-// to four L2 loads in flight.
+// to sixteen L2 loads in flight (one round trip per sixteen partials).
 __device__ __forceinline__ float sum_slots(const float* p, int64_t stride, int nseg) {
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s0 = 0; s0 < nseg; s0 += 4) {
+    float acc = 0.f;
+    for (int s0 = 0; s0 < nseg; s0 += 16) {
+        float v[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (s0 + j < nseg) s4[j] += __ldcg(p + (s0 + j) * stride);
+        for (int j = 0; j < 16; ++j) v[j] = s0 + j < nseg ? __ldcg(p + (s0 + j) * stride) : 0.f;
+#pragma unroll
+        for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+            for (int j = 0; j < w; ++j) v[j] += v[j + w];
+        acc += v[0];
     }
-    return (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    return acc;
 }
 
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
