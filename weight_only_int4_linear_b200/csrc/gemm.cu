@@ -118,7 +118,7 @@ struct PrefillArgs {
     int* fault;
     int M, N, K, G, Mp;
     int m_tiles, n_tiles;       // tiles of 256 tokens x (128 x CTAs per MMA) weight rows
-    int tiles_base, tiles_rem;  // MMA unit (CTA or cluster) b runs tiles_base (+1 for the first tiles_rem) consecutive tiles
+    int tiles, units;           // MMA unit (CTA or cluster) b runs tiles b, b + units, b + 2 units, ...
 };
 
 __device__ __forceinline__ uint32_t magic_pair(uint32_t w) {
@@ -201,6 +201,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// Tile t -> (weight row tile nt, token tile mt).  Groups of kPRaster token tiles are walked with
+// the token tile fastest, so the tiles in flight at once (consecutive t, one per MMA unit) share a
+// few X tiles and a few weight row tiles, and both stay in L2 between their uses.
+#ifndef W4A16_PF_RASTER
+#define W4A16_PF_RASTER 4
+#endif
+constexpr int kPRaster = W4A16_PF_RASTER;
+__device__ __forceinline__ void tile_coords(int t, const PrefillArgs& a, int& nt, int& mt) {
+    const int per_group = kPRaster * a.n_tiles;
+    const int grp = t / per_group, r = t - grp * per_group;
+    const int gm = min(kPRaster, a.m_tiles - grp * kPRaster);  // token tiles in this group (the last may be short)
+    nt = r / gm;
+    mt = grp * kPRaster + (r - nt * gm);
+}
+
 // Arrive on the MMA-issuing CTA's barrier (rank 0 of the cluster; this CTA with one CTA per MMA).
 __device__ __forceinline__ void arrive_issuer(uint64_t* bar) {
     if constexpr (kPCtas == 2)
@@ -225,8 +240,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = kPCtas == 2 ? cluster_ctarank() : 0u;
     const int b = blockIdx.x / kPCtas;  // MMA unit: this CTA or its cluster
-    const int t_first = b * a.tiles_base + min(b, a.tiles_rem);
-    const int ntiles = a.tiles_base + (b < a.tiles_rem ? 1 : 0);
+    const int ntiles = b < a.tiles ? (a.tiles - 1 - b) / a.units + 1 : 0;  // tiles b, b + units, ...
     const int G = a.G;
     const int stages_per_tile = 2 * G;
 
@@ -272,8 +286,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             pdl_wait_primary();  // X comes from the preparation kernel
             int it = 0;
             for (int tt = 0; tt < ntiles; ++tt) {
-                const int tile = t_first + tt;
-                const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+                int nt, mt;
+                tile_coords(b + tt * a.units, a, nt, mt);
                 for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
                     const int s = it % kPStages;
                     if (it >= kPStages && !mbar_wait(&empty[s], ((it / kPStages) - 1) & 1, a.fault, 61)) goto done_tma;
@@ -341,7 +355,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         const int csw = (r >> 2) & 1;
         int it = 0;
         for (int tt = 0; tt < ntiles; ++tt) {
-            const int nt = (t_first + tt) / a.m_tiles;
+            int nt, mt;
+            tile_coords(b + tt * a.units, a, nt, mt);
             const int n = (nt * kPCtas + (int)rank) * kPBM + r;
             uint32_t zc2 = 0x43004300u;  // (128 + c) as a BF16 pair
             for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
@@ -398,8 +413,8 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         int gc = 0;
         bool aborted = false;
         for (int tt = 0; tt < ntiles; ++tt) {
-            const int tile = t_first + tt;
-            const int nt = tile / a.m_tiles, mt = tile - nt * a.m_tiles;
+            int nt, mt;
+            tile_coords(b + tt * a.units, a, nt, mt);
             const int n = (nt * kPCtas + (int)rank) * kPBM + row;
             const int m0 = mt * kPBN + colh * kPFoldCols;
             for (int g = 0; g < G; ++g, ++gc) {
@@ -603,8 +618,8 @@ int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qwei
     int mma_units = prefill_resident_units(cfg);
     if (mma_units <= 0) return W4A16_ERR_CUDA;
     if (mma_units > tiles) mma_units = tiles;
-    args.tiles_base = tiles / mma_units;
-    args.tiles_rem = tiles % mma_units;
+    args.tiles = tiles;
+    args.units = mma_units;
     cfg.gridDim = dim3((unsigned)(mma_units * kPCtas));
     return cudaLaunchKernelEx(&cfg, prefill_kernel, tx, tq, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
