@@ -74,17 +74,7 @@ constexpr int kPABytes = kPBM * kPBK * 2;      // 16 KB
 constexpr int kPCodeBytes = kPBM * kPBK / 2;   // 4 KB
 constexpr int kPStageBytes = kPXBytes + kPABytes + kPCodeBytes;  // 52 KB or 36 KB (1024-aligned)
 static_assert(kPStageBytes % 1024 == 0, "stage alignment");
-// Per-group metadata ring, read by the fold warps: slot = group count % kPMetaSlots holds the 128 rows'
-// (scale, zero point) as FP32 pairs, written by the dequantisers, and the X sums of the tile's 256
-// tokens, copied by TMA.
-#ifndef W4A16_PF_META_SLOTS
-#define W4A16_PF_META_SLOTS (kPCtas == 2 ? 4 : 8)
-#endif
-constexpr int kPMetaSlots = W4A16_PF_META_SLOTS;
-constexpr int kPMetaSzBytes = kPBM * 8;
-constexpr int kPMetaBytes = kPMetaSzBytes + kPBN * 4;  // 2 KB
-constexpr int kPMetaOff = kPStages * kPStageBytes;
-constexpr size_t kPSmem = (size_t)kPMetaOff + kPMetaSlots * kPMetaBytes + 1024;
+constexpr size_t kPSmem = (size_t)kPStages * kPStageBytes + 1024;  // + alignment slack
 static_assert(kPSmem + 512 <= 232448, "shared memory per CTA");
 #ifndef W4A16_PF_FOLD_WARPS
 #define W4A16_PF_FOLD_WARPS 8
@@ -230,12 +220,11 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                                                                const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kPStages], cfull[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
-    __shared__ __align__(8) uint64_t metafull[kPMetaSlots], metafree[kPMetaSlots], drained;
+    __shared__ __align__(8) uint64_t drained;
     __shared__ uint32_t s_tmem;
     const uint32_t raw = smem_u32(smem_raw);
     // identical offsets in both CTAs of a cluster: the pair MMA reads the peer's tiles at this CTA's offsets
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
-    unsigned char* meta = ring + kPMetaOff;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = kPCtas == 2 ? cluster_ctarank() : 0u;
@@ -254,10 +243,6 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         for (int i = 0; i < 2; ++i) {
             mbar_init(&mdone[i], 1);
             mbar_init(&dfree[i], kPFoldWarps * kPCtas);  // the fold warps of every CTA of the MMA
-        }
-        for (int i = 0; i < kPMetaSlots; ++i) {
-            mbar_init(&metafull[i], 4);  // the dequantiser warps, after the TMA copy of the X sums landed
-            mbar_init(&metafree[i], kPFoldWarps);  // the fold warps
         }
         mbar_init(&drained, 1);
         fence_mbar_init();
@@ -292,18 +277,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     const int s = it % kPStages;
                     if (it >= kPStages && !mbar_wait(&empty[s], ((it / kPStages) - 1) & 1, a.fault, 61)) goto done_tma;
                     unsigned char* st = ring + s * kPStageBytes;
-                    const bool first_half = (ks & 1) == 0;  // a group starts: its X sums go to the metadata ring
-                    const int gi = it >> 1, slot = gi % kPMetaSlots;
-                    if (first_half && gi >= kPMetaSlots &&
-                        !mbar_wait(&metafree[slot], ((gi / kPMetaSlots) - 1) & 1, a.fault, 63))
-                        goto done_tma;
-                    mbar_arrive_expect_tx(&full[s], kPXBytes + kPCodeBytes + (first_half ? kPBN * 4 : 0));
+                    mbar_arrive_expect_tx(&full[s], kPXBytes + kPCodeBytes);
                     tma_load_2d(st, &tx, ks * kPBK, mt * kPBN + (int)rank * kPBNc, &full[s]);
                     tma_load_2d(st + kPXBytes + kPABytes, &tq, ks * (kPBK / 8), (nt * kPCtas + (int)rank) * kPBM,
                                 &full[s]);
-                    if (first_half)
-                        bulk_load(meta + slot * kPMetaBytes + kPMetaSzBytes,
-                                  a.xsT + (int64_t)(ks >> 1) * a.Mp + mt * kPBN, kPBN * 4, &full[s]);
                 }
             }
         done_tma:
@@ -361,26 +338,14 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             uint32_t zc2 = 0x43004300u;  // (128 + c) as a BF16 pair
             for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
                 const bool first_half = (ks & 1) == 0;
-                int z = 0;
-                uint32_t sraw = 0;
                 if (first_half) {
-                    z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + (ks >> 1)) : 0;
-                    sraw = n < a.N ? __ldg(a.scales + (int64_t)n * G + (ks >> 1)) : 0;
+                    const int z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + (ks >> 1)) : 0;
                     const int c = (z >= -128 && z <= 128) ? z : 0;
                     const uint32_t cb = __float_as_uint(128.f + (float)c) >> 16;  // exact: |128 + c| <= 256
                     zc2 = cb | (cb << 16);
                 }
                 const int s = it % kPStages;
                 if (!mbar_wait(&full[s], (it / kPStages) & 1, a.fault, 81)) goto done_dq;
-                if (first_half) {
-                    // this row's scale and zero point for the fold warps; the stage's codes barrier also
-                    // covered the TMA copy of the group's X sums into the same slot
-                    const int gi = it >> 1, slot = gi % kPMetaSlots;
-                    reinterpret_cast<float2*>(meta + slot * kPMetaBytes)[r] =
-                        make_float2(bf16_bits_to_float((uint16_t)sraw), (float)z);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&metafull[slot]);
-                }
                 unsigned char* st = ring + s * kPStageBytes;
                 const unsigned char* codes = st + kPXBytes + kPABytes + r * 32;
                 const uint4 c0 = *reinterpret_cast<const uint4*>(codes + 16 * csw);
@@ -412,24 +377,40 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
         for (int j = 0; j < kPFoldCols; ++j) T[j] = 0.f;
         int gc = 0;
         bool aborted = false;
+        // this row's scale and zero point, loaded one group ahead of their use (rows past N: scale 0)
+        auto row_of = [&](int tt2) {
+            int nt2, mt2;
+            tile_coords(b + tt2 * a.units, a, nt2, mt2);
+            return (nt2 * kPCtas + (int)rank) * kPBM + row;
+        };
+        uint32_t s_nx = 0;
+        int z_nx = 0;
+        if (ntiles > 0) {
+            const int n0 = row_of(0);
+            s_nx = n0 < a.N ? __ldg(a.scales + (int64_t)n0 * G) : 0u;
+            z_nx = n0 < a.N ? __ldg(a.zeros + (int64_t)n0 * G) : 0;
+        }
         for (int tt = 0; tt < ntiles; ++tt) {
             int nt, mt;
             tile_coords(b + tt * a.units, a, nt, mt);
             const int n = (nt * kPCtas + (int)rank) * kPBM + row;
+            const int n_next = tt + 1 < ntiles ? row_of(tt + 1) : a.N;  // the next tile's row (a.N: none)
             const int m0 = mt * kPBN + colh * kPFoldCols;
             for (int g = 0; g < G; ++g, ++gc) {
-                const int slot = gc % kPMetaSlots, dbuf = gc & 1;
-                if (!aborted && !mbar_wait(&metafull[slot], (gc / kPMetaSlots) & 1, a.fault, 92)) aborted = true;
+                const int dbuf = gc & 1;
+                const uint32_t s_cur = s_nx;
+                const int z_cur = z_nx;
+                const int nn = g + 1 < G ? n : n_next, gn = g + 1 < G ? g + 1 : 0;
+                s_nx = nn < a.N ? __ldg(a.scales + (int64_t)nn * G + gn) : 0u;
+                z_nx = nn < a.N ? __ldg(a.zeros + (int64_t)nn * G + gn) : 0;
                 if (!aborted && !mbar_wait(&mdone[dbuf], (gc >> 1) & 1, a.fault, 91)) aborted = true;
                 if (!aborted) {
-                    const unsigned char* ms = meta + slot * kPMetaBytes;
-                    const float2 sz = reinterpret_cast<const float2*>(ms)[row];  // rows past N: scale 0
-                    const float sv = sz.x, zv = sz.y;
+                    const float sv = bf16_bits_to_float((uint16_t)s_cur), zv = (float)z_cur;
                     // rows whose zero point was not subtracted by the dequantiser (|z| > 128) fold
-                    // - s (z - c) xsum with c = 0, the X sums of this half's tokens from the ring
-                    const float zr = (zv >= -128.f && zv <= 128.f) ? 0.f : zv;
+                    // - s (z - c) xsum with c = 0, the X sums of this thread's tokens read from global memory
+                    const float zr = (z_cur >= -128 && z_cur <= 128) ? 0.f : zv;
                     const bool need_xs = __any_sync(0xFFFFFFFFu, zr != 0.f);
-                    const float* xs = reinterpret_cast<const float*>(ms + kPMetaSzBytes) + colh * kPFoldCols;
+                    const float* xs = a.xsT + (int64_t)g * a.Mp + m0;
                     tc_fence_after();
 #pragma unroll
                     for (int cc = 0; cc < kPFoldCols / (kPLdCols * kPLdBatch); ++cc) {
@@ -448,7 +429,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                             } else {
 #pragma unroll
                                 for (int j4 = 0; j4 < kPLdCols / 4; ++j4) {
-                                    const float4 xv = *reinterpret_cast<const float4*>(xs + j0 + 4 * j4);
+                                    const float4 xv = __ldg(reinterpret_cast<const float4*>(xs + j0 + 4 * j4));
                                     const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                                     for (int e = 0; e < 4; ++e) {
@@ -462,10 +443,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     tc_fence_before();
                 }
                 __syncwarp();
-                if (lane == 0 && !aborted) {
-                    arrive_issuer(&dfree[dbuf]);
-                    mbar_arrive(&metafree[slot]);
-                }
+                if (lane == 0 && !aborted) arrive_issuer(&dfree[dbuf]);
             }
             // epilogue: this thread's row n, tokens m0 .. m0 + kPFoldCols - 1
             if (n < a.N) {
