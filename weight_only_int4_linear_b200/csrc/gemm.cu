@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                                                                const __grid_constant__ CUtensorMap tq,
                                                                const PrefillArgs a) {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full[kPStages], cfull[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
+    __shared__ __align__(8) uint64_t full[kPStages], afull[kPStages], empty[kPStages], mdone[2], dfree[2];
     __shared__ __align__(8) uint64_t drained;
     __shared__ uint32_t s_tmem;
     const uint32_t raw = smem_u32(smem_raw);
@@ -235,8 +235,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; ++s) {
-            mbar_init(&full[s], 1);   // X tile
-            mbar_init(&cfull[s], 1);  // codes tile (and, at a group's first stage, the group's X sums)
+            mbar_init(&full[s], 1);  // TMA: X and codes tiles
             mbar_init(&afull[s], 4 * kPCtas);  // the dequantiser warps of every CTA of the MMA
             mbar_init(&empty[s], 1);
         }
@@ -287,7 +286,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             // copies in flight land before the CTA may exit
             for (int i = max(0, it - kPStages); i < it; ++i) mbar_wait(&full[i % kPStages], (i / kPStages) & 1, a.fault, 62);
         } else if (warp == kPMmaWarp && lane == 0 && rank == 0) {
-            // afull[s] also stands for full[s] and cfull[s]: every dequantiser warp waited on its CTA's copies
+            // afull[s] also stands for full[s]: every dequantiser warp waited on its CTA's copies first
             int it = 0, gc = 0;
             for (int tt = 0; tt < ntiles; ++tt) {
                 for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
