@@ -42,14 +42,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154180864 + dram__bytes_write.sum 3161856
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154371840 + dram__bytes_write.sum 3226368
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "5e152d4c9e9ee49728f656f5dd80c24d05c7cafb98d86172bb6159a6971d9599",
-                                      "bytes": 157342720},
-    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 8114076160 + write 467899392
+                                      "sha256": "18a05e78ee2f1998d923ba976ebb0fe04afcec9624fe0565177c5f8f1f036fdb",
+                                      "bytes": 157598208},
+    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1111448064 + write 454610944
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
-                                          "sha256": "3b52599ece11483a5179dcf5ffeb0f59761808106138dd5d2dc8c73291b30e73",
-                                          "bytes": 8581975552},
+                                          "sha256": "0a8be340d5196d0f1b2f76571a31a0dbd9b5fb1e01f1b023821b5ec71c9e3bc5",
+                                          "bytes": 1566059008},
 }
 
 

@@ -12,12 +12,11 @@
 //   sum_k (q - z) s x  =  s 2^(-k) ( sum_k q x_int  -  z sum_k x_int ),
 // x_int = x 2^k an integer (k from the exponent of the group's largest |x|).
 // The codes q stay unsigned bytes (w & 0x0F0F0F0F, (w >> 4) & 0x0F0F0F0F); x_int
-// is split into three byte planes, so sum_k q x_int is three exact int32 dot
-// products, combined and scaled in FP32 once per group.  The BF16 scale is never
-// folded into a rounded operand.  Three kernels:
+// is written as three signed base-256 digits, so sum_k q x_int is three exact
+// int32 dot products, combined and scaled in FP32 once per group.  The BF16 scale
+// is never folded into a rounded operand.  Three kernels:
 //   * M <= 2: decode_cc_kernel, the dot products as mma.sync m16n8k32 (codes u8 x
-//     balanced X digits s8, or dp4a on unsigned/signed byte planes in the
-//     W4A16_CC_MMA=0 build) in the warps' registers, X prepared inside the kernel;
+//     X digits s8) in the warps' registers, X prepared inside the kernel;
 //   * 3 <= M <= 32 per launch: decode_tc_kernel, tcgen05.mma kind::i8 with the
 //     codes in tensor memory and the digit planes of all tokens as B;
 //   * prep_x8_kernel: the digit planes for the tensor-core kernel.
@@ -488,42 +487,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 }
 
 // --------------------------------------------------------------------------
-// Single-token decode kernel on the CUDA cores.
+// One- and two-token decode kernel (M <= 2).
 //
-// At M = 1 a tensor-core MMA would waste most of its columns and each MMA
-// instruction costs about a hundred cycles however small, so the dot product
-// runs on the integer dot-product units (dp4a: four 8-bit x 8-bit products
-// added to a 32-bit accumulator), which take four codes per instruction with
-// no conversion.  Codes become bytes with two logical ops per word:
-// w & 0x0F0F0F0F holds codes 0, 2, 4, 6 and (w >> 4) & 0x0F0F0F0F codes
-// 1, 3, 5, 7.  X is expanded exactly into integers per group: with E the
-// exponent of the group's largest |x|, x_int = x * 2^(22 - E) is a signed
-// integer below 2^23 in magnitude (exact for every x within 2^15 of the
-// group maximum, which a BF16 significand of 8 bits needs; smaller values are
-// rounded at 2^(E - 22), far below FP32 accumulation error), split into three
-// byte planes x_int = 65536 p2 + 256 p1 + p0 (p2 signed).  The inner sums
-// sum_k q_k p_k are exact in int32; per group and row they are combined in
-// FP32 as s * 2^(E - 22) * (sum_k q_k x_int_k - z * sum_k x_int_k).
+// At M <= 2 a tcgen05 MMA would waste most of its columns, and its operands
+// would have to pass through tensor memory; the dot products instead run as
+// warp-level mma.sync m16n8k32 in registers: A = 16 rows x 32 codes as
+// unsigned bytes, straight from the packed words (w & 0x0F0F0F0F holds codes
+// 0, 2, 4, 6 and (w >> 4) & 0x0F0F0F0F codes 1, 3, 5, 7), B = 32 codes x 8
+// columns of X digits as signed bytes, D = exact int32 sums.  X is expanded
+// exactly into integers per group: with E the exponent of the group's
+// largest |x|, x_int = x * 2^(21 - E) (exact for every x within 2^14 of the
+// group maximum; smaller values are rounded at 2^(E - 21), far below FP32
+// accumulation error), written in balanced base 256, x_int = 65536 d2 +
+// 256 d1 + d0 with every digit in [-128, 127]; column n = p NT + m of B holds
+// digit plane p of token m (columns past 3 NT are zero).  Per group and row:
+//   acc += s 2^(E - 21) (65536 D2 + 256 D1 + D0 - z sum_k x_int).
+// One MMA takes 32 codes of 16 rows against every plane of both tokens: a
+// compute thread issues 8 MMAs per 128 x 128 unit where byte-plane dp4a would
+// take 96 instructions.
 //
-// X of one group in the layout the kernel reads (400 bytes): four 96-byte
-// quarter blocks (words 4c..4c+3), each word as six 32-bit registers
-// [P0e, P1e, P2e, P0o, P1o, P2o] where Ppe holds plane p of x at k = 0, 2, 4,
-// 6 of the word and Ppo at k = 1, 3, 5, 7 (one byte each), then
-// [sum_k x_int_k (int32), 2^(E - 22) (FP32), -, -].  The 96-byte stride puts
-// the four quarters a warp reads at once in distinct banks.
-constexpr int kQuarterBytes = 96;
-constexpr int kGroupXiBytes = 4 * kQuarterBytes + 16;  // 400 B per group
-
+// X of one group in the layout the kernel reads: 3 NT digit rows of 128 bytes
+// (word w's codes 0,2,4,6 at 8w, codes 1,3,5,7 at 8w + 4: the order in which
+// the two masks above hold the codes, so a lane's B fragment of MMA j is
+// bytes 32 tig + 8 j .. + 7 of its row), then per token (sum_k x_int as FP32,
+// 2^(E - 21)).
 // The CTA streams units (128 rows x one group) through a 4-stage ring:
 //  * warp 4 (one thread) drives TMA: the codes of each unit (8 KB, 64-byte
 //    swizzle) and, once per block of 8 groups of a row tile, that block's
 //    128 x 8 scales and 128 x 8 zero points into one of two metadata slots;
 //  * warp 5 prepares X for each unit's group straight from the BF16 input
-//    (byte planes, the integer group sum and the group's power of two), so
-//    the call is a single launch;
-//  * warps 0-3 compute, thread t taking words 4c..4c+3 (c = t % 4) of rows
-//    t/4 + 32 i, i = 0..3.
-// Up to four CTAs share an SM.
+//    (the digit rows, the group sum and the group's power of two), so the
+//    call is a single launch;
+//  * warps 0-3 compute, warp w taking rows 32 w .. 32 w + 31 of each unit as
+//    two 16-row MMA blocks.
+// Up to four CTAs share an SM: their independent rings keep more loads in
+// flight than one CTA per SM with an in-order ring of the same depth.
 #ifndef W4A16_CC_WARPS
 #define W4A16_CC_WARPS 4
 #endif
@@ -540,10 +538,12 @@ constexpr int kCcThreads = (kCcWarps + 2) * 32;
 constexpr int kCcStages = W4A16_CC_STAGES;
 constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
 constexpr int kCcMaxTokens = 2;                         // tokens per launch of the integer kernel
-constexpr int kCcXOff = kCcCodeBytes;                   // X planes of the group, per token (400 B each)
-// codes + X planes of NT tokens, 512-aligned (the 64-byte swizzle's span)
+constexpr int kCcXOff = kCcCodeBytes;                   // X digit rows of the unit's group, after the codes
+// X of one group (layout above), and codes + X, 512-aligned (the 64-byte swizzle's span)
 template <int NT>
-__host__ __device__ constexpr int cc_stage_bytes() { return (kCcCodeBytes + NT * kGroupXiBytes + 511) / 512 * 512; }
+__host__ __device__ constexpr int cc_x_bytes() { return 3 * NT * 128 + 8 * NT; }
+template <int NT>
+__host__ __device__ constexpr int cc_stage_bytes() { return (kCcCodeBytes + cc_x_bytes<NT>() + 511) / 512 * 512; }
 constexpr int kCcMetaGroups = 8;                        // groups per metadata block
 constexpr int kXAhead = 6;                              // X warp: loads in flight, in units
 constexpr int kCcScBytes = kRowsPerCta * kCcMetaGroups * 2;  // 128 rows x 8 BF16 scales
@@ -559,67 +559,10 @@ __host__ __device__ constexpr size_t cc_smem() { return (size_t)cc_meta_off<NT>(
 // the older block has been released by then.
 static_assert(kCcStages <= kCcMetaGroups, "metadata slot reuse");
 
-__device__ __forceinline__ int dp4a_uu(uint32_t a, uint32_t b, int c) {
-    int d;
-    asm("dp4a.u32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
-    int d;
-    asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
 // This lane's four BF16 values of group g: lane 2w + h holds values 4h..4h+3 of word w.
 __device__ __forceinline__ uint2 load_group_x(const uint16_t* __restrict__ X, int g, int lane) {
     return __ldg(reinterpret_cast<const uint2*>(X + (int64_t)g * kGroup + lane * 4));
 }
-
-// One warp writes a group's X (its lanes' values v from load_group_x) in the layout above.
-__device__ __forceinline__ void prep_group_x(const uint2 v, unsigned char* dst, int lane) {
-    const uint32_t bits[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
-    uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
-    amax = __reduce_max_sync(0xFFFFFFFFu, amax);
-    const int ef = (int)(amax >> 7);            // biased exponent of the largest |x| (0: zero or subnormal)
-    const int E = ef == 0 ? -127 : ef - 127;    // every |x| of the group is below 2^(E + 1)
-    const int k = 22 - E;                       // in [-105, 149]
-    const int k1 = min(k, 127);
-    const float s1 = pow2f(k1), s2 = pow2f(k - k1);  // exact scalings, |x * 2^k| < 2^23
-    int xi[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) xi[i] = __float2int_rn(__uint_as_float(bits[i] << 16) * s1 * s2);
-    // planes of this lane's values: plane p of x_i is byte p of xi (plane 2 signed)
-    uint32_t m[3];
-#pragma unroll
-    for (int p = 0; p < 3; ++p) {
-        const uint32_t b0 = ((uint32_t)xi[0] >> (8 * p)) & 0xFFu, b1 = ((uint32_t)xi[1] >> (8 * p)) & 0xFFu;
-        const uint32_t b2 = ((uint32_t)xi[2] >> (8 * p)) & 0xFFu, b3 = ((uint32_t)xi[3] >> (8 * p)) & 0xFFu;
-        m[p] = b0 | (b2 << 8) | (b1 << 16) | (b3 << 24);  // [even half | odd half]
-    }
-    const int h = lane & 1, w = lane >> 1;
-    uint32_t* out = reinterpret_cast<uint32_t*>(dst + (w >> 2) * kQuarterBytes + (w & 3) * 24 + h * 12);
-#pragma unroll
-    for (int p = 0; p < 3; ++p) {
-        const uint32_t pm = __shfl_xor_sync(0xFFFFFFFFu, m[p], 1);
-        // h = 0 assembles the even register (its values 0, 2 then the partner's 4, 6),
-        // h = 1 the odd one (the partner's 1, 3 then its own 5, 7)
-        out[p] = h ? __byte_perm(pm, m[p], 0x7632) : __byte_perm(m[p], pm, 0x5410);
-    }
-    const int sum = __reduce_add_sync(0xFFFFFFFFu, (xi[0] + xi[1]) + (xi[2] + xi[3]));  // |sum| < 2^30
-    if (lane == 0) {
-        int* ext = reinterpret_cast<int*>(dst + 4 * kQuarterBytes);
-        ext[0] = sum;
-        reinterpret_cast<float*>(ext)[1] = pow2f(E - 22);
-    }
-}
-
-#ifndef W4A16_CC_MMA
-#define W4A16_CC_MMA 1
-#endif
-// 1: the integer dot products run as mma.sync m16n8k32 (codes u8 x balanced X digits s8, int32
-// accumulate) on the warp's registers; 0: as dp4a on X byte planes.
-constexpr bool kCcMma = W4A16_CC_MMA != 0;
 
 // mma.sync m16n8k32, A 16 x 32 unsigned bytes (row-major fragments), B 32 x 8 signed bytes
 // (column-major fragments), D (+)= int32: exact integer dot products.
@@ -631,13 +574,8 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One warp writes token m's balanced base-256 digits of group g (its lanes' values v from
-// load_group_x) as the B operand rows of the MMA layout: row n = p NT + m (digit plane p) holds
-// 128 bytes, word w's codes 0,2,4,6 at 8w and codes 1,3,5,7 at 8w + 4, the order in which
-// w & 0x0F0F0F0F and (w >> 4) & 0x0F0F0F0F hold the codes.  x_int = x 2^(21 - E), E the exponent
-// of the group's largest |x| (exact for every x within 2^14 of it, smaller values rounded at
-// 2^(E - 21)), = 65536 d2 + 256 d1 + d0 with every digit in [-128, 127].  After the 3 NT rows:
-// per token (sum_k x_int as FP32, 2^(E - 21)).
+// One warp writes token m's digits of group g (its lanes' values v from load_group_x) in the layout
+// above: digit row n = p NT + m.
 template <int NT>
 __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst, int lane, int m) {
     const uint32_t bits[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
@@ -773,12 +711,7 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             const int s = i % kCcStages;
             if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
 #pragma unroll
-            for (int m = 0; m < NT; ++m) {
-                if constexpr (kCcMma)
-                    prep_group_x8<NT>(v[m], ring + s * kStageBytes + kCcXOff, lane, m);
-                else
-                    prep_group_x(v[m], ring + s * kStageBytes + kCcXOff + m * kGroupXiBytes, lane);
-            }
+            for (int m = 0; m < NT; ++m) prep_group_x8<NT>(v[m], ring + s * kStageBytes + kCcXOff, lane, m);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         }
@@ -787,190 +720,37 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
 
     // ---------------------------------------------------- compute warps 0-3
     const int t = threadIdx.x;
-    if constexpr (kCcMma) {
-        // Warp w takes rows 32 w .. 32 w + 31 as two 16-row MMA blocks.  Lane (g8, tig) = (lane / 4,
-        // lane % 4) holds, per block, rows g8 and g8 + 8 of its A fragments and words 4 tig .. 4 tig + 3
-        // of each (one 16-byte chunk of the codes tile); MMA j takes word 4 tig + j of every lane, so
-        // its K = 32 codes are words j, 4 + j, 8 + j, 12 + j, and the lane's B fragments are the same
-        // words of digit plane n = g8.  After a unit, D column n = p NT + m of a row is
-        // sum_k q_k d_p(x_k) of token m; lane tig = m gathers its three planes and folds the row.
-        const int g8 = lane >> 2, tig = lane & 3;
-        const int mt = tig < NT ? tig : NT - 1;  // the token this lane folds (lanes tig < NT)
-        const bool owner = tig < NT && tig < a.M;
-        auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
-        int cur_tile = -1;
-        bool aborted = false;
-
-        auto flush = [&](int tile) {
-            const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
-            const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
-            if (first == last) {
-                if (owner) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int n = tile * kRowsPerCta + rrow(k);
-                        if (n < N) a.Y[(int64_t)mt * N + n] = float_to_bf16_bits(y[k]);
-                    }
-                }
-            } else {
-                const int slot = b - first, nseg = last - first + 1;
-                float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * a.M * kRowsPerCta;
-                if (owner) {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) part[mt * kRowsPerCta + rrow(k)] = y[k];
-                }
-                named_barrier_sync(1, kCcWarps * 32);
-                if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
-                named_barrier_sync(1, kCcWarps * 32);
-                if (s_last) {
-                    const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
-                    const float* pb = a.partial + (int64_t)tile * a.max_slots * a.M * kRowsPerCta;
-#pragma unroll
-                    for (int m = 0; m < NT; ++m) {
-                        if (m >= a.M) break;
-                        for (int rl = t; rl < rows; rl += kCcWarps * 32) {
-                            const float sum = sum_slots(pb + (int64_t)m * kRowsPerCta + rl, (int64_t)a.M * kRowsPerCta, nseg);
-                            a.Y[(int64_t)m * N + tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
-                        }
-                    }
-                    if (t == 0) a.counters[tile] = 0;
-                }
-                named_barrier_sync(1, kCcWarps * 32);
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) y[k] = 0.f;
-        };
-
-        UnitCursor uc(u_first, G);
-        int mb = -1;
-        for (int i = 0; i < nunits; ++i, uc.next(G)) {
-            const int tile = uc.tile, g = uc.g;
-            if (i == 0 || (g & (kCcMetaGroups - 1)) == 0) ++mb;
-            if (tile != cur_tile) {
-                if (cur_tile >= 0) flush(cur_tile);
-                cur_tile = tile;
-            }
-            if (aborted) continue;
-            const int s = i % kCcStages;
-            if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 53)) {
-                aborted = true;
-                continue;
-            }
-            const unsigned char* st = ring + s * kStageBytes;
-            // codes: chunk tig of each row, 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3))
-            uint4 cw[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int r = rrow(k);
-                cw[k] = *reinterpret_cast<const uint4*>(st + r * 64 + 16 * (tig ^ ((r >> 1) & 3)));
-            }
-            uint32_t bx[8];
-            if (g8 < 3 * NT) {
-                const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + g8 * 128 + tig * 32);
-                const uint4 u0 = xp[0], u1 = xp[1];
-                bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
-                bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) bx[j] = 0u;
-            }
-            const float* ext = reinterpret_cast<const float*>(st + kCcXOff + 3 * NT * 128);
-            const float xsum = ext[2 * mt], xscale = ext[2 * mt + 1];
-            // this block's metadata (loaded with its first unit, which this warp has already waited for);
-            // rows past N were zero-filled by TMA: s = 0 folds them away
-            const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
-            float sv[4], zv[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int r = rrow(k);
-                sv[k] = bf16_bits_to_float(
-                    *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
-                zv[k] = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
-                                                                 4 * (g & (kCcMetaGroups - 1)));
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
-
-#pragma unroll
-            for (int rb = 0; rb < 2; ++rb) {
-                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
-                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
-                int d[4] = {0, 0, 0, 0};
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_u8s8(d, w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
-                             (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
-                // lane tig holds columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    int P0, P1, P2;
-                    if constexpr (NT == 1) {  // planes 0, 1 at lane tig 0, plane 2 at lane tig 1
-                        P0 = d[2 * h];
-                        P1 = d[2 * h + 1];
-                        P2 = __shfl_sync(0xFFFFFFFFu, d[2 * h], lane | 1);
-                    } else {  // column p NT + m: token 0 planes at (0,0), (1,0), (2,0); token 1 at (0,1), (1,1), (2,1)
-                        const int own = tig == 0 ? d[2 * h] : d[2 * h + 1];
-                        const int x = __shfl_xor_sync(0xFFFFFFFFu, tig == 0 ? d[2 * h + 1] : d[2 * h], 1);
-                        const int t0 = __shfl_sync(0xFFFFFFFFu, d[2 * h], (lane & ~3) | 2);
-                        const int t1 = __shfl_sync(0xFFFFFFFFu, d[2 * h + 1], (lane & ~3) | 2);
-                        P0 = tig == 0 ? own : x;
-                        P1 = tig == 0 ? x : own;
-                        P2 = tig == 0 ? t0 : t1;
-                    }
-                    // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26),
-                    // the rest FP32 with one rounding per step
-                    const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-                    const int k = 2 * rb + h;
-                    y[k] = fmaf(sv[k] * xscale, fmaf(-zv[k], xsum, qx), y[k]);
-                }
-            }
-        }
-        if (cur_tile >= 0) flush(cur_tile);
-        return;
-    }
-    const int c = t & 3;   // words 4c..4c+3 of the group
-    const int rg = t >> 2; // rows rg + kCcRowStep i
-    // the 64-byte swizzle of the codes tile: logical chunk c of row r sits at chunk c ^ ((r >> 1) & 3);
-    // (r >> 1) & 3 is the same for all rows rg + kCcRowStep i (kCcRowStep % 8 == 0)
-    const int code_off = rg * 64 + 16 * (c ^ ((rg >> 1) & 3));
-    float y[kCcRows][NT];
-#pragma unroll
-    for (int i = 0; i < kCcRows; ++i)
-#pragma unroll
-        for (int m = 0; m < NT; ++m) y[i][m] = 0.f;
+    // Warp w takes rows 32 w .. 32 w + 31 as two 16-row MMA blocks.  Lane (g8, tig) = (lane / 4,
+    // lane % 4) holds, per block, rows g8 and g8 + 8 of its A fragments and words 4 tig .. 4 tig + 3
+    // of each (one 16-byte chunk of the codes tile); MMA j takes word 4 tig + j of every lane, so
+    // its K = 32 codes are words j, 4 + j, 8 + j, 12 + j, and the lane's B fragments are the same
+    // words of digit plane n = g8.  After a unit, D column n = p NT + m of a row is
+    // sum_k q_k d_p(x_k) of token m; lane tig = m gathers its three planes and folds the row.
+    const int g8 = lane >> 2, tig = lane & 3;
+    const int mt = tig < NT ? tig : NT - 1;  // the token this lane folds (lanes tig < NT)
+    const bool owner = tig < NT && tig < a.M;
+    auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
+    float y[4] = {0.f, 0.f, 0.f, 0.f};
     int cur_tile = -1;
     bool aborted = false;
 
     auto flush = [&](int tile) {
-#pragma unroll
-        for (int i = 0; i < kCcRows; ++i)  // reduce over the four threads of each row
-#pragma unroll
-            for (int m = 0; m < NT; ++m) {
-                y[i][m] += __shfl_xor_sync(0xFFFFFFFFu, y[i][m], 1);
-                y[i][m] += __shfl_xor_sync(0xFFFFFFFFu, y[i][m], 2);
-            }
         const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
         const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
         if (first == last) {
-            if (c == 0) {
+            if (owner) {
 #pragma unroll
-                for (int i = 0; i < kCcRows; ++i) {
-                    const int n = tile * kRowsPerCta + rg + kCcRowStep * i;
-#pragma unroll
-                    for (int m = 0; m < NT; ++m)
-                        if (n < N && m < a.M) a.Y[(int64_t)m * N + n] = float_to_bf16_bits(y[i][m]);
+                for (int k = 0; k < 4; ++k) {
+                    const int n = tile * kRowsPerCta + rrow(k);
+                    if (n < N) a.Y[(int64_t)mt * N + n] = float_to_bf16_bits(y[k]);
                 }
             }
         } else {
             const int slot = b - first, nseg = last - first + 1;
             float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * a.M * kRowsPerCta;
-            if (c == 0) {
+            if (owner) {
 #pragma unroll
-                for (int i = 0; i < kCcRows; ++i)
-#pragma unroll
-                    for (int m = 0; m < NT; ++m)
-                        if (m < a.M) part[m * kRowsPerCta + rg + kCcRowStep * i] = y[i][m];
+                for (int k = 0; k < 4; ++k) part[mt * kRowsPerCta + rrow(k)] = y[k];
             }
             named_barrier_sync(1, kCcWarps * 32);
             if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
@@ -991,9 +771,7 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             named_barrier_sync(1, kCcWarps * 32);
         }
 #pragma unroll
-        for (int i = 0; i < kCcRows; ++i)
-#pragma unroll
-            for (int m = 0; m < NT; ++m) y[i][m] = 0.f;
+        for (int k = 0; k < 4; ++k) y[k] = 0.f;
     };
 
     UnitCursor uc(u_first, G);
@@ -1012,70 +790,71 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             continue;
         }
         const unsigned char* st = ring + s * kStageBytes;
-        uint4 w[kCcRows];
+        // codes: chunk tig of each row, 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3))
+        uint4 cw[4];
 #pragma unroll
-        for (int r = 0; r < kCcRows; ++r) w[r] = *reinterpret_cast<const uint4*>(st + code_off + 64 * kCcRowStep * r);
-        // X planes of words 4c..4c+3 of token m: word j's registers at xr[m][6j .. 6j+5]
-        uint32_t xr[NT][24];
-        int xsum[NT];
-        float xscale[NT];
-#pragma unroll
-        for (int m = 0; m < NT; ++m) {
-            const unsigned char* xg = st + kCcXOff + m * kGroupXiBytes;
-            const uint4* xq = reinterpret_cast<const uint4*>(xg + c * kQuarterBytes);
-#pragma unroll
-            for (int j = 0; j < 6; ++j) {
-                const uint4 v = xq[j];
-                xr[m][4 * j] = v.x;
-                xr[m][4 * j + 1] = v.y;
-                xr[m][4 * j + 2] = v.z;
-                xr[m][4 * j + 3] = v.w;
-            }
-            const int* ext = reinterpret_cast<const int*>(xg + 4 * kQuarterBytes);
-            xsum[m] = ext[0];
-            xscale[m] = __int_as_float(ext[1]);
+        for (int k = 0; k < 4; ++k) {
+            const int r = rrow(k);
+            cw[k] = *reinterpret_cast<const uint4*>(st + r * 64 + 16 * (tig ^ ((r >> 1) & 3)));
         }
-        // this block's metadata (loaded with its first unit, which this warp has already waited for)
-        const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
-        const unsigned char* scb = ms + rg * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1));
-        const unsigned char* zeb = ms + kCcScBytes + rg * (kCcMetaGroups * 4) + 4 * (g & (kCcMetaGroups - 1));
-        float sv[kCcRows], zv[kCcRows];
+        uint32_t bx[8];
+        if (g8 < 3 * NT) {
+            const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + g8 * 128 + tig * 32);
+            const uint4 u0 = xp[0], u1 = xp[1];
+            bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
+            bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
+        } else {
 #pragma unroll
-        for (int r = 0; r < kCcRows; ++r) {
-            // rows past N were zero-filled by TMA: s = 0 folds them away
-            sv[r] = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(scb + kCcRowStep * kCcMetaGroups * 2 * r));
-            zv[r] = (float)*reinterpret_cast<const int32_t*>(zeb + kCcRowStep * kCcMetaGroups * 4 * r);
+            for (int j = 0; j < 8; ++j) bx[j] = 0u;
+        }
+        const float* ext = reinterpret_cast<const float*>(st + kCcXOff + 3 * NT * 128);
+        const float xsum = ext[2 * mt], xscale = ext[2 * mt + 1];
+        // this block's metadata (loaded with its first unit, which this warp has already waited for);
+        // rows past N were zero-filled by TMA: s = 0 folds them away
+        const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
+        float sv[4], zv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int r = rrow(k);
+            sv[k] = bf16_bits_to_float(
+                *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
+            zv[k] = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
+                                                             4 * (g & (kCcMetaGroups - 1)));
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
 #pragma unroll
-        for (int r = 0; r < kCcRows; ++r) {
-            const uint32_t wr[4] = {w[r].x, w[r].y, w[r].z, w[r].w};
-            int p0[NT], p1[NT], p2[NT];  // sum_k q_k * plane_p(x_k) over this thread's 32 codes, per token
+        for (int rb = 0; rb < 2; ++rb) {
+            const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+            const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
+            int d[4] = {0, 0, 0, 0};
 #pragma unroll
-            for (int m = 0; m < NT; ++m) p0[m] = p1[m] = p2[m] = 0;
+            for (int j = 0; j < 4; ++j)
+                mma_u8s8(d, w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
+                         (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
+            // lane tig holds columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t ce = wr[j] & 0x0F0F0F0Fu, co = (wr[j] >> 4) & 0x0F0F0F0Fu;  // codes 0,2,4,6 / 1,3,5,7
-#pragma unroll
-                for (int m = 0; m < NT; ++m) {
-                    p0[m] = dp4a_uu(ce, xr[m][6 * j], p0[m]);
-                    p1[m] = dp4a_uu(ce, xr[m][6 * j + 1], p1[m]);
-                    p2[m] = dp4a_us(ce, xr[m][6 * j + 2], p2[m]);
-                    p0[m] = dp4a_uu(co, xr[m][6 * j + 3], p0[m]);
-                    p1[m] = dp4a_uu(co, xr[m][6 * j + 4], p1[m]);
-                    p2[m] = dp4a_us(co, xr[m][6 * j + 5], p2[m]);
+            for (int h = 0; h < 2; ++h) {
+                int P0, P1, P2;
+                if constexpr (NT == 1) {  // planes 0, 1 at lane tig 0, plane 2 at lane tig 1
+                    P0 = d[2 * h];
+                    P1 = d[2 * h + 1];
+                    P2 = __shfl_sync(0xFFFFFFFFu, d[2 * h], lane | 1);
+                } else {  // column p NT + m: token 0 planes at (0,0), (1,0), (2,0); token 1 at (0,1), (1,1), (2,1)
+                    const int own = tig == 0 ? d[2 * h] : d[2 * h + 1];
+                    const int x = __shfl_xor_sync(0xFFFFFFFFu, tig == 0 ? d[2 * h + 1] : d[2 * h], 1);
+                    const int t0 = __shfl_sync(0xFFFFFFFFu, d[2 * h], (lane & ~3) | 2);
+                    const int t1 = __shfl_sync(0xFFFFFFFFu, d[2 * h + 1], (lane & ~3) | 2);
+                    P0 = tig == 0 ? own : x;
+                    P1 = tig == 0 ? x : own;
+                    P2 = tig == 0 ? t0 : t1;
                 }
-            }
-#pragma unroll
-            for (int m = 0; m < NT; ++m) {
-                // sum q x_int = 65536 p2 + (256 p1 + p0): the bracket is exact in int32 (< 2^25),
-                // the rest is FP32 with one rounding per step
-                const float qx = fmaf((float)p2[m], 65536.f, (float)(p1[m] * 256 + p0[m]));
-                // y += s 2^(E-22) (sum q x_int  -  [one thread of four] z sum x_int)
-                const float corr = (c == 0) ? (float)xsum[m] : 0.f;
-                y[r][m] = fmaf(sv[r] * xscale[m], fmaf(-zv[r], corr, qx), y[r][m]);
+                // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26),
+                // the rest FP32 with one rounding per step
+                const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+                const int k = 2 * rb + h;
+                y[k] = fmaf(sv[k] * xscale, fmaf(-zv[k], xsum, qx), y[k]);
             }
         }
     }
