@@ -282,26 +282,35 @@ def time_layer_alone(c, torch, w4, stream, min_calls=200):
 
 
 def time_e2e(layers, steps, warmup, torch, w4, stream, path):
-    """Public-API calls with host buffers: pinned H2D of X and D2H of Y every step."""
+    """The C-ABI call with host buffers, once per layer and step: w4a16_linear_host enqueues the
+    pinned H2D copy of X, the layer and the D2H copy of Y on the stream (the automatic path choice,
+    as `path` is for the timed kernels)."""
+    lib = w4.load()
     xs = [torch.from_numpy(L["x_host"].view(np.int16)).pin_memory() for L in layers]
     ys = [torch.empty((L["case"].M, L["case"].N), dtype=torch.int16).pin_memory() for L in layers]
+    calls = []
+    for L, xh, yh in zip(layers, xs, ys):
+        c, pw, ws = L["case"], L["pw"], L["ws"]
+        calls.append((xh.data_ptr(), L["X"].data_ptr(), c.M, c.K, pw.qweight.data_ptr(), pw.scales.data_ptr(),
+                      pw.zeros.data_ptr(), c.N, L["Y"].data_ptr(), yh.data_ptr(),
+                      ws.data_ptr() if ws is not None else None, ws.numel() if ws is not None else 0,
+                      stream.cuda_stream))
+    fn = lib.w4a16_linear_host
 
     def one_step():
-        for L, xh, yh in zip(layers, xs, ys):
-            L["X"].view(torch.int16).copy_(xh, non_blocking=True)
-            _linear_call(w4, L, path)
-            yh.copy_(L["Y"].view(torch.int16), non_blocking=True)
+        for args in calls:
+            st = fn(*args)
+            if st != 0:
+                raise w4.W4A16Error("w4a16_linear_host", st)
 
-    with torch.cuda.stream(stream):
-        for _ in range(warmup):
-            one_step()
+    for _ in range(warmup):
+        one_step()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
-        for _ in range(steps):
-            one_step()
-        end.record(stream)
+    start.record(stream)
+    for _ in range(steps):
+        one_step()
+    end.record(stream)
     torch.cuda.synchronize()
     h2d = sum(L["X"].numel() * 2 for L in layers)
     d2h = sum(L["Y"].numel() * 2 for L in layers)

@@ -132,6 +132,23 @@ W4A16_API int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const u
                       int path, void* stream);
 
 /*
+ * The linear layer on host buffers: one call enqueues, on `stream`, the copy
+ * of X from host to device, w4a16_linear(), and the copy of Y back to the
+ * host (one cudaMemcpyAsync each way), so a caller that holds activations in
+ * host memory pays a single library call per layer.
+ *   X_host    host, bf16 bits [M][K]; page-locked (cudaHostAlloc or
+ *             cudaHostRegister) for the copy to be asynchronous
+ *   X_dev     device, bf16 bits [M][K], the staging buffer X is copied into
+ *   Y_dev     device, bf16 bits [M][N], the layer's output
+ *   Y_host    host, bf16 bits [M][N], page-locked; valid once the stream
+ *             has reached the end of this call's work
+ *   other arguments as w4a16_linear().  The buffers must not overlap.
+ */
+W4A16_API int w4a16_linear_host(const uint16_t* X_host, uint16_t* X_dev, int64_t M, int64_t K, const uint32_t* qweight,
+                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y_dev, uint16_t* Y_host,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Unpack codes ("What the Tensor Types Tell You": two INT4 codes per byte;
  * the word layout above).  codes: device, uint8 [N][K], values 0..15.
  * Test and inspection use.

@@ -229,3 +229,20 @@ def test_zero_points_far_outside_the_code_range(cuda_lib, M, path):
     X = synth.activations_bf16(900 + M, M, K)
     Y = run_linear(X, pw, path)
     assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), f"M={M}")
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 640, 1024), (2, 256, 2048), (96, 384, 1152)])
+def test_host_buffer_entry_matches_device_entry(cuda_lib, M, N, K):
+    """w4a16_linear_host (copies in and out on the stream) gives the same bits as w4a16_linear."""
+    W = synth.weights_f32(M + N + K, synth.TAG_W, N, K)
+    pw = packed_from_host(W)
+    xb = synth.activations_bf16(M + 3, M, K)
+    Y_ref = run_linear(xb, pw)
+    X_host = torch.from_numpy(xb.view(np.int16)).pin_memory()
+    Y_host = torch.full((M, N), -1, dtype=torch.int16).pin_memory()
+    X_dev = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    Y_dev = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(w4.workspace_bytes(M, N, K), 1), dtype=torch.uint8, device="cuda")
+    w4.linear_host(X_host, X_dev, pw.qweight, pw.scales, pw.zeros, Y_dev, Y_host, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y_host, Y_ref.view(torch.int16).cpu())

@@ -50,6 +50,7 @@ SIGNATURES = {
     "w4a16_workspace_init": (_int, [_vp, _sz, _vp]),
     "w4a16_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "w4a16_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
+    "w4a16_linear_host": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "w4a16_unpack": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_dequant": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "w4a16_renorm_rows": (_int, [_vp, _i64, _i64, _vp, _vp]),
@@ -155,6 +156,40 @@ def linear(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: 
         _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N,
         _dev(Y, "Y", torch.bfloat16, (M, N)), ws_ptr, ws_bytes, path, _stream(stream))
     _check("w4a16_linear", st)
+
+
+def _host(t: torch.Tensor, name: str, shape) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype not in (torch.bfloat16, torch.int16):
+        raise TypeError(f"{name} must hold BF16 bits (bfloat16 or int16), got {t.dtype}")
+    if not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be contiguous with shape {tuple(shape)}")
+    return t.data_ptr()
+
+
+def linear_host(X_host: torch.Tensor, X_dev: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                zeros: torch.Tensor, Y_dev: torch.Tensor, Y_host: torch.Tensor,
+                workspace: torch.Tensor | None = None, stream=None) -> None:
+    """w4a16_linear_host: copy X_host to X_dev, run the layer into Y_dev, copy it to Y_host, all
+    enqueued on the stream by one library call (host tensors should be pinned for the copies to be
+    asynchronous; Y_host is valid once the stream has passed this call)."""
+    M, K = X_dev.shape
+    N = qweight.shape[0]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace", torch.uint8)
+        ws_bytes = workspace.numel()
+    st = load().w4a16_linear_host(
+        _host(X_host, "X_host", (M, K)), _dev(X_dev, "X_dev", torch.bfloat16), M, K,
+        _dev(qweight, "qweight", torch.int32, (N, K // 8)),
+        _dev(scales, "scales", torch.bfloat16, (N, K // GROUP)),
+        _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N,
+        _dev(Y_dev, "Y_dev", torch.bfloat16, (M, N)), _host(Y_host, "Y_host", (M, N)), ws_ptr, ws_bytes,
+        _stream(stream))
+    _check("w4a16_linear_host", st)
 
 
 def linear_noalloc(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,

@@ -132,6 +132,22 @@ int w4a16_linear(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweigh
                              stream);
 }
 
+int w4a16_linear_host(const uint16_t* X_host, uint16_t* X_dev, int64_t M, int64_t K, const uint32_t* qweight,
+                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y_dev, uint16_t* Y_host,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    if (!X_host || !Y_host || !X_dev || !Y_dev) return W4A16_ERR_ARG;
+    int st = check_shape(M, N, K);
+    if (st != W4A16_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(X_dev, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return W4A16_ERR_CUDA;
+    st = w4a16_linear_path(X_dev, M, K, qweight, scales, zeros, N, Y_dev, workspace, workspace_bytes, W4A16_PATH_AUTO,
+                           stream);
+    if (st != W4A16_OK) return st;
+    return cudaMemcpyAsync(Y_host, Y_dev, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) == cudaSuccess ? W4A16_OK
+                                                                                                        : W4A16_ERR_CUDA;
+}
+
 int w4a16_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, void* stream) {
     if (!qweight || !codes) return W4A16_ERR_ARG;
     int st = check_shape(1, N, K);
