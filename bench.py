@@ -46,10 +46,10 @@ NCU_TRAFFIC = {
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
                                       "sha256": "18a05e78ee2f1998d923ba976ebb0fe04afcec9624fe0565177c5f8f1f036fdb",
                                       "bytes": 157598208},
-    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1111448064 + write 454610944
+    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1110778880 + write 454575872
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
-                                          "sha256": "0a8be340d5196d0f1b2f76571a31a0dbd9b5fb1e01f1b023821b5ec71c9e3bc5",
-                                          "bytes": 1566059008},
+                                          "sha256": "1eed7b053dbd1150188bcff11bcb6b10faf12c174186544dcacbb0a201dedc7f",
+                                          "bytes": 1565354752},
 }
 
 

@@ -94,10 +94,6 @@ static_assert(32 * (4 * kPRegsDequant + 4 * kPRegsIssue + kPFoldWarps * kPRegsFo
               "setmaxnreg split exceeds the registers the block is launched with");
 static_assert(kPFoldWarps == 8 || kPFoldWarps == 16, "fold warps");
 constexpr int kPLdCols = kPFoldWarps == 16 ? 8 : 16;    // TMEM columns per fold load
-#ifndef W4A16_PF_LD_BATCH
-#define W4A16_PF_LD_BATCH 1
-#endif
-constexpr int kPLdBatch = W4A16_PF_LD_BATCH;            // fold loads in flight per wait
 constexpr uint32_t kPIdesc = idesc_bf16_f32(kPBM * kPCtas, kPBN);
 
 struct PrefillArgs {
@@ -412,29 +408,23 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     const float* xs = a.xsT + (int64_t)g * a.Mp + m0;
                     tc_fence_after();
 #pragma unroll
-                    for (int cc = 0; cc < kPFoldCols / (kPLdCols * kPLdBatch); ++cc) {
-                        uint32_t d[kPLdBatch][kPLdCols];
-#pragma unroll
-                        for (int bt = 0; bt < kPLdBatch; ++bt)
-                            tmem_ldn(tl + dbuf * kPBN + colh * kPFoldCols + (cc * kPLdBatch + bt) * kPLdCols, d[bt]);
+                    for (int cc = 0; cc < kPFoldCols / kPLdCols; ++cc) {
+                        const int j0 = cc * kPLdCols;
+                        uint32_t d[kPLdCols];
+                        tmem_ldn(tl + dbuf * kPBN + colh * kPFoldCols + j0, d);
                         tmem_wait_ld();
+                        if (!need_xs) {
 #pragma unroll
-                        for (int bt = 0; bt < kPLdBatch; ++bt) {
-                            const int j0 = (cc * kPLdBatch + bt) * kPLdCols;
-                            if (!need_xs) {
+                            for (int e = 0; e < kPLdCols; e += 2) fma2_bcast(T[j0 + e], T[j0 + e + 1], sv, d[e], d[e + 1]);
+                        } else {
 #pragma unroll
-                                for (int e = 0; e < kPLdCols; e += 2)
-                                    fma2_bcast(T[j0 + e], T[j0 + e + 1], sv, d[bt][e], d[bt][e + 1]);
-                            } else {
+                            for (int j4 = 0; j4 < kPLdCols / 4; ++j4) {
+                                const float4 xv = __ldg(reinterpret_cast<const float4*>(xs + j0 + 4 * j4));
+                                const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                                for (int j4 = 0; j4 < kPLdCols / 4; ++j4) {
-                                    const float4 xv = __ldg(reinterpret_cast<const float4*>(xs + j0 + 4 * j4));
-                                    const float xq[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) {
-                                        const int j = j0 + 4 * j4 + e;
-                                        T[j] = fmaf(sv, fmaf(-zr, xq[e], __uint_as_float(d[bt][4 * j4 + e])), T[j]);
-                                    }
+                                for (int e = 0; e < 4; ++e) {
+                                    const int j = j0 + 4 * j4 + e;
+                                    T[j] = fmaf(sv, fmaf(-zr, xq[e], __uint_as_float(d[4 * j4 + e])), T[j]);
                                 }
                             }
                         }
