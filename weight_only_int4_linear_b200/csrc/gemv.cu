@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     __shared__ uint32_t s_tmem;
     __shared__ int s_last;
     __shared__ volatile int s_issued;
+    __shared__ float s_split[kRowsPerCta * (NTOK / 2)];  // odd fold warps' row-tile sums (alternate units)
 
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-aligned stages
@@ -228,10 +229,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     const int nunits = a.units_base + (b < a.units_rem ? 1 : 0);
     const int G = a.G;
 
+    // With at most NTOK / 2 tokens the second token half of the fold has nothing to do: the two fold
+    // warps of a lane quadrant then take alternate units instead (four fold warps read each unit).
+    const bool split_units = a.M <= NTOK / 2;
+    const int unit_folders = split_units ? kFoldWarps / 2 : kFoldWarps;
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 4 + 1 + kFoldWarps);  // dequantiser set, MMA commit, fold warps (X sums)
+            mbar_init(&empty[s], 4 + 1 + unit_folders);  // dequantiser set, MMA commit, fold warps (X sums)
         }
         for (int i = 0; i < NA; ++i) {
             mbar_init(&afull[i], 4);
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         }
         for (int i = 0; i < ND; ++i) {
             mbar_init(&mdone[i], 1);
-            mbar_init(&dfree[i], kFoldWarps);
+            mbar_init(&dfree[i], unit_folders);
         }
         s_issued = 0;
         fence_mbar_init();
@@ -345,33 +350,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 
     // ------------------------------------------------------- fold warps 0-7
     constexpr int TH = NTOK / 2;                  // tokens per fold thread
-    const int quad = warp & 3, th = warp >> 2;    // lane quadrant, token half
+    const int quad = warp & 3, th = warp >> 2;    // lane quadrant, token half (or unit parity)
     const int row_local = quad * 32 + lane;
-    const int m_base = th * TH;
+    const int m_base = split_units ? 0 : th * TH;
     const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
     const int N = a.N, M = a.M;
     float acc[TH];
 #pragma unroll
     for (int m = 0; m < TH; ++m) acc[m] = 0.f;
     bool aborted = false;
-    int cur_tile = -1;
+    int cur_tile = (int)(u_first / G);  // the row tile acc accumulates
 
+    // One row tile's sums leave the CTA (every fold thread calls this once per row tile of the CTA's
+    // range, in order).  With alternate units, the odd warps' sums are added to the even warps'.
     auto flush = [&](int tile) {
+        if (split_units) {
+            if (th == 1) {
+#pragma unroll
+                for (int e = 0; e < TH; ++e) s_split[e * kRowsPerCta + row_local] = acc[e];
+            }
+            named_barrier_sync(1, kFoldWarps * 32);
+            if (th == 0) {
+#pragma unroll
+                for (int e = 0; e < TH; ++e) acc[e] += s_split[e * kRowsPerCta + row_local];
+            }
+        }
+        const bool writer = !split_units || th == 0;
         const int n = tile * kRowsPerCta + row_local;
         const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
         const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
         if (first == last) {
-            if (n < N) {
+            if (n < N && writer) {
 #pragma unroll
                 for (int e = 0; e < TH; ++e)
                     if (m_base + e < M) a.Y[(int64_t)(m_base + e) * N + n] = float_to_bf16_bits(acc[e]);
             }
+            if (split_units) named_barrier_sync(1, kFoldWarps * 32);  // s_split is reused by the next tile
         } else {
             const int slot = b - first, nseg = last - first + 1;
             float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * M * kRowsPerCta;
+            if (writer) {
 #pragma unroll
-            for (int e = 0; e < TH; ++e)
-                if (m_base + e < M) part[(m_base + e) * kRowsPerCta + row_local] = acc[e];
+                for (int e = 0; e < TH; ++e)
+                    if (m_base + e < M) part[(m_base + e) * kRowsPerCta + row_local] = acc[e];
+            }
             named_barrier_sync(1, kFoldWarps * 32);
             if (threadIdx.x == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
             named_barrier_sync(1, kFoldWarps * 32);
@@ -401,10 +423,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
     };
 
     auto fold_unit = [&](int j, int tile, float sv, float zv) {
-        if (tile != cur_tile) {
-            if (cur_tile >= 0) flush(cur_tile);
-            cur_tile = tile;
-        }
+        while (cur_tile < tile) flush(cur_tile++);
+        if (split_units && (j & 1) != th) return;  // the other warp of the quadrant folds this unit
         if (aborted) return;
         const int di = j % ND, s = j % S;
         if (!mbar_wait(&mdone[di], (j / ND) & 1, a.fault, 13)) {
@@ -472,7 +492,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             }
         }
     }
-    if (cur_tile >= 0) flush(cur_tile);
+    const int tile_last = nunits > 0 ? (int)((u_first + nunits - 1) / G) : cur_tile - 1;
+    while (cur_tile <= tile_last) flush(cur_tile++);
 
     // teardown: every MMA issued must be complete before the columns are released
     named_barrier_sync(1, kFoldWarps * 32);
