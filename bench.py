@@ -42,10 +42,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154371840 + dram__bytes_write.sum 3226368
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154224384 + dram__bytes_write.sum 4144384
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "18a05e78ee2f1998d923ba976ebb0fe04afcec9624fe0565177c5f8f1f036fdb",
-                                      "bytes": 157598208},
+                                      "sha256": "3a092f494e368178df4636f486048961c4f2b14d6188d7f5ab246b6132a32eb1",
+                                      "bytes": 158368768},
     # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1110778880 + write 454575872
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
                                           "sha256": "1eed7b053dbd1150188bcff11bcb6b10faf12c174186544dcacbb0a201dedc7f",
