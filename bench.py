@@ -665,6 +665,97 @@ def run_profile(spec: str, repeats: int = 4):
         raise SystemExit(1)
 
 
+def _time_graph(torch, stream, body, calls):
+    """Device time per call of `body` (which makes `calls` calls), replayed from a CUDA graph."""
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            body()
+    torch.cuda.synchronize()
+    g = capture(torch, stream, body)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 3
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(reps):
+            g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / (reps * calls)
+
+
+def run_comparators(which: str):
+    """The unfused pipelines the fused kernel replaces ("Quantization I", Concept; "Weight-Only
+    Quantization and Mixed Precision", sections 1 and 7), timed per call beside the fused path, one
+    JSON line per layer:
+      offline_dequant_gemm: W_hat = (q - z) s materialised once in BF16 (not timed), then a cuBLAS
+        BF16 GEMM per call (torch.matmul);
+      naive_three_kernel: per call, unpack to byte codes (w4a16_unpack), dequantise to BF16
+        (w4a16_dequant_codes), cuBLAS BF16 GEMM: every intermediate through HBM.
+    Every call of every variant reads weights past L2 (enough copies rotated)."""
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    w4.load()
+    stream = torch.cuda.Stream()
+    sets = {"decode": workloads.decode_5120(), "prefill": workloads.prefill_8192(ms=[4096])}
+    names = list(sets) if which == "all" else which.split(",")
+    for wl in names:
+        for c in sets[wl]:
+            fused_us, _ = time_layer_alone(c, torch, w4, stream)
+            W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
+            synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+            pw = w4.PackedWeight.from_float(W, stream=stream)
+            torch.cuda.synchronize()
+            del W
+            xb = synth.activations_bf16(c.x_seed, c.M, c.K)
+            X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+            # offline dequantisation: BF16 weights, copies past 3x L2
+            wbytes = c.N * c.K * 2
+            ncopy = max(1, min(16, -(-3 * L2_BYTES // wbytes)))
+            W_hats = [torch.empty((c.N, c.K), dtype=torch.bfloat16, device="cuda") for _ in range(ncopy)]
+            for Wh in W_hats:
+                w4.dequant(pw.qweight, pw.scales, pw.zeros, c.K, Wh)
+            torch.cuda.synchronize()
+
+            def body_gemm():
+                for Wh in W_hats:
+                    torch.matmul(X, Wh.t(), out=Y)
+            gemm_us = _time_graph(torch, stream, body_gemm, ncopy)
+            Y_gemm = Y.clone()
+            del W_hats
+            torch.cuda.empty_cache()
+            # naive three kernels: packed copies past 3x L2, one codes and one W_hat buffer
+            pcopy = max(1, min(16, -(-3 * L2_BYTES // c.code_bytes)))
+            pws = [(pw.qweight, pw.scales, pw.zeros)] + [(pw.qweight.clone(), pw.scales.clone(), pw.zeros.clone())
+                                                         for _ in range(pcopy - 1)]
+            codes = torch.empty((c.N, c.K), dtype=torch.uint8, device="cuda")
+            Wh = torch.empty((c.N, c.K), dtype=torch.bfloat16, device="cuda")
+
+            def body_naive():
+                for qw_, sc_, z_ in pws:
+                    w4.unpack(qw_, c.K, codes)
+                    w4.dequant_codes(codes, sc_, z_, Wh)
+                    torch.matmul(X, Wh.t(), out=Y)
+            naive_us = _time_graph(torch, stream, body_naive, pcopy)
+            torch.cuda.synchronize()
+            agree = bool(torch.equal(Y.view(torch.int16), Y_gemm.view(torch.int16)))
+            line = {"comparators": c.workload, "layer": c.name, "M": c.M, "K": c.K, "N": c.N,
+                    "fused_us": fused_us, "offline_dequant_gemm_us": gemm_us, "naive_three_kernel_us": naive_us,
+                    "fused_speedup_vs_dequant_gemm": gemm_us / fused_us,
+                    "fused_speedup_vs_naive": naive_us / fused_us,
+                    "fused_code_gbs": c.code_bytes / fused_us / 1e3,
+                    "unfused_paths_agree_bitwise": agree, "fault": w4.device_fault()}
+            if c.M >= PREFILL_MIN_M:
+                line.update({"fused_tflops": c.flops / fused_us / 1e6, "dequant_gemm_tflops": c.flops / gemm_us / 1e6,
+                             "naive_tflops": c.flops / naive_us / 1e6})
+            print(json.dumps(line), flush=True)
+            del pws, codes, Wh, pw
+            torch.cuda.empty_cache()
+
+
 def run_sweep(which: str):
     """Per-layer device time of every workload shape (one JSON line each): each
     call reads a different copy of the packed weights, rotating through enough
@@ -710,9 +801,15 @@ def main():
     ap.add_argument("--profile", default=None,
                     help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096, decode:all): run it a few "
                          "times, untimed")
+    ap.add_argument("--comparators", default=None,
+                    help="decode|prefill|all: the unfused pipelines (offline dequant + GEMM, naive three kernels) "
+                         "timed beside the fused path, one JSON line per layer")
     ap.add_argument("--sweep", default=None,
                     help="all, or a comma list of single_gemv, decode, small, prefill: per-layer times, one line each")
     args = ap.parse_args()
+    if args.comparators:
+        run_comparators(args.comparators)
+        return
     if args.sweep:
         run_sweep(args.sweep)
         return

@@ -165,6 +165,17 @@ W4A16_API int w4a16_dequant(const uint32_t* qweight, const uint16_t* scales, con
                   uint16_t* W_hat, void* stream);
 
 /*
+ * Materialise W_hat from unpacked codes (codes: device, uint8 [N][K], values
+ * 0..15, as written by w4a16_unpack): the middle kernel of the unfused
+ * three-kernel pipeline the fused kernel replaces ("Weight-Only Quantization
+ * and Mixed Precision", section 7, "The Pain Point": read and unpack, then
+ * dequantise, then multiply, each through HBM).  Same bits as w4a16_dequant.
+ * Comparison use only.
+ */
+W4A16_API int w4a16_dequant_codes(const uint8_t* codes, const uint16_t* scales, const int32_t* zeros, int64_t N,
+                        int64_t K, uint16_t* W_hat, void* stream);
+
+/*
  * Row renormalisation used between chained layers of the decode-stack
  * workload (not part of the method): out[m][:] = bf16_rne(y[m][:] / rms(y[m][:]))
  * with the sum of squares in FP32; a zero row stays zero.

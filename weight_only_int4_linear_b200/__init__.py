@@ -53,6 +53,7 @@ SIGNATURES = {
     "w4a16_linear_host": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "w4a16_unpack": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_dequant": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
+    "w4a16_dequant_codes": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "w4a16_renorm_rows": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_device_fault": (_int, []),
     "w4a16_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
@@ -226,6 +227,17 @@ def dequant(qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, K:
                               _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N, K,
                               _dev(W_hat, "W_hat", torch.bfloat16, (N, K)), _stream(stream))
     _check("w4a16_dequant", st)
+
+
+def dequant_codes(codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, W_hat: torch.Tensor,
+                  stream=None) -> None:
+    """w4a16_dequant_codes: W_hat bf16 [N, K] from unpacked codes uint8 [N, K] (unfused comparison)."""
+    N, K = codes.shape
+    st = load().w4a16_dequant_codes(_dev(codes, "codes", torch.uint8, (N, K)),
+                                    _dev(scales, "scales", torch.bfloat16, (N, K // GROUP)),
+                                    _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N, K,
+                                    _dev(W_hat, "W_hat", torch.bfloat16, (N, K)), _stream(stream))
+    _check("w4a16_dequant_codes", st)
 
 
 def renorm_rows(y: torch.Tensor, out: torch.Tensor, stream=None) -> None:

@@ -167,6 +167,16 @@ int w4a16_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t
     return launch_dequant(qweight, scales, zeros, N, K, W_hat, (cudaStream_t)stream);
 }
 
+int w4a16_dequant_codes(const uint8_t* codes, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                        uint16_t* W_hat, void* stream) {
+    if (!codes || !scales || !zeros || !W_hat) return W4A16_ERR_ARG;
+    int st = check_shape(1, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(zeros) || !aligned16(W_hat)) return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    return launch_dequant_codes(codes, scales, zeros, N, K, W_hat, (cudaStream_t)stream);
+}
+
 int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, void* stream) {
     if (!y || !out) return W4A16_ERR_ARG;
     if (M < 1 || N < 1) return W4A16_ERR_ARG;

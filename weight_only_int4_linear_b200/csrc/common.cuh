@@ -59,6 +59,8 @@ int launch_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight
 int launch_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, cudaStream_t stream);
 int launch_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
                    uint16_t* out, cudaStream_t stream);
+int launch_dequant_codes(const uint8_t* codes, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                         uint16_t* out, cudaStream_t stream);
 int launch_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, cudaStream_t stream);
 
 // Every workspace starts with the decode path's split-K arrival counters, at

@@ -85,6 +85,36 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ qweight, int64_t word
     }
 }
 
+// Dequantisation from unpacked codes (the middle kernel of the unfused three-kernel
+// W4A16 pipeline, "Weight-Only Quantization and Mixed Precision", section 7): one
+// thread per 16 codes -> 16 BF16 values of (q - z) * s.  (q - z) * s is exact in
+// FP32 (a 5-bit integer times an 8-bit significand), so the one rounding to BF16
+// gives the same bits as dequant_kernel.
+__global__ void dequant_codes_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
+                                     const int32_t* __restrict__ zeros, int64_t chunks, int64_t chunks_per_row,
+                                     uint16_t* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i / chunks_per_row, c = i - n * chunks_per_row;
+        const int64_t grp = n * (chunks_per_row / (kGroup / 16)) + c / (kGroup / 16);
+        const float s = bf16_bits_to_float(scales[grp]);
+        const float z = (float)zeros[grp];
+        const uint4 q = reinterpret_cast<const uint4*>(codes)[i];
+        const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float lo = ((float)((qw[w] >> (16 * h)) & 0xFFu) - z) * s;
+                const float hi = ((float)((qw[w] >> (16 * h + 8)) & 0xFFu) - z) * s;
+                o[2 * w + h] = (uint32_t)float_to_bf16_bits(lo) | ((uint32_t)float_to_bf16_bits(hi) << 16);
+            }
+        uint4* dst = reinterpret_cast<uint4*>(out) + 2 * i;
+        dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+        dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
 // One thread per packed word -> 8 BF16 values of (q - z) * s (exact product in
 // binary64, one rounding to BF16).
 __global__ void dequant_kernel(const uint32_t* __restrict__ qweight, const uint16_t* __restrict__ scales,
@@ -155,6 +185,13 @@ int launch_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight
 int launch_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, cudaStream_t stream) {
     const int64_t words = N * (K / 8);
     unpack_kernel<<<grid_for(words, 256), 256, 0, stream>>>(qweight, words, codes);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+int launch_dequant_codes(const uint8_t* codes, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                         uint16_t* out, cudaStream_t stream) {
+    const int64_t chunks = N * K / 16;
+    dequant_codes_kernel<<<grid_for(chunks, 256), 256, 0, stream>>>(codes, scales, zeros, chunks, K / 16, out);
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
