@@ -52,6 +52,8 @@ def lib():
         L.orc_pack_codes.restype = None
         L.orc_quantize_pack.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.orc_quantize_pack.restype = ctypes.c_int
+        L.orc_quantize_pack_sym.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        L.orc_quantize_pack_sym.restype = ctypes.c_int
         L.orc_unpack.argtypes = [vp, i64, i64, vp]
         L.orc_unpack.restype = None
         L.orc_dequant.argtypes = [vp, vp, vp, i64, i64, vp]
@@ -90,16 +92,18 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def quantize_pack(W: np.ndarray, with_clipped: bool = False):
+def quantize_pack(W: np.ndarray, with_clipped: bool = False, symmetric: bool = False):
     """W float32 [N, K] -> (status, qweight u32 [N, K/8], scales bf16-bits u16 [N, K/128],
-    zeros i32 [N, K/128][, clipped u8 [N, K]])."""
+    zeros i32 [N, K/128][, clipped u8 [N, K]]).  symmetric=True: signed codes
+    q = clamp(rint(w/s), -8, 7) with s = bf16(max|w|/7), stored as q + 8 with zero point 8."""
     W = np.ascontiguousarray(W, dtype=np.float32)
     N, K = W.shape
     qw = np.zeros((N, K // 8), dtype=np.uint32)
     sc = np.zeros((N, max(K // G, 1)), dtype=np.uint16)
     z = np.zeros((N, max(K // G, 1)), dtype=np.int32)
     cl = np.zeros((N, K), dtype=np.uint8) if with_clipped else None
-    st = lib().orc_quantize_pack(_p(W), N, K, _p(qw), _p(sc), _p(z), _p(cl) if cl is not None else None)
+    fn = lib().orc_quantize_pack_sym if symmetric else lib().orc_quantize_pack
+    st = fn(_p(W), N, K, _p(qw), _p(sc), _p(z), _p(cl) if cl is not None else None)
     if with_clipped:
         return st, qw, sc, z, cl
     return st, qw, sc, z

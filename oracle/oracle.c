@@ -27,11 +27,12 @@
  *   z  = rint(-lo / s)                            (ties to even, not clamped)
  *   q  = clamp(rint(w / s) + z, 0, 15)
  * using the stored BF16 scale for z and q so the stored parameters reproduce
- * the codes.  Codes are packed 8 per uint32 word, lowest K index in the lowest
+ * the codes.  The symmetric variant (orc_quantize_pack_sym) is documented at
+ * its definition.  Codes are packed 8 per uint32 word, lowest K index in the lowest
  * nibble.  Group index runs along K, per output row n.
  *
- * Parity status: quantise/pack/unpack/dequant are pinned by hand-worked
- * groups, tie cases, grid round trips and invariants; the matmul by a library
+ * Parity status: quantise/pack/unpack/dequant (both variants) are pinned by
+ * hand-worked groups, tie cases, grid round trips, brute force and invariants; the matmul by a library
  * FP64 matmul of the dequantised weights and one-hot/constant inputs; the
  * row renormalisation by its closed form (unit RMS) on tiny inputs.
  */
@@ -132,10 +133,47 @@ void orc_pack_codes(const uint8_t* codes, int64_t N, int64_t K, uint32_t* qweigh
         }
 }
 
-/* W fp32 [N][K] -> qweight u32 [N][K/8], scales bf16 [N][K/128], zeros i32 [N][K/128].
- * clipped (nullable) u8 [N][K]: 1 where rint(w/s)+z fell outside [0, 15]. */
-int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
-                      int32_t* zeros, uint8_t* clipped) {
+/* Symmetric INT4 ("Quantization I: int8, int4, the basics", Concept: a real
+ * value becomes an integer code through a scale alone; a zero point is what
+ * the affine variants add).  The formula did not survive in the page's text;
+ * the reading implemented is the plainest one for signed 4-bit codes:
+ *   m = max |w| over the group; s = bf16_rne(m / 7)
+ *       (if s == 0: s = bf16_rne(m); if still 0: s = 1)
+ *   q = clamp(rint(w / s), -8, 7)
+ * In the packed container the signed code q is the nibble q + 8 with the zero
+ * point 8, so (nibble - z) * s = q * s and every consumer of the affine format
+ * reads a symmetric weight unchanged. */
+static int orc_quantize_group_sym(const float* w, int64_t G, uint16_t* s_out, int32_t* z_out, uint8_t* q_out,
+                                  uint8_t* clipped) {
+    double m = 0.0;
+    for (int64_t i = 0; i < G; ++i) {
+        if (!isfinite(w[i])) return ORC_ERR_NONFINITE;
+        if (fabs((double)w[i]) > m) m = fabs((double)w[i]);
+    }
+    uint16_t sb = orc_bf16_round(m / 7.0);
+    if (orc_bf16_value(sb) == 0.0) {
+        sb = orc_bf16_round(m);
+        if (orc_bf16_value(sb) == 0.0) sb = 0x3F80; /* 1.0 */
+    }
+    double s = orc_bf16_value(sb);
+    for (int64_t i = 0; i < G; ++i) {
+        double q = nearbyint((double)w[i] / s);
+        int clip = (q < -8.0) || (q > 7.0);
+        if (q < -8.0) q = -8.0;
+        if (q > 7.0) q = 7.0;
+        q_out[i] = (uint8_t)(q + 8.0);
+        if (clipped) clipped[i] = (uint8_t)clip;
+    }
+    *s_out = sb;
+    *z_out = 8;
+    return ORC_OK;
+}
+
+typedef int (*orc_group_quantiser)(const float*, int64_t, uint16_t*, int32_t*, uint8_t*, uint8_t*);
+
+/* Quantise every group of W with `quantise_group` and pack the codes. */
+static int orc_quantize_pack_groups(orc_group_quantiser quantise_group, const float* W, int64_t N, int64_t K,
+                                    uint32_t* qweight, uint16_t* scales, int32_t* zeros, uint8_t* clipped) {
     if (!W || !qweight || !scales || !zeros || N < 1 || K < 1) return ORC_ERR_ARG;
     if (K % ORC_G) return ORC_ERR_SHAPE;
     const int64_t ng = K / ORC_G;
@@ -146,7 +184,7 @@ int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, u
         for (int64_t g = 0; g < ng; ++g) {
             const float* w = W + n * K + g * ORC_G;
             uint8_t* cl = clipped ? clipped + n * K + g * ORC_G : NULL;
-            int st = orc_quantize_group(w, ORC_G, &scales[n * ng + g], &zeros[n * ng + g], q, cl);
+            int st = quantise_group(w, ORC_G, &scales[n * ng + g], &zeros[n * ng + g], q, cl);
             if (st != ORC_OK) {
 #pragma omp critical
                 { if (status == ORC_OK) status = st; }
@@ -162,6 +200,20 @@ int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, u
         }
     }
     return status;
+}
+
+/* W fp32 [N][K] -> qweight u32 [N][K/8], scales bf16 [N][K/128], zeros i32 [N][K/128].
+ * clipped (nullable) u8 [N][K]: 1 where rint(w/s)+z fell outside [0, 15]. */
+int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
+                      int32_t* zeros, uint8_t* clipped) {
+    return orc_quantize_pack_groups(orc_quantize_group, W, N, K, qweight, scales, zeros, clipped);
+}
+
+/* Symmetric variant, same outputs; every zero point is 8.
+ * clipped (nullable) u8 [N][K]: 1 where rint(w/s) fell outside [-8, 7]. */
+int orc_quantize_pack_sym(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
+                          int32_t* zeros, uint8_t* clipped) {
+    return orc_quantize_pack_groups(orc_quantize_group_sym, W, N, K, qweight, scales, zeros, clipped);
 }
 
 /* qweight -> codes u8 [N][K]. */
