@@ -64,6 +64,10 @@ def lib():
         L.orc_linear.restype = None
         L.orc_linear_sampled.argtypes = [vp, i64, i64, vp, vp, vp, i64, vp, i64, vp, i64, vp]
         L.orc_linear_sampled.restype = None
+        L.orc_awq_scale_weights.argtypes = [vp, vp, i64, i64, vp]
+        L.orc_awq_scale_weights.restype = None
+        L.orc_awq_scale_activations.argtypes = [vp, vp, i64, i64, vp]
+        L.orc_awq_scale_activations.restype = None
         L.orc_renorm.argtypes = [vp, i64, i64, vp, vp]
         L.orc_renorm.restype = None
         _lib = L
@@ -182,3 +186,25 @@ def renorm(y_bits: np.ndarray):
     exact = np.zeros((M, N), dtype=np.float64)
     lib().orc_renorm(_p(y_bits), M, N, _p(out), _p(exact))
     return out, exact
+
+
+def awq_scale_weights(W: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """AWQ transform of the weights: W'[n, k] = fp32(W[n, k] * s[k])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    s = np.ascontiguousarray(s, dtype=np.float32)
+    N, K = W.shape
+    assert s.shape == (K,)
+    out = np.empty_like(W)
+    lib().orc_awq_scale_weights(_p(W), _p(s), N, K, _p(out))
+    return out
+
+
+def awq_scale_activations(X: np.ndarray, r: np.ndarray) -> np.ndarray:
+    """AWQ transform of the activations: X'[m, k] = bf16(X[m, k] * r[k]) (bits in, bits out)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    M, K = X.shape
+    assert r.shape == (K,)
+    out = np.empty_like(X)
+    lib().orc_awq_scale_activations(_p(X), _p(r), M, K, _p(out))
+    return out

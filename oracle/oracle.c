@@ -27,14 +27,17 @@
  *   z  = rint(-lo / s)                            (ties to even, not clamped)
  *   q  = clamp(rint(w / s) + z, 0, 15)
  * using the stored BF16 scale for z and q so the stored parameters reproduce
- * the codes.  The symmetric variant (orc_quantize_pack_sym) is documented at
- * its definition.  Codes are packed 8 per uint32 word, lowest K index in the lowest
+ * the codes.  The symmetric variant (orc_quantize_pack_sym) and the AWQ
+ * equivalence transform (orc_awq_scale_*) are documented at their definitions.  Codes are packed 8 per uint32 word, lowest K index in the lowest
  * nibble.  Group index runs along K, per output row n.
  *
  * Parity status: quantise/pack/unpack/dequant (both variants) are pinned by
  * hand-worked groups, tie cases, grid round trips, brute force and invariants; the matmul by a library
  * FP64 matmul of the dequantised weights and one-hot/constant inputs; the
- * row renormalisation by its closed form (unit RMS) on tiny inputs.
+ * row renormalisation by its closed form (unit RMS) on tiny inputs; the AWQ
+ * transform by exact power-of-two equivalence, the rounding bounds of its one
+ * rounding per element, and the error reduction the pages claim for salient
+ * channels.
  */
 #include <math.h>
 #include <stdint.h>
@@ -214,6 +217,27 @@ int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, u
 int orc_quantize_pack_sym(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
                           int32_t* zeros, uint8_t* clipped) {
     return orc_quantize_pack_groups(orc_quantize_group_sym, W, N, K, qweight, scales, zeros, clipped);
+}
+
+/* AWQ equivalence transform ("Axe Corsa 28B" model card, "How the Compression
+ * Works", Stage 1; "Weight-Only Quantization and Mixed Precision", section 3):
+ * input channel k of the weight matrix is multiplied by s_k and the same
+ * channel of the activations by s_k^-1, which leaves X W^T unchanged in exact
+ * arithmetic while moving the salient channels onto a finer part of the
+ * quantisation grid.  The scales are inputs here (the calibration that picks
+ * them is not part of this layer).
+ * W'[n][k] = w[n][k] * s[k], the exact binary64 product rounded once to binary32. */
+void orc_awq_scale_weights(const float* W, const float* s, int64_t N, int64_t K, float* W_out) {
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) W_out[n * K + k] = (float)((double)W[n * K + k] * (double)s[k]);
+}
+
+/* X'[m][k] = x[m][k] * r[k] rounded once to BF16 (nearest, ties to even), with
+ * r[k] the inverse scale as the caller stores it (binary32): the exact product
+ * of a BF16 and a binary32 value fits binary64. */
+void orc_awq_scale_activations(const uint16_t* X, const float* r, int64_t M, int64_t K, uint16_t* X_out) {
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) X_out[m * K + k] = orc_bf16_round(orc_bf16_value(X[m * K + k]) * (double)r[k]);
 }
 
 /* qweight -> codes u8 [N][K]. */
