@@ -756,6 +756,80 @@ def run_comparators(which: str):
             torch.cuda.empty_cache()
 
 
+def awq_channel_scales(K: int, seed: int = 42):
+    """Synthetic AWQ scales: s_k = mean|x_k|^(1/2) over a seeded 64-token calibration batch
+    (salient channels included), normalised to geometric mean 1; r = fp32(1 / s)."""
+    xb = synth.activations_bf16(seed, 64, K)
+    xf = (xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    s = np.sqrt(np.abs(xf).mean(axis=0))
+    s /= np.exp(np.log(s).mean())
+    s = s.astype(np.float32)
+    return s, (1.0 / s.astype(np.float64)).astype(np.float32)
+
+
+def run_variants(which: str):
+    """Weight formats and the AWQ fold on the fused kernels, one JSON line per layer: the
+    affine layer, the same kernels on symmetric-packed weights (zero point 8), and
+    w4a16_linear_awq (activation scaling formed in the kernels' X preparation, weights from
+    w4a16_quantize_pack_awq); device time per call, each call reading a different copy of the
+    weights past L2, replayed from a CUDA graph."""
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    w4.load()
+    stream = torch.cuda.Stream()
+    sets = {"decode": workloads.decode_5120(), "small_batch": workloads.small_batch_8192(),
+            "prefill": workloads.prefill_8192(ms=[4096])}
+    names = list(sets) if which == "all" else which.split(",")
+    for wl in names:
+        for c in sets[wl]:
+            s, r = awq_channel_scales(c.K)
+            s_dev, r_dev = torch.from_numpy(s).cuda(), torch.from_numpy(r).cuda()
+            copies = max(1, min(16, -(-3 * L2_BYTES // c.code_bytes)))
+            W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
+            synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+            packed = {}
+            with torch.cuda.stream(stream):
+                packed["affine"] = [w4.PackedWeight.from_float(W, stream=stream) for _ in range(copies)]
+                packed["symmetric"] = [w4.PackedWeight.from_float(W, stream=stream, symmetric=True)
+                                       for _ in range(copies)]
+                awq = []
+                for _ in range(copies):
+                    pw = w4.PackedWeight(c.N, c.K)
+                    pw.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+                    w4.quantize_pack_awq(W, s_dev, pw.qweight, pw.scales, pw.zeros, pw.status, stream)
+                    awq.append(pw)
+                packed["awq"] = awq
+            torch.cuda.synchronize()
+            del W
+            if any(int(pw.status.item()) != 0 for v in packed.values() for pw in v):
+                raise RuntimeError(f"packing failed for {c.name}")
+            xb = synth.activations_bf16(c.x_seed, c.M, c.K)
+            X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+            ws = torch.zeros(max(w4.workspace_bytes(c.M, c.N, c.K), 256), dtype=torch.uint8, device="cuda")
+            passes = max(1, -(-200 // copies)) if c.M < 512 else 1
+            us = {}
+            for kind, pws in packed.items():
+                def body(pws=pws, kind=kind):
+                    for _ in range(passes):
+                        for pw in pws:
+                            if kind == "awq":
+                                w4.linear_awq(X, r_dev, pw.qweight, pw.scales, pw.zeros, Y, ws)
+                            else:
+                                w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y, ws)
+                us[kind] = _time_graph(torch, stream, body, passes * copies)
+            line = {"variants": c.workload, "layer": c.name, "M": c.M, "K": c.K, "N": c.N,
+                    "affine_us": us["affine"], "symmetric_us": us["symmetric"], "awq_us": us["awq"],
+                    "awq_over_affine": us["awq"] / us["affine"], "fault": w4.device_fault()}
+            if c.M >= PREFILL_MIN_M:
+                line.update({k + "_tflops": c.flops / v / 1e6 for k, v in us.items()})
+            else:
+                line.update({k + "_code_gbs": c.code_bytes / v / 1e3 for k, v in us.items()})
+            print(json.dumps(line), flush=True)
+            del packed, awq, X, Y, ws
+            torch.cuda.empty_cache()
+
+
 def run_sweep(which: str):
     """Per-layer device time of every workload shape (one JSON line each): each
     call reads a different copy of the packed weights, rotating through enough
@@ -804,11 +878,17 @@ def main():
     ap.add_argument("--comparators", default=None,
                     help="decode|prefill|all: the unfused pipelines (offline dequant + GEMM, naive three kernels) "
                          "timed beside the fused path, one JSON line per layer")
+    ap.add_argument("--variants", default=None,
+                    help="decode|small_batch|prefill|all: affine, symmetric-packed and AWQ-folded layers timed "
+                         "on the same kernels, one JSON line per layer")
     ap.add_argument("--sweep", default=None,
                     help="all, or a comma list of single_gemv, decode, small, prefill: per-layer times, one line each")
     args = ap.parse_args()
     if args.comparators:
         run_comparators(args.comparators)
+        return
+    if args.variants:
+        run_variants(args.variants)
         return
     if args.sweep:
         run_sweep(args.sweep)

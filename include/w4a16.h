@@ -95,6 +95,24 @@ W4A16_API int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t
                         int32_t* zeros, int32_t* dev_status, void* stream);
 
 /*
+ * Symmetric INT4 quantise and pack ("Quantization I: int8, int4, the basics",
+ * Concept: a real value maps to an integer code through a scale alone, with
+ * no zero point).  The page's formula did not survive extraction; the reading
+ * implemented, per row n and group g of 128 along K, in binary64:
+ *   m = max |w| over the group; s = bf16_rne(m / 7)
+ *   (if s == 0: s = bf16_rne(m); if still 0: s = 1)
+ *   q = clamp(rint(w / s), -8, 7)   (ties to even; BF16 rounding of s keeps
+ *                                    |w / s| < 7.5, so nothing clips)
+ * The signed code is stored as the nibble q + 8 and every zero point is 8, so
+ * the result is an ordinary packed weight: (nibble - z) * s = q * s, and
+ * w4a16_linear, w4a16_dequant and the other consumers take it unchanged.
+ * Arguments, layouts, ownership and errors as for w4a16_quantize_pack
+ * (W4A16_ERR_ZERO_RANGE cannot occur).
+ */
+W4A16_API int w4a16_quantize_pack_sym(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
+                            int32_t* zeros, int32_t* dev_status, void* stream);
+
+/*
  * Bytes of device workspace w4a16_linear() needs for this shape (0 if none).
  * The workspace starts with a 256 KB area of split-K arrival counters, then
  * holds prepared activations and FP32 split-K partial sums.  The counter area
@@ -130,6 +148,40 @@ W4A16_API int w4a16_linear(const uint16_t* X, int64_t M, int64_t K, const uint32
 W4A16_API int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
                       const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
                       int path, void* stream);
+
+/*
+ * AWQ equivalence transform ("Axe Corsa 28B" model card, "How the Compression
+ * Works", Stage 1; "Weight-Only Quantization and Mixed Precision", section 3):
+ * input channel k of the weight matrix is multiplied by s_k before
+ * quantisation and the same channel of the activations by s_k^-1, so the
+ * product is unchanged in exact arithmetic while the salient channels (large
+ * activations, s_k > 1) land on a finer part of the 4-bit grid.  Choosing s
+ * (calibration) is the caller's; both entries take it as data.
+ *
+ * w4a16_quantize_pack_awq: quantise and pack W'[n][k] = w[n][k] * s[k], the
+ * product rounded once to FP32, exactly as w4a16_quantize_pack would quantise
+ * a W' given directly (asymmetric, group 128).
+ *   s     device, fp32 [K], 16-byte aligned (finite, positive)
+ *   other arguments, errors: as w4a16_quantize_pack (a product that overflows
+ *   to infinity reports W4A16_ERR_NONFINITE).
+ */
+W4A16_API int w4a16_quantize_pack_awq(const float* W, const float* s, int64_t N, int64_t K, uint32_t* qweight,
+                            uint16_t* scales, int32_t* zeros, int32_t* dev_status, void* stream);
+
+/*
+ * w4a16_linear_awq: Y = X' W_hat'^T with X'[m][k] = bf16(x[m][k] * inv_s[k])
+ * (the exact product rounded once to BF16, nearest, ties to even) formed
+ * inside each kernel family's own preparation of X -- no separate pass over X
+ * and no X' in memory -- and W_hat' the packed weights of
+ * w4a16_quantize_pack_awq.  Where a preceding layer already produces X'
+ * (the inverse folded into its weights), call w4a16_linear instead.
+ *   inv_s device, fp32 [K], 16-byte aligned: the inverse scales as the caller
+ *         rounded them (typically fp32(1 / s[k]))
+ *   other arguments, errors: as w4a16_linear_path (path = enum w4a16_path).
+ */
+W4A16_API int w4a16_linear_awq(const uint16_t* X, const float* inv_s, int64_t M, int64_t K, const uint32_t* qweight,
+                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                     size_t workspace_bytes, int path, void* stream);
 
 /*
  * The linear layer on host buffers: one call enqueues, on `stream`, the copy

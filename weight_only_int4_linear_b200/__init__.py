@@ -46,10 +46,13 @@ SIGNATURES = {
     "w4a16_status_string": (ctypes.c_char_p, [_int]),
     "w4a16_version": (_int, []),
     "w4a16_quantize_pack": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_quantize_pack_sym": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "w4a16_workspace_init": (_int, [_vp, _sz, _vp]),
     "w4a16_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "w4a16_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
+    "w4a16_linear_awq": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
+    "w4a16_quantize_pack_awq": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
     "w4a16_linear_host": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "w4a16_unpack": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_dequant": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
@@ -119,17 +122,19 @@ def _dev(t: torch.Tensor, name: str, dtype, shape=None) -> int:
 
 
 def quantize_pack(W: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
-                  dev_status: torch.Tensor, stream=None) -> None:
-    """w4a16_quantize_pack: W fp32 [N, K] -> qweight int32 [N, K/8], scales bf16 [N, K/128],
-    zeros int32 [N, K/128]; dev_status int32 [1] receives device-detected data errors."""
+                  dev_status: torch.Tensor, stream=None, symmetric: bool = False) -> None:
+    """w4a16_quantize_pack (w4a16_quantize_pack_sym when symmetric): W fp32 [N, K] ->
+    qweight int32 [N, K/8], scales bf16 [N, K/128], zeros int32 [N, K/128];
+    dev_status int32 [1] receives device-detected data errors."""
     N, K = W.shape
-    st = load().w4a16_quantize_pack(
+    name = "w4a16_quantize_pack_sym" if symmetric else "w4a16_quantize_pack"
+    st = getattr(load(), name)(
         _dev(W, "W", torch.float32), N, K,
         _dev(qweight, "qweight", torch.int32, (N, K // 8)),
         _dev(scales, "scales", torch.bfloat16, (N, K // GROUP)),
         _dev(zeros, "zeros", torch.int32, (N, K // GROUP)),
         _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream))
-    _check("w4a16_quantize_pack", st)
+    _check(name, st)
 
 
 def workspace_bytes(M: int, N: int, K: int) -> int:
@@ -157,6 +162,39 @@ def linear(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, zeros: 
         _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N,
         _dev(Y, "Y", torch.bfloat16, (M, N)), ws_ptr, ws_bytes, path, _stream(stream))
     _check("w4a16_linear", st)
+
+
+def linear_awq(X: torch.Tensor, inv_s: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+               zeros: torch.Tensor, Y: torch.Tensor, workspace: torch.Tensor | None = None, path: int = PATH_AUTO,
+               stream=None) -> None:
+    """w4a16_linear_awq: Y = bf16(X * inv_s) . W_hat'^T, the activation scaling formed where the
+    kernels prepare X; qweight/scales/zeros from quantize_pack_awq."""
+    M, K = X.shape
+    N = qweight.shape[0]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace", torch.uint8)
+        ws_bytes = workspace.numel()
+    st = load().w4a16_linear_awq(
+        _dev(X, "X", torch.bfloat16), _dev(inv_s, "inv_s", torch.float32, (K,)), M, K,
+        _dev(qweight, "qweight", torch.int32, (N, K // 8)),
+        _dev(scales, "scales", torch.bfloat16, (N, K // GROUP)),
+        _dev(zeros, "zeros", torch.int32, (N, K // GROUP)), N,
+        _dev(Y, "Y", torch.bfloat16, (M, N)), ws_ptr, ws_bytes, path, _stream(stream))
+    _check("w4a16_linear_awq", st)
+
+
+def quantize_pack_awq(W: torch.Tensor, s: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor,
+                      zeros: torch.Tensor, dev_status: torch.Tensor, stream=None) -> None:
+    """w4a16_quantize_pack_awq: quantise and pack fp32(W * s) (s per input channel, [K])."""
+    N, K = W.shape
+    st = load().w4a16_quantize_pack_awq(
+        _dev(W, "W", torch.float32), _dev(s, "s", torch.float32, (K,)), N, K,
+        _dev(qweight, "qweight", torch.int32, (N, K // 8)),
+        _dev(scales, "scales", torch.bfloat16, (N, K // GROUP)),
+        _dev(zeros, "zeros", torch.int32, (N, K // GROUP)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream))
+    _check("w4a16_quantize_pack_awq", st)
 
 
 def _host(t: torch.Tensor, name: str, shape) -> int:
@@ -264,9 +302,10 @@ class PackedWeight:
         self.zeros = torch.empty((N, K // GROUP), dtype=torch.int32, device=device)
 
     @classmethod
-    def from_float(cls, W: torch.Tensor, stream=None) -> "PackedWeight":
+    def from_float(cls, W: torch.Tensor, stream=None, symmetric: bool = False) -> "PackedWeight":
         """Pack W on `stream` (a torch.cuda.Stream, or None for the current one);
-        the status word is cleared on that stream before the kernel runs."""
+        the status word is cleared on that stream before the kernel runs.
+        symmetric=True quantises without a zero point (stored zero points are 8)."""
         N, K = W.shape
         if stream is None:
             stream = torch.cuda.current_stream(W.device)
@@ -275,7 +314,7 @@ class PackedWeight:
         with torch.cuda.stream(stream):
             pw = cls(N, K, device=W.device)
             status = torch.zeros(1, dtype=torch.int32, device=W.device)
-            quantize_pack(W, pw.qweight, pw.scales, pw.zeros, status, stream)
+            quantize_pack(W, pw.qweight, pw.scales, pw.zeros, status, stream, symmetric)
         pw.status = status
         return pw
 

@@ -78,16 +78,33 @@ const char* w4a16_status_string(int status) {
 
 int w4a16_version(void) { return 100; }
 
-int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
-                        int32_t* dev_status, void* stream) {
+static int quantize_pack_entry(const float* W, const float* col_scale, int64_t N, int64_t K, uint32_t* qweight,
+                               uint16_t* scales, int32_t* zeros, int32_t* dev_status, bool symmetric, void* stream) {
     if (!W || !qweight || !scales || !zeros || !dev_status) return W4A16_ERR_ARG;
     int st = check_shape(1, N, K);
     if (st != W4A16_OK) return st;
     if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
-        (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+        (col_scale && !aligned16(col_scale)) || (reinterpret_cast<uintptr_t>(dev_status) & 3u))
         return W4A16_ERR_ALIGN;
     if ((st = check_device()) != W4A16_OK) return st;
-    return launch_quantize_pack(W, N, K, qweight, scales, zeros, dev_status, (cudaStream_t)stream);
+    return launch_quantize_pack(W, col_scale, N, K, qweight, scales, zeros, dev_status, symmetric,
+                                (cudaStream_t)stream);
+}
+
+int w4a16_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
+                        int32_t* dev_status, void* stream) {
+    return quantize_pack_entry(W, nullptr, N, K, qweight, scales, zeros, dev_status, false, stream);
+}
+
+int w4a16_quantize_pack_sym(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
+                            int32_t* zeros, int32_t* dev_status, void* stream) {
+    return quantize_pack_entry(W, nullptr, N, K, qweight, scales, zeros, dev_status, true, stream);
+}
+
+int w4a16_quantize_pack_awq(const float* W, const float* s, int64_t N, int64_t K, uint32_t* qweight,
+                            uint16_t* scales, int32_t* zeros, int32_t* dev_status, void* stream) {
+    if (!s) return W4A16_ERR_ARG;
+    return quantize_pack_entry(W, s, N, K, qweight, scales, zeros, dev_status, false, stream);
 }
 
 size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -106,14 +123,15 @@ int w4a16_workspace_init(void* workspace, size_t bytes, void* stream) {
     return cudaMemsetAsync(workspace, 0, bytes, (cudaStream_t)stream) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
-int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
-                      const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
-                      int path, void* stream) {
+static int linear_entry(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+                        const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                        size_t workspace_bytes, int path, void* stream) {
     if (!X || !qweight || !scales || !zeros || !Y) return W4A16_ERR_ARG;
     if (path < W4A16_PATH_AUTO || path > W4A16_PATH_PREFILL) return W4A16_ERR_ARG;
     int st = check_shape(M, N, K);
     if (st != W4A16_OK) return st;
-    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y))
+    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y) ||
+        (xscale && !aligned16(xscale)))
         return W4A16_ERR_ALIGN;
     if ((st = check_device()) != W4A16_OK) return st;
     const bool prefill = path == W4A16_PATH_PREFILL || (path == W4A16_PATH_AUTO && M >= kPrefillMinM);
@@ -121,8 +139,22 @@ int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* q
     const size_t need = prefill ? prefill_workspace_bytes(M, K) : plan.workspace_bytes();
     if (need > 0 && (!workspace || workspace_bytes < need)) return W4A16_ERR_WORKSPACE;
     if (need > 0 && !aligned16(workspace)) return W4A16_ERR_ALIGN;
-    if (prefill) return launch_prefill(X, M, K, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
-    return launch_decode(X, M, K, qweight, scales, zeros, N, Y, workspace, plan, (cudaStream_t)stream);
+    if (prefill)
+        return launch_prefill(X, xscale, M, K, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
+    return launch_decode(X, xscale, M, K, qweight, scales, zeros, N, Y, workspace, plan, (cudaStream_t)stream);
+}
+
+int w4a16_linear_path(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                      const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                      int path, void* stream) {
+    return linear_entry(X, nullptr, M, K, qweight, scales, zeros, N, Y, workspace, workspace_bytes, path, stream);
+}
+
+int w4a16_linear_awq(const uint16_t* X, const float* inv_s, int64_t M, int64_t K, const uint32_t* qweight,
+                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                     size_t workspace_bytes, int path, void* stream) {
+    if (!inv_s) return W4A16_ERR_ARG;
+    return linear_entry(X, inv_s, M, K, qweight, scales, zeros, N, Y, workspace, workspace_bytes, path, stream);
 }
 
 int w4a16_linear(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,

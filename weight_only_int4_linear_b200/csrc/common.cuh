@@ -48,14 +48,42 @@ __device__ __forceinline__ uint16_t double_to_bf16_bits(double x) {
     return (uint16_t)(sign | r);
 }
 
+// AWQ activation transform of one element: BF16 x times the binary32 inverse
+// channel scale r, rounded once to BF16 (nearest, ties to even).  In FP32:
+// p = fl(x r) and, by an FMA, the residual e = x r - p, which is exact while
+// |p| >= 2^-100 (x r has at most 32 significant bits, so e has at most 9).
+// Rounding p again to BF16 gives the rounding of x r except when p lies
+// exactly halfway between two BF16 values; there the sign of e decides (e = 0
+// is a true tie).  Below 2^-100 that case takes the exact binary64 product.
+__device__ __forceinline__ uint32_t bf16_scaled(uint32_t xbits, float r) {
+    const float x = __uint_as_float(xbits << 16);
+    const float p = __fmul_rn(x, r);
+    const float e = __fmaf_rn(x, r, -p);
+    const uint32_t u = __float_as_uint(p);
+    if ((u & 0x7FFFFFFFu) >= 0x7F800000u) return (u >> 16) | ((u & 0x7FFFFFFFu) > 0x7F800000u ? 0x40u : 0u);
+    uint32_t hi = u >> 16;
+    const uint32_t lo = u & 0xFFFFu;
+    if (lo == 0x8000u) {
+        if ((u & 0x7F800000u) < (27u << 23)) return double_to_bf16_bits((double)x * (double)r);
+        hi += e != 0.f ? (((e > 0.f) == !(u >> 31)) ? 1u : 0u) : (hi & 1u);
+    } else if (lo > 0x8000u) {
+        hi += 1u;
+    }
+    return hi;
+}
+// The same for the two BF16 values of a 32-bit word (low half first along K).
+__device__ __forceinline__ uint32_t bf16x2_scaled(uint32_t pair, float r_lo, float r_hi) {
+    return bf16_scaled(pair & 0xFFFFu, r_lo) | (bf16_scaled(pair >> 16, r_hi) << 16);
+}
+
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace w4a16
 
 // Host-side launch helpers (defined in api.cu).
 namespace w4a16 {
-int launch_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
-                         int32_t* dev_status, cudaStream_t stream);
+int launch_quantize_pack(const float* W, const float* col_scale, int64_t N, int64_t K, uint32_t* qweight,
+                         uint16_t* scales, int32_t* zeros, int32_t* dev_status, bool symmetric, cudaStream_t stream);
 int launch_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, cudaStream_t stream);
 int launch_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
                    uint16_t* out, cudaStream_t stream);
@@ -84,14 +112,17 @@ struct DecodePlan {
     size_t workspace_bytes() const;
 };
 DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms);
-int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
-                  const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, const DecodePlan& plan,
-                  cudaStream_t stream);
+// xscale (nullable, [K] FP32): the AWQ activation transform, x -> bf16(x * xscale[k]), applied
+// where each path prepares X.
+int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+                  const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                  const DecodePlan& plan, cudaStream_t stream);
 int num_sms_current();
 
 // Prefill (tensor-core GEMM) path for large M.
 constexpr int64_t kPrefillMinM = 64;  // W4A16_PATH_AUTO switches to the GEMM at this many tokens
 size_t prefill_workspace_bytes(int64_t M, int64_t K);
-int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
-                   const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, cudaStream_t stream);
+int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                   cudaStream_t stream);
 }  // namespace w4a16

@@ -134,7 +134,9 @@ __device__ __forceinline__ uint4 permute_block(uint4 v) {
 
 // X -> Xp (each 8-block reordered (0,4,1,5,2,6,3,7)) and xsT[g][m] = sum of the group
 // (row stride Mp, a multiple of the 256-token tile so one bulk copy per group and tile reads it).
-__global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __restrict__ X, int M, int K, int Mp,
+// xscale (nullable): each x is first replaced by bf16(x * xscale[k]) (the AWQ activation transform).
+__global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __restrict__ X,
+                                                           const float* __restrict__ xscale, int M, int K, int Mp,
                                                            uint16_t* __restrict__ Xp, float* __restrict__ xsT) {
     pdl_launch_dependents();
     const int G = K / kGroup;
@@ -148,7 +150,13 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __res
         float sum = 0.f;
         if (active) {
             const int64_t off = (int64_t)m * K + (int64_t)g * kGroup + blk * 8;
-            const uint4 v = *reinterpret_cast<const uint4*>(X + off);
+            uint4 v = *reinterpret_cast<const uint4*>(X + off);
+            if (xscale) {
+                const float4* r = reinterpret_cast<const float4*>(xscale + (int64_t)g * kGroup + blk * 8);
+                const float4 r0 = __ldg(r), r1 = __ldg(r + 1);
+                v = make_uint4(bf16x2_scaled(v.x, r0.x, r0.y), bf16x2_scaled(v.y, r0.z, r0.w),
+                               bf16x2_scaled(v.z, r1.x, r1.y), bf16x2_scaled(v.w, r1.z, r1.w));
+            }
             *reinterpret_cast<uint4*>(Xp + off) = permute_block(v);
             sum = (bf16lo(v.x) + bf16hi(v.x)) + (bf16lo(v.y) + bf16hi(v.y)) + (bf16lo(v.z) + bf16hi(v.z)) +
                   (bf16lo(v.w) + bf16hi(v.w));
@@ -526,8 +534,9 @@ size_t prefill_workspace_bytes(int64_t M, int64_t K) {
     return kCounterBytes + align256p((size_t)M * K * 2) + align256p((size_t)(K / kGroup) * Mp * 4);
 }
 
-int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
-                   const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, cudaStream_t stream) {
+int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                   cudaStream_t stream) {
     static bool attr = false;
     if (!attr) {
         if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem) !=
@@ -549,7 +558,7 @@ int launch_prefill(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qwei
     if (pgrid > num_sms_current() * 16) pgrid = num_sms_current() * 16;
     const int Mp = (int)((M + kPBN - 1) / kPBN * kPBN);
     if (Mp > M && cudaMemsetAsync(xsT, 0, (size_t)G * Mp * 4, stream) != cudaSuccess) return W4A16_ERR_CUDA;
-    prefill_prep_kernel<<<pgrid, 256, 0, stream>>>(X, (int)M, (int)K, Mp, Xp, xsT);
+    prefill_prep_kernel<<<pgrid, 256, 0, stream>>>(X, xscale, (int)M, (int)K, Mp, Xp, xsT);
     if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
 
     PrefillArgs args;

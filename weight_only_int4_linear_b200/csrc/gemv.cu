@@ -20,6 +20,11 @@
 //   * 3 <= M <= 32 per launch: decode_tc_kernel, tcgen05.mma kind::i8 with the
 //     codes in tensor memory and the digit planes of all tokens as B;
 //   * prep_x8_kernel: the digit planes for the tensor-core kernel.
+// With AWQ inverse channel scales (the activation half of the equivalence
+// transform), X' = bf16(x * inv_s[k]) is formed where X is prepared: inside
+// prep_x8_kernel, and for M <= 2 by awq_prescale_kernel ahead of the integer
+// kernel, which then reads X' (doing it in the kernel's single X warp made
+// that warp the bottleneck).
 //
 // Work decomposition: a unit is 128 weight rows x one group (8 KB of codes).
 // Units are numbered row tile by row tile and dealt out to a persistent grid
@@ -143,9 +148,11 @@ __device__ __forceinline__ void umma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uin
 
 // One warp per (group g, token m < NTOK): lane l holds x at k = 4l .. 4l + 3 (word w = l / 2,
 // half h = l % 2).  Tokens m >= M get zero planes.
+// xscale (nullable): each x is first replaced by bf16(x * xscale[k]) (the AWQ activation transform).
 template <int NTOK>
-__global__ void __launch_bounds__(256) prep_x8_kernel(const uint16_t* __restrict__ X, int M, int K,
-                                                      uint8_t* __restrict__ planes, float* __restrict__ xs) {
+__global__ void __launch_bounds__(256) prep_x8_kernel(const uint16_t* __restrict__ X, const float* __restrict__ xscale,
+                                                      int M, int K, uint8_t* __restrict__ planes,
+                                                      float* __restrict__ xs) {
     pdl_launch_dependents();
     const int G = K / kGroup;
     const int lane = threadIdx.x & 31;
@@ -160,6 +167,13 @@ __global__ void __launch_bounds__(256) prep_x8_kernel(const uint16_t* __restrict
             bits[1] = v.x >> 16;
             bits[2] = v.y & 0xFFFFu;
             bits[3] = v.y >> 16;
+            if (xscale) {
+                const float4 r = __ldg(reinterpret_cast<const float4*>(xscale + (int64_t)g * kGroup + lane * 4));
+                bits[0] = bf16_scaled(bits[0], r.x);
+                bits[1] = bf16_scaled(bits[1], r.y);
+                bits[2] = bf16_scaled(bits[2], r.z);
+                bits[3] = bf16_scaled(bits[3], r.w);
+            }
         }
         uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
         amax = __reduce_max_sync(0xFFFFFFFFu, amax);
@@ -1022,18 +1036,38 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.max_slots = (int)((G - 1) / p.units_base + 2);
     // the CUDA-core kernel prepares X itself; the tensor-core kernel reads X digit planes and
     // per-token sums and scales prepared per launch
-    p.ws_xp_bytes = p.cc_tokens ? 0 : align256((size_t)G * 3 * p.nt * 128);
+    // the integer kernel reads X itself; its area holds X' = bf16(X * inv_s) for the AWQ entry
+    p.ws_xp_bytes = p.cc_tokens ? align256((size_t)M * K * 2) : align256((size_t)G * 3 * p.nt * 128);
     p.ws_xs_bytes = p.cc_tokens ? 0 : align256((size_t)G * 2 * p.nt * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
     p.ws_counter_bytes = align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
     return p;
 }
 
+// X' = bf16(x * xscale[k]) ahead of the integer kernel, 8 values per thread.  The dependent
+// layer kernel is released first, so it streams weights while this waits for X; its X warp
+// reads X' only after this grid has completed.
+__global__ void __launch_bounds__(256) awq_prescale_kernel(const uint16_t* __restrict__ X,
+                                                           const float* __restrict__ xscale, int64_t n8, int K,
+                                                           uint16_t* __restrict__ Xs) {
+    pdl_launch_dependents();
+    pdl_wait_primary();  // X may come from the preceding kernel
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const int k = (int)((i * 8) % K);
+        const uint4 v = reinterpret_cast<const uint4*>(X)[i];
+        const float4 r0 = __ldg(reinterpret_cast<const float4*>(xscale + k));
+        const float4 r1 = __ldg(reinterpret_cast<const float4*>(xscale + k + 4));
+        reinterpret_cast<uint4*>(Xs)[i] =
+            make_uint4(bf16x2_scaled(v.x, r0.x, r0.y), bf16x2_scaled(v.y, r0.z, r0.w),
+                       bf16x2_scaled(v.z, r1.x, r1.y), bf16x2_scaled(v.w, r1.z, r1.w));
+    }
+}
+
 size_t DecodePlan::workspace_bytes() const { return ws_xp_bytes + ws_xs_bytes + ws_partial_bytes + ws_counter_bytes; }
 
-int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
-                  const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, const DecodePlan& plan,
-                  cudaStream_t stream) {
+int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+                  const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                  const DecodePlan& plan, cudaStream_t stream) {
     CUtensorMap tq;
     if (!cached_tmap(0, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
     int* fault = fault_word();
@@ -1054,13 +1088,31 @@ int launch_decode(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweig
             int prep_grid = (int)ceil_div(prep_threads, 256);
             if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
             if (plan.nt == 16)
-                prep_x8_kernel<16><<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, planes, xs);
+                prep_x8_kernel<16><<<prep_grid, 256, 0, stream>>>(X + m0 * K, xscale, Mc, (int)K, planes, xs);
             else
-                prep_x8_kernel<32><<<prep_grid, 256, 0, stream>>>(X + m0 * K, Mc, (int)K, planes, xs);
+                prep_x8_kernel<32><<<prep_grid, 256, 0, stream>>>(X + m0 * K, xscale, Mc, (int)K, planes, xs);
             if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
         }
         DecodeArgs args;
         args.Xp = X + m0 * K;  // read by the CUDA-core kernel; the tensor-core kernel reads the planes
+        if (plan.cc_tokens && xscale) {
+            uint16_t* Xs = reinterpret_cast<uint16_t*>(planes);
+            const int64_t n8 = (int64_t)Mc * K / 8;
+            int pgrid = (int)ceil_div(n8, 256);
+            if (pgrid > num_sms_current()) pgrid = num_sms_current();
+            cudaLaunchConfig_t pcfg = {};
+            pcfg.gridDim = dim3((unsigned)pgrid);
+            pcfg.blockDim = dim3(256);
+            pcfg.stream = stream;
+            cudaLaunchAttribute pattr[1];
+            pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            pattr[0].val.programmaticStreamSerializationAllowed = 1;
+            pcfg.attrs = pattr;
+            pcfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&pcfg, awq_prescale_kernel, X + m0 * K, xscale, n8, (int)K, Xs) != cudaSuccess)
+                return W4A16_ERR_CUDA;
+            args.Xp = Xs;
+        }
         args.xs = xs;
         args.scales = scales;
         args.zeros = zeros;

@@ -95,5 +95,5 @@ extern "C" int w4a16_linear_noalloc(const uint16_t* X, int64_t M, int64_t K, con
     // the buffer keeps the previous call's contents: the arrival counters must start at zero
     // counters lead the layout; only this call's row tiles need clearing
     if (cudaMemsetAsync(scratch, 0, (size_t)plan.row_tiles * 4, s) != cudaSuccess) return W4A16_ERR_CUDA;
-    return launch_decode(X, M, K, qweight, scales, zeros, N, Y, scratch, plan, s);
+    return launch_decode(X, nullptr, M, K, qweight, scales, zeros, N, Y, scratch, plan, s);
 }

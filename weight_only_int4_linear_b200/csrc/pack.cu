@@ -4,7 +4,9 @@
 // Quantise + pack follows the "Axe Corsa 28B" model card, "How the Compression
 // Works" (asymmetric INT4, one scale and one zero point per 128 consecutive
 // weights, all 16 levels used) under the min/max affine reading documented in
-// include/w4a16.h.  Every decision that sets a code or a stored parameter is
+// include/w4a16.h; the symmetric variant ("Quantization I: int8, int4, the
+// basics", Concept: a scale and no zero point) stores signed codes as q + 8
+// with the zero point 8, so the linear kernels read both formats unchanged.  Every decision that sets a code or a stored parameter is
 // taken in binary64 with IEEE division and round-half-even, so the packed
 // output is bit-exact with any correct implementation of the same reading.
 #include "common.cuh"
@@ -12,7 +14,12 @@
 namespace w4a16 {
 
 // One warp per group of 128 weights: lane l holds w[4l .. 4l+3].
-__global__ void __launch_bounds__(256) quantize_pack_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+// kSym: s = bf16(max|w| / 7), q = clamp(rint(w / s), -8, 7) stored as q + 8, z = 8.
+// col_scale (nullable): the AWQ transform, w[n][k] * col_scale[k] rounded once to FP32, is
+// quantised in place of w.
+template <bool kSym>
+__global__ void __launch_bounds__(256) quantize_pack_kernel(const float* __restrict__ W,
+                                                            const float* __restrict__ col_scale, int64_t N, int64_t K,
                                                             uint32_t* __restrict__ qweight,
                                                             uint16_t* __restrict__ scales,
                                                             int32_t* __restrict__ zeros, int32_t* status) {
@@ -22,7 +29,11 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const float* __restr
     const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
     for (int64_t grp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; grp < total; grp += warps) {
         const int64_t n = grp / ng, g = grp % ng;
-        const float4 v = reinterpret_cast<const float4*>(W + n * K + g * kGroup)[lane];
+        float4 v = reinterpret_cast<const float4*>(W + n * K + g * kGroup)[lane];
+        if (col_scale) {
+            const float4 c = reinterpret_cast<const float4*>(col_scale + g * kGroup)[lane];
+            v = make_float4(__fmul_rn(v.x, c.x), __fmul_rn(v.y, c.y), __fmul_rn(v.z, c.z), __fmul_rn(v.w, c.w));
+        }
         const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
         if (!__all_sync(0xFFFFFFFFu, finite)) {
             if (lane == 0) {
@@ -40,13 +51,15 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const float* __restr
             lo = fminf(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
             hi = fmaxf(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
         }
-        uint16_t sb = double_to_bf16_bits(__ddiv_rn(__dsub_rn((double)hi, (double)lo), 15.0));
+        const double mag = fmax(fabs((double)lo), fabs((double)hi));
+        uint16_t sb = double_to_bf16_bits(kSym ? __ddiv_rn(mag, 7.0)
+                                               : __ddiv_rn(__dsub_rn((double)hi, (double)lo), 15.0));
         if ((sb & 0x7FFFu) == 0) {
-            sb = double_to_bf16_bits(fmax(fabs((double)lo), fabs((double)hi)));
+            sb = double_to_bf16_bits(mag);
             if ((sb & 0x7FFFu) == 0) sb = 0x3F80u;  // 1.0
         }
         const double s = (double)bf16_bits_to_float(sb);
-        const double z = rint(__ddiv_rn(-(double)lo, s));
+        const double z = kSym ? 8.0 : rint(__ddiv_rn(-(double)lo, s));
         if (z > 2147483647.0 || z < -2147483648.0) {
             if (lane == 0) {
                 atomicCAS(status, 0, (int)W4A16_ERR_ZERO_RANGE);
@@ -174,11 +187,15 @@ static int grid_for(int64_t items, int threads) {
     return (int)blocks;
 }
 
-int launch_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
-                         int32_t* dev_status, cudaStream_t stream) {
+int launch_quantize_pack(const float* W, const float* col_scale, int64_t N, int64_t K, uint32_t* qweight,
+                         uint16_t* scales, int32_t* zeros, int32_t* dev_status, bool symmetric, cudaStream_t stream) {
     if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), stream) != cudaSuccess) return W4A16_ERR_CUDA;
     const int64_t groups = N * (K / kGroup);
-    quantize_pack_kernel<<<grid_for(groups * 32, 256), 256, 0, stream>>>(W, N, K, qweight, scales, zeros, dev_status);
+    const int grid = grid_for(groups * 32, 256);
+    if (symmetric)
+        quantize_pack_kernel<true><<<grid, 256, 0, stream>>>(W, col_scale, N, K, qweight, scales, zeros, dev_status);
+    else
+        quantize_pack_kernel<false><<<grid, 256, 0, stream>>>(W, col_scale, N, K, qweight, scales, zeros, dev_status);
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
