@@ -68,6 +68,10 @@ def lib():
         L.orc_awq_scale_weights.restype = None
         L.orc_awq_scale_activations.argtypes = [vp, vp, i64, i64, vp]
         L.orc_awq_scale_activations.restype = None
+        L.orc_w8_quantize.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.orc_w8_quantize.restype = ctypes.c_int
+        L.orc_w8_linear.argtypes = [vp, i64, i64, vp, vp, i64, vp]
+        L.orc_w8_linear.restype = None
         L.orc_renorm.argtypes = [vp, i64, i64, vp, vp]
         L.orc_renorm.restype = None
         _lib = L
@@ -208,3 +212,27 @@ def awq_scale_activations(X: np.ndarray, r: np.ndarray) -> np.ndarray:
     out = np.empty_like(X)
     lib().orc_awq_scale_activations(_p(X), _p(r), M, K, _p(out))
     return out
+
+
+def w8_quantize(W: np.ndarray, with_clipped: bool = False):
+    """W float32 [N, K] -> (status, q int8 [N, K], scales bf16-bits u16 [N][, clipped u8 [N, K]]):
+    symmetric INT8, one scale per output row."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    q = np.zeros((N, K), dtype=np.int8)
+    sc = np.zeros(N, dtype=np.uint16)
+    cl = np.zeros((N, K), dtype=np.uint8) if with_clipped else None
+    st = lib().orc_w8_quantize(_p(W), N, K, _p(q), _p(sc), _p(cl) if cl is not None else None)
+    return (st, q, sc, cl) if with_clipped else (st, q, sc)
+
+
+def w8_linear(X: np.ndarray, q: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """X bf16 bits [M, K], q int8 [N, K], scales bf16 bits [N] -> Y float64 [M, N] (unrounded)."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    M, K = X.shape
+    N = q.shape[0]
+    Y = np.empty((M, N), dtype=np.float64)
+    lib().orc_w8_linear(_p(X), M, K, _p(q), _p(scales), N, _p(Y))
+    return Y

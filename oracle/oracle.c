@@ -27,8 +27,9 @@
  *   z  = rint(-lo / s)                            (ties to even, not clamped)
  *   q  = clamp(rint(w / s) + z, 0, 15)
  * using the stored BF16 scale for z and q so the stored parameters reproduce
- * the codes.  The symmetric variant (orc_quantize_pack_sym) and the AWQ
- * equivalence transform (orc_awq_scale_*) are documented at their definitions.  Codes are packed 8 per uint32 word, lowest K index in the lowest
+ * the codes.  The symmetric variant (orc_quantize_pack_sym), the AWQ
+ * equivalence transform (orc_awq_scale_*) and the INT8 per-channel weights of
+ * W8A16 (orc_w8_*) are documented at their definitions.  Codes are packed 8 per uint32 word, lowest K index in the lowest
  * nibble.  Group index runs along K, per output row n.
  *
  * Parity status: quantise/pack/unpack/dequant (both variants) are pinned by
@@ -238,6 +239,71 @@ void orc_awq_scale_weights(const float* W, const float* s, int64_t N, int64_t K,
 void orc_awq_scale_activations(const uint16_t* X, const float* r, int64_t M, int64_t K, uint16_t* X_out) {
     for (int64_t m = 0; m < M; ++m)
         for (int64_t k = 0; k < K; ++k) X_out[m * K + k] = orc_bf16_round(orc_bf16_value(X[m * K + k]) * (double)r[k]);
+}
+
+/* W8A16: INT8 weights against BF16 activations ("Weight-Only Quantization and
+ * Mixed Precision", section 5, the INT8-weight / 16-bit-activation row of the
+ * selection matrix, and section 8: INT8 needs no grouping; "Weight-Only
+ * Quantisation", Notes: weights stored in INT8 or INT4, activations and
+ * accumulation in higher precision).  The pages give no INT8 formula; the
+ * reading implemented is symmetric per output channel ("Quantization I: int8,
+ * int4, the basics", Concept: a scale and no zero point), per row n:
+ *   m = max_k |w[n][k]|; s = bf16_rne(m / 127)
+ *       (if s == 0: s = bf16_rne(m); if still 0: s = 1)
+ *   q = clamp(rint(w / s), -127, 127)
+ * and w_hat = q s.  clipped (nullable) u8 [N][K]: 1 where rint(w / s) fell
+ * outside [-127, 127]. */
+int orc_w8_quantize(const float* W, int64_t N, int64_t K, int8_t* q, uint16_t* scales, uint8_t* clipped) {
+    if (!W || !q || !scales || N < 1 || K < 1) return ORC_ERR_ARG;
+    int status = ORC_OK;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        const float* w = W + n * K;
+        double m = 0.0;
+        int finite = 1;
+        for (int64_t k = 0; k < K; ++k) {
+            if (!isfinite(w[k])) finite = 0;
+            else if (fabs((double)w[k]) > m) m = fabs((double)w[k]);
+        }
+        if (!finite) {
+#pragma omp critical
+            { if (status == ORC_OK) status = ORC_ERR_NONFINITE; }
+            memset(q + n * K, 0, (size_t)K);
+            scales[n] = 0;
+            continue;
+        }
+        uint16_t sb = orc_bf16_round(m / 127.0);
+        if (orc_bf16_value(sb) == 0.0) {
+            sb = orc_bf16_round(m);
+            if (orc_bf16_value(sb) == 0.0) sb = 0x3F80; /* 1.0 */
+        }
+        const double sv = orc_bf16_value(sb);
+        for (int64_t k = 0; k < K; ++k) {
+            double t = nearbyint((double)w[k] / sv);
+            int clip = (t < -127.0) || (t > 127.0);
+            if (t < -127.0) t = -127.0;
+            if (t > 127.0) t = 127.0;
+            q[n * K + k] = (int8_t)t;
+            if (clipped) clipped[n * K + k] = (uint8_t)clip;
+        }
+        scales[n] = sb;
+    }
+    return status;
+}
+
+/* Y[m][n] = sum_k x[m][k] * q[n][k] * s[n] in binary64 (unrounded); X is BF16
+ * bits [M][K], q int8 [N][K], scales BF16 bits [N]. */
+void orc_w8_linear(const uint16_t* X, int64_t M, int64_t K, const int8_t* q, const uint16_t* scales, int64_t N,
+                   double* Y) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        const double sv = orc_bf16_value(scales[n]);
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += orc_bf16_value(X[m * K + k]) * ((double)q[n * K + k] * sv);
+            Y[m * N + n] = acc;
+        }
+    }
 }
 
 /* qweight -> codes u8 [N][K]. */
