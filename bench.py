@@ -18,6 +18,7 @@ host cores as a CPU baseline.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -42,14 +43,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154224384 + dram__bytes_write.sum 4144384
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 154467840 + dram__bytes_write.sum 3280640
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "3a092f494e368178df4636f486048961c4f2b14d6188d7f5ab246b6132a32eb1",
-                                      "bytes": 158368768},
-    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1110778880 + write 454575872
+                                      "sha256": "bc06683cdc622171ecaebade07dcd0b65f720115eabae56e48b5e191760da7ec",
+                                      "bytes": 157748480},
+    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1110334976 + write 453940736
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
-                                          "sha256": "1eed7b053dbd1150188bcff11bcb6b10faf12c174186544dcacbb0a201dedc7f",
-                                          "bytes": 1565354752},
+                                          "sha256": "d4c1912d8becaa47d896b612c0d94f643d9e1e0a739372ec447659743f2ea05d",
+                                          "bytes": 1564275712},
 }
 
 
@@ -771,8 +772,8 @@ def run_variants(which: str):
     """Weight formats and the AWQ fold on the fused kernels, one JSON line per layer: the
     affine layer, the same kernels on symmetric-packed weights (zero point 8), and
     w4a16_linear_awq (activation scaling formed in the kernels' X preparation, weights from
-    w4a16_quantize_pack_awq); device time per call, each call reading a different copy of the
-    weights past L2, replayed from a CUDA graph."""
+    w4a16_quantize_pack_awq); device time per call (median of three rounds in rotated order),
+    each call reading a different copy of the weights past L2, replayed from a CUDA graph."""
     import torch
     import weight_only_int4_linear_b200 as w4
     w4.load()
@@ -808,16 +809,23 @@ def run_variants(which: str):
             Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
             ws = torch.zeros(max(w4.workspace_bytes(c.M, c.N, c.K), 256), dtype=torch.uint8, device="cuda")
             passes = max(1, -(-200 // copies)) if c.M < 512 else 1
-            us = {}
-            for kind, pws in packed.items():
-                def body(pws=pws, kind=kind):
-                    for _ in range(passes):
-                        for pw in pws:
-                            if kind == "awq":
-                                w4.linear_awq(X, r_dev, pw.qweight, pw.scales, pw.zeros, Y, ws)
-                            else:
-                                w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y, ws)
-                us[kind] = _time_graph(torch, stream, body, passes * copies)
+            # three rounds in rotated order, median per variant: under a sustained load the clock
+            # drifts down, which would otherwise favour whichever variant is timed first
+            samples = {kind: [] for kind in packed}
+            kinds = list(packed)
+            for rnd in range(3):
+                for kind in kinds[rnd:] + kinds[:rnd]:
+                    pws = packed[kind]
+
+                    def body(pws=pws, kind=kind):
+                        for _ in range(passes):
+                            for pw in pws:
+                                if kind == "awq":
+                                    w4.linear_awq(X, r_dev, pw.qweight, pw.scales, pw.zeros, Y, ws)
+                                else:
+                                    w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y, ws)
+                    samples[kind].append(_time_graph(torch, stream, body, passes * copies))
+            us = {kind: statistics.median(v) for kind, v in samples.items()}
             line = {"variants": c.workload, "layer": c.name, "M": c.M, "K": c.K, "N": c.N,
                     "affine_us": us["affine"], "symmetric_us": us["symmetric"], "awq_us": us["awq"],
                     "awq_over_affine": us["awq"] / us["affine"], "fault": w4.device_fault()}
@@ -828,6 +836,63 @@ def run_variants(which: str):
             print(json.dumps(line), flush=True)
             del packed, awq, X, Y, ws
             torch.cuda.empty_cache()
+
+
+def run_w8(which: str):
+    """W8A16 ("Weight-Only Quantization and Mixed Precision", sections 5 and 8: INT8 weights,
+    16-bit activations, no grouping) beside the W4A16 layer and a cuBLAS BF16 GEMM on the same
+    shapes, one JSON line per layer and token count: device time per call, each call reading a
+    different copy of the weights past L2, replayed from a CUDA graph.  The W8 roofline bytes are
+    N K code bytes + 2 N scale bytes (+ X and Y)."""
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    w4.load()
+    stream = torch.cuda.Stream()
+    ms = [int(m) for m in which.split(",")] if which not in ("decode", "all") else [1, 2]
+    for c in workloads.decode_5120():
+        w8_bytes = c.N * c.K + 2 * c.N
+        copies8 = max(1, min(16, -(-3 * L2_BYTES // w8_bytes)))
+        copies16 = max(1, min(16, -(-3 * L2_BYTES // (2 * c.N * c.K))))
+        W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
+        synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+        with torch.cuda.stream(stream):
+            p8 = [w4.PackedW8.from_float(W, stream) for _ in range(copies8)]
+            W16 = [W.to(torch.bfloat16) for _ in range(copies16)]
+        torch.cuda.synchronize()
+        del W
+        if any(int(p.status.item()) != 0 for p in p8):
+            raise RuntimeError(f"W8 quantisation failed for {c.name}")
+        for M in ms:
+            cm = dataclasses.replace(c, M=M)
+            xb = synth.activations_bf16(c.x_seed, M, c.K)
+            X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            Y = torch.empty((M, c.N), dtype=torch.bfloat16, device="cuda")
+            ws = torch.zeros(max(w4.w8_workspace_bytes(M, c.N, c.K), 256), dtype=torch.uint8, device="cuda")
+            passes8 = max(1, -(-200 // copies8))
+
+            def body8():
+                for _ in range(passes8):
+                    for p in p8:
+                        w4.w8_linear(X, p.qweight, p.scales, Y, ws)
+            us8 = _time_graph(torch, stream, body8, passes8 * copies8)
+            passes16 = max(1, -(-100 // copies16))
+
+            def body16():
+                for _ in range(passes16):
+                    for Wb in W16:
+                        torch.matmul(X, Wb.t(), out=Y)
+            us16 = _time_graph(torch, stream, body16, passes16 * copies16)
+            us4, _ = time_layer_alone(cm, torch, w4, stream)
+            line = {"w8a16": c.workload, "layer": c.name, "M": M, "K": c.K, "N": c.N,
+                    "w8_us": us8, "w8_gbs": (w8_bytes + 2 * M * (c.K + c.N)) / us8 / 1e3,
+                    "w8_frac_of_hbm": (w8_bytes + 2 * M * (c.K + c.N)) / us8 / 1e3 / load_peaks()[0]["hbm_gbs"],
+                    "bf16_cublas_us": us16, "w8_speedup_vs_bf16": us16 / us8,
+                    "w4_us": us4, "w4_speedup_vs_bf16": us16 / us4,
+                    "fault": w4.device_fault()}
+            print(json.dumps(line), flush=True)
+            del X, Y, ws
+        del p8, W16
+        torch.cuda.empty_cache()
 
 
 def run_sweep(which: str):
@@ -878,6 +943,9 @@ def main():
     ap.add_argument("--comparators", default=None,
                     help="decode|prefill|all: the unfused pipelines (offline dequant + GEMM, naive three kernels) "
                          "timed beside the fused path, one JSON line per layer")
+    ap.add_argument("--w8", default=None,
+                    help="decode, or a comma list of token counts: W8A16 layers timed beside W4A16 and a cuBLAS "
+                         "BF16 GEMM on the decode shapes, one JSON line each")
     ap.add_argument("--variants", default=None,
                     help="decode|small_batch|prefill|all: affine, symmetric-packed and AWQ-folded layers timed "
                          "on the same kernels, one JSON line per layer")
@@ -889,6 +957,9 @@ def main():
         return
     if args.variants:
         run_variants(args.variants)
+        return
+    if args.w8:
+        run_w8(args.w8)
         return
     if args.sweep:
         run_sweep(args.sweep)

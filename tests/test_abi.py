@@ -1,4 +1,4 @@
-"""The C-ABI library: it loads, exports every symbol include/w4a16.h declares,
+"""The C-ABI library: it loads, exports every symbol the headers under include/ declare,
 and rejects bad arguments on the host before touching a device.  No compute
 calls here (no GPU needed)."""
 import ctypes
@@ -22,9 +22,15 @@ def lib():
     return w4.load()
 
 
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
+
+
 def declared_functions():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"W4A16_API\s+[\w\s\*]+?\b(w4a16_\w+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        names |= set(re.findall(r"W4A16_API\s+[\w\s\*]+?\b(w[48]a16_\w+)\s*\(", open(h).read()))
+    return sorted(names)
 
 
 def test_header_declares_entry_points():
@@ -36,7 +42,7 @@ def test_header_declares_entry_points():
 
 def test_library_exports_every_declared_symbol(lib):
     out = subprocess.check_output(["nm", "-D", "--defined-only", w4.LIB_PATH]).decode()
-    exported = set(re.findall(r"\bT (w4a16_\w+)", out))
+    exported = set(re.findall(r"\bT (w[48]a16_\w+)", out))
     missing = [n for n in declared_functions() if n not in exported]
     assert not missing, f"declared but not exported: {missing}"
     for n in declared_functions():
@@ -47,7 +53,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_header_compiles_as_c(tmp_path):
     src = tmp_path / "t.c"
-    src.write_text('#include "w4a16.h"\nint main(void){return W4A16_OK + W4A16_PATH_AUTO;}\n')
+    src.write_text('#include "w4a16.h"\n#include "w8a16.h"\nint main(void){return W4A16_OK + W4A16_PATH_AUTO;}\n')
     subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-c",
                            str(src), "-o", str(tmp_path / "t.o")])
 
@@ -77,6 +83,13 @@ def test_host_validation_without_device(lib):
     assert lib.w4a16_unpack(P, 4, 128, U, None) == w4.ERR_ALIGN
     assert lib.w4a16_dequant(P, P, None, 4, 128, P, None) == w4.ERR_ARG
     assert lib.w4a16_renorm_rows(P, 0, 8, P, None) == w4.ERR_ARG
+    assert lib.w8a16_linear(None, 1, 128, P, P, 16, P, P, 1 << 20, None) == w4.ERR_ARG
+    assert lib.w8a16_linear(P, 1, 100, P, P, 16, P, P, 1 << 20, None) == w4.ERR_SHAPE
+    assert lib.w8a16_linear(P, 1, 128, U, P, 16, P, P, 1 << 20, None) == w4.ERR_ALIGN
+    assert lib.w8a16_quantize(P, 0, 128, P, P, P, None) == w4.ERR_ARG
+    assert lib.w8a16_quantize(P, 4, 128, P, P, None, None) == w4.ERR_ARG
+    assert lib.w8a16_dequant(P, U, 4, 128, P, None) == w4.ERR_ALIGN
+    assert lib.w8a16_workspace_bytes(1, 16, 100) == 0
     if not torch.cuda.is_available():
         # well-formed arguments reach the device check, which fails without a GPU
         assert lin(P, 1, 128, P, P, P, 16, P, None, 0, 0, None) == w4.ERR_DEVICE

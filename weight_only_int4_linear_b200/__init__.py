@@ -53,6 +53,10 @@ SIGNATURES = {
     "w4a16_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
     "w4a16_linear_awq": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
     "w4a16_quantize_pack_awq": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "w8a16_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "w8a16_dequant": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
+    "w8a16_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "w8a16_linear": (_int, [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "w4a16_linear_host": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "w4a16_unpack": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_dequant": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
@@ -195,6 +199,58 @@ def quantize_pack_awq(W: torch.Tensor, s: torch.Tensor, qweight: torch.Tensor, s
         _dev(zeros, "zeros", torch.int32, (N, K // GROUP)),
         _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream))
     _check("w4a16_quantize_pack_awq", st)
+
+
+def w8_quantize(W: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, dev_status: torch.Tensor,
+                stream=None) -> None:
+    """w8a16_quantize: W fp32 [N, K] -> qweight int8 [N, K], scales bf16 [N] (symmetric per row)."""
+    N, K = W.shape
+    st = load().w8a16_quantize(
+        _dev(W, "W", torch.float32), N, K, _dev(qweight, "qweight", torch.int8, (N, K)),
+        _dev(scales, "scales", torch.bfloat16, (N,)), _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream))
+    _check("w8a16_quantize", st)
+
+
+def w8_dequant(qweight: torch.Tensor, scales: torch.Tensor, W_hat: torch.Tensor, stream=None) -> None:
+    N, K = qweight.shape
+    st = load().w8a16_dequant(_dev(qweight, "qweight", torch.int8, (N, K)),
+                              _dev(scales, "scales", torch.bfloat16, (N,)), N, K,
+                              _dev(W_hat, "W_hat", torch.bfloat16, (N, K)), _stream(stream))
+    _check("w8a16_dequant", st)
+
+
+def w8_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(load().w8a16_workspace_bytes(M, N, K))
+
+
+def w8_linear(X: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, Y: torch.Tensor,
+              workspace: torch.Tensor, stream=None) -> None:
+    """w8a16_linear: Y[M, N] = X[M, K] . (q s)^T (BF16 out, FP32 accumulation)."""
+    M, K = X.shape
+    N = qweight.shape[0]
+    st = load().w8a16_linear(
+        _dev(X, "X", torch.bfloat16), M, K, _dev(qweight, "qweight", torch.int8, (N, K)),
+        _dev(scales, "scales", torch.bfloat16, (N,)), N, _dev(Y, "Y", torch.bfloat16, (M, N)),
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream))
+    _check("w8a16_linear", st)
+
+
+class PackedW8:
+    """Device buffers of one INT8 weight matrix (plumbing: allocation via torch)."""
+
+    def __init__(self, N: int, K: int, device="cuda"):
+        self.N, self.K = N, K
+        self.qweight = torch.empty((N, K), dtype=torch.int8, device=device)
+        self.scales = torch.empty((N,), dtype=torch.bfloat16, device=device)
+
+    @classmethod
+    def from_float(cls, W: torch.Tensor, stream=None) -> "PackedW8":
+        N, K = W.shape
+        pw = cls(N, K, device=W.device)
+        pw.status = torch.zeros(1, dtype=torch.int32, device=W.device)
+        w8_quantize(W, pw.qweight, pw.scales, pw.status, stream)
+        return pw
 
 
 def _host(t: torch.Tensor, name: str, shape) -> int:

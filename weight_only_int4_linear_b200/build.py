@@ -13,8 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libw4a16.so")
 OBJ_DIR = os.path.join(PKG, "_build")
-SOURCES = ["api.cu", "runtime.cu", "pack.cu", "gemv.cu", "gemm.cu", "noalloc.cu"]
-HEADERS = ["common.cuh", "sm100.cuh"]
+SOURCES = ["api.cu", "runtime.cu", "pack.cu", "gemv.cu", "gemm.cu", "noalloc.cu", "w8.cu"]
+HEADERS = ["common.cuh", "sm100.cuh", "decode_units.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -33,7 +33,7 @@ def _stale(target: str, deps) -> bool:
 
 def build(force: bool = False, verbose: bool = False) -> str:
     os.makedirs(OBJ_DIR, exist_ok=True)
-    headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", "w4a16.h")]
+    headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(ROOT, "include", h) for h in ("w4a16.h", "w8a16.h")]
     objs = []
     for src in SOURCES:
         path = os.path.join(CSRC, src)

@@ -5,6 +5,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "w8a16.h"
 
 namespace w4a16 {
 
@@ -216,6 +217,48 @@ int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, vo
     int st = check_device();
     if (st != W4A16_OK) return st;
     return launch_renorm(y, M, N, out, (cudaStream_t)stream);
+}
+
+int w8a16_quantize(const float* W, int64_t N, int64_t K, int8_t* qweight, uint16_t* scales, int32_t* dev_status,
+                   void* stream) {
+    if (!W || !qweight || !scales || !dev_status) return W4A16_ERR_ARG;
+    if (N < 1 || K < 1) return W4A16_ERR_ARG;
+    if (N > kMaxDim || K > kMaxDim) return W4A16_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+        return W4A16_ERR_ALIGN;
+    int st = check_device();
+    if (st != W4A16_OK) return st;
+    return launch_w8_quantize(W, N, K, qweight, scales, dev_status, (cudaStream_t)stream);
+}
+
+int w8a16_dequant(const int8_t* qweight, const uint16_t* scales, int64_t N, int64_t K, uint16_t* W_hat,
+                  void* stream) {
+    if (!qweight || !scales || !W_hat) return W4A16_ERR_ARG;
+    if (N < 1 || K < 1) return W4A16_ERR_ARG;
+    if (N > kMaxDim || K > kMaxDim) return W4A16_ERR_SHAPE;
+    if (!aligned16(qweight) || !aligned16(scales) || !aligned16(W_hat)) return W4A16_ERR_ALIGN;
+    int st = check_device();
+    if (st != W4A16_OK) return st;
+    return launch_w8_dequant(qweight, scales, N, K, W_hat, (cudaStream_t)stream);
+}
+
+size_t w8a16_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (check_shape(M, N, K) != W4A16_OK) return 0;
+    check_device();  // caches the SM count the plan depends on
+    return w8_workspace_bytes(M, N, K);
+}
+
+int w8a16_linear(const uint16_t* X, int64_t M, int64_t K, const int8_t* qweight, const uint16_t* scales, int64_t N,
+                 uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!X || !qweight || !scales || !Y) return W4A16_ERR_ARG;
+    int st = check_shape(M, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(Y)) return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    const size_t need = w8_workspace_bytes(M, N, K);
+    if (!workspace || workspace_bytes < need) return W4A16_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return W4A16_ERR_ALIGN;
+    return launch_w8(X, M, K, qweight, scales, N, Y, workspace, (cudaStream_t)stream);
 }
 
 }  // extern "C"

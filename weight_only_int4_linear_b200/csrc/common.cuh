@@ -125,4 +125,13 @@ size_t prefill_workspace_bytes(int64_t M, int64_t K);
 int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                    const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                    cudaStream_t stream);
+
+// W8A16: INT8 weights with one BF16 scale per row (w8.cu).
+size_t w8_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int launch_w8(const uint16_t* X, int64_t M, int64_t K, const int8_t* q, const uint16_t* scales, int64_t N,
+              uint16_t* Y, void* workspace, cudaStream_t stream);
+int launch_w8_quantize(const float* W, int64_t N, int64_t K, int8_t* q, uint16_t* scales, int32_t* status,
+                       cudaStream_t stream);
+int launch_w8_dequant(const int8_t* q, const uint16_t* scales, int64_t N, int64_t K, uint16_t* out,
+                      cudaStream_t stream);
 }  // namespace w4a16

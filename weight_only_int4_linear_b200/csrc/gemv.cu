@@ -32,6 +32,7 @@
 // of bytes.  A row tile split between CTAs is reduced by the last CTA to
 // finish it (arrival counter), summing the partials in a fixed order.
 #include "common.cuh"
+#include "decode_units.cuh"
 #include "sm100.cuh"
 
 #include <mutex>
@@ -57,28 +58,6 @@ struct DecodeArgs {
     int max_slots;
 };
 
-__device__ __forceinline__ int cta_of_unit(int64_t u, int base, int rem) {
-    const int64_t big = (int64_t)(base + 1) * rem;
-    if (u < big) return (int)(u / (base + 1));
-    return rem + (int)((u - big) / base);
-}
-
-// Walks units in order without a division per step: unit = (row tile, group).
-struct UnitCursor {
-    int tile, g;
-    __device__ __forceinline__ UnitCursor(int64_t u, int G) : tile((int)(u / G)), g((int)(u - (u / G) * G)) {}
-    __device__ __forceinline__ void next(int G) {
-        if (++g == G) {
-            g = 0;
-            ++tile;
-        }
-    }
-};
-
-// 2^e as FP32 for e in [-149, 127] (subnormal below -126).
-__device__ __forceinline__ float pow2f(int e) {
-    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
-}
 
 // --------------------------------------------------------------------------
 // Tensor-core decode kernel (tcgen05, 8-bit integer MMA), one persistent CTA
@@ -653,11 +632,6 @@ __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst,
     }
 }
 
-// All lanes wait; the warp gives up together if any lane's wait ran out.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, int parity, int* fault, int site) {
-    const bool ok = mbar_wait(bar, parity, fault, site);
-    return __all_sync(0xFFFFFFFFu, ok);
-}
 
 template <int NT>
 #ifndef W4A16_CC2_MIN_BLOCKS
@@ -1034,9 +1008,8 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.units_base = (int)(units / grid);
     p.units_rem = (int)(units % grid);
     p.max_slots = (int)((G - 1) / p.units_base + 2);
-    // the CUDA-core kernel prepares X itself; the tensor-core kernel reads X digit planes and
-    // per-token sums and scales prepared per launch
-    // the integer kernel reads X itself; its area holds X' = bf16(X * inv_s) for the AWQ entry
+    // the integer kernel reads X itself (its area holds X' = bf16(X * inv_s) for the AWQ entry);
+    // the tensor-core kernel reads X digit planes and per-token sums and scales prepared per launch
     p.ws_xp_bytes = p.cc_tokens ? align256((size_t)M * K * 2) : align256((size_t)G * 3 * p.nt * 128);
     p.ws_xs_bytes = p.cc_tokens ? 0 : align256((size_t)G * 2 * p.nt * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
