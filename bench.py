@@ -650,6 +650,27 @@ def run_profile(spec: str, repeats: int = 4):
     import weight_only_int4_linear_b200 as w4
     w4.load()
     wl, name = spec.split(":")
+    if wl == "w8":  # the W8A16 layer on a decode shape (hidden 5120, M = 1)
+        stream = torch.cuda.Stream()
+        for c in [c for c in workloads.decode_5120() if name in (c.name, "all")]:
+            W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
+            synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+            p8 = w4.PackedW8.from_float(W, stream)
+            xb = synth.activations_bf16(c.x_seed, c.M, c.K)
+            X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+            ws = torch.zeros(w4.w8_workspace_bytes(c.M, c.N, c.K), dtype=torch.uint8, device="cuda")
+            torch.cuda.synchronize()
+            del W
+            with torch.cuda.stream(stream):
+                for _ in range(repeats):
+                    w4.w8_linear(X, p8.qweight, p8.scales, Y, ws)
+            torch.cuda.synchronize()
+        fault = w4.device_fault()
+        print(json.dumps({"profiled": spec, "repeats": repeats, "fault": fault}))
+        if fault:
+            raise SystemExit(1)
+        return
     cases = {"decode": workloads.decode_5120(), "small": workloads.small_batch_8192(),
              "prefill": workloads.prefill_8192(ms=[4096])}[wl]
     chosen = cases if name == "all" else [c for c in cases if c.name == name]
@@ -938,7 +959,7 @@ def main():
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes per launch of the dominant kernel from an ncu capture of this build")
     ap.add_argument("--profile", default=None,
-                    help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096, decode:all): run it a few "
+                    help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096, decode:all, w8:gate_up): run it a few "
                          "times, untimed")
     ap.add_argument("--comparators", default=None,
                     help="decode|prefill|all: the unfused pipelines (offline dequant + GEMM, naive three kernels) "
