@@ -54,6 +54,12 @@ def lib():
         L.orc_quantize_pack.restype = ctypes.c_int
         L.orc_quantize_pack_sym.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.orc_quantize_pack_sym.restype = ctypes.c_int
+        L.orc_quantize_pack_g.argtypes = [vp, i64, i64, i64, ctypes.c_int, vp, vp, vp, vp]
+        L.orc_quantize_pack_g.restype = ctypes.c_int
+        L.orc_dequant_g.argtypes = [vp, vp, vp, i64, i64, i64, vp]
+        L.orc_dequant_g.restype = None
+        L.orc_linear_g.argtypes = [vp, i64, i64, vp, vp, vp, i64, i64, vp]
+        L.orc_linear_g.restype = None
         L.orc_unpack.argtypes = [vp, i64, i64, vp]
         L.orc_unpack.restype = None
         L.orc_dequant.argtypes = [vp, vp, vp, i64, i64, vp]
@@ -235,4 +241,42 @@ def w8_linear(X: np.ndarray, q: np.ndarray, scales: np.ndarray) -> np.ndarray:
     N = q.shape[0]
     Y = np.empty((M, N), dtype=np.float64)
     lib().orc_w8_linear(_p(X), M, K, _p(q), _p(scales), N, _p(Y))
+    return Y
+
+
+def quantize_pack_g(W: np.ndarray, group: int, symmetric: bool = False, with_clipped: bool = False):
+    """As quantize_pack with groups of `group` (32, 64 or 128) consecutive weights along K:
+    scales and zeros [N, K/group]."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    qw = np.zeros((N, K // 8), dtype=np.uint32)
+    sc = np.zeros((N, max(K // group, 1)), dtype=np.uint16)
+    z = np.zeros((N, max(K // group, 1)), dtype=np.int32)
+    cl = np.zeros((N, K), dtype=np.uint8) if with_clipped else None
+    st = lib().orc_quantize_pack_g(_p(W), N, K, group, int(symmetric), _p(qw), _p(sc), _p(z),
+                                   _p(cl) if cl is not None else None)
+    return (st, qw, sc, z, cl) if with_clipped else (st, qw, sc, z)
+
+
+def dequant_g(qweight, scales, zeros, K: int) -> np.ndarray:
+    """W_hat float64 [N, K]; the group size is K / scales.shape[1]."""
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    zeros = np.ascontiguousarray(zeros, dtype=np.int32)
+    N = qweight.shape[0]
+    out = np.zeros((N, K), dtype=np.float64)
+    lib().orc_dequant_g(_p(qweight), _p(scales), _p(zeros), N, K, K // scales.shape[1], _p(out))
+    return out
+
+
+def linear_g(X: np.ndarray, qweight, scales, zeros) -> np.ndarray:
+    """Y_ref float64 [M, N] (unrounded); the group size is K / scales.shape[1]."""
+    X = np.ascontiguousarray(X, dtype=np.uint16)
+    qweight = np.ascontiguousarray(qweight, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    zeros = np.ascontiguousarray(zeros, dtype=np.int32)
+    M, K = X.shape
+    N = qweight.shape[0]
+    Y = np.zeros((M, N), dtype=np.float64)
+    lib().orc_linear_g(_p(X), M, K, _p(qweight), _p(scales), _p(zeros), N, K // scales.shape[1], _p(Y))
     return Y

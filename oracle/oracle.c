@@ -47,7 +47,7 @@
 #include <omp.h>
 #endif
 
-#define ORC_G 128
+#define ORC_G 128 /* the format's group size; the _g entry points take 32, 64 or 128 */
 
 enum {
     ORC_OK = 0,
@@ -175,20 +175,26 @@ static int orc_quantize_group_sym(const float* w, int64_t G, uint16_t* s_out, in
 
 typedef int (*orc_group_quantiser)(const float*, int64_t, uint16_t*, int32_t*, uint8_t*, uint8_t*);
 
-/* Quantise every group of W with `quantise_group` and pack the codes. */
+/* Quantise every group of G consecutive weights of W with `quantise_group` and
+ * pack the codes.  G = 128 is the format of the model card; 32 and 64 are the
+ * smaller groups of "Quantization I: int8, int4, the basics", Concept (groups
+ * of 32-128 values) and "Weight-Only Quantization and Mixed Precision",
+ * section 8 (32/64/128), with the same per-group rule. */
 static int orc_quantize_pack_groups(orc_group_quantiser quantise_group, const float* W, int64_t N, int64_t K,
-                                    uint32_t* qweight, uint16_t* scales, int32_t* zeros, uint8_t* clipped) {
+                                    int64_t G, uint32_t* qweight, uint16_t* scales, int32_t* zeros,
+                                    uint8_t* clipped) {
     if (!W || !qweight || !scales || !zeros || N < 1 || K < 1) return ORC_ERR_ARG;
-    if (K % ORC_G) return ORC_ERR_SHAPE;
-    const int64_t ng = K / ORC_G;
+    if (G != 32 && G != 64 && G != 128) return ORC_ERR_ARG;
+    if (K % G) return ORC_ERR_SHAPE;
+    const int64_t ng = K / G;
     int status = ORC_OK;
 #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t n = 0; n < N; ++n) {
         uint8_t q[ORC_G];
         for (int64_t g = 0; g < ng; ++g) {
-            const float* w = W + n * K + g * ORC_G;
-            uint8_t* cl = clipped ? clipped + n * K + g * ORC_G : NULL;
-            int st = quantise_group(w, ORC_G, &scales[n * ng + g], &zeros[n * ng + g], q, cl);
+            const float* w = W + n * K + g * G;
+            uint8_t* cl = clipped ? clipped + n * K + g * G : NULL;
+            int st = quantise_group(w, G, &scales[n * ng + g], &zeros[n * ng + g], q, cl);
             if (st != ORC_OK) {
 #pragma omp critical
                 { if (status == ORC_OK) status = st; }
@@ -196,10 +202,10 @@ static int orc_quantize_pack_groups(orc_group_quantiser quantise_group, const fl
                 scales[n * ng + g] = 0;
                 zeros[n * ng + g] = 0;
             }
-            for (int j = 0; j < ORC_G / 8; ++j) {
+            for (int j = 0; j < G / 8; ++j) {
                 uint32_t word = 0;
                 for (int i = 0; i < 8; ++i) word |= ((uint32_t)q[8 * j + i]) << (4 * i);
-                qweight[n * (K / 8) + g * (ORC_G / 8) + j] = word;
+                qweight[n * (K / 8) + g * (G / 8) + j] = word;
             }
         }
     }
@@ -210,14 +216,21 @@ static int orc_quantize_pack_groups(orc_group_quantiser quantise_group, const fl
  * clipped (nullable) u8 [N][K]: 1 where rint(w/s)+z fell outside [0, 15]. */
 int orc_quantize_pack(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
                       int32_t* zeros, uint8_t* clipped) {
-    return orc_quantize_pack_groups(orc_quantize_group, W, N, K, qweight, scales, zeros, clipped);
+    return orc_quantize_pack_groups(orc_quantize_group, W, N, K, ORC_G, qweight, scales, zeros, clipped);
 }
 
 /* Symmetric variant, same outputs; every zero point is 8.
  * clipped (nullable) u8 [N][K]: 1 where rint(w/s) fell outside [-8, 7]. */
 int orc_quantize_pack_sym(const float* W, int64_t N, int64_t K, uint32_t* qweight, uint16_t* scales,
                           int32_t* zeros, uint8_t* clipped) {
-    return orc_quantize_pack_groups(orc_quantize_group_sym, W, N, K, qweight, scales, zeros, clipped);
+    return orc_quantize_pack_groups(orc_quantize_group_sym, W, N, K, ORC_G, qweight, scales, zeros, clipped);
+}
+
+/* Either quantiser with groups of G in {32, 64, 128}; scales and zeros [N][K/G]. */
+int orc_quantize_pack_g(const float* W, int64_t N, int64_t K, int64_t G, int symmetric, uint32_t* qweight,
+                        uint16_t* scales, int32_t* zeros, uint8_t* clipped) {
+    return orc_quantize_pack_groups(symmetric ? orc_quantize_group_sym : orc_quantize_group, W, N, K, G, qweight,
+                                    scales, zeros, clipped);
 }
 
 /* AWQ equivalence transform ("Axe Corsa 28B" model card, "How the Compression
@@ -312,13 +325,19 @@ void orc_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes) {
         for (int64_t k = 0; k < K; ++k) codes[n * K + k] = (uint8_t)((qweight[n * (K / 8) + k / 8] >> (4 * (k % 8))) & 15u);
 }
 
-/* Exact dequantised weight of one element: (q - z) * s, exact in binary64. */
+/* Exact dequantised weight of one element with groups of G: (q - z) * s, exact
+ * in binary64. */
+static double orc_w_hat_g(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t K,
+                          int64_t G, int64_t n, int64_t k) {
+    int64_t ng = K / G;
+    uint32_t q = (qweight[n * (K / 8) + k / 8] >> (4 * (k % 8))) & 15u;
+    int64_t g = k / G;
+    return ((double)q - (double)zeros[n * ng + g]) * orc_bf16_value(scales[n * ng + g]);
+}
+
 static double orc_w_hat(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t K,
                         int64_t n, int64_t k) {
-    int64_t ng = K / ORC_G;
-    uint32_t q = (qweight[n * (K / 8) + k / 8] >> (4 * (k % 8))) & 15u;
-    int64_t g = k / ORC_G;
-    return ((double)q - (double)zeros[n * ng + g]) * orc_bf16_value(scales[n * ng + g]);
+    return orc_w_hat_g(qweight, scales, zeros, K, ORC_G, n, k);
 }
 
 /* W_hat f64 [N][K]. */
@@ -327,6 +346,34 @@ void orc_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_t*
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k) W_hat[n * K + k] = orc_w_hat(qweight, scales, zeros, K, n, k);
+}
+
+/* W_hat f64 [N][K] with groups of G. */
+void orc_dequant_g(const uint32_t* qweight, const uint16_t* scales, const int32_t* zeros, int64_t N, int64_t K,
+                   int64_t G, double* W_hat) {
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) W_hat[n * K + k] = orc_w_hat_g(qweight, scales, zeros, K, G, n, k);
+}
+
+/* Y_ref [M][N] in binary64 with groups of G: the sum of x * w_hat over k,
+ * one group at a time. */
+void orc_linear_g(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                  const int32_t* zeros, int64_t N, int64_t G, double* Y) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t n = 0; n < N; ++n) {
+        double w[ORC_G];
+        for (int64_t m = 0; m < M; ++m) Y[m * N + n] = 0.0;
+        for (int64_t k0 = 0; k0 < K; k0 += G) {
+            for (int64_t t = 0; t < G; ++t) w[t] = orc_w_hat_g(qweight, scales, zeros, K, G, n, k0 + t);
+            for (int64_t m = 0; m < M; ++m) {
+                const uint16_t* x = X + m * K + k0;
+                double acc = 0.0;
+                for (int64_t t = 0; t < G; ++t) acc += orc_bf16_value(x[t]) * w[t];
+                Y[m * N + n] += acc;
+            }
+        }
+    }
 }
 
 /* W_hat rounded to BF16 (nearest, ties to even) [N][K]. */
