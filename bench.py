@@ -916,6 +916,53 @@ def run_w8(which: str):
         torch.cuda.empty_cache()
 
 
+def run_groups(which: str):
+    """Quantisation groups of 32, 64 and 128 weights on the decode shapes (hidden 5120, M = 1),
+    one JSON line per layer: device time per call (w4a16_linear_g), each call reading a different
+    copy of the packed weights past L2, replayed from a CUDA graph; GB/s of code bytes and of
+    all weight bytes (codes + 6 B of metadata per group)."""
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    w4.load()
+    stream = torch.cuda.Stream()
+    for c in workloads.decode_5120():
+        W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
+        synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
+        xb = synth.activations_bf16(c.x_seed, c.M, c.K)
+        X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+        Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
+        line = {"groups": c.workload, "layer": c.name, "M": c.M, "K": c.K, "N": c.N}
+        for group in (128, 64, 32):
+            wbytes = c.code_bytes + c.N * (c.K // group) * 6
+            copies = max(1, min(16, -(-3 * L2_BYTES // wbytes)))
+            pws = []
+            with torch.cuda.stream(stream):
+                for _ in range(copies):
+                    pw = w4.PackedWeight(c.N, c.K, group=group)
+                    pw.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+                    w4.quantize_pack_g(W, group, pw.qweight, pw.scales, pw.zeros, pw.status, stream=stream)
+                    pws.append(pw)
+            torch.cuda.synchronize()
+            if any(int(p.status.item()) != 0 for p in pws):
+                raise RuntimeError(f"packing failed for {c.name}, group {group}")
+            ws = torch.zeros(max(w4.workspace_bytes_g(c.M, c.N, c.K, group), 256), dtype=torch.uint8, device="cuda")
+            passes = max(1, -(-200 // copies))
+
+            def body(pws=pws, group=group, ws=ws):
+                for _ in range(passes):
+                    for p in pws:
+                        w4.linear_g(X, group, p.qweight, p.scales, p.zeros, Y, ws)
+            us = _time_graph(torch, stream, body, passes * copies)
+            line.update({f"g{group}_us": us, f"g{group}_code_gbs": c.code_bytes / us / 1e3,
+                         f"g{group}_all_gbs": wbytes / us / 1e3})
+            del pws, ws
+            torch.cuda.empty_cache()
+        line["fault"] = w4.device_fault()
+        print(json.dumps(line), flush=True)
+        del W, X, Y
+        torch.cuda.empty_cache()
+
+
 def run_sweep(which: str):
     """Per-layer device time of every workload shape (one JSON line each): each
     call reads a different copy of the packed weights, rotating through enough
@@ -967,6 +1014,8 @@ def main():
     ap.add_argument("--w8", default=None,
                     help="decode, or a comma list of token counts: W8A16 layers timed beside W4A16 and a cuBLAS "
                          "BF16 GEMM on the decode shapes, one JSON line each")
+    ap.add_argument("--groups", default=None,
+                    help="decode: quantisation groups of 32, 64 and 128 timed on the decode shapes, one line each")
     ap.add_argument("--variants", default=None,
                     help="decode|small_batch|prefill|all: affine, symmetric-packed and AWQ-folded layers timed "
                          "on the same kernels, one JSON line per layer")
@@ -978,6 +1027,9 @@ def main():
         return
     if args.variants:
         run_variants(args.variants)
+        return
+    if args.groups:
+        run_groups(args.groups)
         return
     if args.w8:
         run_w8(args.w8)

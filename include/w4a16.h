@@ -113,6 +113,35 @@ W4A16_API int w4a16_quantize_pack_sym(const float* W, int64_t N, int64_t K, uint
                             int32_t* zeros, int32_t* dev_status, void* stream);
 
 /*
+ * Quantisation groups of 32 or 64 weights ("Quantization I: int8, int4, the
+ * basics", Concept: groups of 32-128 values, finer fit for more metadata;
+ * "Weight-Only Quantization and Mixed Precision", section 8: group size
+ * 32/64/128).  The rule per group is the one above (symmetric != 0: the
+ * symmetric rule of w4a16_quantize_pack_sym); codes are packed as for groups of
+ * 128; scales and zeros are [N][K/group].  group = 128 is w4a16_quantize_pack /
+ * w4a16_quantize_pack_sym.  K must be a multiple of 128; other arguments and
+ * errors as w4a16_quantize_pack (W4A16_ERR_ARG for another group size).
+ */
+W4A16_API int w4a16_quantize_pack_g(const float* W, int64_t N, int64_t K, int group, int symmetric, uint32_t* qweight,
+                          uint16_t* scales, int32_t* zeros, int32_t* dev_status, void* stream);
+
+/* Workspace bytes of w4a16_linear_g (0 for an invalid shape or group). */
+W4A16_API size_t w4a16_workspace_bytes_g(int64_t M, int64_t N, int64_t K, int group);
+
+/*
+ * The linear layer on weights packed with groups of `group` (32, 64 or 128;
+ * 128 is w4a16_linear).  For 32 and 64: the integer GEMV with the sub-groups of
+ * each 128-K tile kept apart in the X operand (each digit plane split per
+ * sub-group), one token per launch (larger M runs as consecutive launches:
+ * decode is the intended use), K a multiple of 512 (W4A16_ERR_SHAPE otherwise).
+ * Arguments, layouts and errors otherwise as w4a16_linear, with scales and
+ * zeros [N][K/group] and workspace >= w4a16_workspace_bytes_g(M, N, K, group).
+ */
+W4A16_API int w4a16_linear_g(const uint16_t* X, int64_t M, int64_t K, int group, const uint32_t* qweight,
+                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device workspace w4a16_linear() needs for this shape (0 if none).
  * The workspace starts with a 256 KB area of split-K arrival counters, then
  * holds prepared activations and FP32 split-K partial sums.  The counter area

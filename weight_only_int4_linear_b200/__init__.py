@@ -53,6 +53,9 @@ SIGNATURES = {
     "w4a16_linear_path": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
     "w4a16_linear_awq": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _int, _vp]),
     "w4a16_quantize_pack_awq": (_int, [_vp, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_quantize_pack_g": (_int, [_vp, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp]),
+    "w4a16_workspace_bytes_g": (_sz, [_i64, _i64, _i64, _int]),
+    "w4a16_linear_g": (_int, [_vp, _i64, _i64, _int, _vp, _vp, _vp, _i64, _vp, _vp, _sz, _vp]),
     "w8a16_quantize": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _vp]),
     "w8a16_dequant": (_int, [_vp, _vp, _i64, _i64, _vp, _vp]),
     "w8a16_workspace_bytes": (_sz, [_i64, _i64, _i64]),
@@ -199,6 +202,39 @@ def quantize_pack_awq(W: torch.Tensor, s: torch.Tensor, qweight: torch.Tensor, s
         _dev(zeros, "zeros", torch.int32, (N, K // GROUP)),
         _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream))
     _check("w4a16_quantize_pack_awq", st)
+
+
+def quantize_pack_g(W: torch.Tensor, group: int, qweight: torch.Tensor, scales: torch.Tensor,
+                    zeros: torch.Tensor, dev_status: torch.Tensor, symmetric: bool = False, stream=None) -> None:
+    """w4a16_quantize_pack_g: groups of `group` (32, 64, 128) weights; scales/zeros [N, K/group]."""
+    N, K = W.shape
+    st = load().w4a16_quantize_pack_g(
+        _dev(W, "W", torch.float32), N, K, group, int(symmetric),
+        _dev(qweight, "qweight", torch.int32, (N, K // 8)),
+        _dev(scales, "scales", torch.bfloat16, (N, K // group)),
+        _dev(zeros, "zeros", torch.int32, (N, K // group)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream))
+    _check("w4a16_quantize_pack_g", st)
+
+
+def workspace_bytes_g(M: int, N: int, K: int, group: int) -> int:
+    return int(load().w4a16_workspace_bytes_g(M, N, K, group))
+
+
+def linear_g(X: torch.Tensor, group: int, qweight: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+             Y: torch.Tensor, workspace: torch.Tensor | None = None, stream=None) -> None:
+    """w4a16_linear_g: the layer on weights packed with groups of `group`."""
+    M, K = X.shape
+    N = qweight.shape[0]
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr = _dev(workspace, "workspace", torch.uint8)
+        ws_bytes = workspace.numel()
+    st = load().w4a16_linear_g(
+        _dev(X, "X", torch.bfloat16), M, K, group, _dev(qweight, "qweight", torch.int32, (N, K // 8)),
+        _dev(scales, "scales", torch.bfloat16, (N, K // group)), _dev(zeros, "zeros", torch.int32, (N, K // group)),
+        N, _dev(Y, "Y", torch.bfloat16, (M, N)), ws_ptr, ws_bytes, _stream(stream))
+    _check("w4a16_linear_g", st)
 
 
 def w8_quantize(W: torch.Tensor, qweight: torch.Tensor, scales: torch.Tensor, dev_status: torch.Tensor,
@@ -349,13 +385,15 @@ def device_fault() -> int:
 class PackedWeight:
     """Device buffers of one packed weight matrix (plumbing: allocation via torch)."""
 
-    def __init__(self, N: int, K: int, device="cuda"):
+    def __init__(self, N: int, K: int, device="cuda", group: int = GROUP):
         if K % GROUP:
             raise ValueError("K must be a multiple of 128")
-        self.N, self.K = N, K
+        if group not in (32, 64, 128):
+            raise ValueError("group must be 32, 64 or 128")
+        self.N, self.K, self.group = N, K, group
         self.qweight = torch.empty((N, K // 8), dtype=torch.int32, device=device)
-        self.scales = torch.empty((N, K // GROUP), dtype=torch.bfloat16, device=device)
-        self.zeros = torch.empty((N, K // GROUP), dtype=torch.int32, device=device)
+        self.scales = torch.empty((N, K // group), dtype=torch.bfloat16, device=device)
+        self.zeros = torch.empty((N, K // group), dtype=torch.int32, device=device)
 
     @classmethod
     def from_float(cls, W: torch.Tensor, stream=None, symmetric: bool = False) -> "PackedWeight":

@@ -219,6 +219,49 @@ int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, vo
     return launch_renorm(y, M, N, out, (cudaStream_t)stream);
 }
 
+int w4a16_quantize_pack_g(const float* W, int64_t N, int64_t K, int group, int symmetric, uint32_t* qweight,
+                          uint16_t* scales, int32_t* zeros, int32_t* dev_status, void* stream) {
+    if (group == 128) return quantize_pack_entry(W, nullptr, N, K, qweight, scales, zeros, dev_status, symmetric != 0,
+                                                 stream);
+    if (group != 32 && group != 64) return W4A16_ERR_ARG;
+    if (!W || !qweight || !scales || !zeros || !dev_status) return W4A16_ERR_ARG;
+    int st = check_shape(1, N, K);
+    if (st != W4A16_OK) return st;
+    if (!aligned16(W) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+        (reinterpret_cast<uintptr_t>(dev_status) & 3u))
+        return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    return launch_quantize_pack_small(W, N, K, group, symmetric != 0, qweight, scales, zeros, dev_status,
+                                      (cudaStream_t)stream);
+}
+
+size_t w4a16_workspace_bytes_g(int64_t M, int64_t N, int64_t K, int group) {
+    if (group == 128) return w4a16_workspace_bytes(M, N, K);
+    if ((group != 32 && group != 64) || check_shape(M, N, K) != W4A16_OK || K % 512 != 0) return 0;
+    check_device();
+    return decode_sub_workspace_bytes(N, K, group);
+}
+
+int w4a16_linear_g(const uint16_t* X, int64_t M, int64_t K, int group, const uint32_t* qweight,
+                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    if (group == 128)
+        return linear_entry(X, nullptr, M, K, qweight, scales, zeros, N, Y, workspace, workspace_bytes,
+                            W4A16_PATH_AUTO, stream);
+    if (group != 32 && group != 64) return W4A16_ERR_ARG;
+    if (!X || !qweight || !scales || !zeros || !Y) return W4A16_ERR_ARG;
+    int st = check_shape(M, N, K);
+    if (st != W4A16_OK) return st;
+    if (K % 512 != 0) return W4A16_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y))
+        return W4A16_ERR_ALIGN;
+    if ((st = check_device()) != W4A16_OK) return st;
+    const size_t need = decode_sub_workspace_bytes(N, K, group);
+    if (!workspace || workspace_bytes < need) return W4A16_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return W4A16_ERR_ALIGN;
+    return launch_decode_sub(X, M, K, group, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
+}
+
 int w8a16_quantize(const float* W, int64_t N, int64_t K, int8_t* qweight, uint16_t* scales, int32_t* dev_status,
                    void* stream) {
     if (!W || !qweight || !scales || !dev_status) return W4A16_ERR_ARG;

@@ -126,6 +126,15 @@ int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K,
                    const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                    cudaStream_t stream);
 
+// Quantisation groups of 32 or 64 weights (pack.cu, gemv.cu): the quantiser, and the integer
+// GEMV one token per launch.
+int launch_quantize_pack_small(const float* W, int64_t N, int64_t K, int group, bool symmetric, uint32_t* qweight,
+                               uint16_t* scales, int32_t* zeros, int32_t* dev_status, cudaStream_t stream);
+size_t decode_sub_workspace_bytes(int64_t N, int64_t K, int group);
+int launch_decode_sub(const uint16_t* X, int64_t M, int64_t K, int group, const uint32_t* qweight,
+                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                      cudaStream_t stream);
+
 // W8A16: INT8 weights with one BF16 scale per row (w8.cu).
 size_t w8_workspace_bytes(int64_t M, int64_t N, int64_t K);
 int launch_w8(const uint16_t* X, int64_t M, int64_t K, const int8_t* q, const uint16_t* scales, int64_t N,

@@ -87,6 +87,68 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(const float* __restr
     }
 }
 
+// Groups of GS = 32 or 64 weights ("Quantization I: int8, int4, the basics", Concept: groups of
+// 32-128 values; "Weight-Only Quantization and Mixed Precision", section 8), same per-group rule
+// as quantize_pack_kernel.  One warp per 128 weights (lane l holds w[4l .. 4l+3]); each group is
+// a segment of GS/4 lanes and every collective runs on the segment's mask, so a failing group
+// leaves its neighbours alone.  Scales and zero points are [N][K/GS].
+template <bool kSym, int GS>
+__global__ void __launch_bounds__(256) quantize_pack_small_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+                                                                  uint32_t* __restrict__ qweight,
+                                                                  uint16_t* __restrict__ scales,
+                                                                  int32_t* __restrict__ zeros, int32_t* status) {
+    constexpr int kLanes = GS / 4;
+    const int lane = threadIdx.x & 31;
+    const unsigned seg = ((1u << kLanes) - 1u) << (lane & ~(kLanes - 1));
+    const bool leader = (lane & (kLanes - 1)) == 0;
+    const int64_t blocks_per_row = K / 128, groups_per_row = K / GS;
+    const int64_t total = N * blocks_per_row;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+    for (int64_t blk = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; blk < total; blk += warps) {
+        const int64_t n = blk / blocks_per_row, b = blk % blocks_per_row;
+        const int64_t grp = n * groups_per_row + (b * 128 + 4 * lane) / GS;
+        const int64_t word = n * (K / 8) + b * 16 + lane / 2;
+        const float4 v = reinterpret_cast<const float4*>(W + n * K + b * 128)[lane];
+        const bool finite = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+        const bool ok = __all_sync(seg, finite);
+        float lo = fminf(fminf(v.x, v.y), fminf(v.z, v.w));
+        float hi = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+#pragma unroll
+        for (int o = kLanes / 2; o > 0; o >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(seg, lo, o));
+            hi = fmaxf(hi, __shfl_xor_sync(seg, hi, o));
+        }
+        const double mag = fmax(fabs((double)lo), fabs((double)hi));
+        uint16_t sb = double_to_bf16_bits(kSym ? __ddiv_rn(mag, 7.0)
+                                               : __ddiv_rn(__dsub_rn((double)hi, (double)lo), 15.0));
+        if ((sb & 0x7FFFu) == 0) {
+            sb = double_to_bf16_bits(mag);
+            if ((sb & 0x7FFFu) == 0) sb = 0x3F80u;  // 1.0
+        }
+        const double s = (double)bf16_bits_to_float(sb);
+        const double z = kSym ? 8.0 : rint(__ddiv_rn(-(double)lo, s));
+        const bool z_ok = z <= 2147483647.0 && z >= -2147483648.0;
+        uint32_t half = 0;
+        if (ok && z_ok) {
+            const float w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                double t = __dadd_rn(rint(__ddiv_rn((double)w4[i], s)), z);
+                t = fmin(fmax(t, 0.0), 15.0);
+                half |= ((uint32_t)t) << (4 * i);
+            }
+        }
+        // word j = codes of lanes 2j (low half) and 2j + 1 (high half), both in one segment
+        const uint32_t upper = __shfl_xor_sync(seg, half, 1);
+        if ((lane & 1) == 0) qweight[word] = half | (upper << 16);
+        if (leader) {
+            if (!ok || !z_ok) atomicCAS(status, 0, ok ? (int)W4A16_ERR_ZERO_RANGE : (int)W4A16_ERR_NONFINITE);
+            scales[grp] = ok && z_ok ? sb : (uint16_t)0;
+            zeros[grp] = ok && z_ok ? (int32_t)z : 0;
+        }
+    }
+}
+
 // One thread per packed word -> 8 codes.
 __global__ void unpack_kernel(const uint32_t* __restrict__ qweight, int64_t words, uint8_t* __restrict__ codes) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words; i += (int64_t)gridDim.x * blockDim.x) {
@@ -196,6 +258,24 @@ int launch_quantize_pack(const float* W, const float* col_scale, int64_t N, int6
         quantize_pack_kernel<true><<<grid, 256, 0, stream>>>(W, col_scale, N, K, qweight, scales, zeros, dev_status);
     else
         quantize_pack_kernel<false><<<grid, 256, 0, stream>>>(W, col_scale, N, K, qweight, scales, zeros, dev_status);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+
+int launch_quantize_pack_small(const float* W, int64_t N, int64_t K, int group, bool symmetric, uint32_t* qweight,
+                               uint16_t* scales, int32_t* zeros, int32_t* dev_status, cudaStream_t stream) {
+    if (cudaMemsetAsync(dev_status, 0, sizeof(int32_t), stream) != cudaSuccess) return W4A16_ERR_CUDA;
+    const int grid = grid_for(N * (K / 128) * 32, 256);
+    if (group == 64) {
+        if (symmetric)
+            quantize_pack_small_kernel<true, 64><<<grid, 256, 0, stream>>>(W, N, K, qweight, scales, zeros, dev_status);
+        else
+            quantize_pack_small_kernel<false, 64><<<grid, 256, 0, stream>>>(W, N, K, qweight, scales, zeros, dev_status);
+    } else {
+        if (symmetric)
+            quantize_pack_small_kernel<true, 32><<<grid, 256, 0, stream>>>(W, N, K, qweight, scales, zeros, dev_status);
+        else
+            quantize_pack_small_kernel<false, 32><<<grid, 256, 0, stream>>>(W, N, K, qweight, scales, zeros, dev_status);
+    }
     return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
