@@ -90,6 +90,19 @@ def test_host_validation_without_device(lib):
     assert lib.w8a16_quantize(P, 4, 128, P, P, None, None) == w4.ERR_ARG
     assert lib.w8a16_dequant(P, U, 4, 128, P, None) == w4.ERR_ALIGN
     assert lib.w8a16_workspace_bytes(1, 16, 100) == 0
+    # symmetric packing, the AWQ entries and the group-size entries validate the same way
+    assert lib.w4a16_quantize_pack_sym(P, 4, 96, P, P, P, P, None) == w4.ERR_SHAPE
+    assert lib.w4a16_quantize_pack_awq(P, None, 4, 128, P, P, P, P, None) == w4.ERR_ARG
+    assert lib.w4a16_quantize_pack_awq(P, U, 4, 128, P, P, P, P, None) == w4.ERR_ALIGN
+    assert lib.w4a16_linear_awq(P, None, 1, 128, P, P, P, 16, P, None, 0, 0, None) == w4.ERR_ARG
+    assert lib.w4a16_linear_awq(P, U, 1, 128, P, P, P, 16, P, None, 0, 0, None) == w4.ERR_ALIGN
+    assert lib.w4a16_quantize_pack_g(P, 4, 128, 48, 0, P, P, P, P, None) == w4.ERR_ARG
+    assert lib.w4a16_quantize_pack_g(P, 4, 96, 64, 0, P, P, P, P, None) == w4.ERR_SHAPE
+    assert lib.w4a16_linear_g(P, 1, 512, 48, P, P, P, 16, P, P, 1 << 20, None) == w4.ERR_ARG
+    assert lib.w4a16_linear_g(P, 1, 384, 64, P, P, P, 16, P, P, 1 << 20, None) == w4.ERR_SHAPE
+    assert lib.w4a16_linear_g(P, 1, 512, 32, U, P, P, 16, P, P, 1 << 20, None) == w4.ERR_ALIGN
+    assert lib.w4a16_workspace_bytes_g(1, 16, 384, 64) == 0
+    assert lib.w4a16_workspace_bytes_g(1, 16, 512, 48) == 0
     if not torch.cuda.is_available():
         # well-formed arguments reach the device check, which fails without a GPU
         assert lin(P, 1, 128, P, P, P, 16, P, None, 0, 0, None) == w4.ERR_DEVICE
