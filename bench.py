@@ -1004,7 +1004,7 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=90.0,
                     help="reference arm: approximate host seconds for warm-up + timed steps")
     ap.add_argument("--traffic", type=float, default=None,
-                    help="dram bytes per launch of the dominant kernel from an ncu capture of this build")
+                    help="dram bytes per launch of the dominant kernel, from an ncu capture of the current sources")
     ap.add_argument("--profile", default=None,
                     help="workload:layer (e.g. decode:gate_up, prefill:o_proj_m4096, decode:all, w8:gate_up): run it a few "
                          "times, untimed")
