@@ -275,9 +275,16 @@ W4A16_API int w4a16_renorm_rows(const uint16_t* y, int64_t M, int64_t N, uint16_
  * file-scope device array of w4a16_noalloc_scratch_bytes() bytes (16 MiB) that
  * every process loading the library holds on each GPU it uses until exit.  It
  * allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
- *  - Arguments, layouts and results are those of w4a16_linear().
- *  - A problem whose scratch (w4a16_workspace_bytes(M, N, K)) exceeds the
- *    array returns W4A16_ERR_WORKSPACE and launches nothing.
+ *  - Arguments and layouts are those of w4a16_linear().  It always runs the
+ *    decode path, in tiles of 32 tokens for M > 32, with results identical
+ *    bit for bit to w4a16_linear_path(..., W4A16_PATH_DECODE, ...); for
+ *    M >= 64, where w4a16_linear would choose the GEMM, the results agree
+ *    with it within the layer's tolerance but are not the same bits.
+ *  - The limit is the decode path's own scratch (prepared X, split-K
+ *    partial sums, counters), which grows with N and K and with M only up
+ *    to 32 tokens; a problem whose decode scratch exceeds the array returns
+ *    W4A16_ERR_WORKSPACE and launches nothing.  (w4a16_workspace_bytes()
+ *    also counts the GEMM's needs and can be larger for M >= 64.)
  *  - The first call on a device looks up the array's device address (once per
  *    device, with that device current); make that first call before any
  *    stream capture.
@@ -299,9 +306,33 @@ W4A16_API size_t w4a16_noalloc_scratch_bytes(void);
  * call, a positive site code when one did (its outputs are then invalid),
  * or -1 if the device could not be queried.  Kernels never trap or spin
  * forever: a pipeline wait that exceeds about two seconds records its site
- * here and the kernel returns.
+ * here and the kernel returns.  Only the first site is kept until the word
+ * is read.
+ * After a non-zero result, zero every workspace the failed calls used
+ * (w4a16_workspace_init) before its next use: a kernel that gave up may have
+ * left split-K arrival counters non-zero.  (w4a16_linear_noalloc clears the
+ * counters it needs on every call.)
  */
 W4A16_API int w4a16_device_fault(void);
+
+/* Site code that w4a16_selftest_wait() records. */
+#define W4A16_SELFTEST_SITE 900
+/* Largest wait limit w4a16_selftest_wait() accepts, in SM cycles (about one second). */
+#define W4A16_SELFTEST_MAX_CYCLES 2000000000LL
+
+/*
+ * Test of the failure path (the pages have no counterpart; this checks the
+ * library's own error reporting).  Launches one CTA of 32 threads that waits,
+ * with the library's bounded mbarrier wait, on a barrier phase nothing will
+ * complete -- no copy, MMA or other thread is attached to it -- and gives up
+ * after `limit_cycles` SM cycles (1 .. W4A16_SELFTEST_MAX_CYCLES): it records
+ * W4A16_SELFTEST_SITE in the fault word and returns, exactly as a pipeline
+ * wait of the linear kernels does on a timeout.  The GPU context stays
+ * usable; w4a16_device_fault() then returns W4A16_SELFTEST_SITE.
+ * Returns W4A16_ERR_ARG for a limit out of range, W4A16_ERR_DEVICE if the
+ * current device is not sm_100.  Asynchronous on `stream`.
+ */
+W4A16_API int w4a16_selftest_wait(int64_t limit_cycles, void* stream);
 
 #ifdef __cplusplus
 }

@@ -103,10 +103,20 @@ def test_host_validation_without_device(lib):
     assert lib.w4a16_linear_g(P, 1, 512, 32, U, P, P, 16, P, P, 1 << 20, None) == w4.ERR_ALIGN
     assert lib.w4a16_workspace_bytes_g(1, 16, 384, 64) == 0
     assert lib.w4a16_workspace_bytes_g(1, 16, 512, 48) == 0
+    # the failure-path self-test checks its limit before touching a device
+    assert lib.w4a16_selftest_wait(0, None) == w4.ERR_ARG
+    assert lib.w4a16_selftest_wait(2_000_000_001, None) == w4.ERR_ARG
     if not torch.cuda.is_available():
+        assert lib.w4a16_selftest_wait(1000, None) == w4.ERR_DEVICE
         # well-formed arguments reach the device check, which fails without a GPU
         assert lin(P, 1, 128, P, P, P, 16, P, None, 0, 0, None) == w4.ERR_DEVICE
         assert lib.w4a16_workspace_init(P, 64, None) == w4.ERR_DEVICE
+
+
+def test_selftest_constants_match_the_header():
+    text = open(HEADER).read()
+    assert re.search(r"#define W4A16_SELFTEST_SITE (\d+)", text).group(1) == str(w4.SELFTEST_SITE)
+    assert int(re.search(r"#define W4A16_SELFTEST_MAX_CYCLES (\d+)LL", text).group(1)) == 2_000_000_000
 
 
 def test_workspace_bytes(lib):

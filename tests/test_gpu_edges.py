@@ -1,0 +1,170 @@
+"""Activations with extreme per-group dynamic range through every kernel family,
+against the FP64 oracle under the stated tolerance, one token row at a time.
+
+The decode kernels write each group of 128 activations as the integer
+x * 2^(21 - E) in three signed base-256 digits (E the exponent of the group's
+largest magnitude): exact for values within 2^14 of that maximum, rounded at
+2^(E - 21) below it.  The activations themselves are never quantised ("Axe
+Corsa 28B" model card, "How the Compression Works": activations stay BF16), so
+this rounding must stay inside the tolerance whatever the group holds: values
+twenty binades below the group maximum, exact and signed zeros, all-zero
+groups and rows, negative maxima, BF16 subnormals, the smallest normal
+binades, magnitudes near 2^100 and the largest finite BF16.
+
+Each row is compared against its own oracle row (the tolerance's rms taken over
+that row), so a row of tiny values is held to a bound of its own size."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_int4_linear_b200 as w4
+from synth import edge
+from tests._parity import assert_close, bf16_dev_to_f64, bits_to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+ALL = list(edge.KINDS)
+# The GEMM multiplies BF16 (q - z) by BF16 x in FP32 before the scale: |x| * 15 must stay below the FP32
+# maximum, so activations of magnitude 2^124 and above are outside its range (the decode paths take every
+# finite BF16 value).
+PREFILL_KINDS = [k for k in ALL if k != "max_finite"]
+# x * inv_s of the largest finite BF16 overflows for inv_s > 1: the transformed activation is not finite.
+AWQ_KINDS = [k for k in ALL if k != "max_finite"]
+
+
+def _pack(N, K, seed, group=128):
+    W = synth.weights_f32(seed, synth.TAG_W, N, K)
+    W[: min(3, N), :K // 2] += np.float32(0.3)  # a few one-signed groups: zero points outside 0..15
+    Wd = torch.from_numpy(np.ascontiguousarray(W)).cuda()
+    if group == 128:
+        pw = w4.PackedWeight.from_float(Wd)
+        st, qw, sc, z = oracle.quantize_pack(W)
+    else:
+        pw = w4.PackedWeight(N, K, group=group)
+        pw.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        w4.quantize_pack_g(Wd, group, pw.qweight, pw.scales, pw.zeros, pw.status)
+        st, qw, sc, z = oracle.quantize_pack_g(W, group)
+    torch.cuda.synchronize()
+    assert int(pw.status.item()) == 0 and st == oracle.OK
+    return pw, (qw, sc, z)
+
+
+def _check_rows(Y: torch.Tensor, Y_ref: np.ndarray, kinds, what: str):
+    got = bf16_dev_to_f64(Y)
+    for m, kind in enumerate(kinds):
+        assert_close(got[m], Y_ref[m], f"{what} row {m} ({kind})")
+
+
+def _linear(X_bits, pw, path):
+    M, K = X_bits.shape
+    Y = torch.full((M, pw.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    nbytes = w4.workspace_bytes(M, pw.N, K)
+    ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+    w4.linear(bits_to_dev_bf16(X_bits), pw.qweight, pw.scales, pw.zeros, Y, ws, path=path)
+    torch.cuda.synchronize()
+    assert w4.device_fault() == 0
+    return Y
+
+
+@pytest.mark.parametrize("N,K", [(200, 1024), (136, 5120)])
+@pytest.mark.parametrize("kind", ALL)
+def test_one_token(cuda_lib, N, K, kind):
+    """M = 1: the integer GEMV for one token (X digits formed inside the kernel)."""
+    pw, (qw, sc, z) = _pack(N, K, 11)
+    X = edge.activations_bf16(101 + ALL.index(kind), [kind], K)
+    Y = _linear(X, pw, w4.PATH_AUTO)
+    _check_rows(Y, oracle.linear(X, qw, sc, z), [kind], f"M=1 N={N} K={K}")
+
+
+@pytest.mark.parametrize("pair", [(ALL[i], ALL[(i + 1) % len(ALL)]) for i in range(len(ALL))])
+def test_two_tokens(cuda_lib, pair):
+    """M = 2: the integer GEMV for two tokens."""
+    N, K = 200, 2048
+    pw, (qw, sc, z) = _pack(N, K, 12)
+    X = edge.activations_bf16(202, list(pair), K)
+    Y = _linear(X, pw, w4.PATH_AUTO)
+    _check_rows(Y, oracle.linear(X, qw, sc, z), pair, "M=2")
+
+
+@pytest.mark.parametrize("M", [3, 11, 16, 40])
+def test_tensor_core_gemv(cuda_lib, M):
+    """3 <= M <= 63: digit planes prepared per launch, tcgen05 kind::i8 (16- and 32-token tiles; M = 40 runs
+    a 32-token and an 8-token launch)."""
+    N, K = 200, 2048
+    kinds = [ALL[m % len(ALL)] for m in range(M)]
+    pw, (qw, sc, z) = _pack(N, K, 13)
+    X = edge.activations_bf16(300 + M, kinds, K)
+    Y = _linear(X, pw, w4.PATH_DECODE)
+    _check_rows(Y, oracle.linear(X, qw, sc, z), kinds, f"M={M}")
+
+
+@pytest.mark.parametrize("group", [32, 64])
+def test_small_groups(cuda_lib, group):
+    """Groups of 32 and 64: the integer GEMV with per-sub-group digit rows, one token per launch."""
+    N, K = 200, 1024
+    kinds = ALL
+    pw, (qw, sc, z) = _pack(N, K, 14, group)
+    X = edge.activations_bf16(400 + group, kinds, K)
+    M = len(kinds)
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(w4.workspace_bytes_g(M, N, K, group), 256), dtype=torch.uint8, device="cuda")
+    w4.linear_g(bits_to_dev_bf16(X), group, pw.qweight, pw.scales, pw.zeros, Y, ws)
+    torch.cuda.synchronize()
+    assert w4.device_fault() == 0
+    _check_rows(Y, oracle.linear_g(X, qw, sc, z), kinds, f"group {group}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 10])
+def test_awq_activation_scaling(cuda_lib, M):
+    """w4a16_linear_awq: X' = bf16(x * r) formed ahead of (M <= 2) or inside (M >= 3) the X preparation."""
+    N, K = 200, 1024
+    kinds = [AWQ_KINDS[(m + 1) % len(AWQ_KINDS)] for m in range(M)]
+    W = synth.weights_f32(15, synth.TAG_W, N, K)
+    rng = np.random.default_rng(15)
+    s = np.exp2(rng.uniform(-1.5, 1.5, size=K)).astype(np.float32)
+    r = (1.0 / s.astype(np.float64)).astype(np.float32)
+    pw = w4.PackedWeight(N, K)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w4.quantize_pack_awq(torch.from_numpy(W).cuda(), torch.from_numpy(s).cuda(), pw.qweight, pw.scales,
+                         pw.zeros, status)
+    st, qw, sc, z = oracle.quantize_pack(oracle.awq_scale_weights(W, s))
+    X = edge.activations_bf16(500 + M, kinds, K)
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(w4.workspace_bytes(M, N, K), 256), dtype=torch.uint8, device="cuda")
+    w4.linear_awq(bits_to_dev_bf16(X), torch.from_numpy(r).cuda(), pw.qweight, pw.scales, pw.zeros, Y, ws,
+                  path=w4.PATH_DECODE)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0 and st == oracle.OK and w4.device_fault() == 0
+    Xs = oracle.awq_scale_activations(X, r)
+    _check_rows(Y, oracle.linear(Xs, qw, sc, z), kinds, f"AWQ M={M}")
+
+
+def test_prefill_gemm(cuda_lib):
+    """M >= 64: BF16 tiles of (q - z) against BF16 X on the tensor cores (exact products, FP32 sums)."""
+    N, K = 300, 1024
+    kinds = [PREFILL_KINDS[m % len(PREFILL_KINDS)] for m in range(70)]
+    pw, (qw, sc, z) = _pack(N, K, 16)
+    X = edge.activations_bf16(600, kinds, K)
+    Y = _linear(X, pw, w4.PATH_PREFILL)
+    _check_rows(Y, oracle.linear(X, qw, sc, z), kinds, "prefill M=70")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3])
+def test_w8a16(cuda_lib, M):
+    """W8A16: the one-byte-code GEMV with the same digit representation of X."""
+    N, K = 200, 1024
+    W = synth.weights_f32(17, synth.TAG_W, N, K)
+    pw = w4.PackedW8.from_float(torch.from_numpy(W).cuda())
+    st, q, sc = oracle.w8_quantize(W)
+    torch.cuda.synchronize()
+    for start in range(0, len(ALL), M):
+        kinds = [ALL[(start + i) % len(ALL)] for i in range(M)]
+        X = edge.activations_bf16(700 + start, kinds, K)
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ws = torch.zeros(max(w4.w8_workspace_bytes(M, N, K), 256), dtype=torch.uint8, device="cuda")
+        w4.w8_linear(bits_to_dev_bf16(X), pw.qweight, pw.scales, Y, ws)
+        torch.cuda.synchronize()
+        assert w4.device_fault() == 0
+        _check_rows(Y, oracle.w8_linear(X, q, sc), kinds, f"W8 M={M}")

@@ -66,6 +66,7 @@ SIGNATURES = {
     "w4a16_dequant_codes": (_int, [_vp, _vp, _vp, _i64, _i64, _vp, _vp]),
     "w4a16_renorm_rows": (_int, [_vp, _i64, _i64, _vp, _vp]),
     "w4a16_device_fault": (_int, []),
+    "w4a16_selftest_wait": (_int, [_i64, _vp]),
     "w4a16_linear_noalloc": (_int, [_vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp]),
     "w4a16_noalloc_scratch_bytes": (_sz, []),
 }
@@ -380,6 +381,15 @@ def renorm_rows(y: torch.Tensor, out: torch.Tensor, stream=None) -> None:
 def device_fault() -> int:
     """Synchronise, then read and clear the device fault word (0 = no bounded wait gave up)."""
     return int(load().w4a16_device_fault())
+
+
+SELFTEST_SITE = 900
+
+
+def selftest_wait(limit_cycles: int, stream=None) -> None:
+    """w4a16_selftest_wait: one CTA's bounded wait on a barrier phase nothing completes; it gives up
+    after limit_cycles, records SELFTEST_SITE in the fault word and returns."""
+    _check("w4a16_selftest_wait", load().w4a16_selftest_wait(int(limit_cycles), _stream(stream)))
 
 
 class PackedWeight:

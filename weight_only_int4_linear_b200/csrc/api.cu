@@ -15,6 +15,7 @@ std::atomic<int> g_device_ok[kMaxDevices];  // 0 unknown, 1 sm_100, 2 rejected
 std::atomic<int> g_num_sms[kMaxDevices];
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}  // namespace
 
 int check_device() {
     int dev = -1;
@@ -37,6 +38,7 @@ int check_device() {
     return state == 1 ? W4A16_OK : W4A16_ERR_DEVICE;
 }
 
+namespace {
 // Shape limits: indices inside the kernels are 32-bit for M, N, K and 64-bit
 // for element offsets.
 constexpr int64_t kMaxDim = (int64_t)1 << 30;

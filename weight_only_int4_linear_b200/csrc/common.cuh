@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/w4a16.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -82,6 +84,44 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { ret
 
 // Host-side launch helpers (defined in api.cu).
 namespace w4a16 {
+// Identity of the current CUDA context (0 while none is current).  Kernel attributes, occupancy
+// and the device addresses of file-scope symbols belong to a context: they differ between devices
+// and do not survive cudaDeviceReset, so the library's caches of them are keyed by it (runtime.cu).
+uint64_t context_key();
+
+// A value computed once per context: get(make) returns the value cached for the current device if
+// it was made in the current context, else calls make() (a zero result is not cached).
+template <class T>
+class PerContext {
+  public:
+    template <class F>
+    T get(F&& make) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) {
+            cudaGetLastError();
+            return T{};
+        }
+        std::lock_guard<std::mutex> lk(mu_);
+        const uint64_t key = context_key();
+        if (key != 0 && key_[dev] == key) return val_[dev];
+        const T v = make();
+        const uint64_t after = context_key();  // make() may have created the context
+        if (v != T{} && after != 0) {
+            key_[dev] = after;
+            val_[dev] = v;
+        }
+        return v;
+    }
+
+  private:
+    static constexpr int kDevices = 64;
+    std::mutex mu_;
+    uint64_t key_[kDevices] = {};
+    T val_[kDevices] = {};
+};
+
+// The current device is sm_100: W4A16_OK (its SM count cached), else W4A16_ERR_DEVICE (api.cu).
+int check_device();
 int launch_quantize_pack(const float* W, const float* col_scale, int64_t N, int64_t K, uint32_t* qweight,
                          uint16_t* scales, int32_t* zeros, int32_t* dev_status, bool symmetric, cudaStream_t stream);
 int launch_unpack(const uint32_t* qweight, int64_t N, int64_t K, uint8_t* codes, cudaStream_t stream);

@@ -506,24 +506,23 @@ bool prefill_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtenso
 
 size_t align256p(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// MMA units of the prefill kernel that fit on the current device at once (cached per device).
+// MMA units of the prefill kernel that fit on the current device at once (cached per context).
 int prefill_resident_units(const cudaLaunchConfig_t& cfg) {
-    static std::mutex mu;
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-    std::lock_guard<std::mutex> lk(mu);
-    if (cache[dev] > 0) return cache[dev];
-    int units = 0;
-    if constexpr (kPCtas == 1) {
-        units = num_sms_current();
-    } else {
-        cudaLaunchConfig_t q = cfg;
-        q.gridDim = dim3((unsigned)(kPCtas * num_sms_current()));
-        if (cudaOccupancyMaxActiveClusters(&units, prefill_kernel, &q) != cudaSuccess) return -1;
-    }
-    cache[dev] = units;
-    return units;
+    static PerContext<int> cache;
+    return cache.get([&]() -> int {
+        int units = 0;
+        if constexpr (kPCtas == 1) {
+            units = num_sms_current();
+        } else {
+            cudaLaunchConfig_t q = cfg;
+            q.gridDim = dim3((unsigned)(kPCtas * num_sms_current()));
+            if (cudaOccupancyMaxActiveClusters(&units, prefill_kernel, &q) != cudaSuccess) {
+                cudaGetLastError();
+                return 0;
+            }
+        }
+        return units;
+    });
 }
 
 }  // namespace
@@ -537,13 +536,12 @@ size_t prefill_workspace_bytes(int64_t M, int64_t K) {
 int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                    const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                    cudaStream_t stream) {
-    static bool attr = false;
-    if (!attr) {
-        if (cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem) !=
-            cudaSuccess)
-            return W4A16_ERR_CUDA;
-        attr = true;
-    }
+    static PerContext<int> attr;  // the attribute belongs to a context
+    if (!attr.get([]() -> int {
+            return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem) ==
+                   cudaSuccess;
+        }))
+        return W4A16_ERR_CUDA;
     int* fault = fault_word();
     if (!fault) return W4A16_ERR_CUDA;
     char* ws = reinterpret_cast<char*>(workspace) + kCounterBytes;

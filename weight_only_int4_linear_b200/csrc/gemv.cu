@@ -450,9 +450,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             const float xsc[8] = {xc0.x, xc0.y, xc0.z, xc0.w, xc1.x, xc1.y, xc1.z, xc1.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                // sum q x_int = 65536 D2 + 256 D1 + D0
+                // sum q x_int = 65536 D2 + 256 D1 + D0; the power of two last, so that a group of
+                // tiny activations does not underflow in s 2^(E - 21)
                 const float qx = fmaf(to_f(d2[e]), 65536.f, fmaf(to_f(d1[e]), 256.f, to_f(d0[e])));
-                acc[h * 8 + e] = fmaf(sv * xsc[e], fmaf(-zv, xsum[e], qx), acc[h * 8 + e]);
+                acc[h * 8 + e] = fmaf(sv * fmaf(-zv, xsum[e], qx), xsc[e], acc[h * 8 + e]);
             }
         }
         __syncwarp();
@@ -863,7 +864,9 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
                 // the rest FP32 with one rounding per step
                 const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
                 const int k = 2 * rb + h;
-                y[k] = fmaf(sv[k] * xscale, fmaf(-zv[k], xsum, qx), y[k]);
+                // s (sum (q - z) x_int), then the power of two: neither product leaves the FP32 range
+                // unless the group's result itself does
+                y[k] = fmaf(sv[k] * fmaf(-zv[k], xsum, qx), xscale, y[k]);
             }
         }
     }
@@ -872,8 +875,8 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
 
 template <int NTOK>
 int occupancy_nt() {
-    static int occ = 0;
-    if (occ == 0) {
+    static PerContext<int> cache;  // the attribute belongs to a context
+    return cache.get([]() -> int {
         if (cudaFuncSetAttribute(decode_tc_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)TcCfg<NTOK>::kSmem) != cudaSuccess)
             return 0;
@@ -882,26 +885,24 @@ int occupancy_nt() {
                                                           TcCfg<NTOK>::kSmem) != cudaSuccess ||
             o < 1)
             return 0;
-        occ = 1;  // one CTA per SM: it owns all 512 TMEM columns
-    }
-    return occ;
+        return 1;  // one CTA per SM: it owns all 512 TMEM columns
+    });
 }
 
 template <int NT>
 int occupancy_cc() {
-    static int occ = 0;
-    if (occ == 0) {
-        if (cudaFuncSetAttribute(decode_cc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cc_smem<NT>()) !=
-            cudaSuccess)
+    static PerContext<int> cache;  // the attribute and occupancy belong to a context
+    return cache.get([]() -> int {
+        if (cudaFuncSetAttribute(decode_cc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)cc_smem<NT>()) != cudaSuccess)
             return 0;
         int o = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel<NT>, kCcThreads, cc_smem<NT>()) !=
                 cudaSuccess ||
             o < 1)
             return 0;
-        occ = o;
-    }
-    return occ;
+        return o;
+    });
 }
 
 // cc_tokens > 0: the integer CUDA-core kernel for that many tokens; else the tensor-core kernel with MMA N = ntok

@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
                 }
                 const float qx = fmaf((float)P[2], 65536.f, (float)(P[1] * 256 + P[0]));
                 const int k = 2 * rb + hh;
-                if (folder) y[k] = fmaf(sv[k] * xscale, fmaf(-zv[k], xsum, qx), y[k]);
+                if (folder) y[k] = fmaf(sv[k] * fmaf(-zv[k], xsum, qx), xscale, y[k]);  // power of two last
             }
         }
     }
@@ -382,8 +382,8 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
 
 template <int GS>
 int occupancy_sub() {
-    static int occ = 0;
-    if (occ == 0) {
+    static PerContext<int> cache;  // the attribute and occupancy belong to a context
+    return cache.get([]() -> int {
         if (cudaFuncSetAttribute(decode_sub_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)SubCfg<GS>::kSmem) != cudaSuccess)
             return 0;
@@ -392,9 +392,8 @@ int occupancy_sub() {
                 cudaSuccess ||
             o < 1)
             return 0;
-        occ = o;
-    }
-    return occ;
+        return o;
+    });
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }

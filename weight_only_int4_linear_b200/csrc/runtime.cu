@@ -25,10 +25,39 @@ void resolve_encode() {
 }
 
 __device__ int g_fault;  // bounded-wait fault word: 0 = none, else the site that gave up
-constexpr int kMaxDev = 64;
-int* g_fault_addr[kMaxDev];
-std::mutex g_fault_mu;
+PerContext<int*> g_fault_addr;
+
+typedef CUresult (*PFN_ctx_get_current)(CUcontext*);
+typedef CUresult (*PFN_ctx_get_id)(CUcontext, unsigned long long*);
+PFN_ctx_get_current g_ctx_current = nullptr;
+PFN_ctx_get_id g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+void resolve_ctx() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_current = reinterpret_cast<PFN_ctx_get_current>(fn);
+    else
+        cudaGetLastError();
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_id = reinterpret_cast<PFN_ctx_get_id>(fn);
+    else
+        cudaGetLastError();
+}
 }  // namespace
+
+uint64_t context_key() {
+    std::call_once(g_ctx_once, resolve_ctx);
+    if (!g_ctx_current || !g_ctx_id) return 0;
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return (uint64_t)id + 1;  // context IDs are unique over the process; 0 stays "none"
+}
 
 bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
@@ -45,21 +74,48 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
 }
 
 int* fault_word() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-    std::lock_guard<std::mutex> lk(g_fault_mu);
-    if (!g_fault_addr[dev]) {
+    return g_fault_addr.get([]() -> int* {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_fault) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
-        g_fault_addr[dev] = static_cast<int*>(p);
-    }
-    return g_fault_addr[dev];
+        return static_cast<int*>(p);
+    });
 }
 
 }  // namespace w4a16
+
+namespace w4a16 {
+namespace {
+// One CTA waits on a phase of an mbarrier that nothing will complete (no copy, no MMA and no other
+// thread is ever attached to it), with the caller's limit: the bounded wait runs out, records
+// kSelftestSite and the kernel returns, as every pipeline wait of the library does on a timeout.
+__global__ void __launch_bounds__(32) selftest_wait_kernel(long long limit, int* fault) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, fault, W4A16_SELFTEST_SITE, limit);
+}
+}  // namespace
+}  // namespace w4a16
+
+extern "C" W4A16_API int w4a16_selftest_wait(int64_t limit_cycles, void* stream) {
+    if (limit_cycles < 1 || limit_cycles > W4A16_SELFTEST_MAX_CYCLES) return W4A16_ERR_ARG;
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess || major != 10) {
+        cudaGetLastError();
+        return W4A16_ERR_DEVICE;
+    }
+    int* fault = w4a16::fault_word();
+    if (!fault) return W4A16_ERR_CUDA;
+    w4a16::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((long long)limit_cycles, fault);
+    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
 
 extern "C" W4A16_API int w4a16_device_fault(void) {
     int* p = w4a16::fault_word();

@@ -53,17 +53,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitCycles, records `site` in *fault and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* fault, int site) {
+// `limit` SM cycles, records `site` in *fault (unless an earlier site is
+// already there) and returns false.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, int* fault, int site,
+                                                long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             atomicCAS(fault, 0, site);
             return false;
         }
     }
     return true;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* fault, int site) {
+    return mbar_wait_limit(bar, parity, fault, site, kWaitLimitCycles);
 }
 
 // ---------------------------------------------------- 2-CTA clusters -----

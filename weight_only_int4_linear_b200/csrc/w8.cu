@@ -196,7 +196,16 @@ __global__ void __launch_bounds__(kW8Threads, w8_min_blocks<NT>()) w8_decode_ker
     int cur_tile = -1;
     bool aborted = false;
 
-    auto row_scale = [&](int n) { return bf16_bits_to_float(a.scales[n]); };
+    // the row scale enters every block's fold (s P, then the power of two), so that no partial sum
+    // leaves the FP32 range unless the result does; rows past N fold with s = 0
+    float sn[4] = {0.f, 0.f, 0.f, 0.f};
+    auto load_row_scales = [&](int tile) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int n = tile * kW8Rows + rrow(k);
+            sn[k] = n < N ? bf16_bits_to_float(a.scales[n]) : 0.f;
+        }
+    };
     auto flush = [&](int tile) {
         const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
         const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
@@ -205,7 +214,7 @@ __global__ void __launch_bounds__(kW8Threads, w8_min_blocks<NT>()) w8_decode_ker
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int n = tile * kW8Rows + rrow(k);
-                    if (n < N) a.Y[(int64_t)mt * N + n] = float_to_bf16_bits(y[k] * row_scale(n));
+                    if (n < N) a.Y[(int64_t)mt * N + n] = float_to_bf16_bits(y[k]);
                 }
             }
         } else {
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(kW8Threads, w8_min_blocks<NT>()) w8_decode_ker
                     for (int rl = t; rl < rows; rl += kW8Warps * 32) {
                         const float sum = sum_slots(pb + (int64_t)m * kW8Rows + rl, (int64_t)a.M * kW8Rows, nseg);
                         const int n = tile * kW8Rows + rl;
-                        a.Y[(int64_t)m * N + n] = float_to_bf16_bits(sum * row_scale(n));
+                        a.Y[(int64_t)m * N + n] = float_to_bf16_bits(sum);
                     }
                 }
                 if (t == 0) a.counters[tile] = 0;
@@ -244,6 +253,7 @@ __global__ void __launch_bounds__(kW8Threads, w8_min_blocks<NT>()) w8_decode_ker
         if (tile != cur_tile) {
             if (cur_tile >= 0) flush(cur_tile);
             cur_tile = tile;
+            load_row_scales(tile);
         }
         if (aborted) continue;
         const int s = i % kW8Stages;
@@ -304,7 +314,7 @@ __global__ void __launch_bounds__(kW8Threads, w8_min_blocks<NT>()) w8_decode_ker
                 }
                 // |P| <= 128 * 127 * 128 < 2^21: 256 P1 + P0 is exact in int32, the rest FP32
                 const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-                y[2 * rb + h] = fmaf(xscale, qx, y[2 * rb + h]);
+                y[2 * rb + h] = fmaf(sn[2 * rb + h] * qx, xscale, y[2 * rb + h]);
             }
         }
     }
@@ -313,8 +323,8 @@ __global__ void __launch_bounds__(kW8Threads, w8_min_blocks<NT>()) w8_decode_ker
 
 template <int NT>
 int w8_occupancy() {
-    static int occ = 0;
-    if (occ == 0) {
+    static PerContext<int> cache;  // the attribute and occupancy belong to a context
+    return cache.get([]() -> int {
         if (cudaFuncSetAttribute(w8_decode_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)w8_smem<NT>()) != cudaSuccess)
             return 0;
@@ -323,9 +333,8 @@ int w8_occupancy() {
                 cudaSuccess ||
             o < 1)
             return 0;
-        occ = o;
-    }
-    return occ;
+        return o;
+    });
 }
 
 struct W8Plan {
