@@ -12,7 +12,12 @@ groups and rows, negative maxima, BF16 subnormals, the smallest normal
 binades, magnitudes near 2^100 and the largest finite BF16.
 
 Each row is compared against its own oracle row (the tolerance's rms taken over
-that row), so a row of tiny values is held to a bound of its own size."""
+that row), so a row of tiny values is held to a bound of its own size.  Rows of
+subnormal activations times ordinary weights give outputs below the smallest
+normal BF16, where the output's own spacing (2^-133) is coarser than the
+relative bound; there the tolerance's absolute term of half that spacing
+decides, and a separate case scales the weights by 2^20 so that subnormal
+inputs give normal outputs, held to the relative bound alone."""
 import numpy as np
 import pytest
 import torch
@@ -34,8 +39,8 @@ PREFILL_KINDS = [k for k in ALL if k != "max_finite"]
 AWQ_KINDS = [k for k in ALL if k != "max_finite"]
 
 
-def _pack(N, K, seed, group=128):
-    W = synth.weights_f32(seed, synth.TAG_W, N, K)
+def _pack(N, K, seed, group=128, w_scale=1.0):
+    W = synth.weights_f32(seed, synth.TAG_W, N, K) * np.float32(w_scale)
     W[: min(3, N), :K // 2] += np.float32(0.3)  # a few one-signed groups: zero points outside 0..15
     Wd = torch.from_numpy(np.ascontiguousarray(W)).cuda()
     if group == 128:
@@ -76,6 +81,20 @@ def test_one_token(cuda_lib, N, K, kind):
     X = edge.activations_bf16(101 + ALL.index(kind), [kind], K)
     Y = _linear(X, pw, w4.PATH_AUTO)
     _check_rows(Y, oracle.linear(X, qw, sc, z), [kind], f"M=1 N={N} K={K}")
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 40, 70])
+def test_subnormal_inputs_normal_outputs(cuda_lib, M):
+    """Subnormal activations against weights of magnitude ~2^14: outputs in the normal range, so the
+    relative bound applies in full; every kernel family (M = 70 is the GEMM)."""
+    N, K = 200, 2048
+    kinds = ["subnormal" if m % 2 == 0 else "subnormal_mixed" for m in range(M)]
+    pw, (qw, sc, z) = _pack(N, K, 18, w_scale=2.0 ** 20)
+    X = edge.activations_bf16(800 + M, kinds, K)
+    Y = _linear(X, pw, w4.PATH_AUTO)
+    Y_ref = oracle.linear(X, qw, sc, z)
+    assert np.abs(Y_ref[0]).max() > 2.0 ** -120  # outputs in the normal BF16 range
+    _check_rows(Y, Y_ref, kinds, f"subnormal x large weights M={M}")
 
 
 @pytest.mark.parametrize("pair", [(ALL[i], ALL[(i + 1) % len(ALL)]) for i in range(len(ALL))])
