@@ -179,12 +179,13 @@ PREFILL_MIN_M = 64  # the library's automatic path choice: M >= 64 takes the ten
 
 def launches_per_call(c) -> int:
     """Our kernels per linear call: X preparation + GEMM (M >= 64); one
-    single-token GEMV (M = 1, K/128 a multiple of 8, X prepared inside it);
-    else X preparation + GEMV per 32-token chunk."""
+    integer GEMV for one or two tokens (K/128 a multiple of 8, X prepared
+    inside it); X preparation + integer GEMV per 16-token chunk (K/128 a
+    multiple of 8); else X preparation + tensor-core GEMV per 32-token chunk."""
     if c.M >= PREFILL_MIN_M:
         return 2
-    if c.M == 1 and (c.K // 128) % 8 == 0:
-        return 1
+    if (c.K // 128) % 8 == 0:
+        return 1 if c.M <= 2 else 2 * ((c.M + 15) // 16)
     return 2 * ((c.M + 31) // 32)
 
 
@@ -199,26 +200,27 @@ def capture(torch, stream, body):
     return g
 
 
-def time_steps(layers, steps, warmup, torch, w4, stream, path, block=50):
-    """Device time of exactly `steps` passes over the layer set, replayed from CUDA
-    graphs of `block` steps (launch overhead off the timed path)."""
-    with torch.cuda.stream(stream):
-        for _ in range(max(warmup, 1)):
-            for L in layers:
+def _step_body(sets, path, w4, n):
+    """n steps; step i runs every layer once on weight copy i % len(sets)."""
+    def f():
+        for i in range(n):
+            for L in sets[i % len(sets)]:
                 _linear_call(w4, L, path)
+    return f
+
+
+def time_steps(sets, steps, warmup, torch, w4, stream, path, block=50):
+    """Device time of exactly `steps` steps (step i on weight copy i % len(sets)), replayed from CUDA
+    graphs of `block` steps (launch overhead off the timed path), after `warmup` untimed steps."""
+    with torch.cuda.stream(stream):
+        _step_body(sets, path, w4, max(warmup, 1))()
     torch.cuda.synchronize()
     block = max(1, min(block, steps))
+    if block > len(sets):
+        block -= block % len(sets)  # every graph starts on copy 0, so blocks keep the rotation
     full, rest = divmod(steps, block)
-
-    def body(n):
-        def f():
-            for _ in range(n):
-                for L in layers:
-                    _linear_call(w4, L, path)
-        return f
-
-    g_full = capture(torch, stream, body(block))
-    g_rest = capture(torch, stream, body(rest)) if rest else None
+    g_full = capture(torch, stream, _step_body(sets, path, w4, block))
+    g_rest = capture(torch, stream, _step_body(sets, path, w4, rest)) if rest else None
     with torch.cuda.stream(stream):
         g_full.replay()  # graph warm-up
     torch.cuda.synchronize()
@@ -236,19 +238,59 @@ def time_steps(layers, steps, warmup, torch, w4, stream, path, block=50):
     return total_ms
 
 
-def time_layer_alone(c, torch, w4, stream, min_calls=200):
-    """Device time of one call of layer `c` (CUDA events on the launching
-    stream): back-to-back calls replayed from a CUDA graph, each call reading a
-    different copy of the packed weights, rotating through enough copies that
-    their codes exceed 3x L2.  Returns (us per call, copies)."""
+def protocol_blocks(sets, torch, w4, stream, path, seconds, min_blocks=50, block=20):
+    """Repeated timing of the same step outside the headline region: a CUDA graph of `block` steps
+    replayed back to back, each replay bracketed by events on the launching stream, until at least
+    `min_blocks` replays and `seconds` of device time.  Returns the per-step microseconds of every
+    replay."""
+    g = capture(torch, stream, _step_body(sets, path, w4, block))
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    per_step, total_ms = [], 0.0
+    while len(per_step) < min_blocks or total_ms < seconds * 1e3:
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(51)]
+        ev[0].record(stream)
+        with torch.cuda.stream(stream):
+            for j in range(50):
+                g.replay()
+                ev[j + 1].record(stream)
+        torch.cuda.synchronize()
+        for j in range(50):
+            ms = ev[j].elapsed_time(ev[j + 1])
+            per_step.append(ms * 1e3 / block)
+            total_ms += ms
+    del g
+    return per_step
+
+
+def _quantiles(xs):
+    q = np.quantile(np.asarray(xs), [0.1, 0.5, 0.9])
+    return {"p10": float(q[0]), "median": float(q[1]), "p90": float(q[2]), "n": len(xs)}
+
+
+def packed_copies(c, torch, w4, stream, max_copies=48):
+    """Copies of layer c's packed weights, enough that their codes exceed 3x L2 (at most max_copies)."""
     W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
     synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
-    copies = max(1, min(32, -(-3 * L2_BYTES // c.code_bytes)))
+    copies = max(1, min(max_copies, -(-3 * L2_BYTES // c.code_bytes)))
     pws = [w4.PackedWeight.from_float(W, stream=stream) for _ in range(copies)]
     torch.cuda.synchronize()
     del W
     if any(int(pw.status.item()) != 0 for pw in pws):
         raise RuntimeError(f"packing failed for {c.name}")
+    return pws
+
+
+def time_layer_alone(c, torch, w4, stream, min_calls=200, pws=None):
+    """Device time of one call of layer `c` (CUDA events on the launching
+    stream): back-to-back calls replayed from a CUDA graph, each call reading a
+    different copy of the packed weights, rotating through enough copies that
+    their codes exceed 3x L2.  Returns (us per call, copies)."""
+    own = pws is None
+    if own:
+        pws = packed_copies(c, torch, w4, stream)
+    copies = len(pws)
     xb = synth.activations_bf16(c.x_seed, c.M, c.K)
     X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
     Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
@@ -277,9 +319,67 @@ def time_layer_alone(c, torch, w4, stream, min_calls=200):
     e1.record(stream)
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / (reps * passes * copies)
-    del g, pws, X, Y, ws
+    del g, X, Y, ws
+    if own:
+        del pws
     torch.cuda.empty_cache()
     return us, copies
+
+
+def layer_roofline(c, us, peaks, peak_src, kernel):
+    """One layer's measured rate against the copy bandwidth (HBM-bound GEMV) or the dense BF16 peak (GEMM)."""
+    if c.M >= PREFILL_MIN_M:
+        achieved = c.flops / us / 1e6
+        return {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "per_call_us": us,
+                "peak_source": peak_src}
+    achieved = c.code_bytes / us / 1e3
+    return {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "per_call_us": us, "algorithmic_bytes_per_launch": c.code_bytes,
+            "peak_source": peak_src}
+
+
+def decode_kernel_name(c) -> str:
+    if c.M >= PREFILL_MIN_M:
+        return "prefill_kernel"
+    if (c.K // 128) % 8 == 0:
+        if c.M <= 2:
+            return f"decode_cc_kernel<{c.M}>"
+        nt = [t for t in (4, 8, 16) if min(c.M, 16) <= t][0]
+        return f"decode_mt_kernel<{nt}>" + (" per 16-token chunk" if c.M > 16 else "")
+    return "decode_tc_kernel<16>" if min(c.M, 32) <= 16 else "decode_tc_kernel<32>"
+
+
+def run_layer_tables(torch, w4, stream, peaks, peak_src, prefill_ms=(512, 2048)):
+    """The other workloads, each layer alone with its weights rotated past 3x L2: the single 4096 x 4096
+    GEMV, the small-batch sweep M in {2, 4, 8, 16, 32} and the prefill GEMM at M in prefill_ms, on the
+    hidden-8192 shapes (one set of packed copies per shape serves every M)."""
+    out = {}
+    c1 = workloads.single_gemv()[0]
+    us, copies = time_layer_alone(c1, torch, w4, stream)
+    out["single_gemv_4096"] = {"workload": c1.workload, "M": 1, "K": c1.K, "N": c1.N, "weight_copies": copies,
+                               "roofline": layer_roofline(c1, us, peaks, peak_src, decode_kernel_name(c1))}
+    small = workloads.small_batch_8192()
+    pre = workloads.prefill_8192(ms=list(prefill_ms))
+    rows_small, rows_pre = [], []
+    def base(c):
+        return c.name.rsplit("_m", 1)[0]
+    for shape in [name for name, _, _ in workloads.HIDDEN_8192]:
+        cs = [c for c in small if base(c) == shape]
+        pws = packed_copies(cs[0], torch, w4, stream, max_copies=12)
+        for c in cs:
+            us, copies = time_layer_alone(c, torch, w4, stream, pws=pws)
+            rows_small.append({"layer": c.name, "M": c.M, "K": c.K, "N": c.N, "weight_copies": copies,
+                               "roofline": layer_roofline(c, us, peaks, peak_src, decode_kernel_name(c))})
+        for c in [c for c in pre if base(c) == shape]:
+            us, copies = time_layer_alone(c, torch, w4, stream, pws=pws[:1])
+            rows_pre.append({"layer": c.name, "M": c.M, "K": c.K, "N": c.N,
+                             "roofline": layer_roofline(c, us, peaks, peak_src, decode_kernel_name(c))})
+        del pws
+        torch.cuda.empty_cache()
+    out["small_batch_8192"] = rows_small
+    out["prefill_8192_other_m"] = rows_pre
+    return out
 
 
 def time_e2e(layers, steps, warmup, torch, w4, stream, path):
@@ -464,25 +564,35 @@ def run_ours(args):
     stream = torch.cuda.Stream()
     peaks, peak_src = load_peaks()
 
+    # the hidden-5120 layer set at M = 1, two copies of its packed weights: step i runs copy i % 2, so
+    # 2 x 251 MB of weights pass between reuses (4x the 126 MB L2)
     cases = workloads.decode_5120()
-    layers = setup_layers(cases, torch, w4, stream)
+    sets = [setup_layers(cases, torch, w4, stream) for _ in range(2)]
     code_bytes = sum(c.code_bytes for c in cases)
     all_bytes = sum(c.code_bytes + c.meta_bytes + 2 * c.M * (c.K + c.N) for c in cases)
 
-    # warm-up + timed region (device time, CUDA events on the launching stream)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
+    # Clock samples cover a window of the same steps around the timed region: repeated blocks of the
+    # step (the timing protocol's spread) before and after it, so the sampler (one sample per 200 ms)
+    # sees the clocks the timed steps ran at.
     with ClockSampler(local) as clk:
-        total_ms = time_steps(layers, args.steps, args.warmup, torch, w4, stream, w4.PATH_AUTO)
+        proto = protocol_blocks(sets, torch, w4, stream, w4.PATH_AUTO, seconds=args.protocol_seconds / 2)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        total_ms = time_steps(sets, args.steps, args.warmup, torch, w4, stream, w4.PATH_AUTO)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        proto += protocol_blocks(sets, torch, w4, stream, w4.PATH_AUTO, seconds=args.protocol_seconds / 2)
     total_ms = max_over_ranks(total_ms, "cuda")
     value = whole_job_rate(code_bytes, args.steps, total_ms, world)
+    pq = _quantiles(proto)
 
     # end to end through the public API with host buffers
-    e2e_ms, h2d, d2h = time_e2e(layers, args.steps, args.warmup, torch, w4, stream, w4.PATH_AUTO)
+    e2e_ms, h2d, d2h = time_e2e(sets[0], args.steps, args.warmup, torch, w4, stream, w4.PATH_AUTO)
     e2e_ms = max_over_ranks(e2e_ms, "cuda")
     e2e_value = whole_job_rate(code_bytes, args.steps, e2e_ms, world)
-    del layers
+    del sets
     torch.cuda.empty_cache()
 
     # each layer's kernel alone (an M = 1 call is one launch); dominant kernel: gate+up
@@ -500,7 +610,7 @@ def run_ours(args):
     if not args.no_prefill:
         pcases = workloads.prefill_8192(ms=[4096])
         players = setup_layers(pcases, torch, w4, stream)
-        p_ms = time_steps(players, args.prefill_steps, 1, torch, w4, stream, w4.PATH_AUTO, block=1)
+        p_ms = time_steps([players], args.prefill_steps, 1, torch, w4, stream, w4.PATH_AUTO, block=1)
         del players
         torch.cuda.empty_cache()
         flops = sum(c.flops for c in pcases)
@@ -518,6 +628,8 @@ def run_ours(args):
                                 "traffic": ncu_traffic("prefill_kernel", pcases[pdom].name),
                                 "per_call_us": pdom_us, "timed": "whole call: X preparation (about 2% of it) + GEMM",
                                 "peak_source": peak_src}}
+
+    tables = None if args.no_tables else run_layer_tables(torch, w4, stream, peaks, peak_src)
 
     stack = None
     if not args.no_stack:
@@ -549,11 +661,15 @@ def run_ours(args):
         "config": {"workload": "decode_hidden5120_m1", "M": 1,
                    "shapes_KxN": [[c.K, c.N] for c in cases], "group": 128,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {all_bytes / 1e6:.0f} MB read per step vs "
-                         f"{L2_BYTES / 1e6:.0f} MB L2, layers run in sequence"},
+                   "l2": f"inputs larger than L2: two copies of the layer set's weights alternate by step, "
+                         f"{2 * all_bytes / 1e6:.0f} MB read between reuses vs {L2_BYTES / 1e6:.0f} MB L2"},
         "frac_of_hbm_peak": value / world / peaks["hbm_gbs"],
         "all_bytes_gbs": world * all_bytes * args.steps / (total_ms * 1e-3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": f"decode GEMV on {cases[dom].name} "
+        "protocol": {"us_per_step": pq, "gbs_median": code_bytes / pq["median"] / 1e3,
+                     "frac_median": code_bytes / pq["median"] / 1e3 / peaks["hbm_gbs"],
+                     "how": "CUDA graphs of 20 steps replayed back to back around the timed region, "
+                            "each replay bracketed by events; weights rotated as above"},
+        "roofline": {"bound": "hbm", "kernel": f"{decode_kernel_name(cases[dom])} on {cases[dom].name} "
                                                 f"({cases[dom].K}x{cases[dom].N})",
                      "achieved": dom_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": dom_gbs / peaks["hbm_gbs"],
@@ -566,6 +682,7 @@ def run_ours(args):
                 "ms_per_step": e2e_ms / args.steps},
         "prefill": prefill,
         "stack": stack,
+        "configs": tables,
         "gpu_launches": launches,
         "cpu_baseline": cpu,
         "clocks": clk.summary(),
@@ -999,6 +1116,9 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--stack-steps", type=int, default=20)
     ap.add_argument("--no-stack", action="store_true")
+    ap.add_argument("--no-tables", action="store_true", help="skip the single-GEMV, small-batch and other-M tables")
+    ap.add_argument("--protocol-seconds", type=float, default=1.0,
+                    help="device seconds of repeated step blocks around the timed region (spread and clocks)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0,

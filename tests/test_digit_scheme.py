@@ -60,3 +60,65 @@ def test_plane_sums_stay_exact_in_int32():
     worst8 = 128 * 127 * 128
     assert worst4 < 2 ** 21 and worst8 < 2 ** 21
     assert 256 * worst8 + worst8 < 2 ** 31
+
+
+# ---------------------------------------------------------------------------------------------
+# The same scheme as the GPU writes it: the 3-16-token integer GEMV prepares each launch's digit
+# rows once, in its caller's workspace, and reads them back with bulk copies.  White-box check of
+# that preparation, bit for bit, against the host statement above: the workspace layout is
+# [256 KB of split-K counters][per group g: digit rows of 128 bytes, then (sum x_int, 2^(E - 21)) per
+# token as FP32].  Within a row, bytes 8w .. 8w + 3 hold the digits of codes 0, 2, 4, 6 of packed
+# word w (K = 128 g + 8 w + {0, 2, 4, 6}) and bytes 8w + 4 .. 8w + 7 those of codes 1, 3, 5, 7.
+# Row of plane p, token m: 2m + p (p < 2) or 8 + 2m (p = 2) for 4-token tiles, p NT + m otherwise.
+
+import pytest  # noqa: E402
+
+
+def _mt_row(nt, p, m):
+    return (2 * m + p if p < 2 else 8 + 2 * m) if nt == 4 else p * nt + m
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,nt", [(3, 4), (4, 4), (6, 8), (13, 16)])
+def test_gpu_digit_rows_match_the_scheme(cuda_lib, M, nt):
+    import torch
+    import weight_only_int4_linear_b200 as w4
+    from tests._parity import bits_to_dev_bf16
+    from synth import edge
+    N, K = 256, 1024
+    G = K // 128
+    kinds = [edge.KINDS[m % len(edge.KINDS)] for m in range(M)]
+    kinds[0] = "control"
+    Xb = edge.activations_bf16(77 + M, kinds, K)
+    W = synth.weights_f32(5, synth.TAG_W, N, K)
+    pw = w4.PackedWeight.from_float(torch.from_numpy(W).cuda())
+    nbytes = w4.workspace_bytes(M, N, K)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    w4.linear(bits_to_dev_bf16(Xb), pw.qweight, pw.scales, pw.zeros, Y, ws, path=w4.PATH_DECODE)
+    torch.cuda.synchronize()
+    rows = {4: 16, 8: 24, 16: 48}[nt]
+    xbytes = rows * 128 + 8 * nt
+    counters = 256 * 1024
+    raw = ws.cpu().numpy()
+    assert not raw[:counters].any()  # every counter back at zero
+    order = np.array([[8 * w + i for i in (0, 2, 4, 6, 1, 3, 5, 7)] for w in range(16)]).reshape(-1)
+    for g in range(G):
+        blk = raw[counters + g * xbytes: counters + (g + 1) * xbytes]
+        planes = blk[: rows * 128].reshape(rows, 128).view(np.int8)
+        ext = blk[rows * 128:].view(np.float32)
+        used = np.zeros(rows, dtype=bool)
+        for m in range(nt):
+            if m < M:
+                E, x, xi, d0, d1, d2 = _digits(Xb[m, 128 * g:128 * (g + 1)])
+                want = [d0, d1, d2]
+                assert ext[2 * m] == float(xi.sum()), (g, m)
+                assert ext[2 * m + 1] == np.ldexp(1.0, E - 21), (g, m)
+            else:
+                want = [np.zeros(128, dtype=np.int64)] * 3
+                assert ext[2 * m] == 0 and ext[2 * m + 1] == 0
+            for p in range(3):
+                r = _mt_row(nt, p, m)
+                used[r] = True
+                np.testing.assert_array_equal(planes[r].astype(np.int64), want[p][order], err_msg=f"g={g} m={m} p={p}")
+        assert not planes[~used].any()  # padding rows stay zero

@@ -53,6 +53,20 @@ def test_small_shapes_all_outputs(cuda_lib, M, N, K, path):
     assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), f"M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("M", [3, 4, 5, 7, 8, 9, 12, 15, 16, 17, 20, 24, 31, 33, 48, 63])
+def test_small_batch_token_counts_all_outputs(cuda_lib, M):
+    """Every token count of the 3-16-token integer GEMV (tiles of 4, 8 and 16 tokens; M > 16 in chunks of
+    16 with a smaller last tile), K / 128 a multiple of 8, ragged N."""
+    N, K = 200, 1024
+    W = synth.weights_f32(3000 + M, synth.TAG_W, N, K)
+    X = synth.activations_bf16(3100 + M, M, K)
+    pw = packed_from_host(W)
+    st, qw, sc, z = oracle.quantize_pack(W)
+    Y = run_linear(X, pw, w4.PATH_DECODE)
+    assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), f"M={M} N={N} K={K}")
+    assert w4.device_fault() == 0
+
+
 @pytest.mark.parametrize("path", PATHS)
 def test_one_hot_inputs_pick_weight_columns(cuda_lib, path):
     """x = e_k must give Y[:, n] = bf16(w_hat[n][k]) exactly: pins nibble order,

@@ -748,7 +748,10 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
         const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
         const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
         if (first == last) {
-            if (owner) {
+            if constexpr (NT == 1) {  // lane tig holds row rrow(tig)
+                const int n = tile * kRowsPerCta + rrow(tig);
+                if (n < N) a.Y[n] = float_to_bf16_bits(y[0]);
+            } else if (owner) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int n = tile * kRowsPerCta + rrow(k);
@@ -758,7 +761,9 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
         } else {
             const int slot = b - first, nseg = last - first + 1;
             float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * a.M * kRowsPerCta;
-            if (owner) {
+            if constexpr (NT == 1) {
+                part[rrow(tig)] = y[0];
+            } else if (owner) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) part[mt * kRowsPerCta + rrow(k)] = y[k];
             }
@@ -808,8 +813,11 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             cw[k] = *reinterpret_cast<const uint4*>(st + r * 64 + 16 * (tig ^ ((r >> 1) & 3)));
         }
         uint32_t bx[8];
-        if (g8 < 3 * NT) {
-            const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + g8 * 128 + tig * 32);
+        // one token: B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of
+        // the second row block and each lane of a quad can fold one of its four rows
+        const int xrow = NT == 1 ? (g8 & 3) : g8;
+        if (xrow < 3 * NT) {
+            const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + xrow * 128 + tig * 32);
             const uint4 u0 = xp[0], u1 = xp[1];
             bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
             bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
@@ -824,8 +832,8 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
         const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
         float sv[4], zv[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = rrow(k);
+        for (int k = 0; k < (NT == 1 ? 1 : 4); ++k) {
+            const int r = NT == 1 ? rrow(tig) : rrow(k);
             sv[k] = bf16_bits_to_float(
                 *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
             zv[k] = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
@@ -834,39 +842,67 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
+        if constexpr (NT == 1) {
+            int d[2][4];
 #pragma unroll
-        for (int rb = 0; rb < 2; ++rb) {
-            const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
-            const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
-            int d[4] = {0, 0, 0, 0};
+            for (int rb = 0; rb < 2; ++rb) {
+                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_u8s8(d, w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
-                         (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
-            // lane tig holds columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3)
+                for (int j = 0; j < 4; ++j) d[rb][j] = 0;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                int P0, P1, P2;
-                if constexpr (NT == 1) {  // planes 0, 1 at lane tig 0, plane 2 at lane tig 1
-                    P0 = d[2 * h];
-                    P1 = d[2 * h + 1];
-                    P2 = __shfl_sync(0xFFFFFFFFu, d[2 * h], lane | 1);
-                } else {  // column p NT + m: token 0 planes at (0,0), (1,0), (2,0); token 1 at (0,1), (1,1), (2,1)
-                    const int own = tig == 0 ? d[2 * h] : d[2 * h + 1];
-                    const int x = __shfl_xor_sync(0xFFFFFFFFu, tig == 0 ? d[2 * h + 1] : d[2 * h], 1);
-                    const int t0 = __shfl_sync(0xFFFFFFFFu, d[2 * h], (lane & ~3) | 2);
-                    const int t1 = __shfl_sync(0xFFFFFFFFu, d[2 * h + 1], (lane & ~3) | 2);
-                    P0 = tig == 0 ? own : x;
-                    P1 = tig == 0 ? x : own;
-                    P2 = tig == 0 ? t0 : t1;
+                for (int j = 0; j < 4; ++j)
+                    mma_u8s8(d[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
+                             (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
+            }
+            // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes
+            // (0, 1) at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block
+            // tig >> 1 (its own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour
+            // completes its planes.
+            const bool hi = tig >> 1, even = !(tig & 1);
+            int e[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) e[j] = hi ? d[1][j] : d[0][j];
+            const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
+            const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
+            const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
+            const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+            y[0] = fmaf(sv[0] * fmaf(-zv[0], xsum, qx), xscale, y[0]);
+        } else {
+    #pragma unroll
+            for (int rb = 0; rb < 2; ++rb) {
+                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
+                int d[4] = {0, 0, 0, 0};
+    #pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    mma_u8s8(d, w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
+                             (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
+                // lane tig holds columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3)
+    #pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    int P0, P1, P2;
+                    if constexpr (NT == 1) {  // planes 0, 1 at lane tig 0, plane 2 at lane tig 1
+                        P0 = d[2 * h];
+                        P1 = d[2 * h + 1];
+                        P2 = __shfl_sync(0xFFFFFFFFu, d[2 * h], lane | 1);
+                    } else {  // column p NT + m: token 0 planes at (0,0), (1,0), (2,0); token 1 at (0,1), (1,1), (2,1)
+                        const int own = tig == 0 ? d[2 * h] : d[2 * h + 1];
+                        const int x = __shfl_xor_sync(0xFFFFFFFFu, tig == 0 ? d[2 * h + 1] : d[2 * h], 1);
+                        const int t0 = __shfl_sync(0xFFFFFFFFu, d[2 * h], (lane & ~3) | 2);
+                        const int t1 = __shfl_sync(0xFFFFFFFFu, d[2 * h + 1], (lane & ~3) | 2);
+                        P0 = tig == 0 ? own : x;
+                        P1 = tig == 0 ? x : own;
+                        P2 = tig == 0 ? t0 : t1;
+                    }
+                    // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26),
+                    // the rest FP32 with one rounding per step
+                    const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+                    const int k = 2 * rb + h;
+                    // s (sum (q - z) x_int), then the power of two: neither product leaves the FP32 range
+                    // unless the group's result itself does
+                    y[k] = fmaf(sv[k] * fmaf(-zv[k], xsum, qx), xscale, y[k]);
                 }
-                // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26),
-                // the rest FP32 with one rounding per step
-                const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-                const int k = 2 * rb + h;
-                // s (sum (q - z) x_int), then the power of two: neither product leaves the FP32 range
-                // unless the group's result itself does
-                y[k] = fmaf(sv[k] * fmaf(-zv[k], xsum, qx), xscale, y[k]);
             }
         }
     }
@@ -998,8 +1034,17 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     // the integer CUDA-core kernel for M <= kCcMaxTokens (needs 16-byte metadata rows: G % 8 == 0);
     // else the tensor-core kernel with MMA N = 16 or 32
     p.cc_tokens = (M <= kCcMaxTokens && G % 8 == 0) ? (int)M : 0;
+    p.mt = !p.cc_tokens && mt_supported(K);
     p.nt = p.cc_tokens ? 1 : (Mc <= 16 ? 16 : 32);
     p.row_tiles = (int)ceil_div(N, kRowsPerCta);
+    if (p.mt) {  // the 3-16-token integer GEMV keeps its own plan per chunk; only its scratch is sized here
+        p.ws_xp_bytes = mt_workspace_bytes(M, N, K, num_sms);
+        p.ws_xs_bytes = 0;
+        p.ws_partial_bytes = 0;
+        p.ws_counter_bytes =
+            align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
+        return p;
+    }
     const int64_t units = (int64_t)p.row_tiles * G;
     int occ = occupancy(p.cc_tokens, p.nt);
     if (occ < 1) occ = 1;
@@ -1042,6 +1087,9 @@ size_t DecodePlan::workspace_bytes() const { return ws_xp_bytes + ws_xs_bytes + 
 int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                   const DecodePlan& plan, cudaStream_t stream) {
+    if (plan.mt)
+        return launch_decode_mt(X, xscale, M, K, qweight, scales, zeros, N, Y, reinterpret_cast<int*>(workspace),
+                                reinterpret_cast<char*>(workspace) + plan.ws_counter_bytes, stream);
     CUtensorMap tq;
     if (!cached_tmap(0, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
     int* fault = fault_word();

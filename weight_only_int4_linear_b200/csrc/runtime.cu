@@ -73,6 +73,43 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
     return r == CUDA_SUCCESS;
 }
 
+namespace {
+struct TmapKey {
+    const void* base;
+    uint64_t inner, outer, row_bytes;
+    uint32_t box_inner, box_outer;
+    int dtype, swizzle;
+    bool operator==(const TmapKey& o) const {
+        return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+               box_inner == o.box_inner && box_outer == o.box_outer && dtype == o.dtype && swizzle == o.swizzle;
+    }
+};
+constexpr int kTmapSlots = 256;
+TmapKey g_tkeys[kTmapSlots];
+CUtensorMap g_tmaps[kTmapSlots];
+int g_tnext = 0, g_tused = 0;
+std::mutex g_tmu;
+}  // namespace
+
+bool tmap_2d_cached(CUtensorMap* out, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+    const TmapKey key{base, inner, outer, row_bytes, box_inner, box_outer, (int)dtype, (int)swizzle};
+    std::lock_guard<std::mutex> lk(g_tmu);
+    for (int i = 0; i < g_tused; ++i)
+        if (g_tkeys[i] == key) {
+            *out = g_tmaps[i];
+            return true;
+        }
+    CUtensorMap m;
+    if (!encode_tmap_2d(&m, dtype, base, inner, outer, row_bytes, box_inner, box_outer, swizzle)) return false;
+    g_tkeys[g_tnext] = key;
+    g_tmaps[g_tnext] = m;
+    g_tnext = (g_tnext + 1) % kTmapSlots;
+    if (g_tused < kTmapSlots) ++g_tused;
+    *out = m;
+    return true;
+}
+
 int* fault_word() {
     return g_fault_addr.get([]() -> int* {
         void* p = nullptr;

@@ -298,6 +298,13 @@ bool encode_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* bas
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
+// A 2-D tensor map as encode_tmap_2d makes it, encoded once per (base, shape, type, box, swizzle)
+// and kept in a process-wide cache (the map describes global addresses only, so it stays valid for
+// any context in which the base address is).  Returns false on failure.
+bool tmap_2d_cached(CUtensorMap* out, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
+
 // Device address of the current device's fault word (set up once per device).
 int* fault_word();
 
