@@ -178,14 +178,15 @@ PREFILL_MIN_M = 64  # the library's automatic path choice: M >= 64 takes the ten
 
 
 def launches_per_call(c) -> int:
-    """Our kernels per linear call: X preparation + GEMM (M >= 64); one
-    integer GEMV for one or two tokens (K/128 a multiple of 8, X prepared
-    inside it); X preparation + integer GEMV per 16-token chunk (K/128 a
-    multiple of 8); else X preparation + tensor-core GEMV per 32-token chunk."""
+    """Our kernels per linear call: X preparation + GEMM (M >= 64); with K/128
+    a multiple of 8, the one-token integer GEMV + its split-K reduction
+    (M = 1, X prepared inside the GEMV), or X preparation + integer GEMV +
+    reduction (2 <= M <= 8); otherwise X preparation + tensor-core GEMV per
+    32-token chunk."""
     if c.M >= PREFILL_MIN_M:
         return 2
-    if (c.K // 128) % 8 == 0:
-        return 1 if c.M <= 2 else 2 * ((c.M + 15) // 16)
+    if (c.K // 128) % 8 == 0 and c.M <= 8:
+        return 2 if c.M == 1 else 3
     return 2 * ((c.M + 31) // 32)
 
 
@@ -342,11 +343,8 @@ def layer_roofline(c, us, peaks, peak_src, kernel):
 def decode_kernel_name(c) -> str:
     if c.M >= PREFILL_MIN_M:
         return "prefill_kernel"
-    if (c.K // 128) % 8 == 0:
-        if c.M <= 2:
-            return f"decode_cc_kernel<{c.M}>"
-        nt = [t for t in (4, 8, 16) if min(c.M, 16) <= t][0]
-        return f"decode_mt_kernel<{nt}>" + (" per 16-token chunk" if c.M > 16 else "")
+    if (c.K // 128) % 8 == 0 and c.M <= 8:
+        return "decode_cc_kernel<1>" if c.M == 1 else f"decode_mt_kernel<{4 if c.M <= 4 else 8}>"
     return "decode_tc_kernel<16>" if min(c.M, 32) <= 16 else "decode_tc_kernel<32>"
 
 
@@ -1034,49 +1032,66 @@ def run_w8(which: str):
 
 
 def run_groups(which: str):
-    """Quantisation groups of 32, 64 and 128 weights on the decode shapes (hidden 5120, M = 1),
-    one JSON line per layer: device time per call (w4a16_linear_g), each call reading a different
-    copy of the packed weights past L2, replayed from a CUDA graph; GB/s of code bytes and of
-    all weight bytes (codes + 6 B of metadata per group)."""
+    """Quantisation groups of 32, 64 and 128 weights, one JSON line per layer and token count: device
+    time per call (w4a16_linear_g), each call reading a different copy of the packed weights past L2,
+    replayed from a CUDA graph.  "decode": the hidden-5120 shapes at M = 1 (GB/s of code bytes and of
+    all weight bytes, codes + 6 B of metadata per group); "batched": the hidden-8192 shapes at M in
+    {4, 16, 40, 512} (GB/s of code bytes, and TFLOP/s at M = 512); "all": both."""
     import torch
     import weight_only_int4_linear_b200 as w4
     w4.load()
     stream = torch.cuda.Stream()
-    for c in workloads.decode_5120():
-        W = torch.empty((c.N, c.K), dtype=torch.float32, device="cuda")
-        synth.fill_weights_device(c.w_seed, c.w_tag, W.data_ptr(), c.N * c.K, stream=stream.cuda_stream)
-        xb = synth.activations_bf16(c.x_seed, c.M, c.K)
-        X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
-        Y = torch.empty((c.M, c.N), dtype=torch.bfloat16, device="cuda")
-        line = {"groups": c.workload, "layer": c.name, "M": c.M, "K": c.K, "N": c.N}
+    runs = []
+    if which in ("decode", "all"):
+        runs += [(c, [1]) for c in workloads.decode_5120()]
+    if which in ("batched", "all"):
+        runs += [(c, [4, 16, 40, 512]) for c in workloads.small_batch_8192(ms=[2])]
+    for c0, ms in runs:
+        W = torch.empty((c0.N, c0.K), dtype=torch.float32, device="cuda")
+        synth.fill_weights_device(c0.w_seed, c0.w_tag, W.data_ptr(), c0.N * c0.K, stream=stream.cuda_stream)
+        packs = {}
         for group in (128, 64, 32):
-            wbytes = c.code_bytes + c.N * (c.K // group) * 6
+            wbytes = c0.code_bytes + c0.N * (c0.K // group) * 6
             copies = max(1, min(16, -(-3 * L2_BYTES // wbytes)))
             pws = []
             with torch.cuda.stream(stream):
                 for _ in range(copies):
-                    pw = w4.PackedWeight(c.N, c.K, group=group)
+                    pw = w4.PackedWeight(c0.N, c0.K, group=group)
                     pw.status = torch.zeros(1, dtype=torch.int32, device="cuda")
                     w4.quantize_pack_g(W, group, pw.qweight, pw.scales, pw.zeros, pw.status, stream=stream)
                     pws.append(pw)
             torch.cuda.synchronize()
             if any(int(p.status.item()) != 0 for p in pws):
-                raise RuntimeError(f"packing failed for {c.name}, group {group}")
-            ws = torch.zeros(max(w4.workspace_bytes_g(c.M, c.N, c.K, group), 256), dtype=torch.uint8, device="cuda")
-            passes = max(1, -(-200 // copies))
+                raise RuntimeError(f"packing failed for {c0.name}, group {group}")
+            packs[group] = (pws, wbytes)
+        del W
+        torch.cuda.empty_cache()
+        for M in ms:
+            name = c0.name.rsplit("_m", 1)[0]
+            xb = synth.activations_bf16(c0.x_seed + M, M, c0.K)
+            X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+            Y = torch.empty((M, c0.N), dtype=torch.bfloat16, device="cuda")
+            line = {"groups": c0.workload, "layer": name, "M": M, "K": c0.K, "N": c0.N}
+            for group in (128, 64, 32):
+                pws, wbytes = packs[group]
+                ws = torch.zeros(max(w4.workspace_bytes_g(M, c0.N, c0.K, group), 256), dtype=torch.uint8,
+                                 device="cuda")
+                passes = max(1, -(-200 // len(pws))) if M < 512 else 1
 
-            def body(pws=pws, group=group, ws=ws):
-                for _ in range(passes):
-                    for p in pws:
-                        w4.linear_g(X, group, p.qweight, p.scales, p.zeros, Y, ws)
-            us = _time_graph(torch, stream, body, passes * copies)
-            line.update({f"g{group}_us": us, f"g{group}_code_gbs": c.code_bytes / us / 1e3,
-                         f"g{group}_all_gbs": wbytes / us / 1e3})
-            del pws, ws
-            torch.cuda.empty_cache()
-        line["fault"] = w4.device_fault()
-        print(json.dumps(line), flush=True)
-        del W, X, Y
+                def body(pws=pws, group=group, ws=ws):
+                    for _ in range(passes):
+                        for p in pws:
+                            w4.linear_g(X, group, p.qweight, p.scales, p.zeros, Y, ws)
+                us = _time_graph(torch, stream, body, passes * len(pws))
+                line.update({f"g{group}_us": us, f"g{group}_code_gbs": c0.code_bytes / us / 1e3,
+                             f"g{group}_all_gbs": wbytes / us / 1e3})
+                if M >= 64:
+                    line[f"g{group}_tflops"] = 2 * M * c0.N * c0.K / us / 1e6
+                del ws
+            line["fault"] = w4.device_fault()
+            print(json.dumps(line), flush=True)
+            del X, Y
+        del packs
         torch.cuda.empty_cache()
 
 
@@ -1135,7 +1150,8 @@ def main():
                     help="decode, or a comma list of token counts: W8A16 layers timed beside W4A16 and a cuBLAS "
                          "BF16 GEMM on the decode shapes, one JSON line each")
     ap.add_argument("--groups", default=None,
-                    help="decode: quantisation groups of 32, 64 and 128 timed on the decode shapes, one line each")
+                    help="decode|batched|all: quantisation groups of 32, 64 and 128 timed on the decode shapes "
+                         "(M = 1) and the hidden-8192 shapes (M = 4, 16, 40, 512), one line each")
     ap.add_argument("--variants", default=None,
                     help="decode|small_batch|prefill|all: affine, symmetric-packed and AWQ-folded layers timed "
                          "on the same kernels, one JSON line per layer")

@@ -63,7 +63,9 @@ typedef enum {
 /* Kernel family selection for w4a16_linear_path(). */
 typedef enum {
     W4A16_PATH_AUTO = 0,    /* decode GEMV for small M, tensor-core GEMM for large M */
-    W4A16_PATH_DECODE = 1,  /* split-K GEMV: register dequantisation, any M (tiles of 32 tokens) */
+    W4A16_PATH_DECODE = 1,  /* split-K GEMVs, any M: integer mma.sync (codes x digit planes of X) for
+                               M <= 8, tcgen05 (8-bit, codes from tensor memory) for more, in chunks of
+                               32 tokens */
     W4A16_PATH_PREFILL = 2  /* TMA + tcgen05/TMEM GEMM on BF16 tiles dequantised in shared memory */
 } w4a16_path;
 
@@ -130,10 +132,12 @@ W4A16_API size_t w4a16_workspace_bytes_g(int64_t M, int64_t N, int64_t K, int gr
 
 /*
  * The linear layer on weights packed with groups of `group` (32, 64 or 128;
- * 128 is w4a16_linear).  For 32 and 64: the integer GEMV with the sub-groups of
- * each 128-K tile kept apart in the X operand (each digit plane split per
- * sub-group), one token per launch (larger M runs as consecutive launches:
- * decode is the intended use), K a multiple of 512 (W4A16_ERR_SHAPE otherwise).
+ * 128 is w4a16_linear).  For 32 and 64, K a multiple of 512 (W4A16_ERR_SHAPE
+ * otherwise): M = 1 runs the integer GEMV with the sub-groups of each 128-K
+ * tile kept apart in the X operand (each digit plane split per sub-group);
+ * M >= 2 runs the BF16 tensor-core GEMV with one FP32 accumulator per
+ * quantisation group, in chunks of 32 tokens (also for M >= 64, where the
+ * group-128 layer takes the GEMM).
  * Arguments, layouts and errors otherwise as w4a16_linear, with scales and
  * zeros [N][K/group] and workspace >= w4a16_workspace_bytes_g(M, N, K, group).
  */
@@ -168,6 +172,9 @@ W4A16_API int w4a16_workspace_init(void* workspace, size_t bytes, void* stream);
  *   zeros     device, int32 [N][K/128]
  *   Y         device, bf16 bits [M][N] (written; must not overlap the inputs)
  *   workspace device, >= w4a16_workspace_bytes(M, N, K) bytes (NULL allowed when that is 0)
+ * Activations: the decode GEMVs take every finite BF16 value; the GEMM
+ * (M >= 64) sums (q - c) x in FP32 before the scale and needs |x| < 2^113.
+ * Results are the same bits on every run.
  */
 W4A16_API int w4a16_linear(const uint16_t* X, int64_t M, int64_t K, const uint32_t* qweight, const uint16_t* scales,
                  const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, size_t workspace_bytes,

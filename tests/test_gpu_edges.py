@@ -31,10 +31,12 @@ from tests._parity import assert_close, bf16_dev_to_f64, bits_to_dev_bf16
 pytestmark = pytest.mark.gpu
 
 ALL = list(edge.KINDS)
-# The GEMM multiplies BF16 (q - z) by BF16 x in FP32 before the scale: |x| * 15 must stay below the FP32
-# maximum, so activations of magnitude 2^124 and above are outside its range (the decode paths take every
+# The kernels on BF16 operands -- the GEMM, and the tensor-core GEMV for groups of 32/64 beyond one
+# token -- multiply BF16 (q - c) by BF16 x and sum in FP32 before the scale: activations must stay below
+# 2^113 in magnitude, so the largest finite BF16 is outside their range (the integer GEMVs take every
 # finite BF16 value).
 PREFILL_KINDS = [k for k in ALL if k != "max_finite"]
+BF16_KINDS = PREFILL_KINDS
 # x * inv_s of the largest finite BF16 overflows for inv_s > 1: the transformed activation is not finite.
 AWQ_KINDS = [k for k in ALL if k != "max_finite"]
 
@@ -107,10 +109,21 @@ def test_two_tokens(cuda_lib, pair):
     _check_rows(Y, oracle.linear(X, qw, sc, z), pair, "M=2")
 
 
-@pytest.mark.parametrize("M", [3, 11, 16, 40])
+@pytest.mark.parametrize("M", [3, 5, 8])
+def test_small_batch_integer_gemv(cuda_lib, M):
+    """2 <= M <= 8: digit planes prepared once per launch (4- and 8-token tiles), mma.sync u8 x s8."""
+    N, K = 200, 2048
+    kinds = [ALL[m % len(ALL)] for m in range(M)]
+    pw, (qw, sc, z) = _pack(N, K, 13)
+    X = edge.activations_bf16(300 + M, kinds, K)
+    Y = _linear(X, pw, w4.PATH_DECODE)
+    _check_rows(Y, oracle.linear(X, qw, sc, z), kinds, f"M={M}")
+
+
+@pytest.mark.parametrize("M", [9, 11, 16, 40])
 def test_tensor_core_gemv(cuda_lib, M):
-    """3 <= M <= 63: digit planes prepared per launch, tcgen05 kind::i8 (16- and 32-token tiles; M = 40 runs
-    a 32-token and an 8-token launch)."""
+    """9 <= M <= 63: the codes as 8-bit A operands in tensor memory against the digit planes of every token,
+    tcgen05 kind::i8 (16- and 32-token tiles; M = 40 runs a 32-token and an 8-token launch)."""
     N, K = 200, 2048
     kinds = [ALL[m % len(ALL)] for m in range(M)]
     pw, (qw, sc, z) = _pack(N, K, 13)
@@ -120,16 +133,22 @@ def test_tensor_core_gemv(cuda_lib, M):
 
 
 @pytest.mark.parametrize("group", [32, 64])
-def test_small_groups(cuda_lib, group):
-    """Groups of 32 and 64: the integer GEMV with per-sub-group digit rows, one token per launch."""
+@pytest.mark.parametrize("batched", [False, True])
+def test_small_groups(cuda_lib, group, batched):
+    """Groups of 32 and 64: one token per call on the integer GEMV with per-sub-group digit rows (every
+    kind), or all rows in one call on the BF16 tensor-core GEMV (every kind but the largest finite)."""
     N, K = 200, 1024
-    kinds = ALL
+    kinds = BF16_KINDS if batched else ALL
     pw, (qw, sc, z) = _pack(N, K, 14, group)
     X = edge.activations_bf16(400 + group, kinds, K)
     M = len(kinds)
     Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     ws = torch.zeros(max(w4.workspace_bytes_g(M, N, K, group), 256), dtype=torch.uint8, device="cuda")
-    w4.linear_g(bits_to_dev_bf16(X), group, pw.qweight, pw.scales, pw.zeros, Y, ws)
+    if batched:
+        w4.linear_g(bits_to_dev_bf16(X), group, pw.qweight, pw.scales, pw.zeros, Y, ws)
+    else:
+        for m in range(M):
+            w4.linear_g(bits_to_dev_bf16(X[m:m + 1]), group, pw.qweight, pw.scales, pw.zeros, Y[m:m + 1], ws)
     torch.cuda.synchronize()
     assert w4.device_fault() == 0
     _check_rows(Y, oracle.linear_g(X, qw, sc, z), kinds, f"group {group}")

@@ -86,6 +86,22 @@ def test_linear_small_shapes_all_outputs(cuda_lib, G, M, N, K):
 
 
 @pytest.mark.parametrize("G", GROUPS)
+@pytest.mark.parametrize("M", [2, 4, 9, 16, 17, 40, 512])
+def test_batched_token_counts_all_outputs(cuda_lib, G, M):
+    """Batched decode and prefill token counts on the BF16 tensor-core GEMV with one accumulator per
+    quantisation group (tiles of 16 and 32 tokens, M > 32 in chunks of 32)."""
+    N, K = 200, 1024
+    W = synth.weights_f32(7000 + M + G, synth.TAG_W, N, K)
+    W[: N // 5] += np.float32(0.05)
+    W[0, :256] += np.float32(2.0)  # one-signed groups: zero points far outside 0..15
+    X = synth.activations_bf16(7100 + M, M, K)
+    pw = _pack(torch.from_numpy(W).cuda(), G)
+    st, qw, sc, z = oracle.quantize_pack_g(W, G)
+    assert np.abs(z).max() > 128  # the fold's zero-point branch is exercised
+    assert_close(bf16_dev_to_f64(_linear(X, pw)), oracle.linear_g(X, qw, sc, z), f"G={G} M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("G", GROUPS)
 def test_one_hot_inputs_pick_weight_columns(cuda_lib, G):
     """x = e_k gives Y[:, n] = bf16(w_hat[n][k]) exactly: pins the sub-group split of the X
     operand, the per-lane fold and the metadata addressing of every sub-group."""

@@ -13,8 +13,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libw4a16.so")
 OBJ_DIR = os.path.join(PKG, "_build")
-SOURCES = ["api.cu", "runtime.cu", "pack.cu", "gemv.cu", "gemv_mt.cu", "gemv_sub.cu", "gemm.cu", "noalloc.cu",
-           "w8.cu"]
+SOURCES = ["api.cu", "runtime.cu", "pack.cu", "gemv.cu", "gemv_mt.cu", "gemv_bf.cu", "gemv_sub.cu", "gemm.cu",
+           "noalloc.cu", "w8.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "decode_units.cuh"]
 
 NVCC_FLAGS = [

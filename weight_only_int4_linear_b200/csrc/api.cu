@@ -241,7 +241,10 @@ size_t w4a16_workspace_bytes_g(int64_t M, int64_t N, int64_t K, int group) {
     if (group == 128) return w4a16_workspace_bytes(M, N, K);
     if ((group != 32 && group != 64) || check_shape(M, N, K) != W4A16_OK || K % 512 != 0) return 0;
     check_device();
-    return decode_sub_workspace_bytes(N, K, group);
+    // one token: the integer GEMV with per-sub-group digit rows; more: the BF16 tensor-core GEMV (its
+    // scratch after the shared counter area, which it leaves untouched)
+    if (M == 1) return decode_sub_workspace_bytes(N, K, group);
+    return kCounterBytes + bf_workspace_bytes(M, N, K, group, num_sms_current());
 }
 
 int w4a16_linear_g(const uint16_t* X, int64_t M, int64_t K, int group, const uint32_t* qweight,
@@ -258,10 +261,12 @@ int w4a16_linear_g(const uint16_t* X, int64_t M, int64_t K, int group, const uin
     if (!aligned16(X) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(Y))
         return W4A16_ERR_ALIGN;
     if ((st = check_device()) != W4A16_OK) return st;
-    const size_t need = decode_sub_workspace_bytes(N, K, group);
+    const size_t need = w4a16_workspace_bytes_g(M, N, K, group);
     if (!workspace || workspace_bytes < need) return W4A16_ERR_WORKSPACE;
     if (!aligned16(workspace)) return W4A16_ERR_ALIGN;
-    return launch_decode_sub(X, M, K, group, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
+    if (M == 1) return launch_decode_sub(X, M, K, group, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
+    return launch_decode_bf(X, nullptr, M, K, group, qweight, scales, zeros, N, Y,
+                            reinterpret_cast<char*>(workspace) + kCounterBytes, (cudaStream_t)stream);
 }
 
 int w8a16_quantize(const float* W, int64_t N, int64_t K, int8_t* qweight, uint16_t* scales, int32_t* dev_status,

@@ -141,7 +141,8 @@ constexpr size_t kCounterBytes = (size_t)kSharedCounterTiles * 4;  // 256 KB
 
 struct DecodePlan {
     int cc_tokens;    // > 0: the integer CUDA-core kernel for this many tokens (M <= 2)
-    bool mt;          // the integer GEMV for 3-16 tokens per launch (gemv_mt.cu), in chunks of 16 tokens
+    bool mt;          // the integer GEMV for 2-16 tokens per launch (gemv_mt.cu), in chunks of 16 tokens
+    bool bf;          // the BF16 tensor-core GEMV (gemv_bf.cu), in chunks of 32 tokens
     int nt;           // tensor-core kernel: MMA N (16 or 32 tokens per launch); 1 with cc_tokens
     int row_tiles;    // 128-row tiles along N
     int grid;         // persistent CTAs
@@ -160,13 +161,25 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
                   const DecodePlan& plan, cudaStream_t stream);
 int num_sms_current();
 
-// The integer GEMV for 3-16 tokens per launch (gemv_mt.cu): needs K / 128 to be a multiple of 8;
+// The BF16 tensor-core GEMV (gemv_bf.cu) for quantisation groups of `group` (32, 64, 128) weights:
+// scratch = bf_workspace_bytes (after the shared counters); runs M in chunks of 32 tokens.
+size_t bf_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int num_sms);
+int launch_decode_bf(const uint16_t* X, const float* xscale, int64_t M, int64_t K, int group, const uint32_t* qweight,
+                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* scratch,
+                     cudaStream_t stream);
+
+// Split-K reduction of the decode GEMVs (gemv.cu): a dependent grid of one CTA per 128-row tile that
+// adds the partial-sum slots of every tile the GEMV's CTAs shared, in slot order, into Y.
+int launch_decode_reduce(const float* partial, uint16_t* Y, int64_t N, int M, int G, int units_base, int units_rem,
+                         int max_slots, int row_tiles, cudaStream_t stream);
+
+// The integer GEMV for 2-16 tokens per launch (gemv_mt.cu): needs K / 128 to be a multiple of 8;
 // scratch (after the shared counters) = mt_workspace_bytes; runs M in chunks of 16 tokens.
 bool mt_supported(int64_t K);
 size_t mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 int launch_decode_mt(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
-                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, int* counters,
-                     void* scratch, cudaStream_t stream);
+                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* scratch,
+                     cudaStream_t stream);
 
 // Prefill (tensor-core GEMM) path for large M.
 constexpr int64_t kPrefillMinM = 64;  // W4A16_PATH_AUTO switches to the GEMM at this many tokens

@@ -43,6 +43,9 @@ namespace {
 constexpr int kRowsPerCta = 128;
 constexpr int kStageWords = kRowsPerCta * kWordsPerGroup;  // 2048 words = 8 KB
 constexpr int kMaxTokens = 32;  // tokens per launch
+// Token counts up to this take the integer mma.sync GEMV (when K / 128 is a multiple of 8): its MMAs grow
+// with 3 digit planes per token and bound it beyond 8 tokens, where the tcgen05 GEMV is as fast.
+constexpr int64_t kMtMaxTokens = 8;
 
 struct DecodeArgs {
     const uint16_t* Xp;  // [Mc][K] BF16, 8-blocks reordered (0,4,1,5,2,6,3,7); the input X itself for M = 1
@@ -502,9 +505,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 }
 
 // --------------------------------------------------------------------------
-// One- and two-token decode kernel (M <= 2).
+// One-token decode kernel (M = 1).
 //
-// At M <= 2 a tcgen05 MMA would waste most of its columns, and its operands
+// At M = 1 a tcgen05 MMA would waste most of its columns, and its operands
 // would have to pass through tensor memory; the dot products instead run as
 // warp-level mma.sync m16n8k32 in registers: A = 16 rows x 32 codes as
 // unsigned bytes, straight from the packed words (w & 0x0F0F0F0F holds codes
@@ -514,12 +517,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // largest |x|, x_int = x * 2^(21 - E) (exact for every x within 2^14 of the
 // group maximum; smaller values are rounded at 2^(E - 21), far below FP32
 // accumulation error), written in balanced base 256, x_int = 65536 d2 +
-// 256 d1 + d0 with every digit in [-128, 127]; column n = p NT + m of B holds
-// digit plane p of token m (columns past 3 NT are zero).  Per group and row:
-//   acc += s 2^(E - 21) (65536 D2 + 256 D1 + D0 - z sum_k x_int).
-// One MMA takes 32 codes of 16 rows against every plane of both tokens: a
-// compute thread issues 8 MMAs per 128 x 128 unit where byte-plane dp4a would
-// take 96 instructions.
+// 256 d1 + d0 with every digit in [-128, 127]; columns 0-2 of B hold digit
+// planes 0-2, columns 4-6 the same planes again (so that the lanes holding
+// accumulator columns 4-7 have every plane of the second row block), columns
+// 3 and 7 are zero.  Per group and row:
+//   acc += s (65536 D2 + 256 D1 + D0 - z sum_k x_int) 2^(E - 21).
+// One MMA takes 32 codes of 16 rows against every plane: a compute thread
+// issues 8 MMAs per 128 x 128 unit where byte-plane dp4a would take 96
+// instructions, and each lane of a quad folds one of the quad's four rows.
 //
 // X of one group in the layout the kernel reads: 3 NT digit rows of 128 bytes
 // (word w's codes 0,2,4,6 at 8w, codes 1,3,5,7 at 8w + 4: the order in which
@@ -536,7 +541,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 //  * warps 0-3 compute, warp w taking rows 32 w .. 32 w + 31 of each unit as
 //    two 16-row MMA blocks.
 // Up to four CTAs share an SM: their independent rings keep more loads in
-// flight than one CTA per SM with an in-order ring of the same depth.
+// flight than one CTA per SM with an in-order ring of the same depth.  A row
+// tile whose units two CTAs share is written by each as a partial-sum slot,
+// and decode_reduce_kernel, launched as a dependent grid, adds the slots in a
+// fixed order: no CTA waits on another or on an atomic at its end, and each
+// CTA frees its SM for the next layer's weight stream as soon as it is done.
 #ifndef W4A16_CC_WARPS
 #define W4A16_CC_WARPS 4
 #endif
@@ -552,7 +561,6 @@ constexpr int kCcXWarp = kCcWarps + 1;                  // warp 5
 constexpr int kCcThreads = (kCcWarps + 2) * 32;
 constexpr int kCcStages = W4A16_CC_STAGES;
 constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
-constexpr int kCcMaxTokens = 2;                         // tokens per launch of the integer kernel
 constexpr int kCcXOff = kCcCodeBytes;                   // X digit rows of the unit's group, after the codes
 // X of one group (layout above), and codes + X, 512-aligned (the 64-byte swizzle's span)
 template <int NT>
@@ -591,30 +599,39 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
 
 // One warp writes token m's digits of group g (its lanes' values v from load_group_x) in the layout
 // above: digit row n = p NT + m.
+//
+// x_int = rint(x 2^kx) comes from one FFMA with the 1.5 2^23 magic constant (|x 2^kx| < 2^22, so the
+// sum's last place is 1 and its rounding is the rounding to the nearest integer, ties to even), and
+// x_int + 0x808080 = (d0 + 128) + 256 (d1 + 128) + 65536 (d2 + 128) holds the three balanced base-256
+// digits, each plus 128, in its three low bytes: the digit bytes are that word XOR 0x808080.
 template <int NT>
 __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst, int lane, int m) {
-    const uint32_t bits[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
-    uint32_t amax = max(max(bits[0] & 0x7FFFu, bits[1] & 0x7FFFu), max(bits[2] & 0x7FFFu, bits[3] & 0x7FFFu));
+    const uint32_t a2 = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    uint32_t amax = max(a2 & 0xFFFFu, a2 >> 16);
     amax = __reduce_max_sync(0xFFFFFFFFu, amax);
     const int ef = (int)(amax >> 7);
     const int E = ef == 0 ? -127 : ef - 127;  // every |x| of the group is below 2^(E + 1)
     const int kx = 21 - E;                    // in [-106, 148]
     const int k1 = min(kx, 127);
     const float s1 = pow2f(k1), s2 = pow2f(kx - k1);  // exact scalings, |x * 2^kx| < 2^22
-    int xi[4];
-    uint32_t dg[3] = {0u, 0u, 0u};  // this lane's digit bytes per plane, as (i0, i2, i1, i3)
+    const float xv[4] = {__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                         __uint_as_float(v.y & 0xFFFF0000u)};
+    uint32_t D[4];
+    int sum4 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        xi[i] = __float2int_rn(__uint_as_float(bits[i] << 16) * s1 * s2);
-        const int d0 = ((xi[i] + 128) & 255) - 128;
-        const int t = (xi[i] - d0) >> 8;
-        const int d1 = ((t + 128) & 255) - 128;
-        const int d2 = (t - d1) >> 8;
-        const int pos = (i & 1) ? 16 + 8 * (i >> 1) : 8 * (i >> 1);  // i0 -> 0, i2 -> 8, i1 -> 16, i3 -> 24
-        dg[0] |= (uint32_t)(d0 & 255) << pos;
-        dg[1] |= (uint32_t)(d1 & 255) << pos;
-        dg[2] |= (uint32_t)(d2 & 255) << pos;
+        const float f = __fmaf_rn(xv[i] * s1, s2, 12582912.f);  // 1.5 2^23 + x_int
+        const uint32_t yb = __float_as_uint(f) - (0x4B400000u - 0x808080u);  // x_int + 0x808080
+        sum4 += (int)yb;
+        D[i] = yb ^ 0x808080u;  // bytes 0..2: digits d0, d1, d2 as signed bytes
     }
+    // planes as (i0, i2, i1, i3): P = [d0 i0, d0 i2, d1 i0, d1 i2], Q = the same for i1, i3; R, S plane 2
+    const uint32_t P = __byte_perm(D[0], D[2], 0x5140), Q = __byte_perm(D[1], D[3], 0x5140);
+    const uint32_t R = __byte_perm(D[0], D[2], 0x0062), S = __byte_perm(D[1], D[3], 0x0062);
+    uint32_t dg[3];
+    dg[0] = __byte_perm(P, Q, 0x5410);
+    dg[1] = __byte_perm(P, Q, 0x7632);
+    dg[2] = __byte_perm(R, S, 0x5410);
     // lane (w, h) holds codes 4h .. 4h + 3 of word w; h = 0 assembles the even-code register
     // (its codes 0, 2, the partner's 4, 6), h = 1 the odd one (the partner's 1, 3, its own 5, 7)
     const int h = lane & 1, w = lane >> 1;
@@ -625,7 +642,7 @@ __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst,
         const uint32_t out = h ? __byte_perm(lo, hi, 0x7632) : __byte_perm(lo, hi, 0x5410);
         *reinterpret_cast<uint32_t*>(dst + (p * NT + m) * 128 + 8 * w + 4 * h) = out;
     }
-    const int sum = __reduce_add_sync(0xFFFFFFFFu, (xi[0] + xi[1]) + (xi[2] + xi[3]));  // |sum| < 2^29
+    const int sum = __reduce_add_sync(0xFFFFFFFFu, sum4) - 128 * (int)0x808080;  // |sum| < 2^29
     if (lane == 0) {
         float* ext = reinterpret_cast<float*>(dst + 3 * NT * 128);
         ext[2 * m] = (float)sum;
@@ -635,16 +652,13 @@ __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst,
 
 
 template <int NT>
-#ifndef W4A16_CC2_MIN_BLOCKS
-#define W4A16_CC2_MIN_BLOCKS 3
-#endif
-__global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
-                                                               const __grid_constant__ CUtensorMap tsc,
-                                                               const __grid_constant__ CUtensorMap tze,
-                                                               const DecodeArgs a) {
+__global__ void __launch_bounds__(kCcThreads, 4) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
+                                                                  const __grid_constant__ CUtensorMap tsc,
+                                                                  const __grid_constant__ CUtensorMap tze,
+                                                                  const DecodeArgs a) {
+    static_assert(NT == 1, "one token per launch");
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages];
-    __shared__ int s_last;
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((512u - (raw & 511u)) & 511u);  // 512-aligned stages
     constexpr int kStageBytes = cc_stage_bytes<NT>();
@@ -729,7 +743,6 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
     }
 
     // ---------------------------------------------------- compute warps 0-3
-    const int t = threadIdx.x;
     // Warp w takes rows 32 w .. 32 w + 31 as two 16-row MMA blocks.  Lane (g8, tig) = (lane / 4,
     // lane % 4) holds, per block, rows g8 and g8 + 8 of its A fragments and words 4 tig .. 4 tig + 3
     // of each (one 16-byte chunk of the codes tile); MMA j takes word 4 tig + j of every lane, so
@@ -737,56 +750,23 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
     // words of digit plane n = g8.  After a unit, D column n = p NT + m of a row is
     // sum_k q_k d_p(x_k) of token m; lane tig = m gathers its three planes and folds the row.
     const int g8 = lane >> 2, tig = lane & 3;
-    const int mt = tig < NT ? tig : NT - 1;  // the token this lane folds (lanes tig < NT)
-    const bool owner = tig < NT && tig < a.M;
     auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
+    float y = 0.f;  // row rrow(tig) of the current row tile
     int cur_tile = -1;
     bool aborted = false;
 
+    // A row tile leaves the CTA as Y (the CTA holds all of its units) or as this CTA's partial-sum slot
+    // (decode_reduce_kernel adds the slots).
     auto flush = [&](int tile) {
         const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
         const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
         if (first == last) {
-            if constexpr (NT == 1) {  // lane tig holds row rrow(tig)
-                const int n = tile * kRowsPerCta + rrow(tig);
-                if (n < N) a.Y[n] = float_to_bf16_bits(y[0]);
-            } else if (owner) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int n = tile * kRowsPerCta + rrow(k);
-                    if (n < N) a.Y[(int64_t)mt * N + n] = float_to_bf16_bits(y[k]);
-                }
-            }
+            const int n = tile * kRowsPerCta + rrow(tig);
+            if (n < N) a.Y[n] = float_to_bf16_bits(y);
         } else {
-            const int slot = b - first, nseg = last - first + 1;
-            float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * a.M * kRowsPerCta;
-            if constexpr (NT == 1) {
-                part[rrow(tig)] = y[0];
-            } else if (owner) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) part[mt * kRowsPerCta + rrow(k)] = y[k];
-            }
-            named_barrier_sync(1, kCcWarps * 32);
-            if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
-            named_barrier_sync(1, kCcWarps * 32);
-            if (s_last) {
-                const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
-                const float* pb = a.partial + (int64_t)tile * a.max_slots * a.M * kRowsPerCta;
-#pragma unroll
-                for (int m = 0; m < NT; ++m) {
-                    if (m >= a.M) break;
-                    for (int rl = t; rl < rows; rl += kCcWarps * 32) {
-                        const float sum = sum_slots(pb + (int64_t)m * kRowsPerCta + rl, (int64_t)a.M * kRowsPerCta, nseg);
-                        a.Y[(int64_t)m * N + tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
-                    }
-                }
-                if (t == 0) a.counters[tile] = 0;
-            }
-            named_barrier_sync(1, kCcWarps * 32);
+            a.partial[((int64_t)tile * a.max_slots + (b - first)) * kRowsPerCta + rrow(tig)] = y;
         }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) y[k] = 0.f;
+        y = 0.f;
     };
 
     UnitCursor uc(u_first, G);
@@ -812,11 +792,11 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
             const int r = rrow(k);
             cw[k] = *reinterpret_cast<const uint4*>(st + r * 64 + 16 * (tig ^ ((r >> 1) & 3)));
         }
+        // B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of the second
+        // row block and each lane of a quad can fold one of its four rows; columns 3 and 7 are zero
         uint32_t bx[8];
-        // one token: B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of
-        // the second row block and each lane of a quad can fold one of its four rows
-        const int xrow = NT == 1 ? (g8 & 3) : g8;
-        if (xrow < 3 * NT) {
+        const int xrow = g8 & 3;
+        if (xrow < 3) {
             const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + xrow * 128 + tig * 32);
             const uint4 u0 = xp[0], u1 = xp[1];
             bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
@@ -825,86 +805,46 @@ __global__ void __launch_bounds__(kCcThreads, NT == 1 ? 4 : W4A16_CC2_MIN_BLOCKS
 #pragma unroll
             for (int j = 0; j < 8; ++j) bx[j] = 0u;
         }
-        const float* ext = reinterpret_cast<const float*>(st + kCcXOff + 3 * NT * 128);
-        const float xsum = ext[2 * mt], xscale = ext[2 * mt + 1];
-        // this block's metadata (loaded with its first unit, which this warp has already waited for);
-        // rows past N were zero-filled by TMA: s = 0 folds them away
+        const float* ext = reinterpret_cast<const float*>(st + kCcXOff + 3 * 128);
+        const float xsum = ext[0], xscale = ext[1];
+        // this lane's row's metadata, from the block loaded with the block's first unit (which this warp
+        // has already waited for); rows past N were zero-filled by TMA: s = 0 folds them away
         const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
-        float sv[4], zv[4];
-#pragma unroll
-        for (int k = 0; k < (NT == 1 ? 1 : 4); ++k) {
-            const int r = NT == 1 ? rrow(tig) : rrow(k);
-            sv[k] = bf16_bits_to_float(
-                *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
-            zv[k] = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
-                                                             4 * (g & (kCcMetaGroups - 1)));
-        }
+        const int r = rrow(tig);
+        const float sv = bf16_bits_to_float(
+            *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
+        const float zv = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
+                                                                  4 * (g & (kCcMetaGroups - 1)));
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
-        if constexpr (NT == 1) {
-            int d[2][4];
+        int d[2][4];
 #pragma unroll
-            for (int rb = 0; rb < 2; ++rb) {
-                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
-                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
+        for (int rb = 0; rb < 2; ++rb) {
+            const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+            const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) d[rb][j] = 0;
+            for (int j = 0; j < 4; ++j) d[rb][j] = 0;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_u8s8(d[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
-                             (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
-            }
-            // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes
-            // (0, 1) at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block
-            // tig >> 1 (its own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour
-            // completes its planes.
-            const bool hi = tig >> 1, even = !(tig & 1);
-            int e[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) e[j] = hi ? d[1][j] : d[0][j];
-            const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
-            const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
-            const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
-            const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-            y[0] = fmaf(sv[0] * fmaf(-zv[0], xsum, qx), xscale, y[0]);
-        } else {
-    #pragma unroll
-            for (int rb = 0; rb < 2; ++rb) {
-                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
-                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
-                int d[4] = {0, 0, 0, 0};
-    #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_u8s8(d, w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
-                             (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
-                // lane tig holds columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3)
-    #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    int P0, P1, P2;
-                    if constexpr (NT == 1) {  // planes 0, 1 at lane tig 0, plane 2 at lane tig 1
-                        P0 = d[2 * h];
-                        P1 = d[2 * h + 1];
-                        P2 = __shfl_sync(0xFFFFFFFFu, d[2 * h], lane | 1);
-                    } else {  // column p NT + m: token 0 planes at (0,0), (1,0), (2,0); token 1 at (0,1), (1,1), (2,1)
-                        const int own = tig == 0 ? d[2 * h] : d[2 * h + 1];
-                        const int x = __shfl_xor_sync(0xFFFFFFFFu, tig == 0 ? d[2 * h + 1] : d[2 * h], 1);
-                        const int t0 = __shfl_sync(0xFFFFFFFFu, d[2 * h], (lane & ~3) | 2);
-                        const int t1 = __shfl_sync(0xFFFFFFFFu, d[2 * h + 1], (lane & ~3) | 2);
-                        P0 = tig == 0 ? own : x;
-                        P1 = tig == 0 ? x : own;
-                        P2 = tig == 0 ? t0 : t1;
-                    }
-                    // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26),
-                    // the rest FP32 with one rounding per step
-                    const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-                    const int k = 2 * rb + h;
-                    // s (sum (q - z) x_int), then the power of two: neither product leaves the FP32 range
-                    // unless the group's result itself does
-                    y[k] = fmaf(sv[k] * fmaf(-zv[k], xsum, qx), xscale, y[k]);
-                }
-            }
+            for (int j = 0; j < 4; ++j)
+                mma_u8s8(d[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
+                         (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
         }
+        // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes (0, 1)
+        // at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block tig >> 1 (its
+        // own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour completes its planes.
+        const bool hi = tig >> 1, even = !(tig & 1);
+        int e[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) e[j] = hi ? d[1][j] : d[0][j];
+        const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
+        const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
+        const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
+        // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26); then
+        // s (sum (q - z) x_int) and the power of two last, so that neither product leaves the FP32 range
+        // unless the group's result itself does
+        const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+        y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
     }
     if (cur_tile >= 0) flush(cur_tile);
 }
@@ -944,7 +884,6 @@ int occupancy_cc() {
 // cc_tokens > 0: the integer CUDA-core kernel for that many tokens; else the tensor-core kernel with MMA N = ntok
 int occupancy(int cc_tokens, int ntok) {
     if (cc_tokens == 1) return occupancy_cc<1>();
-    if (cc_tokens == 2) return occupancy_cc<2>();
     return ntok == 16 ? occupancy_nt<16>() : occupancy_nt<32>();
 }
 
@@ -1027,18 +966,67 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 }  // namespace
 
+// Split-K reduction of the decode GEMVs: a tile whose units one CTA held was written as Y by that CTA; a
+// tile shared by CTAs first .. last is the sum of their partial-sum slots, added here in slot order (the
+// same bits on every run).  A dependent grid of at most one small CTA per SM, looping over the row
+// tiles: it fits beside the GEMV's CTAs, so all of it is resident (and has released its own dependents)
+// while the GEMV still runs, and it waits for the GEMV only when it reaches a shared tile.
+__global__ void __launch_bounds__(128) decode_reduce_kernel(const float* __restrict__ partial, uint16_t* __restrict__ Y,
+                                                            int N, int M, int G, int units_base, int units_rem,
+                                                            int max_slots, int row_tiles) {
+    pdl_launch_dependents();
+    bool waited = false;
+    for (int tile = blockIdx.x; tile < row_tiles; tile += gridDim.x) {
+        const int first = cta_of_unit((int64_t)tile * G, units_base, units_rem);
+        const int last = cta_of_unit((int64_t)tile * G + G - 1, units_base, units_rem);
+        if (first == last) continue;
+        if (!waited) {
+            pdl_wait_primary();
+            waited = true;
+        }
+        const int nseg = last - first + 1, rows = min(kRowsPerCta, N - tile * kRowsPerCta);
+        const float* pb = partial + (int64_t)tile * max_slots * M * kRowsPerCta;
+        for (int idx = threadIdx.x; idx < M * rows; idx += 128) {
+            const int m = idx / rows, rl = idx - m * rows;
+            const float sum = sum_slots(pb + (int64_t)m * kRowsPerCta + rl, (int64_t)M * kRowsPerCta, nseg);
+            Y[(int64_t)m * N + tile * kRowsPerCta + rl] = float_to_bf16_bits(sum);
+        }
+    }
+}
+
+int launch_decode_reduce(const float* partial, uint16_t* Y, int64_t N, int M, int G, int units_base, int units_rem,
+                         int max_slots, int row_tiles, cudaStream_t stream) {
+    const int sms = num_sms_current();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(row_tiles < sms ? row_tiles : sms));
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_reduce_kernel, partial, Y, (int)N, M, G, units_base, units_rem, max_slots,
+                              row_tiles) == cudaSuccess
+               ? W4A16_OK
+               : W4A16_ERR_CUDA;
+}
+
 DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     DecodePlan p{};
     const int64_t Mc = M < kMaxTokens ? M : kMaxTokens;
     const int64_t G = K / kGroup;
-    // the integer CUDA-core kernel for M <= kCcMaxTokens (needs 16-byte metadata rows: G % 8 == 0);
+    // the one-token integer kernel for M = 1 (needs 16-byte metadata rows: G % 8 == 0);
     // else the tensor-core kernel with MMA N = 16 or 32
-    p.cc_tokens = (M <= kCcMaxTokens && G % 8 == 0) ? (int)M : 0;
-    p.mt = !p.cc_tokens && mt_supported(K);
+    p.cc_tokens = (M <= 1 && G % 8 == 0) ? (int)M : 0;
+    p.mt = !p.cc_tokens && mt_supported(K) && M <= kMtMaxTokens;
+    // 9 or more tokens (or K / 128 not a multiple of 8): the 8-bit tensor-core GEMV below; the BF16
+    // tensor-core GEMV (gemv_bf.cu) serves quantisation groups of 32 and 64
+    p.bf = false;
     p.nt = p.cc_tokens ? 1 : (Mc <= 16 ? 16 : 32);
     p.row_tiles = (int)ceil_div(N, kRowsPerCta);
-    if (p.mt) {  // the 3-16-token integer GEMV keeps its own plan per chunk; only its scratch is sized here
-        p.ws_xp_bytes = mt_workspace_bytes(M, N, K, num_sms);
+    if (p.mt || p.bf) {  // these GEMVs keep their own plans per chunk; only their scratch is sized here
+        p.ws_xp_bytes = p.mt ? mt_workspace_bytes(M, N, K, num_sms) : bf_workspace_bytes(M, N, K, kGroup, num_sms);
         p.ws_xs_bytes = 0;
         p.ws_partial_bytes = 0;
         p.ws_counter_bytes =
@@ -1088,7 +1076,10 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                   const DecodePlan& plan, cudaStream_t stream) {
     if (plan.mt)
-        return launch_decode_mt(X, xscale, M, K, qweight, scales, zeros, N, Y, reinterpret_cast<int*>(workspace),
+        return launch_decode_mt(X, xscale, M, K, qweight, scales, zeros, N, Y,
+                                reinterpret_cast<char*>(workspace) + plan.ws_counter_bytes, stream);
+    if (plan.bf)
+        return launch_decode_bf(X, xscale, M, K, kGroup, qweight, scales, zeros, N, Y,
                                 reinterpret_cast<char*>(workspace) + plan.ws_counter_bytes, stream);
     CUtensorMap tq;
     if (!cached_tmap(0, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
@@ -1153,10 +1144,14 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
         if (plan.cc_tokens && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze)))
             return W4A16_ERR_CUDA;
         const int st = plan.cc_tokens == 1   ? launch_cc<1>(tq, tsc, tze, args, plan.grid, stream)
-                       : plan.cc_tokens == 2 ? launch_cc<2>(tq, tsc, tze, args, plan.grid, stream)
                        : plan.nt == 16       ? launch_tc<16>(tq, tx, args, plan.grid, stream)
                                              : launch_tc<32>(tq, tx, args, plan.grid, stream);
         if (st != W4A16_OK) return st;
+        if (plan.cc_tokens) {
+            const int st2 = launch_decode_reduce(partial, args.Y, N, Mc, G, plan.units_base, plan.units_rem,
+                                                 plan.max_slots, plan.row_tiles, stream);
+            if (st2 != W4A16_OK) return st2;
+        }
     }
     return W4A16_OK;
 }

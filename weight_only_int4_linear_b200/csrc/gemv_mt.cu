@@ -85,7 +85,6 @@ struct MtArgs {
     const int32_t* zeros;
     uint16_t* Y;           // [M][N]
     float* partial;        // [row_tiles][max_slots][M][128]
-    int* counters;         // [row_tiles]
     int* fault;
     int M, N, G;
     int units_base, units_rem;
@@ -155,7 +154,6 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mt_kernel(const __grid_con
     constexpr int TPL = C::kTokPerLane;
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
-    __shared__ int s_last;
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((512u - (raw & 511u)) & 511u);  // 512-aligned stages
     unsigned char* meta = ring + C::kMetaOff;
@@ -222,7 +220,6 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mt_kernel(const __grid_con
     }
 
     // -------------------------------------------------------------------- compute warps 0-3
-    const int t = threadIdx.x;
     // Warp w takes rows 16 kRB w .. as kRB 16-row MMA blocks; lane (g8, tig) = (lane / 4, lane % 4)
     // holds rows g8 and g8 + 8 of each block and words 4 tig .. 4 tig + 3 of each row's codes (one
     // 16-byte chunk); MMA j takes word 4 tig + j of every lane, and the lane's B fragments are the same
@@ -253,9 +250,8 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mt_kernel(const __grid_con
                     }
                 }
             }
-        } else {
-            const int slot = b - first, nseg = last - first + 1;
-            float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * M * kRows;
+        } else {  // this CTA's partial-sum slot of the tile (decode_reduce_kernel adds the slots)
+            float* part = a.partial + ((int64_t)tile * a.max_slots + (b - first)) * M * kRows;
 #pragma unroll
             for (int q = 0; q < TPL; ++q) {
                 const int m = mt_token<NT>(tig, q);
@@ -264,20 +260,6 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mt_kernel(const __grid_con
                     for (int k = 0; k < KR; ++k) part[m * kRows + rrow(k)] = y[k][q];
                 }
             }
-            named_barrier_sync(1, kWarps * 32);
-            if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
-            named_barrier_sync(1, kWarps * 32);
-            if (s_last) {
-                const int rows = min(kRows, N - tile * kRows);
-                const float* pb = a.partial + (int64_t)tile * a.max_slots * M * kRows;
-                for (int idx = t; idx < M * rows; idx += kWarps * 32) {
-                    const int m = idx / rows, rl = idx - m * rows;
-                    const float sum = sum_slots(pb + (int64_t)m * kRows + rl, (int64_t)M * kRows, nseg);
-                    a.Y[(int64_t)m * N + tile * kRows + rl] = float_to_bf16_bits(sum);
-                }
-                if (t == 0) a.counters[tile] = 0;
-            }
-            named_barrier_sync(1, kWarps * 32);
         }
 #pragma unroll
         for (int k = 0; k < KR; ++k)
@@ -504,8 +486,8 @@ size_t mt_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 }
 
 int launch_decode_mt(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
-                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, int* counters,
-                     void* scratch, cudaStream_t stream) {
+                     const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* scratch,
+                     cudaStream_t stream) {
     const int G = (int)(K / kGroup);
     CUtensorMap tq, tsc, tze;
     if (!tmap_2d_cached(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight, (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2,
@@ -536,7 +518,6 @@ int launch_decode_mt(const uint16_t* X, const float* xscale, int64_t M, int64_t 
         args.zeros = zeros;
         args.Y = Y + m0 * N;
         args.partial = partial;
-        args.counters = counters;
         args.fault = fault;
         args.M = Mc;
         args.N = (int)N;
@@ -547,6 +528,9 @@ int launch_decode_mt(const uint16_t* X, const float* xscale, int64_t M, int64_t 
         st = nt == 4   ? launch_mt_kernel<4>(tq, tsc, tze, args, p.grid, stream)
              : nt == 8 ? launch_mt_kernel<8>(tq, tsc, tze, args, p.grid, stream)
                        : launch_mt_kernel<16>(tq, tsc, tze, args, p.grid, stream);
+        if (st != W4A16_OK) return st;
+        st = launch_decode_reduce(partial, args.Y, N, Mc, G, p.units_base, p.units_rem, p.max_slots, p.row_tiles,
+                                  stream);
         if (st != W4A16_OK) return st;
     }
     return W4A16_OK;
