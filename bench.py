@@ -287,7 +287,8 @@ def time_layer_alone(c, torch, w4, stream, min_calls=200, pws=None):
     """Device time of one call of layer `c` (CUDA events on the launching
     stream): back-to-back calls replayed from a CUDA graph, each call reading a
     different copy of the packed weights, rotating through enough copies that
-    their codes exceed 3x L2.  Returns (us per call, copies)."""
+    their codes exceed 3x L2; the median over seven replays of the graph.
+    Returns (us per call, copies)."""
     own = pws is None
     if own:
         pws = packed_copies(c, torch, w4, stream)
@@ -311,15 +312,16 @@ def time_layer_alone(c, torch, w4, stream, min_calls=200, pws=None):
     with torch.cuda.stream(stream):
         g.replay()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 3
-    e0.record(stream)
+    # median over replays, each bracketed by events on the launching stream
+    reps = 7
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record(stream)
     with torch.cuda.stream(stream):
-        for _ in range(reps):
+        for r in range(reps):
             g.replay()
-    e1.record(stream)
+            ev[r + 1].record(stream)
     torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / (reps * passes * copies)
+    us = statistics.median(ev[r].elapsed_time(ev[r + 1]) for r in range(reps)) * 1e3 / (passes * copies)
     del g, X, Y, ws
     if own:
         del pws

@@ -86,10 +86,11 @@ def test_linear_small_shapes_all_outputs(cuda_lib, G, M, N, K):
 
 
 @pytest.mark.parametrize("G", GROUPS)
-@pytest.mark.parametrize("M", [2, 4, 9, 16, 17, 40, 512])
+@pytest.mark.parametrize("M", [2, 4, 9, 16, 17, 40, 70, 300, 512])
 def test_batched_token_counts_all_outputs(cuda_lib, G, M):
-    """Batched decode and prefill token counts on the BF16 tensor-core GEMV with one accumulator per
-    quantisation group (tiles of 16 and 32 tokens, M > 32 in chunks of 32)."""
+    """Batched decode and prefill token counts: the BF16 tensor-core GEMV with one accumulator per
+    quantisation group (tiles of 16 and 32 tokens, M > 32 in chunks of 32), and for groups of 64 at
+    M >= 64 the GEMM with one fold per 64-K stage."""
     N, K = 200, 1024
     W = synth.weights_f32(7000 + M + G, synth.TAG_W, N, K)
     W[: N // 5] += np.float32(0.05)

@@ -143,7 +143,7 @@ static int linear_entry(const uint16_t* X, const float* xscale, int64_t M, int64
     if (need > 0 && (!workspace || workspace_bytes < need)) return W4A16_ERR_WORKSPACE;
     if (need > 0 && !aligned16(workspace)) return W4A16_ERR_ALIGN;
     if (prefill)
-        return launch_prefill(X, xscale, M, K, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
+        return launch_prefill(X, xscale, M, K, kGroup, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
     return launch_decode(X, xscale, M, K, qweight, scales, zeros, N, Y, workspace, plan, (cudaStream_t)stream);
 }
 
@@ -244,6 +244,7 @@ size_t w4a16_workspace_bytes_g(int64_t M, int64_t N, int64_t K, int group) {
     // one token: the integer GEMV with per-sub-group digit rows; more: the BF16 tensor-core GEMV (its
     // scratch after the shared counter area, which it leaves untouched)
     if (M == 1) return decode_sub_workspace_bytes(N, K, group);
+    if (group == 64 && M >= kPrefillMinM) return prefill_workspace_bytes(M, K, group);  // the GEMM
     return kCounterBytes + bf_workspace_bytes(M, N, K, group, num_sms_current());
 }
 
@@ -265,6 +266,8 @@ int w4a16_linear_g(const uint16_t* X, int64_t M, int64_t K, int group, const uin
     if (!workspace || workspace_bytes < need) return W4A16_ERR_WORKSPACE;
     if (!aligned16(workspace)) return W4A16_ERR_ALIGN;
     if (M == 1) return launch_decode_sub(X, M, K, group, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
+    if (group == 64 && M >= kPrefillMinM)
+        return launch_prefill(X, nullptr, M, K, group, qweight, scales, zeros, N, Y, workspace, (cudaStream_t)stream);
     return launch_decode_bf(X, nullptr, M, K, group, qweight, scales, zeros, N, Y,
                             reinterpret_cast<char*>(workspace) + kCounterBytes, (cudaStream_t)stream);
 }

@@ -145,6 +145,7 @@ struct DecodePlan {
     bool bf;          // the BF16 tensor-core GEMV (gemv_bf.cu), in chunks of 32 tokens
     int nt;           // tensor-core kernel: MMA N (16 or 32 tokens per launch); 1 with cc_tokens
     int row_tiles;    // 128-row tiles along N
+    int unit_groups;  // units per row tile (a unit: 128 rows x one or two quantisation groups)
     int grid;         // persistent CTAs
     int units_base;   // each CTA streams units_base (+1 for the first units_rem CTAs) units
     int units_rem;
@@ -183,8 +184,9 @@ int launch_decode_mt(const uint16_t* X, const float* xscale, int64_t M, int64_t 
 
 // Prefill (tensor-core GEMM) path for large M.
 constexpr int64_t kPrefillMinM = 64;  // W4A16_PATH_AUTO switches to the GEMM at this many tokens
-size_t prefill_workspace_bytes(int64_t M, int64_t K);
-int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+// group: quantisation group size, 128 or 64 (one or two folds per 128 K).
+size_t prefill_workspace_bytes(int64_t M, int64_t K, int group = kGroup);
+int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, int group, const uint32_t* qweight,
                    const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                    cudaStream_t stream);
 

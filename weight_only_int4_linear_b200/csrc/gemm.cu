@@ -132,9 +132,10 @@ __device__ __forceinline__ uint4 permute_block(uint4 v) {
     return o;
 }
 
-// X -> Xp (each 8-block reordered (0,4,1,5,2,6,3,7)) and xsT[g][m] = sum of the group
-// (row stride Mp, a multiple of the 256-token tile so one bulk copy per group and tile reads it).
-// xscale (nullable): each x is first replaced by bf16(x * xscale[k]) (the AWQ activation transform).
+// X -> Xp (each 8-block reordered (0,4,1,5,2,6,3,7)) and xsT[g][m] = sum of quantisation group g of
+// GS weights (row stride Mp, a multiple of the 256-token tile so one bulk copy per group and tile
+// reads it).  xscale (nullable): each x is first replaced by bf16(x * xscale[k]) (AWQ).
+template <int GS>
 __global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __restrict__ X,
                                                            const float* __restrict__ xscale, int M, int K, int Mp,
                                                            uint16_t* __restrict__ Xp, float* __restrict__ xsT) {
@@ -161,9 +162,10 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(const uint16_t* __res
             sum = (bf16lo(v.x) + bf16hi(v.x)) + (bf16lo(v.y) + bf16hi(v.y)) + (bf16lo(v.z) + bf16hi(v.z)) +
                   (bf16lo(v.w) + bf16hi(v.w));
         }
+        constexpr int LPG = GS / 8;  // lanes (8-blocks) per quantisation group, aligned in the block of 16
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
-        if (active && blk == 0) xsT[(int64_t)g * Mp + m] = sum;
+        for (int o = LPG / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (active && blk % LPG == 0) xsT[((int64_t)g * (kGroup / GS) + blk / LPG) * Mp + m] = sum;
     }
 }
 
@@ -219,6 +221,8 @@ __device__ __forceinline__ void arrive_issuer(uint64_t* bar) {
 }
 
 
+// GS: quantisation group size, 128 (two 64-K stages per group) or 64 (one stage per group).
+template <int GS>
 __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_constant__ CUtensorMap tx,
                                                                const __grid_constant__ CUtensorMap tq,
                                                                const PrefillArgs a) {
@@ -234,8 +238,10 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
     const uint32_t rank = kPCtas == 2 ? cluster_ctarank() : 0u;
     const int b = blockIdx.x / kPCtas;  // MMA unit: this CTA or its cluster
     const int ntiles = b < a.tiles ? (a.tiles - 1 - b) / a.units + 1 : 0;  // tiles b, b + units, ...
-    const int G = a.G;
-    const int stages_per_tile = 2 * G;
+    constexpr int kSpg = GS / kPBK;  // 64-K stages per quantisation group
+    static_assert(kSpg * kPBK == GS && kSpg >= 1, "group size");
+    const int G = a.G;               // quantisation groups per row
+    const int stages_per_tile = kSpg * G;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPStages; ++s) {
@@ -295,7 +301,7 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             for (int tt = 0; tt < ntiles; ++tt) {
                 for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
                     const int s = it % kPStages;
-                    const int half = ks & 1;
+                    const int half = ks % kSpg;  // stage within the quantisation group
                     const int dbuf = gc & 1;
                     if (half == 0 && gc >= 2 && !mbar_wait(&dfree[dbuf], ((gc >> 1) - 1) & 1, a.fault, 71)) goto done_mma;
                     if (!mbar_wait(&afull[s], (it / kPStages) & 1, a.fault, 73)) goto done_mma;
@@ -312,12 +318,12 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
                     }
                     if constexpr (kPCtas == 2) {
                         umma_commit_pair(&empty[s], 0x3);
-                        if (half == 1) umma_commit_pair(&mdone[dbuf], 0x3);
+                        if (half == kSpg - 1) umma_commit_pair(&mdone[dbuf], 0x3);
                     } else {
                         umma_commit(&empty[s]);
-                        if (half == 1) umma_commit(&mdone[dbuf]);
+                        if (half == kSpg - 1) umma_commit(&mdone[dbuf]);
                     }
-                    if (half == 1) ++gc;
+                    if (half == kSpg - 1) ++gc;
                 }
             }
         done_mma:
@@ -340,9 +346,9 @@ __global__ void __launch_bounds__(kPThreads, 1) prefill_kernel(const __grid_cons
             const int n = (nt * kPCtas + (int)rank) * kPBM + r;
             uint32_t zc2 = 0x43004300u;  // (128 + c) as a BF16 pair
             for (int ks = 0; ks < stages_per_tile; ++ks, ++it) {
-                const bool first_half = (ks & 1) == 0;
+                const bool first_half = ks % kSpg == 0;  // first stage of a quantisation group
                 if (first_half) {
-                    const int z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + (ks >> 1)) : 0;
+                    const int z = n < a.N ? __ldg(a.zeros + (int64_t)n * G + ks / kSpg) : 0;
                     const int c = (z >= -128 && z <= 128) ? z : 0;
                     const uint32_t cb = __float_as_uint(128.f + (float)c) >> 16;  // exact: |128 + c| <= 256
                     zc2 = cb | (cb << 16);
@@ -507,8 +513,9 @@ bool prefill_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtenso
 size_t align256p(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // MMA units of the prefill kernel that fit on the current device at once (cached per context).
-int prefill_resident_units(const cudaLaunchConfig_t& cfg) {
-    static PerContext<int> cache;
+template <class Kern>
+int prefill_resident_units(const cudaLaunchConfig_t& cfg, Kern kernel) {
+    static PerContext<int> cache;  // the same for both group sizes: same resources
     return cache.get([&]() -> int {
         int units = 0;
         if constexpr (kPCtas == 1) {
@@ -516,7 +523,7 @@ int prefill_resident_units(const cudaLaunchConfig_t& cfg) {
         } else {
             cudaLaunchConfig_t q = cfg;
             q.gridDim = dim3((unsigned)(kPCtas * num_sms_current()));
-            if (cudaOccupancyMaxActiveClusters(&units, prefill_kernel, &q) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveClusters(&units, kernel, &q) != cudaSuccess) {
                 cudaGetLastError();
                 return 0;
             }
@@ -527,19 +534,21 @@ int prefill_resident_units(const cudaLaunchConfig_t& cfg) {
 
 }  // namespace
 
-size_t prefill_workspace_bytes(int64_t M, int64_t K) {
+size_t prefill_workspace_bytes(int64_t M, int64_t K, int group) {
     const int64_t Mp = (M + kPBN - 1) / kPBN * kPBN;
     // the decode path's counter area stays untouched at the front (shared workspaces)
-    return kCounterBytes + align256p((size_t)M * K * 2) + align256p((size_t)(K / kGroup) * Mp * 4);
+    return kCounterBytes + align256p((size_t)M * K * 2) + align256p((size_t)(K / group) * Mp * 4);
 }
 
-int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
-                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
-                   cudaStream_t stream) {
+namespace {
+template <int GS>
+int launch_prefill_gs(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
+                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                      cudaStream_t stream) {
     static PerContext<int> attr;  // the attribute belongs to a context
     if (!attr.get([]() -> int {
-            return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPSmem) ==
-                   cudaSuccess;
+            return cudaFuncSetAttribute(prefill_kernel<GS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)kPSmem) == cudaSuccess;
         }))
         return W4A16_ERR_CUDA;
     int* fault = fault_word();
@@ -550,13 +559,13 @@ int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K,
     CUtensorMap tx, tq;
     if (!prefill_tmap(0, Xp, M, K, &tx) || !prefill_tmap(1, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
 
-    const int G = (int)(K / kGroup);
-    const int64_t units = M * G * 16;
+    const int G = (int)(K / GS);  // quantisation groups per row
+    const int64_t units = M * (K / kGroup) * 16;
     int pgrid = (int)ceil_div(units, 256);
     if (pgrid > num_sms_current() * 16) pgrid = num_sms_current() * 16;
     const int Mp = (int)((M + kPBN - 1) / kPBN * kPBN);
     if (Mp > M && cudaMemsetAsync(xsT, 0, (size_t)G * Mp * 4, stream) != cudaSuccess) return W4A16_ERR_CUDA;
-    prefill_prep_kernel<<<pgrid, 256, 0, stream>>>(X, xscale, (int)M, (int)K, Mp, Xp, xsT);
+    prefill_prep_kernel<GS><<<pgrid, 256, 0, stream>>>(X, xscale, (int)M, (int)K, Mp, Xp, xsT);
     if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
 
     PrefillArgs args;
@@ -589,13 +598,22 @@ int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K,
     cfg.numAttrs = 2;
     // persistent: one MMA unit (CTA or 2-CTA cluster) per resident slot, so that every unit runs
     // in the first wave (a cluster needs two free SMs of one GPC, which not every SM count allows)
-    int mma_units = prefill_resident_units(cfg);
+    int mma_units = prefill_resident_units(cfg, prefill_kernel<GS>);
     if (mma_units <= 0) return W4A16_ERR_CUDA;
     if (mma_units > tiles) mma_units = tiles;
     args.tiles = tiles;
     args.units = mma_units;
     cfg.gridDim = dim3((unsigned)(mma_units * kPCtas));
-    return cudaLaunchKernelEx(&cfg, prefill_kernel, tx, tq, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, prefill_kernel<GS>, tx, tq, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+}
+}  // namespace
+
+int launch_prefill(const uint16_t* X, const float* xscale, int64_t M, int64_t K, int group, const uint32_t* qweight,
+                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
+                   cudaStream_t stream) {
+    if (group == 64)
+        return launch_prefill_gs<64>(X, xscale, M, K, qweight, scales, zeros, N, Y, workspace, stream);
+    return launch_prefill_gs<128>(X, xscale, M, K, qweight, scales, zeros, N, Y, workspace, stream);
 }
 
 }  // namespace w4a16

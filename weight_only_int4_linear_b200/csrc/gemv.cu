@@ -510,77 +510,78 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // At M = 1 a tcgen05 MMA would waste most of its columns, and its operands
 // would have to pass through tensor memory; the dot products instead run as
 // warp-level mma.sync m16n8k32 in registers: A = 16 rows x 32 codes as
-// unsigned bytes, straight from the packed words (w & 0x0F0F0F0F holds codes
-// 0, 2, 4, 6 and (w >> 4) & 0x0F0F0F0F codes 1, 3, 5, 7), B = 32 codes x 8
-// columns of X digits as signed bytes, D = exact int32 sums.  X is expanded
-// exactly into integers per group: with E the exponent of the group's
-// largest |x|, x_int = x * 2^(21 - E) (exact for every x within 2^14 of the
-// group maximum; smaller values are rounded at 2^(E - 21), far below FP32
-// accumulation error), written in balanced base 256, x_int = 65536 d2 +
-// 256 d1 + d0 with every digit in [-128, 127]; columns 0-2 of B hold digit
-// planes 0-2, columns 4-6 the same planes again (so that the lanes holding
-// accumulator columns 4-7 have every plane of the second row block), columns
-// 3 and 7 are zero.  Per group and row:
-//   acc += s (65536 D2 + 256 D1 + D0 - z sum_k x_int) 2^(E - 21).
+// unsigned bytes, straight from the packed words, B = 32 codes x 8 columns of
+// X digits as signed bytes, D = exact int32 sums.  Each packed word gives its
+// A bytes in one instruction per half: w & 0x0F0F0F0F holds codes 0, 2, 4, 6,
+// and w & 0xF0F0F0F0 holds 16 times codes 1, 3, 5, 7.  X is expanded into
+// integers per group: with E the exponent of the group's largest |x|, an
+// even code's activation is x_int = rint(x 2^(21 - E)) and an odd code's is
+// rint(x 2^(17 - E)) -- the factor 16 of its A byte makes the product the
+// same q x 2^(21 - E) -- so every activation within 2^10 of the group
+// maximum is exact (within 2^14 for even codes) and smaller ones are rounded
+// at 2^(E - 21) or 2^(E - 17), far below FP32 accumulation error.  x_int is
+// written in balanced base 256, 65536 d2 + 256 d1 + d0 with every digit in
+// [-128, 127]; columns 0-2 of B hold digit planes 0-2, columns 4-6 the same
+// planes again (so that the lanes holding accumulator columns 4-7 have every
+// plane of the second row block), columns 3 and 7 are zero.  Per group and
+// row, with X_k the represented activations (x_int, or 16 x_int for odd codes):
+//   acc += s (65536 D2 + 256 D1 + D0 - z sum_k X_k) 2^(E - 21).
 // One MMA takes 32 codes of 16 rows against every plane: a compute thread
-// issues 8 MMAs per 128 x 128 unit where byte-plane dp4a would take 96
-// instructions, and each lane of a quad folds one of the quad's four rows.
+// issues 8 MMAs per group where byte-plane dp4a would take 96 instructions,
+// and each lane of a quad folds one of the quad's four rows.
 //
-// X of one group in the layout the kernel reads: 3 NT digit rows of 128 bytes
+// X of one group in the layout the kernel reads: 3 digit rows of 128 bytes
 // (word w's codes 0,2,4,6 at 8w, codes 1,3,5,7 at 8w + 4: the order in which
 // the two masks above hold the codes, so a lane's B fragment of MMA j is
-// bytes 32 tig + 8 j .. + 7 of its row), then per token (sum_k x_int as FP32,
-// 2^(E - 21)).
-// The CTA streams units (128 rows x one group) through a 4-stage ring:
-//  * warp 4 (one thread) drives TMA: the codes of each unit (8 KB, 64-byte
+// bytes 32 tig + 8 j .. + 7 of its row), then (sum_k X_k as FP32, 2^(E - 21)),
+// padded to 400 bytes.
+// A unit is 128 rows x one group (8 KB of codes; built with two groups per
+// unit it is 16 KB, which measured slower: fewer stages in flight); the CTA
+// streams units through a 4-stage ring:
+//  * warp 4 (one thread) drives TMA: the codes of each unit (64-byte
 //    swizzle) and, once per block of 8 groups of a row tile, that block's
 //    128 x 8 scales and 128 x 8 zero points into one of two metadata slots;
 //  * warp 5 prepares X for each unit's group straight from the BF16 input
-//    (the digit rows, the group sum and the group's power of two), so the
-//    call is a single launch;
+//    (the digit rows, the group sum and power of two), so the call is a
+//    single launch;
 //  * warps 0-3 compute, warp w taking rows 32 w .. 32 w + 31 of each unit as
 //    two 16-row MMA blocks.
-// Up to four CTAs share an SM: their independent rings keep more loads in
-// flight than one CTA per SM with an in-order ring of the same depth.  A row
-// tile whose units two CTAs share is written by each as a partial-sum slot,
-// and decode_reduce_kernel, launched as a dependent grid, adds the slots in a
+// Four CTAs share an SM: their independent rings keep more loads in flight
+// than one CTA per SM with an in-order ring of the same depth.  A row tile
+// whose units two CTAs share is written by each as a partial-sum slot, and
+// decode_reduce_kernel, launched as a dependent grid, adds the slots in a
 // fixed order: no CTA waits on another or on an atomic at its end, and each
 // CTA frees its SM for the next layer's weight stream as soon as it is done.
-#ifndef W4A16_CC_WARPS
-#define W4A16_CC_WARPS 4
+#ifndef W4A16_CC_UNIT_GROUPS
+#define W4A16_CC_UNIT_GROUPS 1
 #endif
-#ifndef W4A16_CC_STAGES
-#define W4A16_CC_STAGES 4
-#endif
-constexpr int kCcWarps = W4A16_CC_WARPS;                // compute warps
-constexpr int kCcRowStep = kCcWarps * 8;                // rows rg + kCcRowStep * i of one thread
-constexpr int kCcRows = kRowsPerCta / kCcRowStep;       // rows per thread
-static_assert(kCcRows * kCcRowStep == kRowsPerCta && kCcRowStep % 8 == 0, "row split");
-constexpr int kCcTmaWarp = kCcWarps;                    // warp 4
-constexpr int kCcXWarp = kCcWarps + 1;                  // warp 5
+constexpr int kCcUnitGroups = W4A16_CC_UNIT_GROUPS;       // quantisation groups per unit (1 or 2)
+static_assert(kCcUnitGroups == 1 || kCcUnitGroups == 2, "unit size");
+constexpr int kCcWarps = 4;                              // compute warps
+constexpr int kCcTmaWarp = kCcWarps;                     // warp 4
+constexpr int kCcXWarp = kCcWarps + 1;                   // warp 5
 constexpr int kCcThreads = (kCcWarps + 2) * 32;
-constexpr int kCcStages = W4A16_CC_STAGES;
-constexpr int kCcCodeBytes = kStageWords * 4;           // 8 KB, 64-byte swizzle
-constexpr int kCcXOff = kCcCodeBytes;                   // X digit rows of the unit's group, after the codes
-// X of one group (layout above), and codes + X, 512-aligned (the 64-byte swizzle's span)
-template <int NT>
-__host__ __device__ constexpr int cc_x_bytes() { return 3 * NT * 128 + 8 * NT; }
-template <int NT>
-__host__ __device__ constexpr int cc_stage_bytes() { return (kCcCodeBytes + cc_x_bytes<NT>() + 511) / 512 * 512; }
-constexpr int kCcMetaGroups = 8;                        // groups per metadata block
-constexpr int kXAhead = 6;                              // X warp: loads in flight, in units
+constexpr int kCcStages = kCcUnitGroups == 1 ? 4 : 2;    // ring depth: 32 KB of codes in flight per CTA
+constexpr int kCcMinBlocks = 4;                          // CTAs per SM
+constexpr int kCcRowBytes = 64 * kCcUnitGroups;          // codes of one row in a unit
+constexpr int kCcSwizzleSpan = 8 * kCcRowBytes;          // 64- or 128-byte swizzle: 8-row pattern
+constexpr int kCcCodeBytes = kStageWords * 4 * kCcUnitGroups;  // 8 or 16 KB
+constexpr int kCcXOff = kCcCodeBytes;                    // X of the unit's groups, after the codes
+constexpr int kCcXGroupBytes = 400;                      // 3 digit rows + sum and scale, 16-byte aligned
+constexpr int kCcStageBytes =
+    (kCcCodeBytes + kCcUnitGroups * kCcXGroupBytes + kCcSwizzleSpan - 1) / kCcSwizzleSpan * kCcSwizzleSpan;
+constexpr int kCcMetaGroups = 8;                         // groups per metadata block
+constexpr int kXAhead = 4;                               // X warp: loads in flight, in units
 constexpr int kCcScBytes = kRowsPerCta * kCcMetaGroups * 2;  // 128 rows x 8 BF16 scales
 constexpr int kCcZeBytes = kRowsPerCta * kCcMetaGroups * 4;  // 128 rows x 8 int32 zero points
-constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;   // one slot, 6 KB
-template <int NT>
-__host__ __device__ constexpr int cc_meta_off() { return kCcStages * cc_stage_bytes<NT>(); }  // two slots after the ring
-template <int NT>
-__host__ __device__ constexpr size_t cc_smem() { return (size_t)cc_meta_off<NT>() + 2 * kCcMetaBytes + 512; }  // + alignment slack
+constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;    // one slot, 6 KB
+constexpr int kCcMetaOff = kCcStages * kCcStageBytes;    // two slots after the ring
+constexpr size_t kCcSmem = (size_t)kCcMetaOff + 2 * kCcMetaBytes + 1024;  // + alignment slack
 // A metadata slot is rewritten two blocks later.  Blocks are aligned to 8
 // groups inside a row tile (the kernel needs G % 8 == 0), so the block in
-// between has 8 units; with at most kCcStages units in flight, every unit of
+// between has 4 units; with at most kCcStages units in flight, every unit of
 // the older block has been released by then.
-static_assert(kCcStages <= kCcMetaGroups, "metadata slot reuse");
+static_assert(kCcStages <= kCcMetaGroups / kCcUnitGroups, "metadata slot reuse");
 
 // This lane's four BF16 values of group g: lane 2w + h holds values 4h..4h+3 of word w.
 __device__ __forceinline__ uint2 load_group_x(const uint16_t* __restrict__ X, int g, int lane) {
@@ -597,15 +598,13 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// One warp writes token m's digits of group g (its lanes' values v from load_group_x) in the layout
-// above: digit row n = p NT + m.
+// One warp writes the X of one group (its lanes' values v from load_group_x) in the layout above.
 //
-// x_int = rint(x 2^kx) comes from one FFMA with the 1.5 2^23 magic constant (|x 2^kx| < 2^22, so the
-// sum's last place is 1 and its rounding is the rounding to the nearest integer, ties to even), and
+// The integers come from one FFMA with the 1.5 2^23 magic constant (|x 2^k| < 2^22, so the sum's last
+// place is 1 and its rounding is the rounding to the nearest integer, ties to even), and
 // x_int + 0x808080 = (d0 + 128) + 256 (d1 + 128) + 65536 (d2 + 128) holds the three balanced base-256
 // digits, each plus 128, in its three low bytes: the digit bytes are that word XOR 0x808080.
-template <int NT>
-__device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst, int lane, int m) {
+__device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst, int lane) {
     const uint32_t a2 = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
     uint32_t amax = max(a2 & 0xFFFFu, a2 >> 16);
     amax = __reduce_max_sync(0xFFFFFFFFu, amax);
@@ -613,16 +612,17 @@ __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst,
     const int E = ef == 0 ? -127 : ef - 127;  // every |x| of the group is below 2^(E + 1)
     const int kx = 21 - E;                    // in [-106, 148]
     const int k1 = min(kx, 127);
-    const float s1 = pow2f(k1), s2 = pow2f(kx - k1);  // exact scalings, |x * 2^kx| < 2^22
+    const float s1 = pow2f(k1), s2 = pow2f(kx - k1);  // exact scalings, |x 2^kx| < 2^22
+    // lane (w, h) holds codes 4h .. 4h + 3 of word w: values 1 and 3 belong to odd codes (scale 2^(kx - 4))
     const float xv[4] = {__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
                          __uint_as_float(v.y & 0xFFFF0000u)};
     uint32_t D[4];
-    int sum4 = 0;
+    int xi[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float f = __fmaf_rn(xv[i] * s1, s2, 12582912.f);  // 1.5 2^23 + x_int
-        const uint32_t yb = __float_as_uint(f) - (0x4B400000u - 0x808080u);  // x_int + 0x808080
-        sum4 += (int)yb;
+        const float f = __fmaf_rn(xv[i] * s1, (i & 1) ? s2 * 0.0625f : s2, 12582912.f);  // 1.5 2^23 + x_int
+        const uint32_t yb = __float_as_uint(f) - (0x4B400000u - 0x808080u);          // x_int + 0x808080
+        xi[i] = (int)yb - 0x808080;
         D[i] = yb ^ 0x808080u;  // bytes 0..2: digits d0, d1, d2 as signed bytes
     }
     // planes as (i0, i2, i1, i3): P = [d0 i0, d0 i2, d1 i0, d1 i2], Q = the same for i1, i3; R, S plane 2
@@ -632,44 +632,41 @@ __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst,
     dg[0] = __byte_perm(P, Q, 0x5410);
     dg[1] = __byte_perm(P, Q, 0x7632);
     dg[2] = __byte_perm(R, S, 0x5410);
-    // lane (w, h) holds codes 4h .. 4h + 3 of word w; h = 0 assembles the even-code register
-    // (its codes 0, 2, the partner's 4, 6), h = 1 the odd one (the partner's 1, 3, its own 5, 7)
+    // h = 0 assembles the even-code word (its codes 0, 2 and the partner's 4, 6), h = 1 the odd one
+    // (the partner's 1, 3 and its own 5, 7)
     const int h = lane & 1, w = lane >> 1;
 #pragma unroll
     for (int p = 0; p < 3; ++p) {
         const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, dg[p], 1);
         const uint32_t lo = h ? other : dg[p], hi = h ? dg[p] : other;
         const uint32_t out = h ? __byte_perm(lo, hi, 0x7632) : __byte_perm(lo, hi, 0x5410);
-        *reinterpret_cast<uint32_t*>(dst + (p * NT + m) * 128 + 8 * w + 4 * h) = out;
+        *reinterpret_cast<uint32_t*>(dst + p * 128 + 8 * w + 4 * h) = out;
     }
-    const int sum = __reduce_add_sync(0xFFFFFFFFu, sum4) - 128 * (int)0x808080;  // |sum| < 2^29
+    // sum of the represented activations: odd codes' integers count 16 times (|sum| < 2^29)
+    const int sum = __reduce_add_sync(0xFFFFFFFFu, (xi[0] + xi[2]) + 16 * (xi[1] + xi[3]));
     if (lane == 0) {
-        float* ext = reinterpret_cast<float*>(dst + 3 * NT * 128);
-        ext[2 * m] = (float)sum;
-        ext[2 * m + 1] = pow2f(E - 21);
+        float* ext = reinterpret_cast<float*>(dst + 3 * 128);
+        ext[0] = (float)sum;
+        ext[1] = pow2f(E - 21);
     }
 }
 
-
-template <int NT>
-__global__ void __launch_bounds__(kCcThreads, 4) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
+__global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
                                                                   const __grid_constant__ CUtensorMap tsc,
                                                                   const __grid_constant__ CUtensorMap tze,
                                                                   const DecodeArgs a) {
-    static_assert(NT == 1, "one token per launch");
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages];
     const uint32_t raw = smem_u32(smem_raw);
-    unsigned char* ring = smem_raw + ((512u - (raw & 511u)) & 511u);  // 512-aligned stages
-    constexpr int kStageBytes = cc_stage_bytes<NT>();
-    unsigned char* meta = ring + cc_meta_off<NT>();
+    unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-aligned (the swizzle's span)
+    unsigned char* meta = ring + kCcMetaOff;
 
     pdl_launch_dependents();  // the next call may start its weight loads as this grid's CTAs retire
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
     const int64_t u_first = (int64_t)b * a.units_base + min(b, a.units_rem);
     const int nunits = a.units_base + (b < a.units_rem ? 1 : 0);
-    const int G = a.G, N = a.N;
+    const int G2 = a.G, N = a.N;  // units (group pairs) per row tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCcStages; ++s) {
@@ -686,19 +683,20 @@ __global__ void __launch_bounds__(kCcThreads, 4) decode_cc_kernel(const __grid_c
             prefetch_tmap(&tsc);
             prefetch_tmap(&tze);
             // the weights need nothing from the preceding kernel: no PDL wait here
-            UnitCursor cur(u_first, G);
+            UnitCursor cur(u_first, G2);
             int mb = -1, issued = 0;
-            for (int i = 0; i < nunits; ++i, cur.next(G)) {
+            for (int i = 0; i < nunits; ++i, cur.next(G2)) {
                 const int s = i % kCcStages;
                 if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) break;
-                const bool new_block = i == 0 || (cur.g & (kCcMetaGroups - 1)) == 0;
+                const int g0 = cur.g * kCcUnitGroups;  // first group of the unit
+                const bool new_block = i == 0 || (g0 & (kCcMetaGroups - 1)) == 0;
                 if (new_block) ++mb;
-                unsigned char* st = ring + s * kStageBytes;
+                unsigned char* st = ring + s * kCcStageBytes;
                 mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (new_block ? kCcMetaBytes : 0));
-                tma_load_2d(st, &tq, cur.g * kWordsPerGroup, cur.tile * kRowsPerCta, &full[s]);
+                tma_load_2d(st, &tq, g0 * kWordsPerGroup, cur.tile * kRowsPerCta, &full[s]);
                 if (new_block) {
                     unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
-                    const int g8 = cur.g & ~(kCcMetaGroups - 1);
+                    const int g8 = g0 & ~(kCcMetaGroups - 1);
                     tma_load_2d(ms, &tsc, g8, cur.tile * kRowsPerCta, &full[s]);
                     tma_load_2d(ms + kCcScBytes, &tze, g8, cur.tile * kRowsPerCta, &full[s]);
                 }
@@ -715,27 +713,28 @@ __global__ void __launch_bounds__(kCcThreads, 4) decode_cc_kernel(const __grid_c
         pdl_wait_primary();  // X may come from the preceding kernel
         const uint16_t* X = a.Xp;
         // loads run kXAhead units ahead of the preparation, so L2 latency is paid once, not per unit
-        uint2 q[kXAhead][NT];
-        UnitCursor cl(u_first, G);
+        uint2 q[kXAhead][kCcUnitGroups];
+        UnitCursor cl(u_first, G2);
 #pragma unroll
-        for (int j = 0; j < kXAhead; ++j, cl.next(G))
+        for (int j = 0; j < kXAhead; ++j, cl.next(G2))
 #pragma unroll
-            for (int m = 0; m < NT; ++m)
-                q[j][m] = j < nunits && m < a.M ? load_group_x(X + (int64_t)m * a.K, cl.g, lane) : make_uint2(0, 0);
-        for (int i = 0; i < nunits; ++i, cl.next(G)) {
-            uint2 v[NT];
+            for (int gi = 0; gi < kCcUnitGroups; ++gi)
+                q[j][gi] = j < nunits ? load_group_x(X, cl.g * kCcUnitGroups + gi, lane) : make_uint2(0, 0);
+        for (int i = 0; i < nunits; ++i, cl.next(G2)) {
+            uint2 v[kCcUnitGroups];
 #pragma unroll
-            for (int m = 0; m < NT; ++m) {
-                v[m] = q[0][m];
+            for (int gi = 0; gi < kCcUnitGroups; ++gi) {
+                v[gi] = q[0][gi];
 #pragma unroll
-                for (int j = 0; j + 1 < kXAhead; ++j) q[j][m] = q[j + 1][m];
-                q[kXAhead - 1][m] = i + kXAhead < nunits && m < a.M ? load_group_x(X + (int64_t)m * a.K, cl.g, lane)
-                                                                      : make_uint2(0, 0);
+                for (int j = 0; j + 1 < kXAhead; ++j) q[j][gi] = q[j + 1][gi];
+                q[kXAhead - 1][gi] = i + kXAhead < nunits ? load_group_x(X, cl.g * kCcUnitGroups + gi, lane)
+                                                          : make_uint2(0, 0);
             }
             const int s = i % kCcStages;
             if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
 #pragma unroll
-            for (int m = 0; m < NT; ++m) prep_group_x8<NT>(v[m], ring + s * kStageBytes + kCcXOff, lane, m);
+            for (int gi = 0; gi < kCcUnitGroups; ++gi)
+                prep_group_x8(v[gi], ring + s * kCcStageBytes + kCcXOff + gi * kCcXGroupBytes, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
         }
@@ -745,35 +744,35 @@ __global__ void __launch_bounds__(kCcThreads, 4) decode_cc_kernel(const __grid_c
     // ---------------------------------------------------- compute warps 0-3
     // Warp w takes rows 32 w .. 32 w + 31 as two 16-row MMA blocks.  Lane (g8, tig) = (lane / 4,
     // lane % 4) holds, per block, rows g8 and g8 + 8 of its A fragments and words 4 tig .. 4 tig + 3
-    // of each (one 16-byte chunk of the codes tile); MMA j takes word 4 tig + j of every lane, so
+    // of each (one 16-byte chunk of the group's codes); MMA j takes word 4 tig + j of every lane, so
     // its K = 32 codes are words j, 4 + j, 8 + j, 12 + j, and the lane's B fragments are the same
-    // words of digit plane n = g8.  After a unit, D column n = p NT + m of a row is
-    // sum_k q_k d_p(x_k) of token m; lane tig = m gathers its three planes and folds the row.
+    // words of its digit row.
     const int g8 = lane >> 2, tig = lane & 3;
     auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
-    float y = 0.f;  // row rrow(tig) of the current row tile
+    const int r_own = rrow(tig);  // the row this lane folds
+    float y = 0.f;                // row r_own of the current row tile
     int cur_tile = -1;
     bool aborted = false;
 
     // A row tile leaves the CTA as Y (the CTA holds all of its units) or as this CTA's partial-sum slot
     // (decode_reduce_kernel adds the slots).
     auto flush = [&](int tile) {
-        const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
-        const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
+        const int first = cta_of_unit((int64_t)tile * G2, a.units_base, a.units_rem);
+        const int last = cta_of_unit((int64_t)tile * G2 + G2 - 1, a.units_base, a.units_rem);
         if (first == last) {
-            const int n = tile * kRowsPerCta + rrow(tig);
+            const int n = tile * kRowsPerCta + r_own;
             if (n < N) a.Y[n] = float_to_bf16_bits(y);
         } else {
-            a.partial[((int64_t)tile * a.max_slots + (b - first)) * kRowsPerCta + rrow(tig)] = y;
+            a.partial[((int64_t)tile * a.max_slots + (b - first)) * kRowsPerCta + r_own] = y;
         }
         y = 0.f;
     };
 
-    UnitCursor uc(u_first, G);
+    UnitCursor uc(u_first, G2);
     int mb = -1;
-    for (int i = 0; i < nunits; ++i, uc.next(G)) {
-        const int tile = uc.tile, g = uc.g;
-        if (i == 0 || (g & (kCcMetaGroups - 1)) == 0) ++mb;
+    for (int i = 0; i < nunits; ++i, uc.next(G2)) {
+        const int tile = uc.tile, g0 = uc.g * kCcUnitGroups;
+        if (i == 0 || (g0 & (kCcMetaGroups - 1)) == 0) ++mb;
         if (tile != cur_tile) {
             if (cur_tile >= 0) flush(cur_tile);
             cur_tile = tile;
@@ -784,67 +783,76 @@ __global__ void __launch_bounds__(kCcThreads, 4) decode_cc_kernel(const __grid_c
             aborted = true;
             continue;
         }
-        const unsigned char* st = ring + s * kStageBytes;
-        // codes: chunk tig of each row, 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3))
-        uint4 cw[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int r = rrow(k);
-            cw[k] = *reinterpret_cast<const uint4*>(st + r * 64 + 16 * (tig ^ ((r >> 1) & 3)));
-        }
-        // B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of the second
-        // row block and each lane of a quad can fold one of its four rows; columns 3 and 7 are zero
-        uint32_t bx[8];
-        const int xrow = g8 & 3;
-        if (xrow < 3) {
-            const uint4* xp = reinterpret_cast<const uint4*>(st + kCcXOff + xrow * 128 + tig * 32);
-            const uint4 u0 = xp[0], u1 = xp[1];
-            bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
-            bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) bx[j] = 0u;
-        }
-        const float* ext = reinterpret_cast<const float*>(st + kCcXOff + 3 * 128);
-        const float xsum = ext[0], xscale = ext[1];
-        // this lane's row's metadata, from the block loaded with the block's first unit (which this warp
-        // has already waited for); rows past N were zero-filled by TMA: s = 0 folds them away
+        const unsigned char* st = ring + s * kCcStageBytes;
         const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
-        const int r = rrow(tig);
-        const float sv = bf16_bits_to_float(
-            *reinterpret_cast<const uint16_t*>(ms + r * (kCcMetaGroups * 2) + 2 * (g & (kCcMetaGroups - 1))));
-        const float zv = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r * (kCcMetaGroups * 4) +
-                                                                  4 * (g & (kCcMetaGroups - 1)));
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+        for (int gi = 0; gi < kCcUnitGroups; ++gi) {
+            // codes: 16-byte chunk 4 gi + tig of each row; with one group per unit a row is 64 bytes,
+            // 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3)), with two it is 128 bytes, 128-byte
+            // swizzle (chunk c at c ^ (r & 7))
+            uint4 cw[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int r = rrow(k);
+                const int c = kCcUnitGroups == 1 ? (tig ^ ((r >> 1) & 3)) : ((4 * gi + tig) ^ (r & 7));
+                cw[k] = *reinterpret_cast<const uint4*>(st + r * kCcRowBytes + 16 * c);
+            }
+            // B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of the second
+            // row block and each lane of a quad can fold one of its four rows; columns 3 and 7 are zero
+            const unsigned char* xg = st + kCcXOff + gi * kCcXGroupBytes;
+            uint32_t bx[8];
+            const int xrow = g8 & 3;
+            if (xrow < 3) {
+                const uint4* xp = reinterpret_cast<const uint4*>(xg + xrow * 128 + tig * 32);
+                const uint4 u0 = xp[0], u1 = xp[1];
+                bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
+                bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) bx[j] = 0u;
+            }
+            const float* ext = reinterpret_cast<const float*>(xg + 3 * 128);
+            const float xsum = ext[0], xscale = ext[1];
+            // this lane's row's metadata, from the block loaded with the block's first unit (which this
+            // warp has already waited for); rows past N were zero-filled by TMA: s = 0 folds them away
+            const int gb = (g0 + gi) & (kCcMetaGroups - 1);
+            const float sv =
+                bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(ms + r_own * (kCcMetaGroups * 2) + 2 * gb));
+            const float zv = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r_own * (kCcMetaGroups * 4) + 4 * gb);
+            if (gi + 1 == kCcUnitGroups) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+            }
 
-        int d[2][4];
+            int d[2][4];
 #pragma unroll
-        for (int rb = 0; rb < 2; ++rb) {
-            const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
-            const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
+            for (int rb = 0; rb < 2; ++rb) {
+                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) d[rb][j] = 0;
+                for (int j = 0; j < 4; ++j) d[rb][j] = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                mma_u8s8(d[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, (w0[j] >> 4) & 0x0F0F0F0Fu,
-                         (w1[j] >> 4) & 0x0F0F0F0Fu, bx[2 * j], bx[2 * j + 1]);
+                for (int j = 0; j < 4; ++j)
+                    mma_u8s8(d[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, w0[j] & 0xF0F0F0F0u, w1[j] & 0xF0F0F0F0u,
+                             bx[2 * j], bx[2 * j + 1]);
+            }
+            // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes (0, 1)
+            // at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block tig >> 1
+            // (its own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour completes its
+            // planes.
+            const bool hi = tig >> 1, even = !(tig & 1);
+            int e[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) e[j] = hi ? d[1][j] : d[0][j];
+            const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
+            const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
+            const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
+            // sum q X = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26); then
+            // s (sum q X - z sum X) and the power of two last, so that neither product leaves the FP32
+            // range unless the group's result itself does
+            const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+            y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
         }
-        // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes (0, 1)
-        // at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block tig >> 1 (its
-        // own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour completes its planes.
-        const bool hi = tig >> 1, even = !(tig & 1);
-        int e[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) e[j] = hi ? d[1][j] : d[0][j];
-        const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
-        const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
-        const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
-        // sum q x_int = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26); then
-        // s (sum (q - z) x_int) and the power of two last, so that neither product leaves the FP32 range
-        // unless the group's result itself does
-        const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-        y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
     }
     if (cur_tile >= 0) flush(cur_tile);
 }
@@ -865,16 +873,14 @@ int occupancy_nt() {
     });
 }
 
-template <int NT>
 int occupancy_cc() {
     static PerContext<int> cache;  // the attribute and occupancy belong to a context
     return cache.get([]() -> int {
-        if (cudaFuncSetAttribute(decode_cc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)cc_smem<NT>()) != cudaSuccess)
+        if (cudaFuncSetAttribute(decode_cc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kCcSmem) !=
+            cudaSuccess)
             return 0;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel<NT>, kCcThreads, cc_smem<NT>()) !=
-                cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_cc_kernel, kCcThreads, kCcSmem) != cudaSuccess ||
             o < 1)
             return 0;
         return o;
@@ -883,7 +889,7 @@ int occupancy_cc() {
 
 // cc_tokens > 0: the integer CUDA-core kernel for that many tokens; else the tensor-core kernel with MMA N = ntok
 int occupancy(int cc_tokens, int ntok) {
-    if (cc_tokens == 1) return occupancy_cc<1>();
+    if (cc_tokens == 1) return occupancy_cc();
     return ntok == 16 ? occupancy_nt<16>() : occupancy_nt<32>();
 }
 
@@ -911,6 +917,9 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     if (kind == 0)  // packed weights: uint32 [rows = N][cols = K/8], box = one group x 128 rows, 64-B swizzle
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 4, kWordsPerGroup, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_64B);
+    else if (kind == 1)  // packed weights, box = two groups x 128 rows, 128-B swizzle
+        ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, ptr, (uint64_t)cols, (uint64_t)rows,
+                            (uint64_t)cols * 4, kWordsPerGroup * kCcUnitGroups, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
     else if (kind == 2)  // scales: bf16 [rows = N][cols = G], box = 8 groups x 128 rows
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 2, 8, kRowsPerCta);
@@ -930,21 +939,19 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     return true;
 }
 
-template <int NT>
 int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& tze, const DecodeArgs& args, int grid,
               cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kCcThreads);
-    cfg.dynamicSmemBytes = cc_smem<NT>();
+    cfg.dynamicSmemBytes = kCcSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_cc_kernel<NT>, tq, tsc, tze, args) == cudaSuccess ? W4A16_OK
-                                                                                              : W4A16_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, decode_cc_kernel, tq, tsc, tze, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
 template <int NTOK>
@@ -1033,7 +1040,10 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
             align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
         return p;
     }
-    const int64_t units = (int64_t)p.row_tiles * G;
+    // units per row tile: pairs of groups for the one-token kernel, groups for the tensor-core kernel
+    const int64_t ug = p.cc_tokens ? G / kCcUnitGroups : G;
+    p.unit_groups = (int)ug;
+    const int64_t units = (int64_t)p.row_tiles * ug;
     int occ = occupancy(p.cc_tokens, p.nt);
     if (occ < 1) occ = 1;
     int64_t grid = (int64_t)occ * num_sms;
@@ -1041,7 +1051,7 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.grid = (int)grid;
     p.units_base = (int)(units / grid);
     p.units_rem = (int)(units % grid);
-    p.max_slots = (int)((G - 1) / p.units_base + 2);
+    p.max_slots = (int)((ug - 1) / p.units_base + 2);
     // the integer kernel reads X itself (its area holds X' = bf16(X * inv_s) for the AWQ entry);
     // the tensor-core kernel reads X digit planes and per-token sums and scales prepared per launch
     p.ws_xp_bytes = p.cc_tokens ? align256((size_t)M * K * 2) : align256((size_t)G * 3 * p.nt * 128);
@@ -1140,16 +1150,18 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
         args.units_base = plan.units_base;
         args.units_rem = plan.units_rem;
         args.max_slots = plan.max_slots;
-        CUtensorMap tsc, tze;
-        if (plan.cc_tokens && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze)))
+        CUtensorMap tsc, tze, tq1;
+        if (plan.cc_tokens && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze) ||
+                               !cached_tmap(kCcUnitGroups == 1 ? 0 : 1, qweight, N, K / 8, &tq1)))
             return W4A16_ERR_CUDA;
-        const int st = plan.cc_tokens == 1   ? launch_cc<1>(tq, tsc, tze, args, plan.grid, stream)
+        if (plan.cc_tokens) args.G = plan.unit_groups;  // the one-token kernel walks units of two groups
+        const int st = plan.cc_tokens == 1   ? launch_cc(tq1, tsc, tze, args, plan.grid, stream)
                        : plan.nt == 16       ? launch_tc<16>(tq, tx, args, plan.grid, stream)
                                              : launch_tc<32>(tq, tx, args, plan.grid, stream);
         if (st != W4A16_OK) return st;
         if (plan.cc_tokens) {
-            const int st2 = launch_decode_reduce(partial, args.Y, N, Mc, G, plan.units_base, plan.units_rem,
-                                                 plan.max_slots, plan.row_tiles, stream);
+            const int st2 = launch_decode_reduce(partial, args.Y, N, Mc, plan.unit_groups, plan.units_base,
+                                                 plan.units_rem, plan.max_slots, plan.row_tiles, stream);
             if (st2 != W4A16_OK) return st2;
         }
     }
