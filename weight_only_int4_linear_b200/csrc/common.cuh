@@ -162,8 +162,8 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
                   const DecodePlan& plan, cudaStream_t stream);
 int num_sms_current();
 
-// The BF16 tensor-core GEMV (gemv_bf.cu) for quantisation groups of `group` (32, 64, 128) weights:
-// scratch = bf_workspace_bytes (after the shared counters); runs M in chunks of 32 tokens.
+// The BF16 tensor-core GEMV (gemv_bf.cu) for quantisation groups of `group` (32, 64, 128) weights, K / group
+// a multiple of 8: scratch = bf_workspace_bytes (after the shared counters); runs M in chunks of 32 tokens.
 size_t bf_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int num_sms);
 int launch_decode_bf(const uint16_t* X, const float* xscale, int64_t M, int64_t K, int group, const uint32_t* qweight,
                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* scratch,

@@ -12,8 +12,8 @@
 //    subtraction removes 128 + c; exact, since |q - c| <= 256 -- and store the
 //    row's 64 words to tensor memory (the A operand, 128 lanes x 64 columns),
 //    with c = z when |z| <= 128 and c = 0 otherwise;
-//  (scales and zero points are loaded from global memory four units ahead of
-//  their use -- two with groups of 32 -- so their latency is not paid per unit;)
+//  (scales and zero points arrive by TMA with the codes, in blocks of 8
+//  quantisation groups x 128 rows, into a small ring of shared-memory slots;)
 //  * one thread issues eight tcgen05.mma kind::f16 (M = 128, N = tokens,
 //    K = 16), A from tensor memory, B = the tokens' BF16 activations (TMA,
 //    128-byte swizzle, K-major), FP32 accumulation in tensor memory, one
@@ -44,7 +44,9 @@ constexpr int kDqWarps = 8;                             // warps 4-11: lane quad
 constexpr int kMmaWarp = kFoldWarps + kDqWarps;         // 12
 constexpr int kTmaWarp = kMmaWarp + 1;                  // 13
 constexpr int kThreads = (kTmaWarp + 1) * 32;           // 448
-constexpr int kAhead = 4;                               // metadata loads run this many units ahead of use
+constexpr int kMetaGroups = 8;                          // quantisation groups per metadata block
+constexpr int kScBytes = kRows * kMetaGroups * 2;       // 128 rows x 8 BF16 scales
+constexpr int kMetaBytes = kScBytes + kRows * kMetaGroups * 4;  // + 128 rows x 8 int32 zero points
 
 template <int NTOK, int GS>
 struct BfCfg {
@@ -56,7 +58,11 @@ struct BfCfg {
     static constexpr int kXsBytes = SUB * NTOK * 4;          // sum of x per quantisation group and token
     static constexpr int kStageBytes = (kXsOff + kXsBytes + 1023) & ~1023;
     static constexpr int kStages = (200 * 1024) / kStageBytes < 8 ? (200 * 1024) / kStageBytes : 8;
-    static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;  // + alignment slack
+    static constexpr int kUnitsPerBlock = kMetaGroups / SUB;  // units per metadata block
+    // a slot is rewritten when its block's last unit is at least kStages units behind the TMA thread
+    static constexpr int kMetaSlots = 1 + (kStages + kUnitsPerBlock - 1) / kUnitsPerBlock;
+    static constexpr int kMetaOff = kStages * kStageBytes;
+    static constexpr size_t kSmem = (size_t)kMetaOff + (size_t)kMetaSlots * kMetaBytes + 1024;  // + alignment slack
     static constexpr int kACols = 64;                        // 128 rows x 128 BF16
     static constexpr int kNumA = 4;
     static constexpr uint32_t kColD = kNumA * kACols;        // accumulators after the A buffers
@@ -68,12 +74,10 @@ struct BfCfg {
 
 struct BfArgs {
     const float* xs;       // [G][SUB][NTOK]: sums of the launch's activations per quantisation group
-    const uint16_t* scales;
-    const int32_t* zeros;
     uint16_t* Y;           // [M][N]
     float* partial;        // [row_tiles][max_slots][M][128]
     int* fault;
-    int M, N, G;           // G: 128-K units per row (K / 128); scales and zeros have G * SUB columns
+    int M, N, G;           // G: 128-K units per row (K / 128); scales and zeros have G * SUB columns (a multiple of 8)
     int units_base, units_rem;
     int max_slots;
 };
@@ -145,11 +149,13 @@ __global__ void __launch_bounds__(256) prep_bf_kernel(const uint16_t* __restrict
 template <int NTOK, int GS>
 __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_constant__ CUtensorMap tq,
                                                                 const __grid_constant__ CUtensorMap tx,
+                                                                const __grid_constant__ CUtensorMap tsc,
+                                                                const __grid_constant__ CUtensorMap tze,
                                                                 const BfArgs a) {
     using C = BfCfg<NTOK, GS>;
     constexpr int S = C::kStages, NA = C::kNumA, ND = C::kNumD, SUB = C::SUB;
     constexpr uint32_t kIdesc = idesc_bf16_f32(128, NTOK);
-    constexpr int AH = SUB >= 4 ? 2 : kAhead;  // metadata lookahead (registers: AH x SUB values per thread)
+    constexpr int UPB = C::kUnitsPerBlock, NS = C::kMetaSlots;
     extern __shared__ unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t full[S], empty[S], afull[NA], afree[NA], mdone[ND], dfree[ND];
     __shared__ uint32_t s_tmem;
@@ -157,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_con
 
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-aligned stages
+    unsigned char* meta = ring + C::kMetaOff;                                // NS slots of kMetaBytes
 
     pdl_launch_dependents();  // the next call may start its weight loads as this grid's CTAs retire
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -164,7 +171,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_con
     const int64_t u_first = (int64_t)b * a.units_base + min(b, a.units_rem);
     const int nunits = a.units_base + (b < a.units_rem ? 1 : 0);
     const int G = a.G, N = a.N, M = a.M;
-    const int GQ = G * SUB;  // quantisation groups per row
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -191,15 +197,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_con
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tx);
+            prefetch_tmap(&tsc);
+            prefetch_tmap(&tze);
             constexpr uint32_t kTx = C::kXBytes + kCodeBytes + C::kXsBytes;
             const int pre = min(S, nunits);
+            int mb = -1;
+            // codes of unit i and, with the first unit of a block of 8 quantisation groups, the block's scales
+            // and zero points into slot mb % NS
+            auto codes_meta = [&](int i, const UnitCursor& c) {
+                const int s = i % S;
+                const bool new_block = i == 0 || c.g % UPB == 0;
+                if (new_block) ++mb;
+                mbar_arrive_expect_tx(&full[s], kTx + (new_block ? kMetaBytes : 0));
+                tma_load_2d(ring + s * C::kStageBytes + C::kCodeOff, &tq, c.g * kWordsPerGroup, c.tile * kRows, &full[s]);
+                if (new_block) {
+                    unsigned char* ms = meta + (mb % NS) * kMetaBytes;
+                    const int gq8 = (c.g * SUB) & ~(kMetaGroups - 1);
+                    tma_load_2d(ms, &tsc, gq8, c.tile * kRows, &full[s]);
+                    tma_load_2d(ms + kScBytes, &tze, gq8, c.tile * kRows, &full[s]);
+                }
+            };
             // the weights do not depend on the preparation kernel: start streaming them at once
             UnitCursor cur(u_first, G);
-            for (int i = 0; i < pre; ++i, cur.next(G)) {
-                mbar_arrive_expect_tx(&full[i], kTx);
-                tma_load_2d(ring + i * C::kStageBytes + C::kCodeOff, &tq, cur.g * kWordsPerGroup, cur.tile * kRows,
-                            &full[i]);
-            }
+            for (int i = 0; i < pre; ++i, cur.next(G)) codes_meta(i, cur);
             pdl_wait_primary();  // X and its sums come from the preparation kernel
             UnitCursor cx(u_first, G);
             for (int i = 0; i < pre; ++i, cx.next(G)) {
@@ -213,8 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_con
                 const int s = i % S;
                 if (!mbar_wait(&empty[s], ((i / S) - 1) & 1, a.fault, 131)) break;
                 unsigned char* st = ring + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], kTx);
-                tma_load_2d(st + C::kCodeOff, &tq, cur.g * kWordsPerGroup, cur.tile * kRows, &full[s]);
+                codes_meta(i, cur);
                 tma_load_2d(st, &tx, cur.g * kGroup, 0, &full[s]);
                 tma_load_2d(st + C::kXBlock, &tx, cur.g * kGroup + 64, 0, &full[s]);
                 bulk_load(st + C::kXsOff, a.xs + (int64_t)cur.g * SUB * NTOK, C::kXsBytes, &full[s]);
@@ -262,71 +281,50 @@ __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_con
         const int row_local = quad * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(quad * 32) << 16);
         const int sw = (row_local >> 1) & 3;  // 64-byte swizzle of the codes tile
-        // zero points of this row, AH units ahead (rows past N: the last row's -- their codes are
-        // zero-filled and their scale folds them away)
-        auto load_z = [&](const UnitCursor& c, int (&z)[SUB]) {
-            const int n = min(c.tile * kRows + row_local, N - 1);
-#pragma unroll
-            for (int sg = 0; sg < SUB; ++sg) z[sg] = __ldg(a.zeros + (int64_t)n * GQ + c.g * SUB + sg);
-        };
         UnitCursor zc(u_first, G);
-        int zr[AH][SUB];
+        int mb = -1;
+        for (int i = 0; i < nunits; ++i, zc.next(G)) {
+            if (i == 0 || zc.g % UPB == 0) ++mb;
+            const int s = i % S, ai = i % NA;
+            if (i >= NA && !mbar_wait(&afree[ai], ((i / NA) - 1) & 1, a.fault, 151)) break;
+            if (!mbar_wait(&full[s], (i / S) & 1, a.fault, 152)) break;
+            // the zero points of this half's words (quantisation groups (8 half .. 8 half + 7) / (GS / 8)) from
+            // the block's slot; rows past N were zero-filled (c = 0)
+            const int* zrow = reinterpret_cast<const int*>(meta + (mb % NS) * kMetaBytes + kScBytes +
+                                                           row_local * (kMetaGroups * 4)) +
+                              ((zc.g * SUB) & (kMetaGroups - 1));
+            const int q0 = GS == 32 ? 2 * half : (GS == 64 ? half : 0);
+            const uint32_t c2a = zero_pair(zrow[q0]), c2b = GS == 32 ? zero_pair(zrow[q0 + 1]) : c2a;
+            // this half's 8 words (chunks 2 half, 2 half + 1); logical 16-byte chunk q of row r sits at chunk
+            // q ^ ((r >> 1) & 3)
+            const unsigned char* codes = ring + s * C::kStageBytes + C::kCodeOff + row_local * 64;
+            uint32_t w[8];
 #pragma unroll
-        for (int u = 0; u < AH; ++u) {
-            if (u < nunits) load_z(zc, zr[u]);
-            zc.next(G);
-        }
-        bool stop = false;
-        for (int i0 = 0; i0 < nunits && !stop; i0 += AH) {
-#pragma unroll
-            for (int u = 0; u < AH; ++u) {
-                const int i = i0 + u;
-                if (i >= nunits || stop) break;
-                uint32_t cp[SUB];
-#pragma unroll
-                for (int sg = 0; sg < SUB; ++sg) cp[sg] = zero_pair(zr[u][sg]);
-                if (i + AH < nunits) load_z(zc, zr[u]);
-                zc.next(G);
-                const int s = i % S, ai = i % NA;
-                if (i >= NA && !mbar_wait(&afree[ai], ((i / NA) - 1) & 1, a.fault, 151)) {
-                    stop = true;
-                    break;
-                }
-                if (!mbar_wait(&full[s], (i / S) & 1, a.fault, 152)) {
-                    stop = true;
-                    break;
-                }
-                // this half's 8 words (32 codes ... chunks 2 half, 2 half + 1); logical 16-byte chunk q of
-                // row r sits at chunk q ^ ((r >> 1) & 3)
-                const unsigned char* codes = ring + s * C::kStageBytes + C::kCodeOff + row_local * 64;
-                uint32_t w[8];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(codes + 16 * ((2 * half + q) ^ sw));
-                    w[4 * q] = v.x;
-                    w[4 * q + 1] = v.y;
-                    w[4 * q + 2] = v.z;
-                    w[4 * q + 3] = v.w;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                // word j (codes 8j .. 8j + 7, quantisation group j / (GS / 8)) -> columns 4j .. 4j + 3
-                // holding the pairs (q0, q4), (q1, q5), (q2, q6), (q3, q7), each minus its c
-                uint32_t pr[32];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const uint32_t x = w[jj], c2 = cp[(8 * half + jj) / (GS / 8)];
-                    pr[4 * jj] = sub_bf16x2(magic_pair(x), c2);
-                    pr[4 * jj + 1] = sub_bf16x2(magic_pair(x >> 4), c2);
-                    pr[4 * jj + 2] = sub_bf16x2(magic_pair(x >> 8), c2);
-                    pr[4 * jj + 3] = sub_bf16x2(magic_pair(x >> 12), c2);
-                }
-                tmem_st32(tl + ai * C::kACols + 32 * half, pr);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&afull[ai]);
+            for (int q = 0; q < 2; ++q) {
+                const uint4 v = *reinterpret_cast<const uint4*>(codes + 16 * ((2 * half + q) ^ sw));
+                w[4 * q] = v.x;
+                w[4 * q + 1] = v.y;
+                w[4 * q + 2] = v.z;
+                w[4 * q + 3] = v.w;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            // word j (codes 8j .. 8j + 7) -> columns 4j .. 4j + 3 holding the pairs (q0, q4), (q1, q5),
+            // (q2, q6), (q3, q7), each minus its c
+            uint32_t pr[32];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const uint32_t x = w[jj], c2 = jj < 4 ? c2a : c2b;
+                pr[4 * jj] = sub_bf16x2(magic_pair(x), c2);
+                pr[4 * jj + 1] = sub_bf16x2(magic_pair(x >> 4), c2);
+                pr[4 * jj + 2] = sub_bf16x2(magic_pair(x >> 8), c2);
+                pr[4 * jj + 3] = sub_bf16x2(magic_pair(x >> 12), c2);
+            }
+            tmem_st32(tl + ai * C::kACols + 32 * half, pr);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[ai]);
         }
         return;
     }
@@ -362,80 +360,57 @@ __global__ void __launch_bounds__(kThreads, 1) decode_bf_kernel(const __grid_con
         for (int m = 0; m < NTOK; ++m) acc[m] = 0.f;
     };
 
-    // scale and zero point of this row per quantisation group, AH units ahead (raw, converted at use)
-    auto load_meta = [&](const UnitCursor& c, uint32_t (&sr)[SUB], int (&zr)[SUB]) {
-        const int n = min(c.tile * kRows + row_local, N - 1);
+    UnitCursor fc(u_first, G);
+    int mb = -1;
+    for (int i = 0; i < nunits; ++i, fc.next(G)) {
+        if (i == 0 || fc.g % UPB == 0) ++mb;
+        const int tile = fc.tile;
+        while (cur_tile < tile) flush(cur_tile++);
+        if (aborted) continue;
+        const int s = i % S;
+        const float* xsum = reinterpret_cast<const float*>(ring + s * C::kStageBytes + C::kXsOff);
+        // this row's scales and zero points from the block's slot (the MMA that this warp waits for
+        // below was issued after the slot's copy completed); rows past N were zero-filled (s = 0)
+        const unsigned char* ms = meta + (mb % NS) * kMetaBytes;
+        const int gq = (fc.g * SUB) & (kMetaGroups - 1);
 #pragma unroll
         for (int sg = 0; sg < SUB; ++sg) {
-            sr[sg] = __ldg(a.scales + (int64_t)n * GQ + c.g * SUB + sg);
-            zr[sg] = __ldg(a.zeros + (int64_t)n * GQ + c.g * SUB + sg);
-        }
-    };
-    UnitCursor fc(u_first, G), mc(u_first, G);
-    uint32_t sr[AH][SUB];
-    int zr[AH][SUB];
-#pragma unroll
-    for (int u = 0; u < AH; ++u) {
-        if (u < nunits) load_meta(mc, sr[u], zr[u]);
-        mc.next(G);
-    }
-    for (int i0 = 0; i0 < nunits; i0 += AH) {
-#pragma unroll
-        for (int u = 0; u < AH; ++u) {
-            const int i = i0 + u;
-            if (i >= nunits) break;
-            const int tile = fc.tile;
-            while (cur_tile < tile) flush(cur_tile++);
-            const bool row_ok = tile * kRows + row_local < N;
-            float sv[SUB], zv[SUB];
-            bool corr[SUB];
-#pragma unroll
-            for (int sg = 0; sg < SUB; ++sg) {
-                sv[sg] = row_ok ? bf16_bits_to_float((uint16_t)sr[u][sg]) : 0.f;
-                corr[sg] = !(zr[u][sg] >= -128 && zr[u][sg] <= 128);  // zero point left for the fold
-                zv[sg] = (float)zr[u][sg];
+            const int jd = i * SUB + sg, di = jd % ND;
+            if (!mbar_wait(&mdone[di], (jd / ND) & 1, a.fault, 161)) {
+                aborted = true;
+                break;
             }
-            if (i + AH < nunits) load_meta(mc, sr[u], zr[u]);
-            mc.next(G);
-            fc.next(G);
-            if (aborted) continue;
-            const int s = i % S;
-            const float* xsum = reinterpret_cast<const float*>(ring + s * C::kStageBytes + C::kXsOff);
+            tc_fence_after();
+            const float sv = bf16_bits_to_float(
+                *reinterpret_cast<const uint16_t*>(ms + row_local * (kMetaGroups * 2) + 2 * (gq + sg)));
+            const int zi = *reinterpret_cast<const int32_t*>(ms + kScBytes + row_local * (kMetaGroups * 4) + 4 * (gq + sg));
+            const bool corr = !(zi >= -128 && zi <= 128);  // zero point left for the fold
+            const bool any_corr = __any_sync(0xFFFFFFFFu, corr);
+            const float zc = corr ? (float)zi : 0.f;
 #pragma unroll
-            for (int sg = 0; sg < SUB; ++sg) {
-                const int jd = i * SUB + sg, di = jd % ND;
-                if (!mbar_wait(&mdone[di], (jd / ND) & 1, a.fault, 161)) {
-                    aborted = true;
-                    break;
+            for (int c0 = 0; c0 < NTOK; c0 += 16) {  // 16 tokens' sums at a time
+                uint32_t d[16];
+                tmem_ld16(tl + C::kColD + di * NTOK + c0, d);
+                tmem_wait_ld();
+                if (c0 + 16 == NTOK) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&dfree[di]);
                 }
-                tc_fence_after();
-                const bool any_corr = __any_sync(0xFFFFFFFFu, corr[sg]);
-                const float zc = corr[sg] ? zv[sg] : 0.f;
+                if (any_corr) {
 #pragma unroll
-                for (int c0 = 0; c0 < NTOK; c0 += 16) {  // 16 tokens' sums at a time
-                    uint32_t d[16];
-                    tmem_ld16(tl + C::kColD + di * NTOK + c0, d);
-                    tmem_wait_ld();
-                    if (c0 + 16 == NTOK) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&dfree[di]);
-                    }
-                    if (any_corr) {
+                    for (int e = 0; e < 16; ++e)
+                        acc[c0 + e] =
+                            fmaf(sv, fmaf(-zc, xsum[sg * NTOK + c0 + e], __uint_as_float(d[e])), acc[c0 + e]);
+                } else {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            acc[c0 + e] = fmaf(sv[sg], fmaf(-zc, xsum[sg * NTOK + c0 + e], __uint_as_float(d[e])),
-                                               acc[c0 + e]);
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) acc[c0 + e] = fmaf(sv[sg], __uint_as_float(d[e]), acc[c0 + e]);
-                    }
+                    for (int e = 0; e < 16; ++e) acc[c0 + e] = fmaf(sv, __uint_as_float(d[e]), acc[c0 + e]);
                 }
             }
-            if (aborted) continue;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);  // the stage's sums read
         }
+        if (aborted) continue;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // the stage's sums read
     }
     const int tile_last = nunits > 0 ? (int)((u_first + nunits - 1) / G) : cur_tile - 1;
     while (cur_tile <= tile_last) flush(cur_tile++);
@@ -522,8 +497,6 @@ int launch_bf_chunk(const uint16_t* X, const float* xscale, int Mc, int64_t K, c
     }
     BfArgs args;
     args.xs = xs;
-    args.scales = scales;
-    args.zeros = zeros;
     args.Y = Y;
     args.partial = partial;
     args.fault = fault;
@@ -540,7 +513,15 @@ int launch_bf_chunk(const uint16_t* X, const float* xscale, int Mc, int64_t K, c
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, decode_bf_kernel<NTOK, GS>, tq, tx, args) != cudaSuccess) return W4A16_ERR_CUDA;
+    const int GQ = G * (kGroup / GS);  // quantisation groups per row
+    CUtensorMap tsc, tze;
+    if (!tmap_2d_cached(&tsc, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, scales, (uint64_t)GQ, (uint64_t)N, (uint64_t)GQ * 2,
+                        kMetaGroups, kRows) ||
+        !tmap_2d_cached(&tze, CU_TENSOR_MAP_DATA_TYPE_INT32, zeros, (uint64_t)GQ, (uint64_t)N, (uint64_t)GQ * 4,
+                        kMetaGroups, kRows))
+        return W4A16_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, decode_bf_kernel<NTOK, GS>, tq, tx, tsc, tze, args) != cudaSuccess)
+        return W4A16_ERR_CUDA;
     return launch_decode_reduce(partial, Y, N, Mc, G, p.units_base, p.units_rem, p.max_slots, p.row_tiles, stream);
 }
 
@@ -566,6 +547,7 @@ size_t bf_workspace_bytes(int64_t M, int64_t N, int64_t K, int group, int num_sm
 int launch_decode_bf(const uint16_t* X, const float* xscale, int64_t M, int64_t K, int group, const uint32_t* qweight,
                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* scratch,
                      cudaStream_t stream) {
+    if ((K / group) % kMetaGroups != 0) return W4A16_ERR_SHAPE;  // metadata blocks of 8 quantisation groups
     CUtensorMap tq;
     if (!tmap_2d_cached(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight, (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2,
                         kWordsPerGroup, kRows, CU_TENSOR_MAP_SWIZZLE_64B))
