@@ -181,11 +181,11 @@ def launches_per_call(c) -> int:
     """Our kernels per linear call: X preparation + GEMM (M >= 64); with K/128
     a multiple of 8, the one-token integer GEMV + its split-K reduction
     (M = 1, X prepared inside the GEMV), or X preparation + integer GEMV +
-    reduction (2 <= M <= 8); otherwise X preparation + tensor-core GEMV per
+    reduction (2 <= M <= 16); otherwise X preparation + tensor-core GEMV per
     32-token chunk."""
     if c.M >= PREFILL_MIN_M:
         return 2
-    if (c.K // 128) % 8 == 0 and c.M <= 8:
+    if (c.K // 128) % 8 == 0 and c.M <= 16:
         return 2 if c.M == 1 else 3
     return 2 * ((c.M + 31) // 32)
 
@@ -345,8 +345,8 @@ def layer_roofline(c, us, peaks, peak_src, kernel):
 def decode_kernel_name(c) -> str:
     if c.M >= PREFILL_MIN_M:
         return "prefill_kernel"
-    if (c.K // 128) % 8 == 0 and c.M <= 8:
-        return "decode_cc_kernel<1>" if c.M == 1 else f"decode_mt_kernel<{4 if c.M <= 4 else 8}>"
+    if (c.K // 128) % 8 == 0 and c.M <= 16:
+        return "decode_cc_kernel" if c.M == 1 else f"decode_mt_kernel<{4 if c.M <= 4 else 8 if c.M <= 8 else 16}>"
     return "decode_tc_kernel<16>" if min(c.M, 32) <= 16 else "decode_tc_kernel<32>"
 
 

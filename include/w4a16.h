@@ -64,7 +64,7 @@ typedef enum {
 typedef enum {
     W4A16_PATH_AUTO = 0,    /* decode GEMV for small M, tensor-core GEMM for large M */
     W4A16_PATH_DECODE = 1,  /* split-K GEMVs, any M: integer mma.sync (codes x digit planes of X) for
-                               M <= 8, tcgen05 (8-bit, codes from tensor memory) for more, in chunks of
+                               M <= 16, tcgen05 (8-bit, codes from tensor memory) for more, in chunks of
                                32 tokens */
     W4A16_PATH_PREFILL = 2  /* TMA + tcgen05/TMEM GEMM on BF16 tiles dequantised in shared memory */
 } w4a16_path;
@@ -153,8 +153,9 @@ W4A16_API int w4a16_linear_g(const uint16_t* X, int64_t M, int64_t K, int group,
  * call leaves it zero again and no call writes anything else there, so one
  * workspace, sized for the largest shape, can be shared by calls of any
  * shapes that are ordered on one stream.  Exception: a decode call with
- * N > 8,388,608 keeps counters beyond that area and needs a workspace of its
- * own.  Calls that may run concurrently need separate workspaces.
+ * N > 8,388,480 (one token) or N > 8,388,608 (more) keeps counters beyond
+ * that area and needs a workspace of its own.  Calls that may run
+ * concurrently need separate workspaces.
  */
 W4A16_API size_t w4a16_workspace_bytes(int64_t M, int64_t N, int64_t K);
 

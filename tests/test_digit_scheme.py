@@ -79,7 +79,7 @@ def _mt_row(nt, p, m):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M,nt", [(2, 4), (3, 4), (4, 4), (6, 8), (8, 8)])
+@pytest.mark.parametrize("M,nt", [(2, 4), (3, 4), (4, 4), (6, 8), (8, 8), (12, 16), (16, 16)])
 def test_gpu_digit_rows_match_the_scheme(cuda_lib, M, nt):
     import torch
     import weight_only_int4_linear_b200 as w4

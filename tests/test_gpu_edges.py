@@ -109,9 +109,9 @@ def test_two_tokens(cuda_lib, pair):
     _check_rows(Y, oracle.linear(X, qw, sc, z), pair, "M=2")
 
 
-@pytest.mark.parametrize("M", [3, 5, 8])
+@pytest.mark.parametrize("M", [3, 5, 8, 12, 16])
 def test_small_batch_integer_gemv(cuda_lib, M):
-    """2 <= M <= 8: digit planes prepared once per launch (4- and 8-token tiles), mma.sync u8 x s8."""
+    """2 <= M <= 16: digit planes prepared once per launch (4-, 8- and 16-token tiles), mma.sync u8 x s8."""
     N, K = 200, 2048
     kinds = [ALL[m % len(ALL)] for m in range(M)]
     pw, (qw, sc, z) = _pack(N, K, 13)
@@ -120,16 +120,17 @@ def test_small_batch_integer_gemv(cuda_lib, M):
     _check_rows(Y, oracle.linear(X, qw, sc, z), kinds, f"M={M}")
 
 
-@pytest.mark.parametrize("M", [9, 11, 16, 40])
-def test_tensor_core_gemv(cuda_lib, M):
-    """9 <= M <= 63: the codes as 8-bit A operands in tensor memory against the digit planes of every token,
-    tcgen05 kind::i8 (16- and 32-token tiles; M = 40 runs a 32-token and an 8-token launch)."""
-    N, K = 200, 2048
+@pytest.mark.parametrize("M,K", [(9, 640), (16, 640), (17, 2048), (40, 2048)])
+def test_tensor_core_gemv(cuda_lib, M, K):
+    """The codes as 8-bit A operands in tensor memory against the digit planes of every token, tcgen05
+    kind::i8 (16- and 32-token tiles): 17 or more tokens, or any count when K / 128 is not a multiple of 8
+    (M = 40 runs a 32-token and an 8-token launch)."""
+    N = 200
     kinds = [ALL[m % len(ALL)] for m in range(M)]
     pw, (qw, sc, z) = _pack(N, K, 13)
     X = edge.activations_bf16(300 + M, kinds, K)
     Y = _linear(X, pw, w4.PATH_DECODE)
-    _check_rows(Y, oracle.linear(X, qw, sc, z), kinds, f"M={M}")
+    _check_rows(Y, oracle.linear(X, qw, sc, z), kinds, f"M={M} K={K}")
 
 
 @pytest.mark.parametrize("group", [32, 64])

@@ -161,8 +161,8 @@ def test_workspace_reuse_and_errors(cuda_lib):
     w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y2, ws)
     torch.cuda.synchronize()
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))  # deterministic split-K order
-    with pytest.raises(w4.W4A16Error) as e:
-        w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y1, ws[: nbytes - 256])
+    with pytest.raises(w4.W4A16Error) as e:  # not even the 256 KB counter area
+        w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y1, ws[: 128 * 1024])
     assert e.value.status == w4.ERR_WORKSPACE
     with pytest.raises(w4.W4A16Error) as e:
         w4.linear(X, pw.qweight, pw.scales, pw.zeros, Y1, None)

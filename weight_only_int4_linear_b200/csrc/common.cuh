@@ -135,7 +135,8 @@ int launch_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, cudaSt
 // the same place for every shape: each call leaves its counters zero and no
 // call writes anything else below kCounterBytes, so calls of any shapes and
 // paths ordered on one stream can share one workspace (row tiles up to
-// kSharedCounterTiles, i.e. N up to 8,388,608).
+// kSharedCounterTiles, i.e. N up to 8,388,608; the one-token kernel keeps one
+// more counter after its row tiles', so N up to 8,388,480 there).
 constexpr int64_t kSharedCounterTiles = 65536;
 constexpr size_t kCounterBytes = (size_t)kSharedCounterTiles * 4;  // 256 KB
 
@@ -150,6 +151,9 @@ struct DecodePlan {
     int units_base;   // each CTA streams units_base (+1 for the first units_rem CTAs) units
     int units_rem;
     int max_slots;    // partial-sum slots per row tile
+    int cc_units;     // one-token kernel: units (quantisation groups) per chunk, 2 or 4
+    int cc_cpt;       // one-token kernel: chunks per row tile (quantisation groups / cc_units)
+    int cc_chunks;    // one-token kernel: chunks in all
     // workspace layout: [counters][Xp][xs][partials]
     size_t ws_counter_bytes, ws_xp_bytes, ws_xs_bytes, ws_partial_bytes;
     size_t workspace_bytes() const;

@@ -15,22 +15,24 @@
 // is written as three signed base-256 digits, so sum_k q x_int is three exact
 // int32 dot products, combined and scaled in FP32 once per group.  The BF16 scale
 // is never folded into a rounded operand.  Three kernels:
-//   * M <= 2: decode_cc_kernel, the dot products as mma.sync m16n8k32 (codes u8 x
+//   * M = 1: decode_cc_kernel, the dot products as mma.sync m16n8k32 (codes u8 x
 //     X digits s8) in the warps' registers, X prepared inside the kernel;
 //   * 3 <= M <= 32 per launch: decode_tc_kernel, tcgen05.mma kind::i8 with the
 //     codes in tensor memory and the digit planes of all tokens as B;
 //   * prep_x8_kernel: the digit planes for the tensor-core kernel.
 // With AWQ inverse channel scales (the activation half of the equivalence
 // transform), X' = bf16(x * inv_s[k]) is formed where X is prepared: inside
-// prep_x8_kernel, and for M <= 2 by awq_prescale_kernel ahead of the integer
+// prep_x8_kernel, and for M = 1 by awq_prescale_kernel ahead of the integer
 // kernel, which then reads X' (doing it in the kernel's single X warp made
 // that warp the bottleneck).
 //
 // Work decomposition: a unit is 128 weight rows x one group (8 KB of codes).
-// Units are numbered row tile by row tile and dealt out to a persistent grid
-// in contiguous, equal ranges (+-1 unit), so every CTA streams the same number
-// of bytes.  A row tile split between CTAs is reduced by the last CTA to
-// finish it (arrival counter), summing the partials in a fixed order.
+// The tensor-core kernel deals units, numbered row tile by row tile, to a
+// persistent grid in contiguous, equal ranges (+-1 unit), and a row tile split
+// between CTAs is reduced by the last CTA to finish its part (arrival counter);
+// the one-token kernel hands out chunks of 2 or 4 units from a counter and a
+// dependent reduction kernel adds the chunks' partial sums.  Either way the
+// partials are summed in a fixed order.
 #include "common.cuh"
 #include "decode_units.cuh"
 #include "sm100.cuh"
@@ -44,8 +46,9 @@ constexpr int kRowsPerCta = 128;
 constexpr int kStageWords = kRowsPerCta * kWordsPerGroup;  // 2048 words = 8 KB
 constexpr int kMaxTokens = 32;  // tokens per launch
 // Token counts up to this take the integer mma.sync GEMV (when K / 128 is a multiple of 8): its MMAs grow
-// with 3 digit planes per token and bound it beyond 8 tokens, where the tcgen05 GEMV is as fast.
-constexpr int64_t kMtMaxTokens = 8;
+// with 3 digit planes per token; at 9-16 tokens it still beats the tcgen05 GEMV by 8-18 % (gate+up and down
+// at hidden size 8192), and the tcgen05 GEMV takes 17-32 tokens per launch.
+constexpr int64_t kMtMaxTokens = 16;
 
 struct DecodeArgs {
     const uint16_t* Xp;  // [Mc][K] BF16, 8-blocks reordered (0,4,1,5,2,6,3,7); the input X itself for M = 1
@@ -535,53 +538,72 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // the two masks above hold the codes, so a lane's B fragment of MMA j is
 // bytes 32 tig + 8 j .. + 7 of its row), then (sum_k X_k as FP32, 2^(E - 21)),
 // padded to 400 bytes.
-// A unit is 128 rows x one group (8 KB of codes; built with two groups per
-// unit it is 16 KB, which measured slower: fewer stages in flight); the CTA
-// streams units through a 4-stage ring:
-//  * warp 4 (one thread) drives TMA: the codes of each unit (64-byte
-//    swizzle) and, once per block of 8 groups of a row tile, that block's
-//    128 x 8 scales and 128 x 8 zero points into one of two metadata slots;
-//  * warp 5 prepares X for each unit's group straight from the BF16 input
-//    (the digit rows, the group sum and power of two), so the call is a
-//    single launch;
-//  * warps 0-3 compute, warp w taking rows 32 w .. 32 w + 31 of each unit as
-//    two 16-row MMA blocks.
-// Four CTAs share an SM: their independent rings keep more loads in flight
-// than one CTA per SM with an in-order ring of the same depth.  A row tile
-// whose units two CTAs share is written by each as a partial-sum slot, and
-// decode_reduce_kernel, launched as a dependent grid, adds the slots in a
-// fixed order: no CTA waits on another or on an atomic at its end, and each
-// CTA frees its SM for the next layer's weight stream as soon as it is done.
-#ifndef W4A16_CC_UNIT_GROUPS
-#define W4A16_CC_UNIT_GROUPS 1
-#endif
-constexpr int kCcUnitGroups = W4A16_CC_UNIT_GROUPS;       // quantisation groups per unit (1 or 2)
-static_assert(kCcUnitGroups == 1 || kCcUnitGroups == 2, "unit size");
+// A unit is 128 rows x one group (8 KB of codes).  Units are dealt out in
+// chunks of U consecutive groups of one row tile (U = 4, or 2 where the CTAs
+// have fewer than 12 units each): chunk c is row tile c / cpt, groups
+// U (c % cpt) onwards (cpt = G / U chunks per row tile).  CTA b takes chunk b first, then asks a global counter for the
+// next free chunk while it issues the current one, so a CTA that starts early
+// or streams fast takes more chunks and every CTA finishes within about a
+// chunk of the others.  (An equal, static deal left the CTAs that started
+// late -- launched as the preceding call's CTAs freed their SMs -- finishing
+// several microseconds after the rest, and the next call cannot begin its
+// arithmetic until the last one is done.)  Each chunk leaves its 128 partial
+// sums in a slot of its own, and decode_cc_reduce_kernel, launched as a
+// dependent grid, adds each row tile's slots in slot order, so Y has the same
+// bits however the chunks were shared out.  (Adding them inside this kernel,
+// by the CTA that completed a tile's last chunk, measured slower: the arrival
+// and the reads of the last tiles kept CTAs resident for microseconds after
+// their arithmetic ended.)
+// Warp roles (192 threads, four CTAs per SM), with a 4-stage ring:
+//  * warp 4 (one thread) takes chunks and drives TMA: per unit it publishes
+//    (row tile, group, chunk slot, metadata slot) in a descriptor ring, then
+//    loads the codes (64-byte swizzle) and, with a chunk's first unit, the
+//    128 x 8 scales and zero points of the 8-group block that holds the chunk
+//    into one of three metadata slots;
+//  * warp 5 prepares X: the groups of a chunk are loaded at its first unit,
+//    and each unit's digit rows, group sum and power of two are written into
+//    its stage;
+//  * warps 0-3 compute: warp w takes rows 32 w .. 32 w + 31 of each unit as
+//    two 16-row MMA blocks (below); at a chunk's last unit each lane stores
+//    its row's sum into the chunk's slot.
 constexpr int kCcWarps = 4;                              // compute warps
 constexpr int kCcTmaWarp = kCcWarps;                     // warp 4
 constexpr int kCcXWarp = kCcWarps + 1;                   // warp 5
 constexpr int kCcThreads = (kCcWarps + 2) * 32;
-constexpr int kCcStages = kCcUnitGroups == 1 ? 4 : 2;    // ring depth: 32 KB of codes in flight per CTA
+constexpr int kCcStages = 4;                             // ring depth: 32 KB of codes in flight per CTA
 constexpr int kCcMinBlocks = 4;                          // CTAs per SM
-constexpr int kCcRowBytes = 64 * kCcUnitGroups;          // codes of one row in a unit
-constexpr int kCcSwizzleSpan = 8 * kCcRowBytes;          // 64- or 128-byte swizzle: 8-row pattern
-constexpr int kCcCodeBytes = kStageWords * 4 * kCcUnitGroups;  // 8 or 16 KB
-constexpr int kCcXOff = kCcCodeBytes;                    // X of the unit's groups, after the codes
+constexpr int kCcChunkMax = 4;                           // units (groups) per chunk: 2 or 4
+constexpr int kCcRowBytes = 64;                          // codes of one row in a unit
+constexpr int kCcSwizzleSpan = 8 * kCcRowBytes;          // 64-byte swizzle: 8-row pattern
+constexpr int kCcCodeBytes = kStageWords * 4;            // 8 KB
+constexpr int kCcXOff = kCcCodeBytes;                    // X of the unit's group, after the codes
 constexpr int kCcXGroupBytes = 400;                      // 3 digit rows + sum and scale, 16-byte aligned
-constexpr int kCcStageBytes =
-    (kCcCodeBytes + kCcUnitGroups * kCcXGroupBytes + kCcSwizzleSpan - 1) / kCcSwizzleSpan * kCcSwizzleSpan;
+constexpr int kCcStageBytes = (kCcCodeBytes + kCcXGroupBytes + kCcSwizzleSpan - 1) / kCcSwizzleSpan * kCcSwizzleSpan;
 constexpr int kCcMetaGroups = 8;                         // groups per metadata block
-constexpr int kXAhead = 4;                               // X warp: loads in flight, in units
 constexpr int kCcScBytes = kRowsPerCta * kCcMetaGroups * 2;  // 128 rows x 8 BF16 scales
 constexpr int kCcZeBytes = kRowsPerCta * kCcMetaGroups * 4;  // 128 rows x 8 int32 zero points
 constexpr int kCcMetaBytes = kCcScBytes + kCcZeBytes;    // one slot, 6 KB
-constexpr int kCcMetaOff = kCcStages * kCcStageBytes;    // two slots after the ring
-constexpr size_t kCcSmem = (size_t)kCcMetaOff + 2 * kCcMetaBytes + 1024;  // + alignment slack
-// A metadata slot is rewritten two blocks later.  Blocks are aligned to 8
-// groups inside a row tile (the kernel needs G % 8 == 0), so the block in
-// between has 4 units; with at most kCcStages units in flight, every unit of
-// the older block has been released by then.
-static_assert(kCcStages <= kCcMetaGroups / kCcUnitGroups, "metadata slot reuse");
+constexpr int kCcMetaSlots = 3;
+constexpr int kCcMetaOff = kCcStages * kCcStageBytes;    // the metadata slots after the ring
+constexpr size_t kCcSmem = (size_t)kCcMetaOff + kCcMetaSlots * kCcMetaBytes + 1024;  // + alignment slack
+static_assert(kCcMetaGroups % kCcChunkMax == 0, "a chunk lies inside one metadata block");
+// A chunk's block goes into slot (chunk number) % kCcMetaSlots, overwriting the block of the chunk
+// kCcMetaSlots chunks earlier, whose last unit is then at least (kCcMetaSlots - 1) 2 + 1 units back
+// (chunks of 2 or more units); the TMA thread issues a unit only after the unit kCcStages back has been
+// released.
+static_assert((kCcMetaSlots - 1) * 2 + 1 >= kCcStages, "metadata slot reuse");
+
+struct CcArgs {
+    const uint16_t* X;  // [K] BF16: the activations (X' = bf16(x * xscale) for the AWQ entry)
+    uint16_t* Y;        // [N]
+    float* partial;     // [row_tiles][cpt][128]: one slot of sums per chunk
+    int* counters;      // counters[row_tiles]: the chunk counter (the row tiles' own counters stay unused)
+    int* fault;
+    int N, G;           // G: groups per row (a multiple of 8)
+    int U;              // units per chunk (2 or 4)
+    int cpt, chunks;    // chunks per row tile (G / U), chunks in all
+    int row_tiles;
+};
 
 // This lane's four BF16 values of group g: lane 2w + h holds values 4h..4h+3 of word w.
 __device__ __forceinline__ uint2 load_group_x(const uint16_t* __restrict__ X, int g, int lane) {
@@ -654,24 +676,26 @@ __device__ __forceinline__ void prep_group_x8(const uint2 v, unsigned char* dst,
 __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(const __grid_constant__ CUtensorMap tq,
                                                                   const __grid_constant__ CUtensorMap tsc,
                                                                   const __grid_constant__ CUtensorMap tze,
-                                                                  const DecodeArgs a) {
+                                                                  const CcArgs a) {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages];
+    __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages], dready[kCcStages];
+    __shared__ int4 s_desc[kCcStages];   // (row tile, group, chunk slot, flags) of the unit in each stage
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-aligned (the swizzle's span)
     unsigned char* meta = ring + kCcMetaOff;
+    // descriptor flags: first unit of its chunk, last unit of its chunk, end of the stream; metadata slot
+    constexpr int kFirst = 1, kLast = 2, kEnd = 4, kSlotShift = 4;
 
     pdl_launch_dependents();  // the next call may start its weight loads as this grid's CTAs retire
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
-    const int64_t u_first = (int64_t)b * a.units_base + min(b, a.units_rem);
-    const int nunits = a.units_base + (b < a.units_rem ? 1 : 0);
-    const int G2 = a.G, N = a.N;  // units (group pairs) per row tile
+    int* const next_chunk = a.counters + a.row_tiles;  // chunks taken beyond the first gridDim.x
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCcStages; ++s) {
             mbar_init(&full[s], 2);  // TMA thread (with the transaction bytes) + X warp
             mbar_init(&empty[s], kCcWarps);
+            mbar_init(&dready[s], 1);  // TMA thread: the stage's descriptor is written
         }
         fence_mbar_init();
     }
@@ -682,61 +706,86 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
             prefetch_tmap(&tq);
             prefetch_tmap(&tsc);
             prefetch_tmap(&tze);
-            // the weights need nothing from the preceding kernel: no PDL wait here
-            UnitCursor cur(u_first, G2);
-            int mb = -1, issued = 0;
-            for (int i = 0; i < nunits; ++i, cur.next(G2)) {
-                const int s = i % kCcStages;
-                if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) break;
-                const int g0 = cur.g * kCcUnitGroups;  // first group of the unit
-                const bool new_block = i == 0 || (g0 & (kCcMetaGroups - 1)) == 0;
-                if (new_block) ++mb;
-                unsigned char* st = ring + s * kCcStageBytes;
-                mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (new_block ? kCcMetaBytes : 0));
-                tma_load_2d(st, &tq, g0 * kWordsPerGroup, cur.tile * kRowsPerCta, &full[s]);
-                if (new_block) {
-                    unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
-                    const int g8 = g0 & ~(kCcMetaGroups - 1);
-                    tma_load_2d(ms, &tsc, g8, cur.tile * kRowsPerCta, &full[s]);
-                    tma_load_2d(ms + kCcScBytes, &tze, g8, cur.tile * kRowsPerCta, &full[s]);
+            int i = 0, nchunks = 0;  // units and chunks issued
+            bool ok = true;
+            auto issue_chunk = [&](int c) {
+                const int tile = c / a.cpt, k = c - tile * a.cpt;
+                const int mslot = nchunks++ % kCcMetaSlots;
+                for (int u = 0; u < a.U; ++u, ++i) {
+                    const int s = i % kCcStages;
+                    if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) {
+                        ok = false;
+                        return;
+                    }
+                    const int g = k * a.U + u;
+                    s_desc[s] = make_int4(tile, g, k,
+                                          (u == 0 ? kFirst : 0) | (u + 1 == a.U ? kLast : 0) | (mslot << kSlotShift));
+                    mbar_arrive(&dready[s]);
+                    unsigned char* st = ring + s * kCcStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (u == 0 ? kCcMetaBytes : 0));
+                    tma_load_2d(st, &tq, g * kWordsPerGroup, tile * kRowsPerCta, &full[s]);
+                    if (u == 0) {
+                        unsigned char* ms = meta + mslot * kCcMetaBytes;
+                        const int g8 = g & ~(kCcMetaGroups - 1);
+                        tma_load_2d(ms, &tsc, g8, tile * kRowsPerCta, &full[s]);
+                        tma_load_2d(ms + kCcScBytes, &tze, g8, tile * kRowsPerCta, &full[s]);
+                    }
                 }
-                ++issued;
+            };
+            // the weights need nothing from the preceding kernel: the first chunk streams at once
+            issue_chunk(b);  // gridDim.x <= chunks
+            // the chunk counter is this launch's once the preceding launch has completed (which leaves it zero)
+            pdl_wait_primary();
+            // Each CTA takes chunks until the counter runs past the end, so a launch draws exactly `chunks`
+            // values, 0 .. chunks - 1: the CTA that draws the last one is the last to draw at all and
+            // puts the counter back to zero for the next launch.
+            int v = ok ? atomicAdd(next_chunk, 1) : 0;
+            while (ok && (int)gridDim.x + v < a.chunks) {
+                const int c = (int)gridDim.x + v;
+                v = atomicAdd(next_chunk, 1);  // in flight while chunk c is issued
+                issue_chunk(c);
             }
-            // no copy may still be in flight when the CTA exits
-            for (int i = max(0, issued - kCcStages); i < issued; ++i)
-                mbar_wait(&full[i % kCcStages], (i / kCcStages) & 1, a.fault, 52);
+            if (ok && v == a.chunks - 1) *next_chunk = 0;
+            // every copy issued must land before the CTA may exit; then the end of the stream, in the stage
+            // after the last unit (posted after the drain, so that no stage sees a newer phase meanwhile)
+            for (int j = max(0, i - kCcStages); j < i; ++j)
+                mbar_wait(&full[j % kCcStages], (j / kCcStages) & 1, a.fault, 52);
+            if (ok) {
+                const int s = i % kCcStages;
+                if (i < kCcStages || mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) {
+                    s_desc[s] = make_int4(-1, 0, 0, kEnd);
+                    mbar_arrive(&dready[s]);
+                    mbar_arrive(&full[s]);
+                }
+            }
         }
         return;
     }
 
     if (warp == kCcXWarp) {  // ------------------------------------------ X warp
         pdl_wait_primary();  // X may come from the preceding kernel
-        const uint16_t* X = a.Xp;
-        // loads run kXAhead units ahead of the preparation, so L2 latency is paid once, not per unit
-        uint2 q[kXAhead][kCcUnitGroups];
-        UnitCursor cl(u_first, G2);
-#pragma unroll
-        for (int j = 0; j < kXAhead; ++j, cl.next(G2))
-#pragma unroll
-            for (int gi = 0; gi < kCcUnitGroups; ++gi)
-                q[j][gi] = j < nunits ? load_group_x(X, cl.g * kCcUnitGroups + gi, lane) : make_uint2(0, 0);
-        for (int i = 0; i < nunits; ++i, cl.next(G2)) {
-            uint2 v[kCcUnitGroups];
-#pragma unroll
-            for (int gi = 0; gi < kCcUnitGroups; ++gi) {
-                v[gi] = q[0][gi];
-#pragma unroll
-                for (int j = 0; j + 1 < kXAhead; ++j) q[j][gi] = q[j + 1][gi];
-                q[kXAhead - 1][gi] = i + kXAhead < nunits ? load_group_x(X, cl.g * kCcUnitGroups + gi, lane)
-                                                          : make_uint2(0, 0);
-            }
+        uint2 xq[kCcChunkMax];  // the current chunk's groups, loaded together (one L2 round trip per chunk)
+        for (int i = 0;; ++i) {
             const int s = i % kCcStages;
-            if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 54)) break;
+            if (!warp_wait(&dready[s], (i / kCcStages) & 1, a.fault, 54)) break;
+            const int4 d = s_desc[s];
+            if (!(d.w & kEnd)) {
+                if (d.w & kFirst) {
 #pragma unroll
-            for (int gi = 0; gi < kCcUnitGroups; ++gi)
-                prep_group_x8(v[gi], ring + s * kCcStageBytes + kCcXOff + gi * kCcXGroupBytes, lane);
+                    for (int j = 0; j < kCcChunkMax; ++j)
+                        if (j < a.U) xq[j] = load_group_x(a.X, d.y + j, lane);
+                }
+                const int u = d.y & (a.U - 1);
+                uint2 v = xq[0];
+#pragma unroll
+                for (int j = 1; j < kCcChunkMax; ++j)
+                    if (u == j) v = xq[j];
+                // the stage was released before its descriptor was posted
+                prep_group_x8(v, ring + s * kCcStageBytes + kCcXOff, lane);
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
+            if (d.w & kEnd) break;
         }
         return;
     }
@@ -750,112 +799,119 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
     const int g8 = lane >> 2, tig = lane & 3;
     auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
     const int r_own = rrow(tig);  // the row this lane folds
-    float y = 0.f;                // row r_own of the current row tile
-    int cur_tile = -1;
-    bool aborted = false;
-
-    // A row tile leaves the CTA as Y (the CTA holds all of its units) or as this CTA's partial-sum slot
-    // (decode_reduce_kernel adds the slots).
-    auto flush = [&](int tile) {
-        const int first = cta_of_unit((int64_t)tile * G2, a.units_base, a.units_rem);
-        const int last = cta_of_unit((int64_t)tile * G2 + G2 - 1, a.units_base, a.units_rem);
-        if (first == last) {
-            const int n = tile * kRowsPerCta + r_own;
-            if (n < N) a.Y[n] = float_to_bf16_bits(y);
-        } else {
-            a.partial[((int64_t)tile * a.max_slots + (b - first)) * kRowsPerCta + r_own] = y;
-        }
-        y = 0.f;
-    };
-
-    UnitCursor uc(u_first, G2);
-    int mb = -1;
-    for (int i = 0; i < nunits; ++i, uc.next(G2)) {
-        const int tile = uc.tile, g0 = uc.g * kCcUnitGroups;
-        if (i == 0 || (g0 & (kCcMetaGroups - 1)) == 0) ++mb;
-        if (tile != cur_tile) {
-            if (cur_tile >= 0) flush(cur_tile);
-            cur_tile = tile;
-        }
-        if (aborted) continue;
+    float y = 0.f;                // row r_own of the current chunk
+    for (int i = 0;; ++i) {
         const int s = i % kCcStages;
-        if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 53)) {
-            aborted = true;
-            continue;
-        }
+        if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 53)) break;
+        const int4 d = s_desc[s];
+        if (d.w & kEnd) break;
         const unsigned char* st = ring + s * kCcStageBytes;
-        const unsigned char* ms = meta + (mb & 1) * kCcMetaBytes;
+        const unsigned char* ms = meta + ((d.w >> kSlotShift) & 3) * kCcMetaBytes;
+        // codes: 16-byte chunk tig of each 64-byte row, 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3))
+        uint4 cw[4];
 #pragma unroll
-        for (int gi = 0; gi < kCcUnitGroups; ++gi) {
-            // codes: 16-byte chunk 4 gi + tig of each row; with one group per unit a row is 64 bytes,
-            // 64-byte swizzle (chunk c of row r at c ^ ((r >> 1) & 3)), with two it is 128 bytes, 128-byte
-            // swizzle (chunk c at c ^ (r & 7))
-            uint4 cw[4];
+        for (int k = 0; k < 4; ++k) {
+            const int r = rrow(k);
+            cw[k] = *reinterpret_cast<const uint4*>(st + r * kCcRowBytes + 16 * (tig ^ ((r >> 1) & 3)));
+        }
+        // B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of the second
+        // row block and each lane of a quad can fold one of its four rows; columns 3 and 7 are zero
+        const unsigned char* xg = st + kCcXOff;
+        uint32_t bx[8];
+        const int xrow = g8 & 3;
+        if (xrow < 3) {
+            const uint4* xp = reinterpret_cast<const uint4*>(xg + xrow * 128 + tig * 32);
+            const uint4 u0 = xp[0], u1 = xp[1];
+            bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
+            bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
+        } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int r = rrow(k);
-                const int c = kCcUnitGroups == 1 ? (tig ^ ((r >> 1) & 3)) : ((4 * gi + tig) ^ (r & 7));
-                cw[k] = *reinterpret_cast<const uint4*>(st + r * kCcRowBytes + 16 * c);
-            }
-            // B columns 4-6 repeat digit planes 0-2, so that lanes tig = 2, 3 hold every plane of the second
-            // row block and each lane of a quad can fold one of its four rows; columns 3 and 7 are zero
-            const unsigned char* xg = st + kCcXOff + gi * kCcXGroupBytes;
-            uint32_t bx[8];
-            const int xrow = g8 & 3;
-            if (xrow < 3) {
-                const uint4* xp = reinterpret_cast<const uint4*>(xg + xrow * 128 + tig * 32);
-                const uint4 u0 = xp[0], u1 = xp[1];
-                bx[0] = u0.x; bx[1] = u0.y; bx[2] = u0.z; bx[3] = u0.w;
-                bx[4] = u1.x; bx[5] = u1.y; bx[6] = u1.z; bx[7] = u1.w;
-            } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) bx[j] = 0u;
-            }
-            const float* ext = reinterpret_cast<const float*>(xg + 3 * 128);
-            const float xsum = ext[0], xscale = ext[1];
-            // this lane's row's metadata, from the block loaded with the block's first unit (which this
-            // warp has already waited for); rows past N were zero-filled by TMA: s = 0 folds them away
-            const int gb = (g0 + gi) & (kCcMetaGroups - 1);
-            const float sv =
-                bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(ms + r_own * (kCcMetaGroups * 2) + 2 * gb));
-            const float zv = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r_own * (kCcMetaGroups * 4) + 4 * gb);
-            if (gi + 1 == kCcUnitGroups) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-            }
+            for (int j = 0; j < 8; ++j) bx[j] = 0u;
+        }
+        const float* ext = reinterpret_cast<const float*>(xg + 3 * 128);
+        const float xsum = ext[0], xscale = ext[1];
+        // this lane's row's metadata, from the chunk's block (loaded with the chunk's first unit, which
+        // this warp has already waited for); rows past N were zero-filled by TMA: s = 0 folds them away
+        const int gb = d.y & (kCcMetaGroups - 1);
+        const float sv = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(ms + r_own * (kCcMetaGroups * 2) + 2 * gb));
+        const float zv = (float)*reinterpret_cast<const int32_t*>(ms + kCcScBytes + r_own * (kCcMetaGroups * 4) + 4 * gb);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
 
-            int d[2][4];
+        int dd[2][4];
 #pragma unroll
-            for (int rb = 0; rb < 2; ++rb) {
-                const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
-                const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
+        for (int rb = 0; rb < 2; ++rb) {
+            const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
+            const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) d[rb][j] = 0;
+            for (int j = 0; j < 4; ++j) dd[rb][j] = 0;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    mma_u8s8(d[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, w0[j] & 0xF0F0F0F0u, w1[j] & 0xF0F0F0F0u,
-                             bx[2 * j], bx[2 * j + 1]);
-            }
-            // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes (0, 1)
-            // at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block tig >> 1
-            // (its own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour completes its
-            // planes.
-            const bool hi = tig >> 1, even = !(tig & 1);
-            int e[4];
+            for (int j = 0; j < 4; ++j)
+                mma_u8s8(dd[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, w0[j] & 0xF0F0F0F0u, w1[j] & 0xF0F0F0F0u,
+                         bx[2 * j], bx[2 * j + 1]);
+        }
+        // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3): planes (0, 1)
+        // at tig = 0 and 2, (2, -) at tig = 1 and 3.  Lane tig folds row rrow(tig): row block tig >> 1
+        // (its own MMA results) and row g8 + 8 (tig & 1); one exchange with the neighbour completes its
+        // planes.
+        const bool hi = tig >> 1, even = !(tig & 1);
+        int e[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) e[j] = hi ? d[1][j] : d[0][j];
-            const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
-            const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
-            const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
-            // sum q X = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26); then
-            // s (sum q X - z sum X) and the power of two last, so that neither product leaves the FP32
-            // range unless the group's result itself does
-            const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
-            y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
+        for (int j = 0; j < 4; ++j) e[j] = hi ? dd[1][j] : dd[0][j];
+        const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
+        const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
+        const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
+        // sum q X = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26); then
+        // s (sum q X - z sum X) and the power of two last, so that neither product leaves the FP32
+        // range unless the group's result itself does
+        const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+        y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
+
+        if (d.w & kLast) {  // the chunk's sums leave through its slot (decode_cc_reduce_kernel adds them)
+            a.partial[((int64_t)d.x * a.cpt + d.z) * kRowsPerCta + r_own] = y;
+            y = 0.f;
         }
     }
-    if (cur_tile >= 0) flush(cur_tile);
 }
+
+// Split-K sums of the one-token kernel: Y[n] = the sum of row n's chunk slots in slot order.  A
+// dependent grid: its CTAs become resident beside the GEMV's (256 threads of at most 32 registers fit next
+// to four GEMV CTAs) and wait for it to complete.  Per row tile, 128 x P threads: part p adds slots p,
+// p + P, ... of its row (at most 16 loads in flight per thread, so one L2 round trip serves tiles of up to
+// 16 P chunks), then part 0 adds the P part sums in order.
+constexpr int kCcRedParts = 2;
+__global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_kernel(const float* __restrict__ partial,
+                                                                                     uint16_t* __restrict__ Y, int N,
+                                                                                     int cpt, int row_tiles) {
+    __shared__ float s_part[kCcRedParts - 1][kRowsPerCta];
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    const int r = threadIdx.x % kRowsPerCta, p = threadIdx.x / kRowsPerCta;
+    for (int tile = blockIdx.x; tile < row_tiles; tile += gridDim.x) {
+        const float* pb = partial + (int64_t)tile * cpt * kRowsPerCta + r;
+        float acc = 0.f;
+        for (int k0 = p; k0 < cpt; k0 += 16 * kCcRedParts) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int k = k0 + e * kCcRedParts;
+                v[e] = k < cpt ? __ldcg(pb + (int64_t)k * kRowsPerCta) : 0.f;
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc += v[e];
+        }
+        if (p > 0) s_part[p - 1][r] = acc;
+        __syncthreads();
+        if (p == 0) {
+#pragma unroll
+            for (int q = 0; q < kCcRedParts - 1; ++q) acc += s_part[q][r];
+            const int n = tile * kRowsPerCta + r;
+            if (n < N) Y[n] = float_to_bf16_bits(acc);
+        }
+        __syncthreads();
+    }
+}
+
 
 template <int NTOK>
 int occupancy_nt() {
@@ -887,11 +943,6 @@ int occupancy_cc() {
     });
 }
 
-// cc_tokens > 0: the integer CUDA-core kernel for that many tokens; else the tensor-core kernel with MMA N = ntok
-int occupancy(int cc_tokens, int ntok) {
-    if (cc_tokens == 1) return occupancy_cc();
-    return ntok == 16 ? occupancy_nt<16>() : occupancy_nt<32>();
-}
 
 // Tensor maps keyed by base pointer and shape (encoding costs a few
 // microseconds of host time; a decode step reuses the same few tensors).
@@ -917,9 +968,6 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     if (kind == 0)  // packed weights: uint32 [rows = N][cols = K/8], box = one group x 128 rows, 64-B swizzle
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 4, kWordsPerGroup, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_64B);
-    else if (kind == 1)  // packed weights, box = two groups x 128 rows, 128-B swizzle
-        ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_UINT32, ptr, (uint64_t)cols, (uint64_t)rows,
-                            (uint64_t)cols * 4, kWordsPerGroup * kCcUnitGroups, kRowsPerCta, CU_TENSOR_MAP_SWIZZLE_128B);
     else if (kind == 2)  // scales: bf16 [rows = N][cols = G], box = 8 groups x 128 rows
         ok = encode_tmap_2d(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ptr, (uint64_t)cols, (uint64_t)rows,
                             (uint64_t)cols * 2, 8, kRowsPerCta);
@@ -939,7 +987,7 @@ bool cached_tmap(int kind, const void* ptr, int64_t rows, int64_t cols, CUtensor
     return true;
 }
 
-int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& tze, const DecodeArgs& args, int grid,
+int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& tze, const CcArgs& args, int grid,
               cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -1032,6 +1080,22 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.bf = false;
     p.nt = p.cc_tokens ? 1 : (Mc <= 16 ? 16 : 32);
     p.row_tiles = (int)ceil_div(N, kRowsPerCta);
+    if (p.cc_tokens) {  // chunks dealt out by a counter after the row tiles' arrival counters
+        int occ = occupancy_cc();
+        if (occ < 1) occ = 1;
+        const int64_t grid = (int64_t)occ * num_sms;
+        // chunks of 4 units where every CTA streams 12 or more units, else of 2 (finer sharing)
+        p.cc_units = (int64_t)p.row_tiles * G >= 12 * grid ? 4 : 2;
+        p.cc_cpt = (int)(G / p.cc_units);
+        p.cc_chunks = p.row_tiles * p.cc_cpt;
+        p.grid = (int)(grid < p.cc_chunks ? grid : p.cc_chunks);
+        p.ws_xp_bytes = align256((size_t)M * K * 2);  // X' = bf16(X * xscale) for the AWQ entry
+        p.ws_xs_bytes = 0;
+        p.ws_partial_bytes = align256((size_t)p.cc_chunks * kRowsPerCta * 4);
+        const int64_t words = p.row_tiles + 1;
+        p.ws_counter_bytes = align256((size_t)(words > kSharedCounterTiles ? words : kSharedCounterTiles) * 4);
+        return p;
+    }
     if (p.mt || p.bf) {  // these GEMVs keep their own plans per chunk; only their scratch is sized here
         p.ws_xp_bytes = p.mt ? mt_workspace_bytes(M, N, K, num_sms) : bf_workspace_bytes(M, N, K, kGroup, num_sms);
         p.ws_xs_bytes = 0;
@@ -1040,11 +1104,11 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
             align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
         return p;
     }
-    // units per row tile: pairs of groups for the one-token kernel, groups for the tensor-core kernel
-    const int64_t ug = p.cc_tokens ? G / kCcUnitGroups : G;
+    // units per row tile: one per group
+    const int64_t ug = G;
     p.unit_groups = (int)ug;
     const int64_t units = (int64_t)p.row_tiles * ug;
-    int occ = occupancy(p.cc_tokens, p.nt);
+    int occ = p.nt == 16 ? occupancy_nt<16>() : occupancy_nt<32>();
     if (occ < 1) occ = 1;
     int64_t grid = (int64_t)occ * num_sms;
     if (grid > units) grid = units;
@@ -1052,10 +1116,9 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     p.units_base = (int)(units / grid);
     p.units_rem = (int)(units % grid);
     p.max_slots = (int)((ug - 1) / p.units_base + 2);
-    // the integer kernel reads X itself (its area holds X' = bf16(X * inv_s) for the AWQ entry);
     // the tensor-core kernel reads X digit planes and per-token sums and scales prepared per launch
-    p.ws_xp_bytes = p.cc_tokens ? align256((size_t)M * K * 2) : align256((size_t)G * 3 * p.nt * 128);
-    p.ws_xs_bytes = p.cc_tokens ? 0 : align256((size_t)G * 2 * p.nt * 4);
+    p.ws_xp_bytes = align256((size_t)G * 3 * p.nt * 128);
+    p.ws_xs_bytes = align256((size_t)G * 2 * p.nt * 4);
     p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * Mc * kRowsPerCta * 4);
     p.ws_counter_bytes = align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
     return p;
@@ -1082,6 +1145,71 @@ __global__ void __launch_bounds__(256) awq_prescale_kernel(const uint16_t* __res
 
 size_t DecodePlan::workspace_bytes() const { return ws_xp_bytes + ws_xs_bytes + ws_partial_bytes + ws_counter_bytes; }
 
+namespace {
+
+// M = 1: the chunked integer GEMV (after awq_prescale_kernel for the AWQ entry); it adds its own split-K
+// slots, so the call is one launch (two with the prescale).
+int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint32_t* qweight, const uint16_t* scales,
+                   const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, const DecodePlan& plan,
+                   cudaStream_t stream) {
+    const int G = (int)(K / kGroup);
+    CUtensorMap tq, tsc, tze;
+    if (!cached_tmap(0, qweight, N, K / 8, &tq) || !cached_tmap(2, scales, N, G, &tsc) ||
+        !cached_tmap(3, zeros, N, G, &tze))
+        return W4A16_ERR_CUDA;
+    int* fault = fault_word();
+    if (!fault) return W4A16_ERR_CUDA;
+    char* ws = reinterpret_cast<char*>(workspace);
+    CcArgs args;
+    args.X = X;
+    if (xscale) {
+        uint16_t* Xs = reinterpret_cast<uint16_t*>(ws + plan.ws_counter_bytes);
+        const int64_t n8 = K / 8;
+        int pgrid = (int)ceil_div(n8, 256);
+        if (pgrid > num_sms_current()) pgrid = num_sms_current();
+        cudaLaunchConfig_t pcfg = {};
+        pcfg.gridDim = dim3((unsigned)pgrid);
+        pcfg.blockDim = dim3(256);
+        pcfg.stream = stream;
+        cudaLaunchAttribute pattr[1];
+        pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        pattr[0].val.programmaticStreamSerializationAllowed = 1;
+        pcfg.attrs = pattr;
+        pcfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&pcfg, awq_prescale_kernel, X, xscale, n8, (int)K, Xs) != cudaSuccess)
+            return W4A16_ERR_CUDA;
+        args.X = Xs;
+    }
+    args.Y = Y;
+    args.partial = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes + plan.ws_xs_bytes);
+    args.counters = reinterpret_cast<int*>(ws);
+    args.fault = fault;
+    args.N = (int)N;
+    args.G = G;
+    args.U = plan.cc_units;
+    args.cpt = plan.cc_cpt;
+    args.chunks = plan.cc_chunks;
+    args.row_tiles = plan.row_tiles;
+    int st = launch_cc(tq, tsc, tze, args, plan.grid, stream);
+    if (st != W4A16_OK) return st;
+    const int sms = num_sms_current();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(plan.row_tiles < sms ? plan.row_tiles : sms));
+    cfg.blockDim = dim3(kRowsPerCta * kCcRedParts);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, (const float*)args.partial, Y, (int)N, plan.cc_cpt,
+                              plan.row_tiles) == cudaSuccess
+               ? W4A16_OK
+               : W4A16_ERR_CUDA;
+}
+
+}  // namespace
+
 int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
                   const DecodePlan& plan, cudaStream_t stream) {
@@ -1091,6 +1219,7 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
     if (plan.bf)
         return launch_decode_bf(X, xscale, M, K, kGroup, qweight, scales, zeros, N, Y,
                                 reinterpret_cast<char*>(workspace) + plan.ws_counter_bytes, stream);
+    if (plan.cc_tokens) return launch_cc_path(X, xscale, K, qweight, scales, zeros, N, Y, workspace, plan, stream);
     CUtensorMap tq;
     if (!cached_tmap(0, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
     int* fault = fault_word();
@@ -1104,38 +1233,17 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
     for (int64_t m0 = 0; m0 < M; m0 += kMaxTokens) {
         const int Mc = (int)((M - m0) < kMaxTokens ? (M - m0) : kMaxTokens);
         CUtensorMap tx;
-        if (!plan.cc_tokens && !cached_tmap(plan.nt, planes, (int64_t)G * 3 * plan.nt, 128, &tx))
-            return W4A16_ERR_CUDA;
-        if (!plan.cc_tokens) {
-            const int64_t prep_threads = (int64_t)G * plan.nt * 32;
-            int prep_grid = (int)ceil_div(prep_threads, 256);
-            if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
-            if (plan.nt == 16)
-                prep_x8_kernel<16><<<prep_grid, 256, 0, stream>>>(X + m0 * K, xscale, Mc, (int)K, planes, xs);
-            else
-                prep_x8_kernel<32><<<prep_grid, 256, 0, stream>>>(X + m0 * K, xscale, Mc, (int)K, planes, xs);
-            if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
-        }
+        if (!cached_tmap(plan.nt, planes, (int64_t)G * 3 * plan.nt, 128, &tx)) return W4A16_ERR_CUDA;
+        const int64_t prep_threads = (int64_t)G * plan.nt * 32;
+        int prep_grid = (int)ceil_div(prep_threads, 256);
+        if (prep_grid > num_sms_current() * 8) prep_grid = num_sms_current() * 8;
+        if (plan.nt == 16)
+            prep_x8_kernel<16><<<prep_grid, 256, 0, stream>>>(X + m0 * K, xscale, Mc, (int)K, planes, xs);
+        else
+            prep_x8_kernel<32><<<prep_grid, 256, 0, stream>>>(X + m0 * K, xscale, Mc, (int)K, planes, xs);
+        if (cudaGetLastError() != cudaSuccess) return W4A16_ERR_CUDA;
         DecodeArgs args;
-        args.Xp = X + m0 * K;  // read by the CUDA-core kernel; the tensor-core kernel reads the planes
-        if (plan.cc_tokens && xscale) {
-            uint16_t* Xs = reinterpret_cast<uint16_t*>(planes);
-            const int64_t n8 = (int64_t)Mc * K / 8;
-            int pgrid = (int)ceil_div(n8, 256);
-            if (pgrid > num_sms_current()) pgrid = num_sms_current();
-            cudaLaunchConfig_t pcfg = {};
-            pcfg.gridDim = dim3((unsigned)pgrid);
-            pcfg.blockDim = dim3(256);
-            pcfg.stream = stream;
-            cudaLaunchAttribute pattr[1];
-            pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            pattr[0].val.programmaticStreamSerializationAllowed = 1;
-            pcfg.attrs = pattr;
-            pcfg.numAttrs = 1;
-            if (cudaLaunchKernelEx(&pcfg, awq_prescale_kernel, X + m0 * K, xscale, n8, (int)K, Xs) != cudaSuccess)
-                return W4A16_ERR_CUDA;
-            args.Xp = Xs;
-        }
+        args.Xp = X + m0 * K;  // the tensor-core kernel reads the planes
         args.xs = xs;
         args.scales = scales;
         args.zeros = zeros;
@@ -1150,20 +1258,9 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
         args.units_base = plan.units_base;
         args.units_rem = plan.units_rem;
         args.max_slots = plan.max_slots;
-        CUtensorMap tsc, tze, tq1;
-        if (plan.cc_tokens && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze) ||
-                               !cached_tmap(kCcUnitGroups == 1 ? 0 : 1, qweight, N, K / 8, &tq1)))
-            return W4A16_ERR_CUDA;
-        if (plan.cc_tokens) args.G = plan.unit_groups;  // the one-token kernel walks units of two groups
-        const int st = plan.cc_tokens == 1   ? launch_cc(tq1, tsc, tze, args, plan.grid, stream)
-                       : plan.nt == 16       ? launch_tc<16>(tq, tx, args, plan.grid, stream)
-                                             : launch_tc<32>(tq, tx, args, plan.grid, stream);
+        const int st = plan.nt == 16 ? launch_tc<16>(tq, tx, args, plan.grid, stream)
+                                     : launch_tc<32>(tq, tx, args, plan.grid, stream);
         if (st != W4A16_OK) return st;
-        if (plan.cc_tokens) {
-            const int st2 = launch_decode_reduce(partial, args.Y, N, Mc, plan.unit_groups, plan.units_base,
-                                                 plan.units_rem, plan.max_slots, plan.row_tiles, stream);
-            if (st2 != W4A16_OK) return st2;
-        }
     }
     return W4A16_OK;
 }

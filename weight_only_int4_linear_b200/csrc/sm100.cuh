@@ -149,6 +149,9 @@ __device__ __forceinline__ float sum_slots(const float* p, int64_t stride, int n
     return acc;
 }
 
+// Release / acquire fence at GPU scope (cheaper than the sequentially consistent __threadfence()).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
