@@ -592,6 +592,9 @@ static_assert(kCcMetaGroups % kCcChunkMax == 0, "a chunk lies inside one metadat
 // (chunks of 2 or more units); the TMA thread issues a unit only after the unit kCcStages back has been
 // released.
 static_assert((kCcMetaSlots - 1) * 2 + 1 >= kCcStages, "metadata slot reuse");
+// MMA accumulators start at the bits of 1.5 2^23: a plane sum P then ends as the FP32 number 1.5 2^23 + P
+// (|P| < 2^22; here |P| < 2^22 even with the odd codes' factor 16: 128 codes x 240 x 128).
+constexpr int kCcPlaneBias = 0x4B400000;
 
 struct CcArgs {
     const uint16_t* X;  // [K] BF16: the activations (X' = bf16(x * xscale) for the AWQ entry)
@@ -844,7 +847,7 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
             const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
             const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) dd[rb][j] = 0;
+            for (int j = 0; j < 4; ++j) dd[rb][j] = kCcPlaneBias;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 mma_u8s8(dd[rb], w0[j] & 0x0F0F0F0Fu, w1[j] & 0x0F0F0F0Fu, w0[j] & 0xF0F0F0F0u, w1[j] & 0xF0F0F0F0u,
@@ -861,10 +864,13 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
         const int x0 = __shfl_xor_sync(0xFFFFFFFFu, even ? e[2] : e[0], 1);
         const int x1 = __shfl_xor_sync(0xFFFFFFFFu, e[3], 1);
         const int P0 = even ? e[0] : x0, P1 = even ? e[1] : x1, P2 = even ? x0 : e[2];
-        // sum q X = 65536 P2 + (256 P1 + P0): the bracket is exact in int32 (< 2^26); then
-        // s (sum q X - z sum X) and the power of two last, so that neither product leaves the FP32
-        // range unless the group's result itself does
-        const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+        // the plane sums are biased: read as FP32 each is 1.5 2^23 + P exactly (|P| < 2^22), so one
+        // subtraction converts it.  sum q X = 65536 P2 + (256 P1 + P0), the bracket rounded once by the inner
+        // FMA; then s (sum q X - z sum X) and the power of two last, so that neither product leaves the
+        // FP32 range unless the group's result itself does
+        const float F0 = __int_as_float(P0) - 12582912.f, F1 = __int_as_float(P1) - 12582912.f,
+                    F2 = __int_as_float(P2) - 12582912.f;
+        const float qx = fmaf(F2, 65536.f, fmaf(F1, 256.f, F0));
         y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
 
         if (d.w & kLast) {  // the chunk's sums leave through its slot (decode_cc_reduce_kernel adds them)

@@ -54,6 +54,12 @@ constexpr int kMetaBytes = kScBytes + kZeBytes;
 // (G % 8 == 0), so the block in between has 8 units, and at most kStages of them are in flight.
 static_assert(kStages <= kMetaGroups, "metadata slot reuse");
 
+// MMA accumulators start at the bits of 1.5 2^23 (0x4B400000): a plane sum P (|P| < 2^18: 128 codes of at
+// most 15 times digits of at most 128) then ends as the FP32 number 1.5 2^23 + P, exactly, and one
+// subtraction of 1.5 2^23 gives P as a float -- where an integer-to-float conversion would take a
+// quarter-rate instruction per plane.
+constexpr int kPlaneBias = 0x4B400000;
+
 template <int NT>
 struct MtCfg {
     static constexpr int kTiles = NT == 4 ? 2 : 3 * NT / 8;   // n8 tiles of the B operand
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mt_kernel(const __grid_con
 #pragma unroll
                 for (int u = 0; u < NTL; ++u) {
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) d[u][e] = 0;
+                    for (int e = 0; e < 4; ++e) d[u][e] = kPlaneBias;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) mma_u8s8(d[u], A[rb][j], bx[u][2 * j], bx[u][2 * j + 1]);
                 }
@@ -364,8 +370,11 @@ __global__ void __launch_bounds__(kThreads, 3) decode_mt_kernel(const __grid_con
                             P1 = d[1][2 * h + j];
                             P2 = d[2][2 * h + j];
                         }
-                        // 256 P1 + P0 exact in int32 (< 2^26); the power of two last
-                        const float qx = fmaf((float)P2, 65536.f, (float)(P1 * 256 + P0));
+                        // each plane sum is biased: its bits read as FP32 are 1.5 2^23 + P, so one exact
+                        // subtraction converts it; 256 P1 + P0 is rounded once, by the inner FMA
+                        const float F0 = __int_as_float(P0) - 12582912.f, F1 = __int_as_float(P1) - 12582912.f,
+                                    F2 = __int_as_float(P2) - 12582912.f;
+                        const float qx = fmaf(F2, 65536.f, fmaf(F1, 256.f, F0));
                         y[k][q0 + j] = fmaf(sv[k] * fmaf(-zv[k], xs[j], qx), xc[j], y[k][q0 + j]);
                     }
                 }
