@@ -517,7 +517,7 @@ def run_stack(torch, w4, stream, steps):
         raise RuntimeError(f"a kernel gave up a bounded wait (site {fault}) in the stack")
     return {"value": code_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "workload": "decode_stack_80x8192",
             "ms_per_step": ms, "steps": steps, "packed_code_bytes": code_bytes,
-            "launches_per_step": STACK_LAYERS * (4 + 2),
+            "launches_per_step": STACK_LAYERS * (sum(launches_per_call(c) for c in workloads.stack_layer(0)) + 2),
             "note": "aggregate packed-code GB/s over 80 layers x {qkv, o, gate+up, down} chained on one "
                     "stream with the renorm kernels between them (their time included)"}
 
