@@ -883,9 +883,10 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
 // Split-K sums of the one-token kernel: Y[n] = the sum of row n's chunk slots in slot order.  A
 // dependent grid: its CTAs become resident beside the GEMV's (256 threads of at most 32 registers fit next
 // to four GEMV CTAs) and wait for it to complete.  Per row tile, 128 x P threads: part p adds slots p,
-// p + P, ... of its row (at most 16 loads in flight per thread, so one L2 round trip serves tiles of up to
-// 16 P chunks), then part 0 adds the P part sums in order.
+// p + P, ... of its row (at most 32 loads in flight per thread, so one L2 round trip serves tiles of up to
+// 32 P chunks), then part 0 adds the P part sums in order.
 constexpr int kCcRedParts = 2;
+constexpr int kCcRedLoads = 32;
 __global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_kernel(const float* __restrict__ partial,
                                                                                      uint16_t* __restrict__ Y, int N,
                                                                                      int cpt, int row_tiles) {
@@ -896,15 +897,15 @@ __global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_ke
     for (int tile = blockIdx.x; tile < row_tiles; tile += gridDim.x) {
         const float* pb = partial + (int64_t)tile * cpt * kRowsPerCta + r;
         float acc = 0.f;
-        for (int k0 = p; k0 < cpt; k0 += 16 * kCcRedParts) {
-            float v[16];
+        for (int k0 = p; k0 < cpt; k0 += kCcRedLoads * kCcRedParts) {
+            float v[kCcRedLoads];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < kCcRedLoads; ++e) {
                 const int k = k0 + e * kCcRedParts;
                 v[e] = k < cpt ? __ldcg(pb + (int64_t)k * kRowsPerCta) : 0.f;
             }
 #pragma unroll
-            for (int e = 0; e < 16; ++e) acc += v[e];
+            for (int e = 0; e < kCcRedLoads; ++e) acc += v[e];
         }
         if (p > 0) s_part[p - 1][r] = acc;
         __syncthreads();
