@@ -223,8 +223,13 @@ W4A16_API int w4a16_linear_awq(const uint16_t* X, const float* inv_s, int64_t M,
 /*
  * The linear layer on host buffers: one call enqueues, on `stream`, the copy
  * of X from host to device, w4a16_linear(), and the copy of Y back to the
- * host (one cudaMemcpyAsync each way), so a caller that holds activations in
- * host memory pays a single library call per layer.
+ * host, so a caller that holds activations in host memory pays a single
+ * library call per layer.  For one token (M = 1, K a multiple of 1024) with
+ * host buffers mapped into the device's address space (cudaHostAlloc, or
+ * cudaHostRegister with cudaHostRegisterMapped) the two transfers are done
+ * by the library's kernels -- a copy kernel reads X_host, the split-K
+ * reduction also stores Y into Y_host -- so that consecutive calls keep
+ * overlapping on the stream; otherwise one cudaMemcpyAsync each way.
  *   X_host    host, bf16 bits [M][K]; page-locked (cudaHostAlloc or
  *             cudaHostRegister) for the copy to be asynchronous
  *   X_dev     device, bf16 bits [M][K], the staging buffer X is copied into

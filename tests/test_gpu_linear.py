@@ -245,6 +245,37 @@ def test_zero_points_far_outside_the_code_range(cuda_lib, M, path):
     assert_close(bf16_dev_to_f64(Y), oracle.linear(X, qw, sc, z), f"M={M}")
 
 
+def test_host_buffer_entry_chained_through_host(cuda_lib):
+    """Two one-token layers through w4a16_linear_host, the second reading the first's host output: the
+    transfers are kernels of the launch chain (mapped host buffers), so the second call's copy must wait for
+    the first call's stores into host memory.  Same bits as the device-buffer chain."""
+    K1, N1, N2 = 2048, 3072, 1000  # layer 2: K = 3072
+    W1 = synth.weights_f32(31, synth.TAG_W, N1, K1)
+    W2 = synth.weights_f32(32, synth.TAG_W, N2, N1)
+    p1, p2 = packed_from_host(W1), packed_from_host(W2)
+    xb = synth.activations_bf16(33, 1, K1)
+    Y1_ref = run_linear(xb, p1)
+    Y2_ref = run_linear(Y1_ref.view(torch.int16).cpu().numpy().view(np.uint16), p2)
+    X_host = torch.from_numpy(xb.view(np.int16)).pin_memory()
+    H_host = torch.full((1, N1), -1, dtype=torch.int16).pin_memory()
+    Y_host = torch.full((1, N2), -1, dtype=torch.int16).pin_memory()
+    X1 = torch.empty((1, K1), dtype=torch.bfloat16, device="cuda")
+    Y1 = torch.empty((1, N1), dtype=torch.bfloat16, device="cuda")
+    X2 = torch.empty((1, N1), dtype=torch.bfloat16, device="cuda")
+    Y2 = torch.empty((1, N2), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(max(w4.workspace_bytes(1, N1, K1), w4.workspace_bytes(1, N2, N1)), dtype=torch.uint8,
+                     device="cuda")
+    for _ in range(3):
+        H_host.fill_(-1)
+        Y_host.fill_(-1)
+        w4.linear_host(X_host, X1, p1.qweight, p1.scales, p1.zeros, Y1, H_host, ws)
+        w4.linear_host(H_host, X2, p2.qweight, p2.scales, p2.zeros, Y2, Y_host, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(H_host, Y1_ref.view(torch.int16).cpu())
+        assert torch.equal(Y_host, Y2_ref.view(torch.int16).cpu())
+        assert torch.equal(Y2.view(torch.int16), Y2_ref.view(torch.int16))
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 640, 1024), (2, 256, 2048), (96, 384, 1152)])
 def test_host_buffer_entry_matches_device_entry(cuda_lib, M, N, K):
     """w4a16_linear_host (copies in and out on the stream) gives the same bits as w4a16_linear."""

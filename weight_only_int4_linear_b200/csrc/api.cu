@@ -174,6 +174,27 @@ int w4a16_linear_host(const uint16_t* X_host, uint16_t* X_dev, int64_t M, int64_
     int st = check_shape(M, N, K);
     if (st != W4A16_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
+    // One token on the decode path: both transfers as part of the kernels' launch chain (the host buffers
+    // accessed through their mapped device addresses), so that consecutive calls keep overlapping
+    if (M == 1) {
+        void *xh = nullptr, *yh = nullptr;
+        const bool mapped = cudaHostGetDevicePointer(&xh, const_cast<uint16_t*>(X_host), 0) == cudaSuccess &&
+                            cudaHostGetDevicePointer(&yh, Y_host, 0) == cudaSuccess && aligned16(xh);
+        if (!mapped) cudaGetLastError();  // not mapped: the copy-engine transfers below
+        if ((st = check_device()) != W4A16_OK) return st;
+        const DecodePlan plan = plan_decode(M, N, K, num_sms_current());
+        if (mapped && plan.cc_tokens) {
+            if (!qweight || !scales || !zeros) return W4A16_ERR_ARG;
+            if (!aligned16(X_dev) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) ||
+                !aligned16(Y_dev))
+                return W4A16_ERR_ALIGN;
+            const size_t need = plan.workspace_bytes();
+            if (need > 0 && (!workspace || workspace_bytes < need)) return W4A16_ERR_WORKSPACE;
+            if (need > 0 && !aligned16(workspace)) return W4A16_ERR_ALIGN;
+            return launch_decode(X_dev, nullptr, M, K, qweight, scales, zeros, N, Y_dev, workspace, plan, s,
+                                 static_cast<const uint16_t*>(xh), static_cast<uint16_t*>(yh));
+        }
+    }
     if (cudaMemcpyAsync(X_dev, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
         return W4A16_ERR_CUDA;
     st = w4a16_linear_path(X_dev, M, K, qweight, scales, zeros, N, Y_dev, workspace, workspace_bytes, W4A16_PATH_AUTO,

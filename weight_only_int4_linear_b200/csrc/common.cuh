@@ -161,9 +161,12 @@ struct DecodePlan {
 DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms);
 // xscale (nullable, [K] FP32): the AWQ activation transform, x -> bf16(x * xscale[k]), applied
 // where each path prepares X.
+// X_host, Y_host (nullable, one-token plans only): device addresses of mapped page-locked host buffers; X is
+// then first copied from X_host into X by a kernel of the launch chain, and Y is also stored into Y_host.
 int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
-                  const DecodePlan& plan, cudaStream_t stream);
+                  const DecodePlan& plan, cudaStream_t stream, const uint16_t* X_host = nullptr,
+                  uint16_t* Y_host = nullptr);
 int num_sms_current();
 
 // The BF16 tensor-core GEMV (gemv_bf.cu) for quantisation groups of `group` (32, 64, 128) weights, K / group

@@ -880,6 +880,18 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
     }
 }
 
+// Copy of X from mapped host memory into the device buffer, as a kernel in the programmatic-launch chain (a
+// copy-engine transfer would end the chain: the GEMV could no longer start its weight loads early).  It
+// waits for the preceding kernel before reading (X may be that kernel's host-mapped output) and before
+// writing (that kernel may still read the device buffer).
+__global__ void __launch_bounds__(256) h2d_copy_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst,
+                                                       int64_t n16) {
+    pdl_launch_dependents();
+    pdl_wait_primary();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = src[i];
+}
+
 // Split-K sums of the one-token kernel: Y[n] = the sum of row n's chunk slots in slot order.  A
 // dependent grid: its CTAs become resident beside the GEMV's (256 threads of at most 32 registers fit next
 // to four GEMV CTAs) and wait for it to complete.  Per row tile, 128 x P threads: part p adds slots p,
@@ -889,7 +901,8 @@ constexpr int kCcRedParts = 2;
 constexpr int kCcRedLoads = 32;
 __global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_kernel(const float* __restrict__ partial,
                                                                                      uint16_t* __restrict__ Y, int N,
-                                                                                     int cpt, int row_tiles) {
+                                                                                     int cpt, int row_tiles,
+                                                                                     uint16_t* __restrict__ Yh) {
     __shared__ float s_part[kCcRedParts - 1][kRowsPerCta];
     pdl_launch_dependents();
     pdl_wait_primary();
@@ -913,7 +926,11 @@ __global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_ke
 #pragma unroll
             for (int q = 0; q < kCcRedParts - 1; ++q) acc += s_part[q][r];
             const int n = tile * kRowsPerCta + r;
-            if (n < N) Y[n] = float_to_bf16_bits(acc);
+            if (n < N) {
+                const uint16_t yb = float_to_bf16_bits(acc);
+                Y[n] = yb;
+                if (Yh) Yh[n] = yb;  // the host copy, stored straight into mapped host memory
+            }
         }
         __syncthreads();
     }
@@ -1158,7 +1175,7 @@ namespace {
 // slots, so the call is one launch (two with the prescale).
 int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint32_t* qweight, const uint16_t* scales,
                    const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace, const DecodePlan& plan,
-                   cudaStream_t stream) {
+                   cudaStream_t stream, const uint16_t* X_host, uint16_t* Y_host) {
     const int G = (int)(K / kGroup);
     CUtensorMap tq, tsc, tze;
     if (!cached_tmap(0, qweight, N, K / 8, &tq) || !cached_tmap(2, scales, N, G, &tsc) ||
@@ -1167,6 +1184,22 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
     int* fault = fault_word();
     if (!fault) return W4A16_ERR_CUDA;
     char* ws = reinterpret_cast<char*>(workspace);
+    if (X_host) {  // X arrives from host memory by a kernel of the chain
+        const int64_t n16 = K * 2 / 16;
+        int grid = (int)ceil_div(n16, 256 * 4);
+        cudaLaunchConfig_t ccfg = {};
+        ccfg.gridDim = dim3((unsigned)(grid < 1 ? 1 : grid));
+        ccfg.blockDim = dim3(256);
+        ccfg.stream = stream;
+        cudaLaunchAttribute cattr[1];
+        cattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        cattr[0].val.programmaticStreamSerializationAllowed = 1;
+        ccfg.attrs = cattr;
+        ccfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&ccfg, h2d_copy_kernel, reinterpret_cast<const uint4*>(X_host),
+                               reinterpret_cast<uint4*>(const_cast<uint16_t*>(X)), n16) != cudaSuccess)
+            return W4A16_ERR_CUDA;
+    }
     CcArgs args;
     args.X = X;
     if (xscale) {
@@ -1210,7 +1243,7 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, (const float*)args.partial, Y, (int)N, plan.cc_cpt,
-                              plan.row_tiles) == cudaSuccess
+                              plan.row_tiles, Y_host) == cudaSuccess
                ? W4A16_OK
                : W4A16_ERR_CUDA;
 }
@@ -1219,14 +1252,16 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
 
 int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,
-                  const DecodePlan& plan, cudaStream_t stream) {
+                  const DecodePlan& plan, cudaStream_t stream, const uint16_t* X_host, uint16_t* Y_host) {
     if (plan.mt)
         return launch_decode_mt(X, xscale, M, K, qweight, scales, zeros, N, Y,
                                 reinterpret_cast<char*>(workspace) + plan.ws_counter_bytes, stream);
     if (plan.bf)
         return launch_decode_bf(X, xscale, M, K, kGroup, qweight, scales, zeros, N, Y,
                                 reinterpret_cast<char*>(workspace) + plan.ws_counter_bytes, stream);
-    if (plan.cc_tokens) return launch_cc_path(X, xscale, K, qweight, scales, zeros, N, Y, workspace, plan, stream);
+    if (plan.cc_tokens)
+        return launch_cc_path(X, xscale, K, qweight, scales, zeros, N, Y, workspace, plan, stream, X_host, Y_host);
+    if (X_host || Y_host) return W4A16_ERR_ARG;  // host-mapped transfers are the one-token path's
     CUtensorMap tq;
     if (!cached_tmap(0, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
     int* fault = fault_word();
