@@ -199,9 +199,10 @@ def test_one_workspace_shared_by_shapes_and_paths(cuda_lib):
     assert w4.device_fault() == 0
 
 
-def test_renorm_rows(cuda_lib):
+@pytest.mark.parametrize("N", [28672, 1001])  # the wide kernel (N % 8 == 0, values in registers) and the general one
+def test_renorm_rows(cuda_lib, N):
     rng = np.random.default_rng(4)
-    y = torch.from_numpy(rng.standard_normal((3, 28672)).astype(np.float32) * 5).to(torch.bfloat16).cuda()
+    y = torch.from_numpy(rng.standard_normal((3, N)).astype(np.float32) * 5).to(torch.bfloat16).cuda()
     y[2].zero_()
     out = torch.empty_like(y)
     w4.renorm_rows(y, out)

@@ -241,6 +241,62 @@ __global__ void __launch_bounds__(256) renorm_kernel(const uint16_t* __restrict_
     }
 }
 
+// The same for rows of N <= kRenormMaxN values, N a multiple of 8 and 16-byte aligned rows: 1024 threads per
+// row, each holding up to four 8-value chunks in registers (one read of the row), as a kernel of the
+// programmatic-launch chain: the next kernel may start its own loads while this one waits for y.
+constexpr int kRenormThreads = 1024, kRenormChunks = 4;
+constexpr int64_t kRenormMaxN = (int64_t)kRenormThreads * kRenormChunks * 8;
+__global__ void __launch_bounds__(kRenormThreads) renorm_wide_kernel(const uint16_t* __restrict__ y, int64_t N,
+                                                                     uint16_t* __restrict__ out) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // y comes from the preceding kernel
+    const uint4* row = reinterpret_cast<const uint4*>(y + (int64_t)blockIdx.x * N);
+    uint4* orow = reinterpret_cast<uint4*>(out + (int64_t)blockIdx.x * N);
+    const int n8 = (int)(N / 8);
+    uint4 v[kRenormChunks];
+    float ss = 0.f;
+#pragma unroll
+    for (int c = 0; c < kRenormChunks; ++c) {
+        const int j = threadIdx.x + c * kRenormThreads;
+        v[c] = j < n8 ? row[j] : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+            ss = fmaf(lo, lo, ss);
+            ss = fmaf(hi, hi, ss);
+        }
+    }
+    __shared__ float red[32];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float t = red[threadIdx.x];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+        if (threadIdx.x == 0) red[0] = t;
+    }
+    __syncthreads();
+    const float rms = sqrtf(red[0] / (float)N);
+#pragma unroll
+    for (int c = 0; c < kRenormChunks; ++c) {
+        const int j = threadIdx.x + c * kRenormThreads;
+        if (j < n8) {
+            const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+                o4[e] = (uint32_t)float_to_bf16_bits(rms > 0.f ? lo / rms : 0.f) |
+                        ((uint32_t)float_to_bf16_bits(rms > 0.f ? hi / rms : 0.f) << 16);
+            }
+            orow[j] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+    }
+}
+
 static int grid_for(int64_t items, int threads) {
     int64_t blocks = ceil_div(items, threads);
     const int64_t cap = (int64_t)num_sms_current() * 32;
@@ -300,8 +356,21 @@ int launch_dequant(const uint32_t* qweight, const uint16_t* scales, const int32_
 }
 
 int launch_renorm(const uint16_t* y, int64_t M, int64_t N, uint16_t* out, cudaStream_t stream) {
-    renorm_kernel<<<(unsigned)M, 256, 0, stream>>>(y, N, out);
-    return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    const bool wide = N % 8 == 0 && N <= kRenormMaxN && ((uintptr_t)y & 15) == 0 && ((uintptr_t)out & 15) == 0;
+    if (!wide) {
+        renorm_kernel<<<(unsigned)M, 256, 0, stream>>>(y, N, out);
+        return cudaGetLastError() == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)M);
+    cfg.blockDim = dim3(kRenormThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, renorm_wide_kernel, y, N, out) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
 }  // namespace w4a16
