@@ -85,3 +85,35 @@ def test_interleaved_shapes_share_the_counter(cuda_lib):
     X = synth.activations_bf16(21, 1, K)
     ref = _oracle_rows(N, K, 11, X, np.arange(N))
     assert_close(bf16_dev_to_f64(first[0]), ref, "interleaved 1000 x 2048")
+
+
+@pytest.mark.parametrize("group", [64, 32])
+def test_small_group_kernel_chunks_share_the_counter(cuda_lib, group):
+    """The one-token kernel for groups of 64 and 32 deals its chunks from the same counter: repeated calls,
+    interleaved with group-128 calls on one workspace, give the same bits and leave the counters at zero."""
+    N, K = 3000, 4096
+    W = dev_weights(41, synth.TAG_W, N, K)
+    pw = w4.PackedWeight(N, K, group=group)
+    pw.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    w4.quantize_pack_g(W, group, pw.qweight, pw.scales, pw.zeros, pw.status)
+    p128 = _packed(5120, 5120, 42)
+    X = bits_to_dev_bf16(synth.activations_bf16(43, 1, K))
+    X128 = bits_to_dev_bf16(synth.activations_bf16(44, 1, 5120))
+    nbytes = max(w4.workspace_bytes_g(1, N, K, group), w4.workspace_bytes(1, 5120, 5120))
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        Y = torch.full((1, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        w4.linear_g(X, group, pw.qweight, pw.scales, pw.zeros, Y, ws)
+        Y128 = torch.empty((1, 5120), dtype=torch.bfloat16, device="cuda")
+        w4.linear(X128, p128.qweight, p128.scales, p128.zeros, Y128, ws)
+        outs.append(Y)
+    torch.cuda.synchronize()
+    assert int(pw.status.item()) == 0
+    assert not ws[:COUNTER_BYTES].any().item()
+    for Y in outs[1:]:
+        assert torch.equal(Y.view(torch.int16), outs[0].view(torch.int16))
+    Wh = synth.weights_f32(41, synth.TAG_W, N, K)
+    st, qw, sc, z = oracle.quantize_pack_g(Wh, group)
+    assert st == oracle.OK
+    assert_close(bf16_dev_to_f64(outs[0]), oracle.linear_g(synth.activations_bf16(43, 1, K), qw, sc, z), f"G={group}")

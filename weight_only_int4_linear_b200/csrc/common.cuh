@@ -176,6 +176,10 @@ int launch_decode_bf(const uint16_t* X, const float* xscale, int64_t M, int64_t 
                      const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* scratch,
                      cudaStream_t stream);
 
+// Chunk sums of the one-token GEMVs (gemv.cu, gemv_sub.cu): partial [row_tiles][cpt][128] -> Y [N] (and Y_host
+// when given: a mapped host buffer), each row's slots added in slot order; a dependent launch.
+int launch_cc_reduce(const float* partial, uint16_t* Y, int64_t N, int cpt, int row_tiles, cudaStream_t stream,
+                     uint16_t* Y_host = nullptr);
 // Split-K reduction of the decode GEMVs (gemv.cu): a dependent grid of one CTA per 128-row tile that
 // adds the partial-sum slots of every tile the GEMV's CTAs shared, in slot order, into Y.
 int launch_decode_reduce(const float* partial, uint16_t* Y, int64_t N, int M, int G, int units_base, int units_rem,

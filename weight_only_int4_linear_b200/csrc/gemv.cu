@@ -1230,11 +1230,18 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
     args.cpt = plan.cc_cpt;
     args.chunks = plan.cc_chunks;
     args.row_tiles = plan.row_tiles;
-    int st = launch_cc(tq, tsc, tze, args, plan.grid, stream);
+    const int st = launch_cc(tq, tsc, tze, args, plan.grid, stream);
     if (st != W4A16_OK) return st;
+    return launch_cc_reduce(args.partial, Y, N, plan.cc_cpt, plan.row_tiles, stream, Y_host);
+}
+
+}  // namespace
+
+int launch_cc_reduce(const float* partial, uint16_t* Y, int64_t N, int cpt, int row_tiles, cudaStream_t stream,
+                     uint16_t* Y_host) {
     const int sms = num_sms_current();
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(plan.row_tiles < sms ? plan.row_tiles : sms));
+    cfg.gridDim = dim3((unsigned)(row_tiles < sms ? row_tiles : sms));
     cfg.blockDim = dim3(kRowsPerCta * kCcRedParts);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1242,13 +1249,10 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, (const float*)args.partial, Y, (int)N, plan.cc_cpt,
-                              plan.row_tiles, Y_host) == cudaSuccess
+    return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, partial, Y, (int)N, cpt, row_tiles, Y_host) == cudaSuccess
                ? W4A16_OK
                : W4A16_ERR_CUDA;
 }
-
-}  // namespace
 
 int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
                   const uint16_t* scales, const int32_t* zeros, int64_t N, uint16_t* Y, void* workspace,

@@ -23,19 +23,16 @@ constexpr int kCcThreads = (kCcWarps + 2) * 32;
 constexpr int kCcStages = 4;
 constexpr int kCcCodeBytes = kRowsPerCta * kWordsPerGroup * 4;  // 8 KB, 64-byte swizzle
 constexpr int kCcXOff = kCcCodeBytes;                // X digit rows after the codes
-constexpr int kXAhead = 6;                           // X warp: loads in flight, in units
+constexpr int kChunkMax = 4;                         // units per chunk (a metadata block holds 4 units)
 
-struct DecodeArgs {
+struct SubArgs {
     const uint16_t* Xp;  // [K] BF16, this launch's token
-    const uint16_t* scales;
-    const int32_t* zeros;
-    uint16_t* Y;         // [N]
-    float* partial;      // [row_tiles][max_slots][128]
-    int* counters;       // [row_tiles]
+    float* partial;      // [row_tiles][cpt][128]: one slot of sums per chunk
+    int* counters;       // counters[0]: the chunk counter
     int* fault;
-    int M, N, K, G;
-    int units_base, units_rem;
-    int max_slots;
+    int N, G;            // G = 128-K units per row (a multiple of 4)
+    int U;               // units per chunk: 2 or 4 (4 for groups of 32)
+    int cpt, chunks;     // chunks per row tile, chunks in all
 };
 
 // This lane's four BF16 values of 128-K unit g: lane 2w + h holds values 4h..4h+3 of word w.
@@ -109,12 +106,14 @@ struct SubCfg {
     static constexpr int kScBytes = kRowsPerCta * kMetaGroups * 2;
     static constexpr int kMetaBytes = kRowsPerCta * kMetaGroups * 6;
     static constexpr int kMetaOff = kCcStages * kStageBytes;
-    static constexpr size_t kSmem = (size_t)kMetaOff + 2 * kMetaBytes + 512;
+    // chunks of 2 (GS = 64 only) or 4 units; a chunk's block overwrites the slot of the chunk kMetaSlots
+    // chunks earlier, whose last unit is then (kMetaSlots - 1) Umin + 1 units back
+    static constexpr int kUnitsMin = GS == 64 ? 2 : 4;
+    static constexpr int kMetaSlots = GS == 64 ? 3 : 2;
+    static constexpr size_t kSmem = (size_t)kMetaOff + kMetaSlots * kMetaBytes + 512;
     static constexpr int kMinBlocks = GS == 64 ? 4 : 3;
+    static_assert((kMetaSlots - 1) * kUnitsMin + 1 >= kCcStages, "metadata slot reuse");
 };
-// a metadata slot is rewritten two blocks (8 units) later, after every unit of the older block
-// has been released (at most kCcStages units are in flight)
-static_assert(kCcStages <= 4, "metadata slot reuse of the small-group kernel");
 
 // One warp writes the digits of one 128-K unit for groups of GS (layout above).  Within a row,
 // word w's eight digit bytes are stored in the order the codes come out of a packed word
@@ -167,27 +166,27 @@ __device__ __forceinline__ void prep_unit_x8_sub(const uint2 v, unsigned char* d
 template <int GS>
 __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub_kernel(
     const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tsc,
-    const __grid_constant__ CUtensorMap tze, const DecodeArgs a) {
+    const __grid_constant__ CUtensorMap tze, const SubArgs a) {
     using C = SubCfg<GS>;
     constexpr int kSub = C::kSub;
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages];
-    __shared__ int s_last;
+    __shared__ __align__(8) uint64_t full[kCcStages], empty[kCcStages], dready[kCcStages];
+    __shared__ int4 s_desc[kCcStages];  // (row tile, unit, chunk slot, flags) of the unit in each stage
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((512u - (raw & 511u)) & 511u);
     unsigned char* meta = ring + C::kMetaOff;
+    constexpr int kFirst = 1, kLast = 2, kEnd = 4, kSlotShift = 4;
 
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
-    const int64_t u_first = (int64_t)b * a.units_base + min(b, a.units_rem);
-    const int nunits = a.units_base + (b < a.units_rem ? 1 : 0);
-    const int G = a.G, N = a.N;  // G = 128-K units per row
+    int* const next_chunk = a.counters;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCcStages; ++s) {
             mbar_init(&full[s], 2);
             mbar_init(&empty[s], kCcWarps);
+            mbar_init(&dready[s], 1);
         }
         fence_mbar_init();
     }
@@ -198,117 +197,97 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
             prefetch_tmap(&tq);
             prefetch_tmap(&tsc);
             prefetch_tmap(&tze);
-            UnitCursor cur(u_first, G);
-            int mb = -1, issued = 0;
-            for (int i = 0; i < nunits; ++i, cur.next(G)) {
-                const int s = i % kCcStages;
-                if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 111)) break;
-                const bool new_block = i == 0 || (cur.g & 3) == 0;
-                if (new_block) ++mb;
-                unsigned char* st = ring + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (new_block ? C::kMetaBytes : 0));
-                tma_load_2d(st, &tq, cur.g * kWordsPerGroup, cur.tile * kRowsPerCta, &full[s]);
-                if (new_block) {
-                    unsigned char* ms = meta + (mb & 1) * C::kMetaBytes;
-                    const int g0 = (cur.g & ~3) * kSub;
-                    tma_load_2d(ms, &tsc, g0, cur.tile * kRowsPerCta, &full[s]);
-                    tma_load_2d(ms + C::kScBytes, &tze, g0, cur.tile * kRowsPerCta, &full[s]);
+            int i = 0, nchunks = 0;
+            bool ok = true;
+            // the units of chunk c (a chunk lies inside one 4-unit metadata block, loaded with its first unit)
+            auto issue_chunk = [&](int c) {
+                const int tile = c / a.cpt, k = c - tile * a.cpt;
+                const int mslot = nchunks++ % C::kMetaSlots;
+                for (int u = 0; u < a.U; ++u, ++i) {
+                    const int s = i % kCcStages;
+                    if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 111)) {
+                        ok = false;
+                        return;
+                    }
+                    const int g = k * a.U + u;
+                    s_desc[s] = make_int4(tile, g, k,
+                                          (u == 0 ? kFirst : 0) | (u + 1 == a.U ? kLast : 0) | (mslot << kSlotShift));
+                    mbar_arrive(&dready[s]);
+                    unsigned char* st = ring + s * C::kStageBytes;
+                    mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (u == 0 ? C::kMetaBytes : 0));
+                    tma_load_2d(st, &tq, g * kWordsPerGroup, tile * kRowsPerCta, &full[s]);
+                    if (u == 0) {
+                        unsigned char* ms = meta + mslot * C::kMetaBytes;
+                        const int g0 = (g & ~3) * kSub;
+                        tma_load_2d(ms, &tsc, g0, tile * kRowsPerCta, &full[s]);
+                        tma_load_2d(ms + C::kScBytes, &tze, g0, tile * kRowsPerCta, &full[s]);
+                    }
                 }
-                ++issued;
+            };
+            issue_chunk(b);  // gridDim.x <= chunks; the weights need nothing from the preceding kernel
+            pdl_wait_primary();  // the chunk counter is this launch's once the preceding one has completed
+            // a launch draws exactly `chunks` values: the CTA drawing the last one resets the counter
+            int v = ok ? atomicAdd(next_chunk, 1) : 0;
+            while (ok && (int)gridDim.x + v < a.chunks) {
+                const int c = (int)gridDim.x + v;
+                v = atomicAdd(next_chunk, 1);  // in flight while chunk c is issued
+                issue_chunk(c);
             }
-            for (int i = max(0, issued - kCcStages); i < issued; ++i)
-                mbar_wait(&full[i % kCcStages], (i / kCcStages) & 1, a.fault, 112);
+            if (ok && v == a.chunks - 1) *next_chunk = 0;
+            for (int j = max(0, i - kCcStages); j < i; ++j)
+                mbar_wait(&full[j % kCcStages], (j / kCcStages) & 1, a.fault, 112);
+            if (ok) {  // the end of the unit stream, in the stage after the last unit
+                const int s = i % kCcStages;
+                if (i < kCcStages || mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 111)) {
+                    s_desc[s] = make_int4(-1, 0, 0, kEnd);
+                    mbar_arrive(&dready[s]);
+                    mbar_arrive(&full[s]);
+                }
+            }
         }
         return;
     }
 
     if (warp == kCcXWarp) {  // ------------------------------------------ X warp
         pdl_wait_primary();
-        const uint16_t* X = a.Xp;
-        uint2 q[kXAhead];
-        UnitCursor cl(u_first, G);
-#pragma unroll
-        for (int j = 0; j < kXAhead; ++j, cl.next(G)) q[j] = j < nunits ? load_group_x(X, cl.g, lane) : make_uint2(0, 0);
-        for (int i = 0; i < nunits; ++i, cl.next(G)) {
-            const uint2 v = q[0];
-#pragma unroll
-            for (int j = 0; j + 1 < kXAhead; ++j) q[j] = q[j + 1];
-            q[kXAhead - 1] = i + kXAhead < nunits ? load_group_x(X, cl.g, lane) : make_uint2(0, 0);
+        uint2 xq[kChunkMax];  // the chunk's units, loaded together at its first unit
+        for (int i = 0;; ++i) {
             const int s = i % kCcStages;
-            if (i >= kCcStages && !warp_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 114)) break;
-            prep_unit_x8_sub<GS>(v, ring + s * C::kStageBytes + kCcXOff, lane);
+            if (!warp_wait(&dready[s], (i / kCcStages) & 1, a.fault, 114)) break;
+            const int4 d = s_desc[s];
+            if (!(d.w & kEnd)) {
+                if (d.w & kFirst) {
+#pragma unroll
+                    for (int j = 0; j < kChunkMax; ++j)
+                        if (j < a.U) xq[j] = load_group_x(a.Xp, d.y + j, lane);
+                }
+                const int u = d.y & (a.U - 1);
+                uint2 v = xq[0];
+#pragma unroll
+                for (int j = 1; j < kChunkMax; ++j)
+                    if (u == j) v = xq[j];
+                prep_unit_x8_sub<GS>(v, ring + s * C::kStageBytes + kCcXOff, lane);  // the stage is free
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&full[s]);
+            if (d.w & kEnd) break;
         }
         return;
     }
 
     // ---------------------------------------------------- compute warps 0-3
-    const int t = threadIdx.x;
     const int g8 = lane >> 2, tig = lane & 3;
     const bool folder = tig < kSub;               // lane tig folds sub-group tig
     const int jsub = folder ? tig : 0;
     auto rrow = [&](int k) { return 32 * warp + 16 * (k >> 1) + g8 + 8 * (k & 1); };
     float y[4] = {0.f, 0.f, 0.f, 0.f};
-    int cur_tile = -1;
-    bool aborted = false;
 
-    auto flush = [&](int tile) {
-        float tot[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {  // the quad's sub-group sums, in a fixed order
-            tot[k] = y[k] + __shfl_xor_sync(0xFFFFFFFFu, y[k], 1);
-            if constexpr (kSub == 4) tot[k] += __shfl_xor_sync(0xFFFFFFFFu, tot[k], 2);
-        }
-        const bool owner = tig == 0;
-        const int first = cta_of_unit((int64_t)tile * G, a.units_base, a.units_rem);
-        const int last = cta_of_unit((int64_t)tile * G + G - 1, a.units_base, a.units_rem);
-        if (first == last) {
-            if (owner) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int n = tile * kRowsPerCta + rrow(k);
-                    if (n < N) a.Y[n] = float_to_bf16_bits(tot[k]);
-                }
-            }
-        } else {
-            const int slot = b - first, nseg = last - first + 1;
-            float* part = a.partial + ((int64_t)tile * a.max_slots + slot) * kRowsPerCta;
-            if (owner) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) part[rrow(k)] = tot[k];
-            }
-            named_barrier_sync(1, kCcWarps * 32);
-            if (t == 0) s_last = (arrive_acq_rel_gpu(&a.counters[tile]) == nseg - 1);
-            named_barrier_sync(1, kCcWarps * 32);
-            if (s_last) {
-                const int rows = min(kRowsPerCta, N - tile * kRowsPerCta);
-                const float* pb = a.partial + (int64_t)tile * a.max_slots * kRowsPerCta;
-                for (int rl = t; rl < rows; rl += kCcWarps * 32)
-                    a.Y[tile * kRowsPerCta + rl] = float_to_bf16_bits(sum_slots(pb + rl, kRowsPerCta, nseg));
-                if (t == 0) a.counters[tile] = 0;
-            }
-            named_barrier_sync(1, kCcWarps * 32);
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) y[k] = 0.f;
-    };
-
-    UnitCursor uc(u_first, G);
-    int mb = -1;
-    for (int i = 0; i < nunits; ++i, uc.next(G)) {
-        const int tile = uc.tile, g = uc.g;
-        if (i == 0 || (g & 3) == 0) ++mb;
-        if (tile != cur_tile) {
-            if (cur_tile >= 0) flush(cur_tile);
-            cur_tile = tile;
-        }
-        if (aborted) continue;
+    for (int i = 0;; ++i) {
         const int s = i % kCcStages;
-        if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 113)) {
-            aborted = true;
-            continue;
-        }
+        if (!warp_wait(&full[s], (i / kCcStages) & 1, a.fault, 113)) break;
+        const int4 d = s_desc[s];
+        if (d.w & kEnd) break;
+        const int g = d.y;
         const unsigned char* st = ring + s * C::kStageBytes;
         uint4 cw[4];
 #pragma unroll
@@ -333,7 +312,7 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
         }
         const float* ext = reinterpret_cast<const float*>(st + kCcXOff + C::kExt);
         const float xscale = ext[0], xsum = ext[1 + jsub];
-        const unsigned char* ms = meta + (mb & 1) * C::kMetaBytes;
+        const unsigned char* ms = meta + ((d.w >> kSlotShift) & 3) * C::kMetaBytes;
         const int gi = (g & 3) * kSub + jsub;  // this lane's group inside the metadata block
         float sv[4], zv[4];
 #pragma unroll
@@ -349,12 +328,12 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
         for (int rb = 0; rb < 2; ++rb) {
             const uint32_t w0[4] = {cw[2 * rb].x, cw[2 * rb].y, cw[2 * rb].z, cw[2 * rb].w};
             const uint32_t w1[4] = {cw[2 * rb + 1].x, cw[2 * rb + 1].y, cw[2 * rb + 1].z, cw[2 * rb + 1].w};
-            int d[4] = {0, 0, 0, 0}, e[4] = {0, 0, 0, 0};
+            int dd[4] = {0, 0, 0, 0}, e[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint32_t a0 = w0[j] & 0x0F0F0F0Fu, a1 = w1[j] & 0x0F0F0F0Fu;
                 const uint32_t a2 = (w0[j] >> 4) & 0x0F0F0F0Fu, a3 = (w1[j] >> 4) & 0x0F0F0F0Fu;
-                mma_u8s8(d, a0, a1, a2, a3, bx[2 * j], bx[2 * j + 1]);
+                mma_u8s8(dd, a0, a1, a2, a3, bx[2 * j], bx[2 * j + 1]);
                 if constexpr (kSub == 4) mma_u8s8(e, a0, a1, a2, a3, bz[2 * j], bz[2 * j + 1]);
             }
             // lane tig holds D columns 2 tig, 2 tig + 1 of rows g8 (d0, d1) and g8 + 8 (d2, d3); folder j
@@ -367,8 +346,8 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
                     const bool second = kSub == 4 && p == 2;
                     const int col = (p * kSub + jsub) & 7;
                     const int src = (lane & ~3) | (col >> 1);
-                    const int va = __shfl_sync(0xFFFFFFFFu, second ? e[2 * hh] : d[2 * hh], src);
-                    const int vb = __shfl_sync(0xFFFFFFFFu, second ? e[2 * hh + 1] : d[2 * hh + 1], src);
+                    const int va = __shfl_sync(0xFFFFFFFFu, second ? e[2 * hh] : dd[2 * hh], src);
+                    const int vb = __shfl_sync(0xFFFFFFFFu, second ? e[2 * hh + 1] : dd[2 * hh + 1], src);
                     P[p] = (col & 1) ? vb : va;
                 }
                 const float qx = fmaf((float)P[2], 65536.f, (float)(P[1] * 256 + P[0]));
@@ -376,8 +355,17 @@ __global__ void __launch_bounds__(kCcThreads, SubCfg<GS>::kMinBlocks) decode_sub
                 if (folder) y[k] = fmaf(sv[k] * fmaf(-zv[k], xsum, qx), xscale, y[k]);  // power of two last
             }
         }
+        if (d.w & kLast) {  // the chunk's row sums (the quad's sub-groups, in a fixed order) into its slot
+            float* part = a.partial + ((int64_t)d.x * a.cpt + d.z) * kRowsPerCta;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float tot = y[k] + __shfl_xor_sync(0xFFFFFFFFu, y[k], 1);
+                if constexpr (kSub == 4) tot += __shfl_xor_sync(0xFFFFFFFFu, tot, 2);
+                if (tig == 0) part[rrow(k)] = tot;
+                y[k] = 0.f;
+            }
+        }
     }
-    if (cur_tile >= 0) flush(cur_tile);
 }
 
 template <int GS>
@@ -399,31 +387,30 @@ int occupancy_sub() {
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 
-// Unit deal and workspace of the small-group kernel (one token per launch).
+// Chunk deal and workspace of the small-group kernel (one token per launch).
 DecodePlan plan_decode_sub(int64_t N, int64_t K, int group, int num_sms) {
     DecodePlan p{};
-    const int64_t G = K / kGroup;
+    const int64_t G = K / kGroup;  // 128-K units per row (a multiple of 4)
     p.cc_tokens = 1;
     p.nt = 1;
     p.row_tiles = (int)ceil_div(N, kRowsPerCta);
-    const int64_t units = (int64_t)p.row_tiles * G;
     int occ = group == 64 ? occupancy_sub<64>() : occupancy_sub<32>();
     if (occ < 1) occ = 1;
-    int64_t grid = (int64_t)occ * num_sms;
-    if (grid > units) grid = units;
-    p.grid = (int)grid;
-    p.units_base = (int)(units / grid);
-    p.units_rem = (int)(units % grid);
-    p.max_slots = (int)((G - 1) / p.units_base + 2);
+    const int64_t grid = (int64_t)occ * num_sms;
+    // chunks of 4 units where every CTA streams 12 or more units, else of 2 (groups of 32: always 4)
+    p.cc_units = (group == 32 || (int64_t)p.row_tiles * G >= 12 * grid) ? 4 : 2;
+    p.cc_cpt = (int)(G / p.cc_units);
+    p.cc_chunks = p.row_tiles * p.cc_cpt;
+    p.grid = (int)(grid < p.cc_chunks ? grid : p.cc_chunks);
     p.ws_xp_bytes = 0;
     p.ws_xs_bytes = 0;
-    p.ws_partial_bytes = align256((size_t)p.row_tiles * p.max_slots * kRowsPerCta * 4);
-    p.ws_counter_bytes = align256((size_t)(p.row_tiles > kSharedCounterTiles ? p.row_tiles : kSharedCounterTiles) * 4);
+    p.ws_partial_bytes = align256((size_t)p.cc_chunks * kRowsPerCta * 4);
+    p.ws_counter_bytes = kCounterBytes;  // counters[0] is the chunk counter
     return p;
 }
 
 template <int GS>
-int launch_sub(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& tze, const DecodeArgs& args, int grid,
+int launch_sub(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& tze, const SubArgs& args, int grid,
                cudaStream_t stream) {
     if (occupancy_sub<GS>() < 1) return W4A16_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
@@ -459,24 +446,21 @@ int launch_decode_sub(const uint16_t* X, int64_t M, int64_t K, int group, const 
     int* fault = fault_word();
     if (!fault) return W4A16_ERR_CUDA;
     char* ws = reinterpret_cast<char*>(workspace);
-    DecodeArgs args{};
-    args.scales = scales;
-    args.zeros = zeros;
+    SubArgs args{};
     args.partial = reinterpret_cast<float*>(ws + plan.ws_counter_bytes);
     args.counters = reinterpret_cast<int*>(ws);
     args.fault = fault;
-    args.M = 1;
     args.N = (int)N;
-    args.K = (int)K;
     args.G = (int)(K / kGroup);
-    args.units_base = plan.units_base;
-    args.units_rem = plan.units_rem;
-    args.max_slots = plan.max_slots;
-    for (int64_t m = 0; m < M; ++m) {  // one token per launch
+    args.U = plan.cc_units;
+    args.cpt = plan.cc_cpt;
+    args.chunks = plan.cc_chunks;
+    for (int64_t m = 0; m < M; ++m) {  // one token per launch, then its chunk sums
         args.Xp = X + m * K;
-        args.Y = Y + m * N;
-        const int st = group == 64 ? launch_sub<64>(tq, tsc, tze, args, plan.grid, stream)
-                                   : launch_sub<32>(tq, tsc, tze, args, plan.grid, stream);
+        int st = group == 64 ? launch_sub<64>(tq, tsc, tze, args, plan.grid, stream)
+                             : launch_sub<32>(tq, tsc, tze, args, plan.grid, stream);
+        if (st != W4A16_OK) return st;
+        st = launch_cc_reduce(args.partial, Y + m * N, N, plan.cc_cpt, plan.row_tiles, stream);
         if (st != W4A16_OK) return st;
     }
     return W4A16_OK;
