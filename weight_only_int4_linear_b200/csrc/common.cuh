@@ -153,6 +153,8 @@ struct DecodePlan {
     int max_slots;    // partial-sum slots per row tile
     int cc_units;     // one-token kernel: units (quantisation groups) per chunk, 2 or 4
     int cc_cpt;       // one-token kernel: chunks per row tile (quantisation groups / cc_units)
+    int cc_tiles_a;   // one-token kernel: row tiles in chunks of cc_units; the rest in chunks of 2
+    int cc_chunks_a;  // one-token kernel: chunks of the first cc_tiles_a row tiles
     int cc_chunks;    // one-token kernel: chunks in all
     // workspace layout: [counters][Xp][xs][partials]
     size_t ws_counter_bytes, ws_xp_bytes, ws_xs_bytes, ws_partial_bytes;
@@ -178,8 +180,9 @@ int launch_decode_bf(const uint16_t* X, const float* xscale, int64_t M, int64_t 
 
 // Chunk sums of the one-token GEMVs (gemv.cu, gemv_sub.cu): partial [row_tiles][cpt][128] -> Y [N] (and Y_host
 // when given: a mapped host buffer), each row's slots added in slot order; a dependent launch.
+// tiles_a >= 0: row tiles from tiles_a on hold cpt_b slots each, after the first tiles_a * cpt slots.
 int launch_cc_reduce(const float* partial, uint16_t* Y, int64_t N, int cpt, int row_tiles, cudaStream_t stream,
-                     uint16_t* Y_host = nullptr);
+                     uint16_t* Y_host = nullptr, int tiles_a = -1, int cpt_b = 0);
 // Split-K reduction of the decode GEMVs (gemv.cu): a dependent grid of one CTA per 128-row tile that
 // adds the partial-sum slots of every tile the GEMV's CTAs shared, in slot order, into Y.
 int launch_decode_reduce(const float* partial, uint16_t* Y, int64_t N, int M, int G, int units_base, int units_rem,

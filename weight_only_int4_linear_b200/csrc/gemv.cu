@@ -541,7 +541,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 // A unit is 128 rows x one group (8 KB of codes).  Units are dealt out in
 // chunks of U consecutive groups of one row tile (U = 4, or 2 where the CTAs
 // have fewer than 12 units each): chunk c is row tile c / cpt, groups
-// U (c % cpt) onwards (cpt = G / U chunks per row tile).  CTA b takes chunk b first, then asks a global counter for the
+// U (c % cpt) onwards (cpt = G / U chunks per row tile); with U = 4 the last
+// row tiles (about two chunks per CTA) are cut into chunks of 2, so that the
+// chunks drawn last are short.  A chunk's partial sums go to slot c.  CTA b takes chunk b first, then asks a global counter for the
 // next free chunk while it issues the current one, so a CTA that starts early
 // or streams fast takes more chunks and every CTA finishes within about a
 // chunk of the others.  (An equal, static deal left the CTAs that started
@@ -603,8 +605,9 @@ struct CcArgs {
     int* counters;      // counters[row_tiles]: the chunk counter (the row tiles' own counters stay unused)
     int* fault;
     int N, G;           // G: groups per row (a multiple of 8)
-    int U;              // units per chunk (2 or 4)
-    int cpt, chunks;    // chunks per row tile (G / U), chunks in all
+    int U;              // units per chunk in row tiles [0, tiles_a) (2 or 4); 2 in the tiles after them
+    int cpt, chunks;    // chunks per row tile (G / U) in the first region, chunks in all
+    int tiles_a, chunks_a;  // row tiles and chunks of the first region (chunk c is slot c of the partials)
     int row_tiles;
 };
 
@@ -687,7 +690,8 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-aligned (the swizzle's span)
     unsigned char* meta = ring + kCcMetaOff;
     // descriptor flags: first unit of its chunk, last unit of its chunk, end of the stream; metadata slot
-    constexpr int kFirst = 1, kLast = 2, kEnd = 4, kSlotShift = 4;
+    // and the chunk's unit count
+    constexpr int kFirst = 1, kLast = 2, kEnd = 4, kSlotShift = 4, kUnitsShift = 8;
 
     pdl_launch_dependents();  // the next call may start its weight loads as this grid's CTAs retire
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -712,17 +716,29 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
             int i = 0, nchunks = 0;  // units and chunks issued
             bool ok = true;
             auto issue_chunk = [&](int c) {
-                const int tile = c / a.cpt, k = c - tile * a.cpt;
+                // chunk c: U units of one row tile; the row tiles from tiles_a on are cut into chunks of 2
+                int tile, U, g0;
+                if (c < a.chunks_a) {
+                    tile = c / a.cpt;
+                    U = a.U;
+                    g0 = (c - tile * a.cpt) * U;
+                } else {
+                    const int cb = c - a.chunks_a, cpt_b = a.G / 2;
+                    tile = a.tiles_a + cb / cpt_b;
+                    U = 2;
+                    g0 = (cb - (tile - a.tiles_a) * cpt_b) * 2;
+                }
                 const int mslot = nchunks++ % kCcMetaSlots;
-                for (int u = 0; u < a.U; ++u, ++i) {
+                for (int u = 0; u < U; ++u, ++i) {
                     const int s = i % kCcStages;
                     if (i >= kCcStages && !mbar_wait(&empty[s], ((i / kCcStages) - 1) & 1, a.fault, 51)) {
                         ok = false;
                         return;
                     }
-                    const int g = k * a.U + u;
-                    s_desc[s] = make_int4(tile, g, k,
-                                          (u == 0 ? kFirst : 0) | (u + 1 == a.U ? kLast : 0) | (mslot << kSlotShift));
+                    const int g = g0 + u;
+                    s_desc[s] = make_int4(tile, g, c,
+                                          (u == 0 ? kFirst : 0) | (u + 1 == U ? kLast : 0) | (mslot << kSlotShift) |
+                                              (U << kUnitsShift));
                     mbar_arrive(&dready[s]);
                     unsigned char* st = ring + s * kCcStageBytes;
                     mbar_arrive_expect_tx(&full[s], kCcCodeBytes + (u == 0 ? kCcMetaBytes : 0));
@@ -773,12 +789,13 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
             if (!warp_wait(&dready[s], (i / kCcStages) & 1, a.fault, 54)) break;
             const int4 d = s_desc[s];
             if (!(d.w & kEnd)) {
+                const int U = (d.w >> kUnitsShift) & 7;
                 if (d.w & kFirst) {
 #pragma unroll
                     for (int j = 0; j < kCcChunkMax; ++j)
-                        if (j < a.U) xq[j] = load_group_x(a.X, d.y + j, lane);
+                        if (j < U) xq[j] = load_group_x(a.X, d.y + j, lane);
                 }
-                const int u = d.y & (a.U - 1);
+                const int u = d.y & (U - 1);
                 uint2 v = xq[0];
 #pragma unroll
                 for (int j = 1; j < kCcChunkMax; ++j)
@@ -874,7 +891,7 @@ __global__ void __launch_bounds__(kCcThreads, kCcMinBlocks) decode_cc_kernel(con
         y = fmaf(sv * fmaf(-zv, xsum, qx), xscale, y);
 
         if (d.w & kLast) {  // the chunk's sums leave through its slot (decode_cc_reduce_kernel adds them)
-            a.partial[((int64_t)d.x * a.cpt + d.z) * kRowsPerCta + r_own] = y;
+            a.partial[(int64_t)d.z * kRowsPerCta + r_own] = y;  // slot = chunk index
             y = 0.f;
         }
     }
@@ -902,20 +919,24 @@ constexpr int kCcRedLoads = 32;
 __global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_kernel(const float* __restrict__ partial,
                                                                                      uint16_t* __restrict__ Y, int N,
                                                                                      int cpt, int row_tiles,
-                                                                                     uint16_t* __restrict__ Yh) {
+                                                                                     uint16_t* __restrict__ Yh,
+                                                                                     int tiles_a, int cpt_b) {
     __shared__ float s_part[kCcRedParts - 1][kRowsPerCta];
     pdl_launch_dependents();
     pdl_wait_primary();
     const int r = threadIdx.x % kRowsPerCta, p = threadIdx.x / kRowsPerCta;
     for (int tile = blockIdx.x; tile < row_tiles; tile += gridDim.x) {
-        const float* pb = partial + (int64_t)tile * cpt * kRowsPerCta + r;
+        // the tile's slots: cpt from tile * cpt in the first region, cpt_b after the first region's
+        const int64_t first = tile < tiles_a ? (int64_t)tile * cpt : (int64_t)tiles_a * cpt + (int64_t)(tile - tiles_a) * cpt_b;
+        const int nslots = tile < tiles_a ? cpt : cpt_b;
+        const float* pb = partial + first * kRowsPerCta + r;
         float acc = 0.f;
-        for (int k0 = p; k0 < cpt; k0 += kCcRedLoads * kCcRedParts) {
+        for (int k0 = p; k0 < nslots; k0 += kCcRedLoads * kCcRedParts) {
             float v[kCcRedLoads];
 #pragma unroll
             for (int e = 0; e < kCcRedLoads; ++e) {
                 const int k = k0 + e * kCcRedParts;
-                v[e] = k < cpt ? __ldcg(pb + (int64_t)k * kRowsPerCta) : 0.f;
+                v[e] = k < nslots ? __ldcg(pb + (int64_t)k * kRowsPerCta) : 0.f;
             }
 #pragma unroll
             for (int e = 0; e < kCcRedLoads; ++e) acc += v[e];
@@ -1111,7 +1132,16 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
         // chunks of 4 units where every CTA streams 12 or more units, else of 2 (finer sharing)
         p.cc_units = (int64_t)p.row_tiles * G >= 12 * grid ? 4 : 2;
         p.cc_cpt = (int)(G / p.cc_units);
-        p.cc_chunks = p.row_tiles * p.cc_cpt;
+        // with chunks of 4, the last row tiles (about two chunks of 2 per CTA) are cut into chunks of 2, so
+        // that the CTAs' last chunks are short and they finish closer together
+        int tiles_b = 0;
+        if (p.cc_units == 4) {
+            tiles_b = (int)ceil_div(4 * grid, G);
+            if (tiles_b > p.row_tiles / 2) tiles_b = p.row_tiles / 2;
+        }
+        p.cc_tiles_a = p.row_tiles - tiles_b;
+        p.cc_chunks_a = p.cc_tiles_a * p.cc_cpt;
+        p.cc_chunks = p.cc_chunks_a + tiles_b * (int)(G / 2);
         p.grid = (int)(grid < p.cc_chunks ? grid : p.cc_chunks);
         p.ws_xp_bytes = align256((size_t)M * K * 2);  // X' = bf16(X * xscale) for the AWQ entry
         p.ws_xs_bytes = 0;
@@ -1229,16 +1259,19 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
     args.U = plan.cc_units;
     args.cpt = plan.cc_cpt;
     args.chunks = plan.cc_chunks;
+    args.tiles_a = plan.cc_tiles_a;
+    args.chunks_a = plan.cc_chunks_a;
     args.row_tiles = plan.row_tiles;
     const int st = launch_cc(tq, tsc, tze, args, plan.grid, stream);
     if (st != W4A16_OK) return st;
-    return launch_cc_reduce(args.partial, Y, N, plan.cc_cpt, plan.row_tiles, stream, Y_host);
+    return launch_cc_reduce(args.partial, Y, N, plan.cc_cpt, plan.row_tiles, stream, Y_host, plan.cc_tiles_a,
+                            G / 2);
 }
 
 }  // namespace
 
 int launch_cc_reduce(const float* partial, uint16_t* Y, int64_t N, int cpt, int row_tiles, cudaStream_t stream,
-                     uint16_t* Y_host) {
+                     uint16_t* Y_host, int tiles_a, int cpt_b) {
     const int sms = num_sms_current();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(row_tiles < sms ? row_tiles : sms));
@@ -1249,7 +1282,9 @@ int launch_cc_reduce(const float* partial, uint16_t* Y, int64_t N, int cpt, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, partial, Y, (int)N, cpt, row_tiles, Y_host) == cudaSuccess
+    if (tiles_a < 0) tiles_a = row_tiles;  // one region
+    return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, partial, Y, (int)N, cpt, row_tiles, Y_host, tiles_a,
+                              cpt_b) == cudaSuccess
                ? W4A16_OK
                : W4A16_ERR_CUDA;
 }
