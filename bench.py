@@ -43,10 +43,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 143392768 + dram__bytes_write.sum 4161024
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 143394048 + dram__bytes_write.sum 4007936
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "0856580ddb8b3611d54a03d1baf9dec6650626f2e4d82b0e76c0cb1f3c8d93bc",
-                                      "bytes": 147553792},
+                                      "sha256": "a36ce49bcd77d739e40a6d2a74a0f28d59706ecbc13794c556f1dad1543ff49c",
+                                      "bytes": 147401984},
     # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1110334976 + write 453940736
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
                                           "sha256": "d4c1912d8becaa47d896b612c0d94f643d9e1e0a739372ec447659743f2ea05d",

@@ -911,31 +911,35 @@ __global__ void __launch_bounds__(256) h2d_copy_kernel(const uint4* __restrict__
 
 // Split-K sums of the one-token kernel: Y[n] = the sum of row n's chunk slots in slot order.  A
 // dependent grid: its CTAs become resident beside the GEMV's (256 threads of at most 32 registers fit next
-// to four GEMV CTAs) and wait for it to complete.  Per row tile, 128 x P threads: part p adds slots p,
-// p + P, ... of its row (at most 32 loads in flight per thread, so one L2 round trip serves tiles of up to
-// 32 P chunks), then part 0 adds the P part sums in order.
-constexpr int kCcRedParts = 2;
+// to four GEMV CTAs) and wait for it to complete.  An item is 256 / P rows of a row tile, P threads per
+// row: part p adds slots p, p + P, ... of its row (at most 32 loads in flight per thread, so one L2 round
+// trip serves tiles of up to 32 P chunks), then part 0 adds the P part sums in order.  P = 2 (whole row
+// tiles) unless a tile has more than 64 slots, then P = 4 (half tiles).
+constexpr int kCcRedThreads = 256;
 constexpr int kCcRedLoads = 32;
-__global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_kernel(const float* __restrict__ partial,
-                                                                                     uint16_t* __restrict__ Y, int N,
-                                                                                     int cpt, int row_tiles,
-                                                                                     uint16_t* __restrict__ Yh,
-                                                                                     int tiles_a, int cpt_b) {
-    __shared__ float s_part[kCcRedParts - 1][kRowsPerCta];
+template <int P>
+__global__ void __launch_bounds__(kCcRedThreads) decode_cc_reduce_kernel(const float* __restrict__ partial,
+                                                                          uint16_t* __restrict__ Y, int N, int cpt,
+                                                                          int row_tiles, uint16_t* __restrict__ Yh,
+                                                                          int tiles_a, int cpt_b) {
+    constexpr int R = kCcRedThreads / P;   // rows per item
+    constexpr int SUBT = kRowsPerCta / R;  // items per row tile
+    __shared__ float s_part[P - 1][R];
     pdl_launch_dependents();
     pdl_wait_primary();
-    const int r = threadIdx.x % kRowsPerCta, p = threadIdx.x / kRowsPerCta;
-    for (int tile = blockIdx.x; tile < row_tiles; tile += gridDim.x) {
+    const int r = threadIdx.x % R, p = threadIdx.x / R;
+    for (int item = blockIdx.x; item < row_tiles * SUBT; item += gridDim.x) {
+        const int tile = item / SUBT, row = (item % SUBT) * R + r;
         // the tile's slots: cpt from tile * cpt in the first region, cpt_b after the first region's
         const int64_t first = tile < tiles_a ? (int64_t)tile * cpt : (int64_t)tiles_a * cpt + (int64_t)(tile - tiles_a) * cpt_b;
         const int nslots = tile < tiles_a ? cpt : cpt_b;
-        const float* pb = partial + first * kRowsPerCta + r;
+        const float* pb = partial + first * kRowsPerCta + row;
         float acc = 0.f;
-        for (int k0 = p; k0 < nslots; k0 += kCcRedLoads * kCcRedParts) {
+        for (int k0 = p; k0 < nslots; k0 += kCcRedLoads * P) {
             float v[kCcRedLoads];
 #pragma unroll
             for (int e = 0; e < kCcRedLoads; ++e) {
-                const int k = k0 + e * kCcRedParts;
+                const int k = k0 + e * P;
                 v[e] = k < nslots ? __ldcg(pb + (int64_t)k * kRowsPerCta) : 0.f;
             }
 #pragma unroll
@@ -945,8 +949,8 @@ __global__ void __launch_bounds__(kRowsPerCta * kCcRedParts) decode_cc_reduce_ke
         __syncthreads();
         if (p == 0) {
 #pragma unroll
-            for (int q = 0; q < kCcRedParts - 1; ++q) acc += s_part[q][r];
-            const int n = tile * kRowsPerCta + r;
+            for (int q = 0; q < P - 1; ++q) acc += s_part[q][r];
+            const int n = tile * kRowsPerCta + row;
             if (n < N) {
                 const uint16_t yb = float_to_bf16_bits(acc);
                 Y[n] = yb;
@@ -1273,20 +1277,25 @@ int launch_cc_path(const uint16_t* X, const float* xscale, int64_t K, const uint
 int launch_cc_reduce(const float* partial, uint16_t* Y, int64_t N, int cpt, int row_tiles, cudaStream_t stream,
                      uint16_t* Y_host, int tiles_a, int cpt_b) {
     const int sms = num_sms_current();
+    if (tiles_a < 0) tiles_a = row_tiles;  // one region
+    // four parts where a tile has more slots than two parts load in one round trip; at most one CTA per SM
+    // (more would take the places that the next call's GEMV CTAs start in)
+    const bool four = (cpt > cpt_b ? cpt : cpt_b) > 2 * kCcRedLoads;
+    const int64_t items = (int64_t)row_tiles * (four ? 2 : 1);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(row_tiles < sms ? row_tiles : sms));
-    cfg.blockDim = dim3(kRowsPerCta * kCcRedParts);
+    cfg.gridDim = dim3((unsigned)(items < sms ? items : sms));
+    cfg.blockDim = dim3(kCcRedThreads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (tiles_a < 0) tiles_a = row_tiles;  // one region
-    return cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel, partial, Y, (int)N, cpt, row_tiles, Y_host, tiles_a,
-                              cpt_b) == cudaSuccess
-               ? W4A16_OK
-               : W4A16_ERR_CUDA;
+    const cudaError_t e = four ? cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel<4>, partial, Y, (int)N, cpt,
+                                                    row_tiles, Y_host, tiles_a, cpt_b)
+                               : cudaLaunchKernelEx(&cfg, decode_cc_reduce_kernel<2>, partial, Y, (int)N, cpt,
+                                                    row_tiles, Y_host, tiles_a, cpt_b);
+    return e == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
 int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, const uint32_t* qweight,
