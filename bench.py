@@ -47,10 +47,10 @@ NCU_TRAFFIC = {
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
                                       "sha256": "a36ce49bcd77d739e40a6d2a74a0f28d59706ecbc13794c556f1dad1543ff49c",
                                       "bytes": 147401984},
-    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1110334976 + write 453940736
+    # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1108846080 + write 454347264
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
-                                          "sha256": "d4c1912d8becaa47d896b612c0d94f643d9e1e0a739372ec447659743f2ea05d",
-                                          "bytes": 1564275712},
+                                          "sha256": "6e2f2daa7ddb04a9b7ae69d75359c9f4f41576d570171e6775945c9328b4e6e0",
+                                          "bytes": 1563193344},
 }
 
 

@@ -1,5 +1,6 @@
 """The one-token GEMV deals out its work in chunks of 2 or 4 quantisation groups of a 128-row tile, taken
-from a counter in the workspace, and a dependent kernel adds each tile's chunk sums in slot order.
+from a counter in the workspace, and a dependent kernel adds each tile's chunk sums in slot order (two
+parts per row over whole tiles, or four over half tiles where a tile has more than 64 chunks).
 
 Checked here: outputs against the FP64 oracle for both chunk sizes (4 where every CTA streams 12 or more
 units, else 2) and ragged last row tiles; the same bits on every call whichever
@@ -37,7 +38,9 @@ def _oracle_rows(N, K, seed, X, rows):
 @pytest.mark.parametrize("N,K", [(300, 1024),     # 3 row tiles, the last of 44 rows; 8 groups per row
                                  (129, 1024),     # a one-row last tile
                                  (4096, 4096),    # 1024 units: chunks of 2
-                                 (8192, 16384)])  # 8192 units: chunks of 4 on a 148-SM part
+                                 (8192, 16384),   # 8192 units: chunks of 4 on a 148-SM part
+                                 (300, 32768)])   # 128 chunks per tile: the reduction's four parts per row
+                                                  # over half tiles, the last half tile past N
 def test_chunked_one_token_gemv(cuda_lib, N, K):
     seed = 7 + N + K
     pw = _packed(N, K, seed)
