@@ -89,13 +89,25 @@ struct DecodeArgs {
 // the MMAs, 13 drives TMA.  Rings:
 // shared-memory stages (codes, X planes, per token X sums and scales), 4 A
 // buffers and 8 (NTOK = 16) or 4 (NTOK = 32) accumulators, each with a
-// full/free mbarrier pair.
+// full/free mbarrier pair, and (K / 128 a multiple of 8) three slots of
+// scale and zero-point blocks that TMA fills with the codes (per-row loads
+// of the fold warps otherwise: 9-12 % slower on 24 and 32 tokens).
 
 // X planes of one launch, prepared by prep_x8_kernel: for group g, row
 // p NTOK + m of the B tile holds digit plane p of token m (128 bytes, MMA K
 // order); xs holds per group [sum_k x_int (FP32) for each token, then
 // 2^(E - 21) for each token].
-template <int NTOK>
+// Scales and zero points: with TM (K / 128 a multiple of 8, so that their
+// rows are 16-byte aligned) TMA brings them with the codes, in blocks of 8
+// groups x 128 rows (2 KB of BF16 scales, then 4 KB of int32 zero points),
+// into a ring of kMetaSlots shared-memory slots: block b of a CTA's range
+// goes to slot b % kMetaSlots with the first unit of the block; otherwise
+// the fold warps load their rows' values from global memory, a few units
+// ahead.
+constexpr int kTcMetaGroups = 8;
+constexpr int kTcScBytes = 128 * kTcMetaGroups * 2;
+constexpr int kTcMetaBytes = kTcScBytes + 128 * kTcMetaGroups * 4;  // 6 KB
+template <int NTOK, bool TM>
 struct TcCfg {
     static constexpr int kBRows = 3 * NTOK;                  // MMA N
     static constexpr int kBBytes = kBRows * 128;             // one group of K, 128-byte swizzle
@@ -103,8 +115,14 @@ struct TcCfg {
     static constexpr int kXsOff = kCodeOff + kStageWords * 4;
     static constexpr int kXsBytes = 2 * NTOK * 4;
     static constexpr int kStageBytes = (kXsOff + kXsBytes + 1023) & ~1023;
-    static constexpr int kStages = (220 * 1024) / kStageBytes;
-    static constexpr size_t kSmem = (size_t)kStages * kStageBytes + 1024;  // + alignment slack
+    static constexpr int kMetaSlots = TM ? 3 : 0;
+    static constexpr int kStages = (220 * 1024 - kMetaSlots * kTcMetaBytes) / kStageBytes;
+    static constexpr int kMetaOff = kStages * kStageBytes;
+    static constexpr size_t kSmem = (size_t)kMetaOff + (size_t)kMetaSlots * kTcMetaBytes + 1024;  // + alignment slack
+    // A block's slot is rewritten kMetaSlots blocks later, with the first unit of that block; the blocks in
+    // between hold 8 units each (blocks are aligned to 8 groups inside a row tile), and the TMA thread issues
+    // a unit only once the fold is done with the unit kStages back.
+    static_assert(!TM || 8 * (kMetaSlots - 1) >= kStages - 1, "metadata slot reuse");
     static constexpr uint32_t kTmemCols = 512;
     static constexpr int kACols = 32;                        // 128 rows x 128 bytes
     static constexpr int kNumA = 4;                          // A buffers at 0..127
@@ -204,11 +222,14 @@ constexpr int kMmaWarp = kFoldWarps + kDqWarps;  // 12
 constexpr int kTmaWarp = kMmaWarp + 1;           // 13
 constexpr int kTcThreads = (kTmaWarp + 1) * 32;  // 448
 
-template <int NTOK>
+template <int NTOK, bool TM>
 __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_constant__ CUtensorMap tq,
                                                                   const __grid_constant__ CUtensorMap tx,
+                                                                  const __grid_constant__ CUtensorMap tsc,
+                                                                  const __grid_constant__ CUtensorMap tze,
                                                                   const DecodeArgs a) {
-    using C = TcCfg<NTOK>;
+    using C = TcCfg<NTOK, TM>;
+    constexpr int NS = C::kMetaSlots;
     constexpr int S = C::kStages;
     constexpr int NA = C::kNumA, ND = C::kNumD;
     constexpr uint32_t kIdesc = idesc_u8s8_s32(128, C::kBRows);
@@ -221,6 +242,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
 
     const uint32_t raw = smem_u32(smem_raw);
     unsigned char* ring = smem_raw + ((1024u - (raw & 1023u)) & 1023u);  // 1024-aligned stages
+    unsigned char* meta = ring + C::kMetaOff;                                // NS metadata slots (TM)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.x;
@@ -257,15 +279,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         if (lane == 0) {
             prefetch_tmap(&tq);
             prefetch_tmap(&tx);
+            if constexpr (TM) {
+                prefetch_tmap(&tsc);
+                prefetch_tmap(&tze);
+            }
             constexpr uint32_t kTx = C::kBBytes + kStageWords * 4 + C::kXsBytes;
             const int pre = min(S, nunits);
+            int mb = -1;  // metadata blocks started (TM)
+            // codes of unit i into stage s and, with the first unit of a block of 8 groups, the block's scales
+            // and zero points into slot mb % NS
+            auto codes_meta = [&](int i, int s, const UnitCursor& c) {
+                const bool new_block = TM && (i == 0 || (c.g & (kTcMetaGroups - 1)) == 0);
+                if (new_block) ++mb;
+                mbar_arrive_expect_tx(&full[s], kTx + (new_block ? kTcMetaBytes : 0));
+                tma_load_2d(ring + s * C::kStageBytes + C::kCodeOff, &tq, c.g * kWordsPerGroup, c.tile * kRowsPerCta,
+                            &full[s]);
+                if constexpr (TM) {
+                    if (new_block) {
+                        unsigned char* ms = meta + (mb % NS) * kTcMetaBytes;
+                        const int g8 = c.g & ~(kTcMetaGroups - 1);
+                        tma_load_2d(ms, &tsc, g8, c.tile * kRowsPerCta, &full[s]);
+                        tma_load_2d(ms + kTcScBytes, &tze, g8, c.tile * kRowsPerCta, &full[s]);
+                    }
+                }
+            };
             // the weights do not depend on the preparation kernel: start streaming them at once
             UnitCursor cur(u_first, G);
-            for (int i = 0; i < pre; ++i, cur.next(G)) {
-                mbar_arrive_expect_tx(&full[i], kTx);
-                tma_load_2d(ring + i * C::kStageBytes + C::kCodeOff, &tq, cur.g * kWordsPerGroup,
-                            cur.tile * kRowsPerCta, &full[i]);
-            }
+            for (int i = 0; i < pre; ++i, cur.next(G)) codes_meta(i, i, cur);
             pdl_wait_primary();  // X planes come from the preparation kernel
             UnitCursor cx(u_first, G);
             for (int i = 0; i < pre; ++i, cx.next(G)) {
@@ -278,10 +318,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             for (int i = pre; i < nunits; ++i, cur.next(G)) {
                 const int s = i % S;
                 if (!mbar_wait(&empty[s], ((i / S) - 1) & 1, a.fault, 21)) break;
-                const int tile = cur.tile, g = cur.g;
+                const int g = cur.g;
                 unsigned char* st = ring + s * C::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], kTx);
-                tma_load_2d(st + C::kCodeOff, &tq, g * kWordsPerGroup, tile * kRowsPerCta, &full[s]);
+                codes_meta(i, s, cur);
                 tma_load_2d(st, &tx, 0, g * C::kBRows, &full[s]);
                 bulk_load(st + C::kXsOff, a.xs + (int64_t)g * 2 * NTOK, C::kXsBytes, &full[s]);
                 ++issued;
@@ -421,7 +460,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         zraw = __ldg(a.zeros + (int64_t)n * G + g);
     };
 
-    auto fold_unit = [&](int j, int tile, float sv, float zv) {
+    // unit j of row tile `tile`; sv, zv: its scale and zero point, or (TM) read here from metadata slot
+    // `slot`, group g (the MMA waited for below was issued after the slot's copy landed; rows past N were
+    // zero-filled: s = 0)
+    auto fold_unit = [&](int j, int tile, float sv, float zv, int slot, int g) {
         while (cur_tile < tile) flush(cur_tile++);
         if (split_units && (j & 1) != th) return;  // the other warp of the quadrant folds this unit
         if (aborted) return;
@@ -431,6 +473,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             return;
         }
         tc_fence_after();
+        if constexpr (TM) {
+            const unsigned char* ms = meta + slot * kTcMetaBytes;
+            const int gb = g & (kTcMetaGroups - 1);
+            sv = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(ms + row_local * (kTcMetaGroups * 2) + 2 * gb));
+            zv = (float)*reinterpret_cast<const int32_t*>(ms + kTcScBytes + row_local * (kTcMetaGroups * 4) + 4 * gb);
+        }
         const float* xs = reinterpret_cast<const float*>(ring + s * C::kStageBytes + C::kXsOff);
         const uint32_t dcol = tl + C::kColD + di * C::kBRows + m_base;
         // integer -> FP32 by the 2^23 + 2^22 magic (exact for |v| < 2^22; every plane sum is)
@@ -466,29 +514,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         if (lane == 0) mbar_arrive(&empty[s]);  // X sums and scales read
     };
 
-    // metadata loads run kMetaAhead units ahead of the folds (scattered 2- and 4-byte loads of L2
-    // latency): unit j's scale and zero point live in slot j % kMetaAhead of a register ring
-    constexpr int kMetaAhead = 4;
-    UnitCursor fc(u_first, G), mc(u_first, G);
-    uint32_t sr[kMetaAhead];
-    int zr[kMetaAhead];
-#pragma unroll
-    for (int u = 0; u < kMetaAhead; ++u) {
-        load_meta(mc.tile, mc.g, sr[u], zr[u]);
-        mc.next(G);
-    }
-    for (int j0 = 0; j0 < nunits; j0 += kMetaAhead) {
+    if constexpr (TM) {
+        UnitCursor fc(u_first, G);
+        int mb = -1;  // metadata block of unit j, counted as the TMA thread counts them
+        for (int j = 0; j < nunits; ++j, fc.next(G)) {
+            if (j == 0 || (fc.g & (kTcMetaGroups - 1)) == 0) ++mb;
+            fold_unit(j, fc.tile, 0.f, 0.f, mb % NS, fc.g);
+        }
+    } else {
+        // metadata loads run kMetaAhead units ahead of the folds (scattered 2- and 4-byte loads of L2
+        // latency): unit j's scale and zero point live in slot j % kMetaAhead of a register ring
+        constexpr int kMetaAhead = 4;
+        UnitCursor fc(u_first, G), mc(u_first, G);
+        uint32_t sr[kMetaAhead];
+        int zr[kMetaAhead];
 #pragma unroll
         for (int u = 0; u < kMetaAhead; ++u) {
-            const int j = j0 + u;
-            if (j < nunits) {
-                const bool row_ok = fc.tile * kRowsPerCta + row_local < N;
-                const float sv = row_ok ? bf16_bits_to_float((uint16_t)sr[u]) : 0.f;
-                const float zv = (float)zr[u];
-                load_meta(mc.tile, mc.g, sr[u], zr[u]);
-                mc.next(G);
-                fold_unit(j, fc.tile, sv, zv);
-                fc.next(G);
+            load_meta(mc.tile, mc.g, sr[u], zr[u]);
+            mc.next(G);
+        }
+        for (int j0 = 0; j0 < nunits; j0 += kMetaAhead) {
+#pragma unroll
+            for (int u = 0; u < kMetaAhead; ++u) {
+                const int j = j0 + u;
+                if (j < nunits) {
+                    const bool row_ok = fc.tile * kRowsPerCta + row_local < N;
+                    const float sv = row_ok ? bf16_bits_to_float((uint16_t)sr[u]) : 0.f;
+                    const float zv = (float)zr[u];
+                    load_meta(mc.tile, mc.g, sr[u], zr[u]);
+                    mc.next(G);
+                    fold_unit(j, fc.tile, sv, zv, 0, 0);
+                    fc.next(G);
+                }
             }
         }
     }
@@ -966,12 +1023,14 @@ template <int NTOK>
 int occupancy_nt() {
     static PerContext<int> cache;  // the attribute belongs to a context
     return cache.get([]() -> int {
-        if (cudaFuncSetAttribute(decode_tc_kernel<NTOK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)TcCfg<NTOK>::kSmem) != cudaSuccess)
+        if (cudaFuncSetAttribute(decode_tc_kernel<NTOK, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TcCfg<NTOK, false>::kSmem) != cudaSuccess ||
+            cudaFuncSetAttribute(decode_tc_kernel<NTOK, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TcCfg<NTOK, true>::kSmem) != cudaSuccess)
             return 0;
         int o = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_tc_kernel<NTOK>, kTcThreads,
-                                                          TcCfg<NTOK>::kSmem) != cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, decode_tc_kernel<NTOK, false>, kTcThreads,
+                                                          TcCfg<NTOK, false>::kSmem) != cudaSuccess ||
             o < 1)
             return 0;
         return 1;  // one CTA per SM: it owns all 512 TMEM columns
@@ -1051,19 +1110,23 @@ int launch_cc(const CUtensorMap& tq, const CUtensorMap& tsc, const CUtensorMap& 
     return cudaLaunchKernelEx(&cfg, decode_cc_kernel, tq, tsc, tze, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
 }
 
-template <int NTOK>
-int launch_tc(const CUtensorMap& tq, const CUtensorMap& tx, const DecodeArgs& args, int grid, cudaStream_t stream) {
+// tsc, tze: the scales' and zero points' tensor maps with TM (unused, any map, without)
+template <int NTOK, bool TM>
+int launch_tc(const CUtensorMap& tq, const CUtensorMap& tx, const CUtensorMap& tsc, const CUtensorMap& tze,
+              const DecodeArgs& args, int grid, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kTcThreads);
-    cfg.dynamicSmemBytes = TcCfg<NTOK>::kSmem;
+    cfg.dynamicSmemBytes = TcCfg<NTOK, TM>::kSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_tc_kernel<NTOK>, tq, tx, args) == cudaSuccess ? W4A16_OK : W4A16_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, decode_tc_kernel<NTOK, TM>, tq, tx, tsc, tze, args) == cudaSuccess
+               ? W4A16_OK
+               : W4A16_ERR_CUDA;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -1312,6 +1375,11 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
     if (X_host || Y_host) return W4A16_ERR_ARG;  // host-mapped transfers are the one-token path's
     CUtensorMap tq;
     if (!cached_tmap(0, qweight, N, K / 8, &tq)) return W4A16_ERR_CUDA;
+    const int G = (int)(K / kGroup);
+    // scales and zero points by TMA where their rows are 16-byte aligned (G % 8 == 0)
+    const bool tm = G % kTcMetaGroups == 0;
+    CUtensorMap tsc = tq, tze = tq;
+    if (tm && (!cached_tmap(2, scales, N, G, &tsc) || !cached_tmap(3, zeros, N, G, &tze))) return W4A16_ERR_CUDA;
     int* fault = fault_word();
     if (!fault) return W4A16_ERR_CUDA;
     char* ws = reinterpret_cast<char*>(workspace);
@@ -1319,7 +1387,6 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
     uint8_t* planes = reinterpret_cast<uint8_t*>(ws + plan.ws_counter_bytes);
     float* xs = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes);
     float* partial = reinterpret_cast<float*>(ws + plan.ws_counter_bytes + plan.ws_xp_bytes + plan.ws_xs_bytes);
-    const int G = (int)(K / kGroup);
     for (int64_t m0 = 0; m0 < M; m0 += kMaxTokens) {
         const int Mc = (int)((M - m0) < kMaxTokens ? (M - m0) : kMaxTokens);
         CUtensorMap tx;
@@ -1348,8 +1415,10 @@ int launch_decode(const uint16_t* X, const float* xscale, int64_t M, int64_t K, 
         args.units_base = plan.units_base;
         args.units_rem = plan.units_rem;
         args.max_slots = plan.max_slots;
-        const int st = plan.nt == 16 ? launch_tc<16>(tq, tx, args, plan.grid, stream)
-                                     : launch_tc<32>(tq, tx, args, plan.grid, stream);
+        const int st = plan.nt == 16 ? (tm ? launch_tc<16, true>(tq, tx, tsc, tze, args, plan.grid, stream)
+                                           : launch_tc<16, false>(tq, tx, tsc, tze, args, plan.grid, stream))
+                                     : (tm ? launch_tc<32, true>(tq, tx, tsc, tze, args, plan.grid, stream)
+                                           : launch_tc<32, false>(tq, tx, tsc, tze, args, plan.grid, stream));
         if (st != W4A16_OK) return st;
     }
     return W4A16_OK;
