@@ -43,10 +43,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 143392000 + dram__bytes_write.sum 3620864
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 143396352 + dram__bytes_write.sum 3670784
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "7149262b57b435f2f3e2b2cf1153ba3dac818e537cbbbde8b98e74996c7e460a",
-                                      "bytes": 147012864},
+                                      "sha256": "952fab591a4709739c161e413eb4a3aaef1ce6de829ee3159c7c41fbe8407e9a",
+                                      "bytes": 147067136},
     # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1108846080 + write 454347264
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
                                           "sha256": "6e2f2daa7ddb04a9b7ae69d75359c9f4f41576d570171e6775945c9328b4e6e0",

@@ -481,7 +481,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
         }
         const float* xs = reinterpret_cast<const float*>(ring + s * C::kStageBytes + C::kXsOff);
         const uint32_t dcol = tl + C::kColD + di * C::kBRows + m_base;
-        // integer -> FP32 by the 2^23 + 2^22 magic (exact for |v| < 2^22; every plane sum is)
+        // integer -> FP32 by the 2^23 + 2^22 magic (exact for |v| < 2^22; every plane sum is: 128 codes of at
+        // most 15 times digits of at most 128); the two low planes are first combined as the integer
+        // 256 D1 + D0 (|.| < 2^27) and converted once -- the same rounding as the FP32 fma(D1, 256, D0) of the
+        // exact plane values, one instruction for four
         auto to_f = [](uint32_t v) { return __int_as_float((int)v + 0x4B400000) - 12582912.f; };
 #pragma unroll
         for (int h = 0; h < TH / 8; ++h) {  // 8 tokens at a time: their three digit planes
@@ -506,7 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) decode_tc_kernel(const __grid_c
             for (int e = 0; e < 8; ++e) {
                 // sum q x_int = 65536 D2 + 256 D1 + D0; the power of two last, so that a group of
                 // tiny activations does not underflow in s 2^(E - 21)
-                const float qx = fmaf(to_f(d2[e]), 65536.f, fmaf(to_f(d1[e]), 256.f, to_f(d0[e])));
+                const float qx = fmaf(to_f(d2[e]), 65536.f, __int2float_rn((int)d1[e] * 256 + (int)d0[e]));
                 acc[h * 8 + e] = fmaf(sv * fmaf(-zv, xsum[e], qx), xsc[e], acc[h * 8 + e]);
             }
         }
