@@ -43,10 +43,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (summaries under profiles/).  A figure holds only for the kernel source it was taken on,
 # so each carries the sha256 of that source file; after any change it reads as null.
 NCU_TRAFFIC = {
-    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 143396352 + dram__bytes_write.sum 3670784
+    # python bench.py --profile decode:gate_up; dram__bytes_read.sum 143392512 + dram__bytes_write.sum 4034048
     ("decode_cc_kernel", "gate_up"): {"source": "weight_only_int4_linear_b200/csrc/gemv.cu",
-                                      "sha256": "952fab591a4709739c161e413eb4a3aaef1ce6de829ee3159c7c41fbe8407e9a",
-                                      "bytes": 147067136},
+                                      "sha256": "ab8e6f501913c473315e69ad4e443a993bcb8cd4dd825179dd595b891d690b0e",
+                                      "bytes": 147426560},
     # python bench.py --profile prefill:gate_up_m4096; dram__bytes_read.sum 1108846080 + write 454347264
     ("prefill_kernel", "gate_up_m4096"): {"source": "weight_only_int4_linear_b200/csrc/gemm.cu",
                                           "sha256": "6e2f2daa7ddb04a9b7ae69d75359c9f4f41576d570171e6775945c9328b4e6e0",

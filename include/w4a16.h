@@ -64,8 +64,8 @@ typedef enum {
 typedef enum {
     W4A16_PATH_AUTO = 0,    /* decode GEMV for small M, tensor-core GEMM for large M */
     W4A16_PATH_DECODE = 1,  /* split-K GEMVs, any M: integer mma.sync (codes x digit planes of X) for
-                               M <= 16, tcgen05 (8-bit, codes from tensor memory) for more, in chunks of
-                               32 tokens */
+                               M <= 16 when K / 128 is a multiple of 8, tcgen05 (8-bit, codes from tensor
+                               memory) otherwise, in chunks of 32 tokens */
     W4A16_PATH_PREFILL = 2  /* TMA + tcgen05/TMEM GEMM on BF16 tiles dequantised in shared memory */
 } w4a16_path;
 

@@ -63,7 +63,7 @@ def test_plane_sums_stay_exact_in_int32():
 
 
 # ---------------------------------------------------------------------------------------------
-# The same scheme as the GPU writes it: the 2-8-token integer GEMV prepares each launch's digit
+# The same scheme as the GPU writes it: the 2-16-token integer GEMV prepares each launch's digit
 # rows once, in its caller's workspace, and reads them back with bulk copies.  White-box check of
 # that preparation, bit for bit, against the host statement above: the workspace layout is
 # [256 KB of split-K counters][per group g: digit rows of 128 bytes, then (sum x_int, 2^(E - 21)) per

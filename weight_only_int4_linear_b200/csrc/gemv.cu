@@ -1,5 +1,5 @@
-// Decode path of the W4A16 linear layer: persistent split-K GEMV for small M
-// (up to 32 tokens per launch).
+// Decode path of the W4A16 linear layer: persistent split-K GEMVs for small M
+// (up to 32 tokens per launch; more in consecutive launches).
 //
 // Only the packed codes (0.5 byte per weight) and the per-group scale and zero
 // point cross the memory bus; each code is consumed on chip straight from its
@@ -14,12 +14,16 @@
 // The codes q stay unsigned bytes (w & 0x0F0F0F0F, (w >> 4) & 0x0F0F0F0F); x_int
 // is written as three signed base-256 digits, so sum_k q x_int is three exact
 // int32 dot products, combined and scaled in FP32 once per group.  The BF16 scale
-// is never folded into a rounded operand.  Three kernels:
+// is never folded into a rounded operand.  In this file:
 //   * M = 1: decode_cc_kernel, the dot products as mma.sync m16n8k32 (codes u8 x
-//     X digits s8) in the warps' registers, X prepared inside the kernel;
-//   * 3 <= M <= 32 per launch: decode_tc_kernel, tcgen05.mma kind::i8 with the
-//     codes in tensor memory and the digit planes of all tokens as B;
+//     X digits s8) in the warps' registers, X prepared inside the kernel, and
+//     decode_cc_reduce_kernel for its split-K sums;
+//   * 17 or more tokens (32 per launch), and any M when K / 128 is not a
+//     multiple of 8: decode_tc_kernel, tcgen05.mma kind::i8 with the codes in
+//     tensor memory and the digit planes of all tokens as B;
 //   * prep_x8_kernel: the digit planes for the tensor-core kernel.
+// 2-16 tokens run the register-MMA GEMV of gemv_mt.cu; groups of 32 and 64
+// run gemv_sub.cu (one token) and gemv_bf.cu (more).
 // With AWQ inverse channel scales (the activation half of the equivalence
 // transform), X' = bf16(x * inv_s[k]) is formed where X is prepared: inside
 // prep_x8_kernel, and for M = 1 by awq_prescale_kernel ahead of the integer
@@ -67,7 +71,8 @@ struct DecodeArgs {
 
 // --------------------------------------------------------------------------
 // Tensor-core decode kernel (tcgen05, 8-bit integer MMA), one persistent CTA
-// per SM, for 2 <= M <= 32 tokens per launch.
+// per SM, for up to 32 tokens per launch (17 or more tokens; any count when
+// K / 128 is not a multiple of 8).
 //
 // The codes are the A operand as unsigned bytes, exactly: per packed word,
 // w & 0x0F0F0F0F holds codes 0, 2, 4, 6 and (w >> 4) & 0x0F0F0F0F codes
@@ -1186,12 +1191,12 @@ DecodePlan plan_decode(int64_t M, int64_t N, int64_t K, int num_sms) {
     DecodePlan p{};
     const int64_t Mc = M < kMaxTokens ? M : kMaxTokens;
     const int64_t G = K / kGroup;
-    // the one-token integer kernel for M = 1 (needs 16-byte metadata rows: G % 8 == 0);
-    // else the tensor-core kernel with MMA N = 16 or 32
+    // the one-token integer kernel for M = 1 (needs 16-byte metadata rows: G % 8 == 0); the register-MMA
+    // GEMV of gemv_mt.cu for 2-16 tokens (same condition); else the 8-bit tensor-core GEMV below with MMA
+    // N = 3 x 16 or 3 x 32 (17 or more tokens, or K / 128 not a multiple of 8); the BF16 tensor-core GEMV
+    // (gemv_bf.cu) serves quantisation groups of 32 and 64
     p.cc_tokens = (M <= 1 && G % 8 == 0) ? (int)M : 0;
     p.mt = !p.cc_tokens && mt_supported(K) && M <= kMtMaxTokens;
-    // 9 or more tokens (or K / 128 not a multiple of 8): the 8-bit tensor-core GEMV below; the BF16
-    // tensor-core GEMV (gemv_bf.cu) serves quantisation groups of 32 and 64
     p.bf = false;
     p.nt = p.cc_tokens ? 1 : (Mc <= 16 ? 16 : 32);
     p.row_tiles = (int)ceil_div(N, kRowsPerCta);

@@ -1,5 +1,5 @@
-// Integer GEMV for 3 to 16 tokens per launch: the decode path between the
-// one- and two-token kernel and the GEMM ("Weight-Only Quantization and Mixed
+// Integer GEMV for 2 to 16 tokens per launch: the decode path between the
+// one-token kernel and the tensor-core GEMVs ("Weight-Only Quantization and Mixed
 // Precision", sections 1 and 5: decode stays bound by the weight stream for
 // small batches, so the packed codes are read once for every token of the
 // launch and nothing but codes and metadata crosses the memory bus).
