@@ -63,6 +63,85 @@ def test_plane_sums_stay_exact_in_int32():
 
 
 # ---------------------------------------------------------------------------------------------
+# The one-token GEMV's variant.  Its A operand takes the two halves of a packed word as bytes without a
+# shift: w & 0x0F0F0F0F holds codes 0, 2, 4, 6 of the word and w & 0xF0F0F0F0 holds 16 times codes 1, 3, 5, 7.
+# The activations of the odd codes (K odd) are therefore expressed with four fewer fractional bits,
+# x_int = rint(x 2^(17 - E)), those of the even codes as above, rint(x 2^(21 - E)), and the group's
+# represented dot product is 2^(E - 21) (sum_even q x_int + sum_odd 16 q x_int).  Claims checked here: the
+# odd values are exact within 2^10 of the group maximum and within half a step, 2^(E - 18), elsewhere; the
+# digits fit signed bytes and recompose; the plane sums (bytes of at most 240 against digits of at most
+# 128) stay below 2^22, the range in which the accumulators' bias 1.5 2^23 converts them exactly; and the
+# represented product differs from the exact one by no more than the half steps allow.
+
+
+def _one_token_ints(xb):
+    """xb: BF16 bits of one group -> (E, x, x_int) with the even/odd scalings of the one-token kernel."""
+    amax = int((xb & 0x7FFF).max())
+    ef = amax >> 7
+    E = -127 if ef == 0 else ef - 127
+    x = _bf16_to_f32(xb).astype(np.float64)
+    k = np.arange(x.size)
+    shift = np.where(k % 2 == 1, 17 - E, 21 - E)
+    xi = np.rint(np.ldexp(x, shift)).astype(np.int64)
+    return E, x, xi, k % 2 == 1
+
+
+def _balanced_digits(xi):
+    d0 = ((xi + 128) & 255) - 128
+    t = (xi - d0) >> 8
+    d1 = ((t + 128) & 255) - 128
+    d2 = (t - d1) >> 8
+    return d0, d1, d2
+
+
+def test_one_token_odd_codes_exact_within_2_10_and_half_step_elsewhere():
+    rng = np.random.default_rng(11)
+    for _ in range(500):
+        scale = 2.0 ** rng.integers(-30, 30)
+        x = rng.standard_normal(128) * scale * np.exp(rng.uniform(-12, 0, size=128))
+        xb = (x.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+        E, xv, xi, odd = _one_token_ints(xb)
+        rep = np.where(odd, np.ldexp(xi.astype(np.float64), E - 17), np.ldexp(xi.astype(np.float64), E - 21))
+        exact_odd = odd & (np.abs(xv) >= 2.0 ** (E - 10))
+        exact_even = ~odd & (np.abs(xv) >= 2.0 ** (E - 14))
+        np.testing.assert_array_equal(rep[exact_odd], xv[exact_odd])
+        np.testing.assert_array_equal(rep[exact_even], xv[exact_even])
+        assert np.all(np.abs(rep - xv)[odd] <= 2.0 ** (E - 18))
+        assert np.all(np.abs(rep - xv)[~odd] <= 2.0 ** (E - 22))
+
+
+def test_one_token_digits_and_plane_sums_on_edge_activations():
+    from synth import edge
+    kinds = list(edge.KINDS)
+    X = edge.activations_bf16(21, kinds, 1024)
+    rng = np.random.default_rng(12)
+    worst = 64 * 15 * 128 + 64 * 240 * 128  # even bytes q, odd bytes 16 q, digits of magnitude <= 128
+    assert worst < 2 ** 22
+    bias = np.float32(12582912.0)  # 1.5 2^23
+    for row in X:
+        for xb in row.reshape(-1, 128):
+            E, x, xi, odd = _one_token_ints(xb)
+            assert np.abs(xi[odd]).max(initial=0) < 2 ** 18 and np.abs(xi[~odd]).max(initial=0) < 2 ** 22
+            d0, d1, d2 = _balanced_digits(xi)
+            for d in (d0, d1, d2):
+                assert d.min() >= -128 and d.max() <= 127
+            np.testing.assert_array_equal(65536 * d2 + 256 * d1 + d0, xi)
+            q = rng.integers(0, 16, size=128)
+            a = np.where(odd, 16 * q, q)  # the A bytes
+            planes = [int((a * d).sum()) for d in (d0, d1, d2)]
+            for P in planes:
+                assert abs(P) <= worst
+                # the accumulator starts at the bits of 1.5 2^23 and ends as the FP32 number 1.5 2^23 + P
+                assert float(np.float32(bias + np.float32(P)) - bias) == P
+            # the integer identity the fold relies on, and the product within the half-step bound
+            assert 65536 * planes[2] + 256 * planes[1] + planes[0] == int((a * xi).sum())
+            represented = np.ldexp(float((a * xi).sum()), E - 21)
+            exact = float((q * x).sum())
+            bound = float((q[odd] * 2.0 ** (E - 18)).sum() + (q[~odd] * 2.0 ** (E - 22)).sum())
+            assert abs(represented - exact) <= bound + 1e-300
+
+
+# ---------------------------------------------------------------------------------------------
 # The same scheme as the GPU writes it: the 2-16-token integer GEMV prepares each launch's digit
 # rows once, in its caller's workspace, and reads them back with bulk copies.  White-box check of
 # that preparation, bit for bit, against the host statement above: the workspace layout is
